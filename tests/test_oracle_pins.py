@@ -1,0 +1,330 @@
+"""Pins for the CPU oracle: each test checks it against something other than itself.
+
+What the pages fix (Punica README, LoRA paragraph and multi-LoRA paragraph):
+the shapes A [H1, r], B [r, H2]; the identity x@(W + A@B) = x@W + x@A@B; the
+batched definition in which each row uses its own adapter. The pins below are:
+library conversions (numpy float16, torch bfloat16), a hand-worked example,
+exact rational arithmetic, one-hot closed forms, a dense numpy GEMM for the
+Identical distribution, and invariants of the segment semantics. Each is chosen
+so that a plausible slip in the oracle (a transposed operand, a wrong index, a
+dropped term, a sign) fails at least one of them.
+"""
+import json
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from adapter_matmul_b200 import inputs
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def f16_bits(vals):
+    return np.asarray(vals, dtype=np.float64).astype(np.float16).view(np.uint16)
+
+
+def dec(bits, dt):
+    """Independent decode through numpy / torch (not the oracle)."""
+    bits = np.ascontiguousarray(bits, dtype=np.uint16)
+    if dt == "f16":
+        return bits.view(np.float16).astype(np.float64)
+    return torch.from_numpy(bits.view(np.int16).copy()).view(torch.bfloat16).to(torch.float64).numpy()
+
+
+# ---------------------------------------------------------------------------------------------
+# storage conversions
+# ---------------------------------------------------------------------------------------------
+
+def test_f16_decode_all_patterns_match_numpy():
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    got = oracle.decode(bits, "f16")
+    ref = bits.view(np.float16).astype(np.float64)
+    assert np.array_equal(np.isnan(got), np.isnan(ref))
+    m = ~np.isnan(ref)
+    assert np.array_equal(got[m], ref[m])
+    assert np.array_equal(np.signbit(got[m]), np.signbit(ref[m]))
+
+
+def test_bf16_decode_all_patterns_match_torch():
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    got = oracle.decode(bits, "bf16")
+    ref = dec(bits, "bf16")
+    assert np.array_equal(np.isnan(got), np.isnan(ref))
+    m = ~np.isnan(ref)
+    assert np.array_equal(got[m], ref[m])
+    assert np.array_equal(np.signbit(got[m]), np.signbit(ref[m]))
+
+
+def _wide_doubles(n, seed):
+    rng = np.random.default_rng(seed)
+    mant = rng.random(n) * 2 - 1
+    expo = rng.integers(-30, 20, n)
+    v = np.ldexp(mant, expo)
+    extra = [0.0, -0.0, 65504.0, 65519.99, 65520.0, -65520.0, 1e9, 2.0 ** -24, 2.0 ** -25,
+             3 * 2.0 ** -26, 2.0 ** -14, 2.0 ** -14 * (1 - 2 ** -11), np.inf, -np.inf]
+    return np.concatenate([v, np.array(extra)])
+
+
+def test_f16_encode_matches_numpy_rne():
+    v = _wide_doubles(200000, 1)
+    got = oracle.encode(v, "f16")
+    with np.errstate(over="ignore"):
+        ref = v.astype(np.float16).view(np.uint16)  # numpy rounds binary64 -> binary16 to nearest even
+    assert np.array_equal(got, ref)
+
+
+def test_f16_encode_exact_ties_go_to_even():
+    # 1 + k*2^-10 + 2^-11 is exactly halfway between two fp16 neighbours
+    k = np.arange(0, 1024)
+    v = 1.0 + k * 2.0 ** -10 + 2.0 ** -11
+    got = oracle.decode(oracle.encode(v, "f16"), "f16")
+    even = np.where(k % 2 == 0, 1.0 + k * 2.0 ** -10, 1.0 + (k + 1) * 2.0 ** -10)
+    assert np.array_equal(got, even)
+
+
+def test_bf16_encode_matches_torch_rne_on_fp32_values():
+    v32 = _wide_doubles(200000, 2).astype(np.float32)
+    v32 = np.concatenate([v32, np.array([3.3895314e38, -3.3895314e38, 1e-40, -1e-41], dtype=np.float32)])
+    got = oracle.encode(v32.astype(np.float64), "bf16")
+    ref = torch.from_numpy(v32).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(got, ref)
+
+
+def test_bf16_encode_exact_ties_go_to_even():
+    k = np.arange(0, 128)
+    v = 1.0 + k * 2.0 ** -7 + 2.0 ** -8
+    got = oracle.decode(oracle.encode(v, "bf16"), "bf16")
+    even = np.where(k % 2 == 0, 1.0 + k * 2.0 ** -7, 1.0 + (k + 1) * 2.0 ** -7)
+    assert np.array_equal(got, even)
+
+
+# ---------------------------------------------------------------------------------------------
+# the maths of the README
+# ---------------------------------------------------------------------------------------------
+
+def test_hand_worked_example_golden():
+    g = json.load(open(os.path.join(GOLDEN, "lora_worked_example.json")))
+    X = f16_bits(g["X"])
+    A = [f16_bits(a) for a in g["A"]]
+    B = [f16_bits(b) for b in g["B"]]
+    W = np.array(g["W"])
+    xw = dec(X, "f16") @ W
+    # fp32 twin: V exactly as derived by hand, Y = x@W + delta
+    V, sk = oracle.shrink_f32(X, A, g["seg_starts"], g["lora_idx"], g["r"], "f16")
+    assert sk == 0
+    assert np.array_equal(V, np.array(g["V"], dtype=np.float32))
+    Y, _ = oracle.expand_f32(f16_bits(xw), V, B, g["seg_starts"], g["lora_idx"], 1.0, "f16")
+    assert np.array_equal(dec(Y, "f16"), np.array(g["Y"]))
+    Yd, _ = oracle.apply_f32(np.zeros((3, 2), np.uint16), X, A, B, g["seg_starts"], g["lora_idx"], 1.0, "f16")
+    assert np.array_equal(dec(Yd, "f16"), np.array(g["delta"]))
+    # binary64 twin
+    Y64, _ = oracle.apply_f64(xw, X, A, B, g["seg_starts"], g["lora_idx"], 1.0, "f16")
+    assert np.array_equal(Y64, np.array(g["Y"]))
+
+
+@pytest.mark.parametrize("dt", ["f16", "bf16"])
+def test_identity_against_materialised_weight(dt):
+    """x@(W + A@B) == x@W + (x@A)@B, with W + A@B materialised in fp64 by numpy."""
+    rng = np.random.default_rng(7)
+    T, H1, H2, r = 8, 24, 16, 4
+    X = inputs.cast_f32_bits(rng.standard_normal((T, H1)).astype(np.float32), dt)
+    A = [inputs.cast_f32_bits(rng.standard_normal((H1, r)).astype(np.float32) * 0.3, dt) for _ in range(3)]
+    B = [inputs.cast_f32_bits(rng.standard_normal((r, H2)).astype(np.float32) * 0.5, dt) for _ in range(3)]
+    W = rng.standard_normal((H1, H2))
+    seg, idx = [0, 3, 5, 8], [2, 0, 1]
+    x = dec(X, dt)
+    ref = np.zeros((T, H2))
+    for s in range(3):
+        Wp = W + dec(A[idx[s]], dt) @ dec(B[idx[s]], dt)
+        ref[seg[s]:seg[s + 1]] = x[seg[s]:seg[s + 1]] @ Wp
+    got, sk = oracle.apply_f64(x @ W, X, A, B, seg, idx, 1.0, dt)
+    assert sk == 0
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("dt", ["f16", "bf16"])
+def test_one_hot_rows_pick_adapter_rows_and_columns(dt):
+    """X[t] = e_k selects row k of A_i; V = e_j selects row j of B_i. Exact."""
+    rng = np.random.default_rng(11)
+    T, H1, H2, r, nA = 6, 20, 12, 5, 3
+    A = [inputs.cast_f32_bits(rng.standard_normal((H1, r)).astype(np.float32), dt) for _ in range(nA)]
+    B = [inputs.cast_f32_bits(rng.standard_normal((r, H2)).astype(np.float32), dt) for _ in range(nA)]
+    seg, idx = [0, 2, 3, 6], [1, 2, 0]
+    ks = [3, 17, 0, 19, 8, 11]
+    js = [4, 0, 2, 1, 3, 4]
+    one = inputs.cast_f32_bits(np.ones(1, np.float32), dt)[0]
+    X = np.zeros((T, H1), np.uint16)
+    for t, k in enumerate(ks):
+        X[t, k] = one
+    V, _ = oracle.shrink_f32(X, A, seg, idx, r, dt)
+    V64, _ = oracle.shrink_f64(X, A, seg, idx, r, dt)
+    Vs = np.zeros((T, r), np.float32)
+    Y0 = np.zeros((T, H2), np.uint16)
+    for s in range(3):
+        for t in range(seg[s], seg[s + 1]):
+            assert np.array_equal(V[t], dec(A[idx[s]][ks[t]], dt).astype(np.float32))
+            assert np.array_equal(V64[t], dec(A[idx[s]][ks[t]], dt))
+            Vs[t, js[t]] = 1.0
+    Y, _ = oracle.expand_f32(Y0, Vs, B, seg, idx, 1.0, dt)
+    for s in range(3):
+        for t in range(seg[s], seg[s + 1]):
+            assert np.array_equal(Y[t], B[idx[s]][js[t]])
+
+
+@pytest.mark.parametrize("dt", ["f16", "bf16"])
+def test_identical_distribution_equals_dense_gemm(dt):
+    """All tokens on one adapter: SGMV == dense (X@A)@B by numpy in fp64."""
+    rng = np.random.default_rng(3)
+    T, H1, H2, r = 16, 64, 48, 8
+    X = inputs.cast_f32_bits(rng.standard_normal((T, H1)).astype(np.float32), dt)
+    A = [inputs.cast_f32_bits((rng.standard_normal((H1, r)) / 8).astype(np.float32), dt)]
+    B = [inputs.cast_f32_bits((rng.standard_normal((r, H2)) / 3).astype(np.float32), dt)]
+    dense = (dec(X, dt) @ dec(A[0], dt)) @ dec(B[0], dt)
+    got64, _ = oracle.apply_f64(np.zeros((T, H2)), X, A, B, [0, T], [0], 1.0, dt)
+    np.testing.assert_allclose(got64, dense, rtol=1e-12, atol=1e-12)
+    # fp32 twin: within one storage ulp plus the fp32 accumulation bound
+    got32, _ = oracle.apply_f32(np.zeros((T, H2), np.uint16), X, A, B, [0, T], [0], 1.0, dt)
+    ulp = 2.0 ** -10 if dt == "f16" else 2.0 ** -7
+    err = np.abs(dec(got32, dt) - dense)
+    assert np.all(err <= ulp * np.abs(dense) + 1e-5)
+    # Distinct with every adapter equal gives the same fp32 result, row for row
+    Ad = A * T
+    Bd = B * T
+    gotd, _ = oracle.apply_f32(np.zeros((T, H2), np.uint16), X, Ad, Bd, list(range(T + 1)), list(range(T)), 1.0, dt)
+    assert np.array_equal(gotd, got32)
+
+
+def test_brute_force_exact_rationals():
+    """Tiny problem in exact rational arithmetic (Fraction) vs both twins."""
+    rng = np.random.default_rng(5)
+    T, H1, H2, r = 3, 5, 4, 2
+    dt = "f16"
+    X = f16_bits(rng.standard_normal((T, H1)))
+    A = [f16_bits(rng.standard_normal((H1, r))), f16_bits(rng.standard_normal((H1, r)))]
+    B = [f16_bits(rng.standard_normal((r, H2))), f16_bits(rng.standard_normal((r, H2)))]
+    Y0 = f16_bits(rng.standard_normal((T, H2)))
+    seg, idx = [0, 1, 3], [1, 0]
+    F = lambda bits: [[Fraction(float(v)) for v in row] for row in dec(np.atleast_2d(bits), dt)]
+    x, y0 = F(X), F(Y0)
+    exact = [[None] * H2 for _ in range(T)]
+    for s in range(2):
+        a, b = F(A[idx[s]]), F(B[idx[s]])
+        for t in range(seg[s], seg[s + 1]):
+            v = [sum(x[t][k] * a[k][j] for k in range(H1)) for j in range(r)]
+            for c in range(H2):
+                exact[t][c] = y0[t][c] + sum(v[j] * b[j][c] for j in range(r))
+    ex = np.array([[float(v) for v in row] for row in exact])
+    got64, _ = oracle.apply_f64(dec(Y0, dt), X, A, B, seg, idx, 1.0, dt)
+    np.testing.assert_allclose(got64, ex, rtol=1e-14, atol=1e-14)
+    got32, _ = oracle.apply_f32(Y0, X, A, B, seg, idx, 1.0, dt)
+    # fp32 accumulation then one fp16 rounding: within one fp16 ulp of the exact value
+    assert np.all(np.abs(dec(got32, dt) - ex) <= 2.0 ** -10 * np.maximum(np.abs(ex), 2.0 ** -14) * 1.01)
+
+
+# ---------------------------------------------------------------------------------------------
+# segment semantics
+# ---------------------------------------------------------------------------------------------
+
+def _case(dt="f16", T=12, H1=32, H2=24, r=4, nA=4, seed=9):
+    rng = np.random.default_rng(seed)
+    X = inputs.cast_f32_bits(rng.standard_normal((T, H1)).astype(np.float32), dt)
+    A = [inputs.cast_f32_bits((rng.standard_normal((H1, r)) / 5).astype(np.float32), dt) for _ in range(nA)]
+    B = [inputs.cast_f32_bits((rng.standard_normal((r, H2)) / 2).astype(np.float32), dt) for _ in range(nA)]
+    Y = inputs.cast_f32_bits(rng.standard_normal((T, H2)).astype(np.float32) + 0.01, dt)
+    return X, A, B, Y
+
+
+def test_zero_length_segments_are_noops():
+    X, A, B, Y = _case()
+    base, _ = oracle.apply_f32(Y, X, A, B, [0, 5, 12], [1, 3], 1.0, "f16")
+    with_empty, sk = oracle.apply_f32(Y, X, A, B, [0, 0, 5, 5, 5, 12, 12], [2, 1, 0, 3, 3, 1], 1.0, "f16")
+    assert sk == 0
+    assert np.array_equal(base, with_empty)
+
+
+def test_splitting_a_segment_is_bit_identical():
+    X, A, B, Y = _case()
+    one, _ = oracle.apply_f32(Y, X, A, B, [0, 12], [2], 1.0, "f16")
+    split, _ = oracle.apply_f32(Y, X, A, B, [0, 4, 9, 12], [2, 2, 2], 1.0, "f16")
+    assert np.array_equal(one, split)
+
+
+def test_permuting_segments_permutes_rows():
+    X, A, B, Y = _case()
+    seg, idx = [0, 3, 7, 12], [0, 3, 1]
+    out, _ = oracle.apply_f32(Y, X, A, B, seg, idx, 1.0, "f16")
+    order = [2, 0, 1]
+    rows = np.concatenate([np.arange(seg[s], seg[s + 1]) for s in order])
+    lens = [seg[s + 1] - seg[s] for s in order]
+    seg2 = np.concatenate([[0], np.cumsum(lens)])
+    out2, _ = oracle.apply_f32(Y[rows], X[rows], A, B, seg2, [idx[s] for s in order], 1.0, "f16")
+    assert np.array_equal(out2, out[rows])
+
+
+def test_rows_outside_segments_and_bad_segments_untouched():
+    X, A, B, Y = _case()
+    # rows 0..1 and 10..11 in no segment; one segment with a bad adapter id; one reversed
+    seg = [2, 5, 7, 6, 10]
+    idx = [1, 9, 0, 2]
+    out, sk = oracle.apply_f32(Y, X, A, B, seg, idx, 1.0, "f16")
+    assert sk == 2
+    # valid: [2,5) on adapter 1 and [6,10) on adapter 2
+    for t in [0, 1, 5, 10, 11]:
+        assert np.array_equal(out[t], Y[t])
+    ref, _ = oracle.apply_f32(Y, X, A, B, [2, 5, 6, 10], [1, 0, 2], 1.0, "f16")
+    for t in [2, 3, 4, 6, 7, 8, 9]:
+        assert np.array_equal(out[t], ref[t])
+
+
+def test_scale_linearity_powers_of_two_and_zero():
+    X, A, B, Y = _case()
+    Z = np.zeros_like(Y)
+    seg, idx = [0, 6, 12], [3, 1]
+    d1, _ = oracle.apply_f32(Z, X, A, B, seg, idx, 1.0, "f16")
+    for k in (-2, 1, 3):
+        dk, _ = oracle.apply_f32(Z, X, A, B, seg, idx, 2.0 ** k, "f16")
+        a1, ak = dec(d1, "f16"), dec(dk, "f16")
+        normal = np.abs(a1) * 2.0 ** k >= 2.0 ** -14
+        assert np.array_equal(ak[normal], a1[normal] * 2.0 ** k)
+    same, _ = oracle.apply_f32(Y, X, A, B, seg, idx, 0.0, "f16")
+    assert np.array_equal(same, Y)
+
+
+# ---------------------------------------------------------------------------------------------
+# bookkeeping
+# ---------------------------------------------------------------------------------------------
+
+def test_group_segments_tiny_config_printed_segments():
+    w = inputs.tiny()
+    seg, idx, perm = oracle.group_segments(w.ids, w.num_adapters)
+    assert seg.tolist() == [0, 1, 4, 6, 8]
+    assert idx.tolist() == [0, 1, 2, 3]
+    assert perm.tolist() == list(range(8))
+
+
+@pytest.mark.parametrize("maker", [lambda: inputs.uniform(), lambda: inputs.skewed(),
+                                   lambda: inputs.identical(), lambda: inputs.llama70b_decode()])
+def test_group_segments_invariants_and_stable_argsort(maker):
+    w = maker()
+    seg, idx, perm = oracle.group_segments(w.ids, w.num_adapters)
+    T = w.T
+    assert seg[0] == 0 and seg[-1] == T
+    assert np.all(np.diff(seg) > 0)
+    assert np.all(np.diff(idx) > 0)
+    assert np.array_equal(np.sort(perm), np.arange(T))
+    for s in range(len(idx)):
+        part = perm[seg[s]:seg[s + 1]]
+        assert np.all(w.ids[part] == idx[s])
+        assert np.all(np.diff(part) > 0)
+    # independent library routine: a stable argsort by adapter id
+    assert np.array_equal(perm, np.argsort(w.ids, kind="stable"))
+    assert idx.tolist() == sorted(set(w.ids.tolist()))
+
+
+def test_group_segments_rejects_out_of_range_ids():
+    with pytest.raises(ValueError):
+        oracle.group_segments([0, 5, 1], 4)
