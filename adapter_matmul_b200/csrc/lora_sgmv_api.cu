@@ -1,0 +1,389 @@
+// lora_sgmv_api.cu -- C ABI entry points: host-side validation, dispatch, launches.
+//
+// Every entry point validates its host-visible arguments first and returns an
+// error code without launching anything when one is wrong. Arrays that live on
+// the device (segments, adapter tables) are checked by the kernels per segment.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "../../include/lora_sgmv.h"
+#include "sgmv_grouped_tc.cuh"
+#include "sgmv_split.cuh"
+
+namespace {
+
+using sgmv::ExpandParams;
+using sgmv::ShrinkParams;
+
+constexpr int kVersion = 100;  // 0.1.0
+
+// Number of kernels this library has launched successfully in this process.
+std::atomic<uint64_t> g_launches{0};
+
+lora_sgmv_status counted(cudaError_t e) {
+    if (e != cudaSuccess) return LORA_SGMV_ERR_CUDA;
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return LORA_SGMV_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool split_rank(int r) { return r == 8 || r == 16 || r == 32 || r == 64 || r == 128; }
+
+// Lazily filled per-device facts, guarded by a mutex.
+struct DeviceFacts {
+    int sms = 0;
+    int max_smem_optin = 0;
+};
+std::mutex g_mu;
+std::vector<DeviceFacts> g_devices;
+
+lora_sgmv_status device_facts(DeviceFacts& out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return LORA_SGMV_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (dev >= static_cast<int>(g_devices.size())) g_devices.resize(dev + 1);
+    DeviceFacts& f = g_devices[dev];
+    if (f.sms == 0) {
+        if (cudaDeviceGetAttribute(&f.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&f.max_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
+                cudaSuccess) {
+            f.sms = 0;
+            return LORA_SGMV_ERR_CUDA;
+        }
+    }
+    out = f;
+    return LORA_SGMV_OK;
+}
+
+// Opt a kernel into more than 48 KB of dynamic shared memory, once per device.
+template <typename K>
+lora_sgmv_status ensure_smem(K kernel, size_t bytes, int& done_mask) {
+    if (bytes <= 48 * 1024) return LORA_SGMV_OK;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return LORA_SGMV_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_mu);
+    const int bit = 1 << (dev & 31);
+    if (done_mask & bit) return LORA_SGMV_OK;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess)
+        return LORA_SGMV_ERR_CUDA;
+    done_mask |= bit;
+    return LORA_SGMV_OK;
+}
+
+// ---- split path: launch plans ----------------------------------------------------------
+
+int clamp_grid_y(int n) { return std::min(n, 65535); }
+
+// token-chunk slots from a segment-length estimate
+int chunk_slots(int max_len, int tokens_per_chunk, int cap) {
+    const int chunks = (std::max(max_len, 1) + tokens_per_chunk - 1) / tokens_per_chunk;
+    return std::max(1, std::min(chunks, cap));
+}
+
+int cluster_size_for(int H1) {
+    // enough CTAs to split H1 into slices of at least 256 rows, at most 8 (portable cluster)
+    int c = 1;
+    while (c < 8 && H1 / (c * 2) >= 256) c *= 2;
+    return c;
+}
+
+template <typename T, int R>
+lora_sgmv_status launch_shrink(const ShrinkParams& p0, int max_len, cudaStream_t stream) {
+    static int smem_done = 0;
+    ShrinkParams p = p0;
+    const int C = cluster_size_for(p.H1);
+    p.ks = ((p.H1 + C - 1) / C + 7) / 8 * 8;
+    const size_t smem = sgmv::shrink_smem_bytes(p.ks, R);
+    DeviceFacts f;
+    if (device_facts(f) != LORA_SGMV_OK) return LORA_SGMV_ERR_CUDA;
+    if (smem > static_cast<size_t>(f.max_smem_optin)) return LORA_SGMV_ERR_DIM;
+    auto kernel = sgmv::sgmv_shrink_cluster_kernel<T, R>;
+    if (ensure_smem(kernel, smem, smem_done) != LORA_SGMV_OK) return LORA_SGMV_ERR_CUDA;
+
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(C, clamp_grid_y(p.n_segments), chunk_slots(max_len, sgmv::kShrinkTokens, 8));
+    cfg.blockDim = dim3(sgmv::kShrinkThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = C;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return counted(cudaLaunchKernelEx(&cfg, kernel, p));
+}
+
+template <typename T, int R>
+lora_sgmv_status launch_expand(const ExpandParams& p, int max_len, bool after_shrink, cudaStream_t stream) {
+    cudaLaunchConfig_t cfg = {};
+    const int cols_per_cta = sgmv::kExpandThreads * 8;
+    cfg.gridDim = dim3((p.H2 + cols_per_cta - 1) / cols_per_cta, clamp_grid_y(p.n_segments),
+                       chunk_slots(max_len, sgmv::kExpandTokens, 8));
+    cfg.blockDim = dim3(sgmv::kExpandThreads, 1, 1);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = after_shrink ? 1 : 0;
+    return counted(cudaLaunchKernelEx(&cfg, sgmv::sgmv_expand_kernel<T, R>, p));
+}
+
+template <typename T>
+lora_sgmv_status shrink_dispatch_r(const ShrinkParams& p, int r, int max_len, cudaStream_t s) {
+    switch (r) {
+        case 8: return launch_shrink<T, 8>(p, max_len, s);
+        case 16: return launch_shrink<T, 16>(p, max_len, s);
+        case 32: return launch_shrink<T, 32>(p, max_len, s);
+        case 64: return launch_shrink<T, 64>(p, max_len, s);
+        case 128: return launch_shrink<T, 128>(p, max_len, s);
+    }
+    return LORA_SGMV_ERR_UNSUPPORTED;
+}
+
+template <typename T>
+lora_sgmv_status expand_dispatch_r(const ExpandParams& p, int r, int max_len, bool chained, cudaStream_t s) {
+    switch (r) {
+        case 8: return launch_expand<T, 8>(p, max_len, chained, s);
+        case 16: return launch_expand<T, 16>(p, max_len, chained, s);
+        case 32: return launch_expand<T, 32>(p, max_len, chained, s);
+        case 64: return launch_expand<T, 64>(p, max_len, chained, s);
+        case 128: return launch_expand<T, 128>(p, max_len, chained, s);
+    }
+    return LORA_SGMV_ERR_UNSUPPORTED;
+}
+
+lora_sgmv_status shrink_dispatch(const ShrinkParams& p, int r, lora_sgmv_dtype dt, int max_len, cudaStream_t s) {
+    return dt == LORA_SGMV_F16 ? shrink_dispatch_r<__half>(p, r, max_len, s)
+                               : shrink_dispatch_r<__nv_bfloat16>(p, r, max_len, s);
+}
+
+lora_sgmv_status expand_dispatch(const ExpandParams& p, int r, lora_sgmv_dtype dt, int max_len, bool chained,
+                                 cudaStream_t s) {
+    return dt == LORA_SGMV_F16 ? expand_dispatch_r<__half>(p, r, max_len, chained, s)
+                               : expand_dispatch_r<__nv_bfloat16>(p, r, max_len, chained, s);
+}
+
+int estimate_max_len(int max_seg_len, int T, int n) {
+    if (max_seg_len > 0) return std::min(max_seg_len, std::max(T, 1));
+    return n > 0 ? (T + n - 1) / n : T;
+}
+
+lora_sgmv_status check_common(int32_t n_segments, int32_t num_adapters, int32_t T, lora_sgmv_dtype dtype) {
+    if (dtype != LORA_SGMV_F16 && dtype != LORA_SGMV_BF16) return LORA_SGMV_ERR_DTYPE;
+    if (n_segments < 0 || T < 0 || num_adapters < 0) return LORA_SGMV_ERR_DIM;
+    return LORA_SGMV_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t lora_sgmv_version(void) { return kVersion; }
+
+uint64_t lora_sgmv_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+int32_t lora_sgmv_rank_supported(int32_t r, lora_sgmv_variant variant) {
+    switch (variant) {
+        case LORA_SGMV_VARIANT_AUTO:
+        case LORA_SGMV_VARIANT_SPLIT: return split_rank(r) ? 1 : 0;
+        case LORA_SGMV_VARIANT_GROUPED_TC: return sgmv::grouped_tc_rank(r) ? 1 : 0;
+    }
+    return 0;
+}
+
+const char* lora_sgmv_status_string(lora_sgmv_status status) {
+    switch (status) {
+        case LORA_SGMV_OK: return "ok";
+        case LORA_SGMV_ERR_NULL: return "a required pointer is NULL";
+        case LORA_SGMV_ERR_DIM: return "invalid size";
+        case LORA_SGMV_ERR_ALIGN: return "pointer or row pitch not 16-byte aligned";
+        case LORA_SGMV_ERR_DTYPE: return "unknown storage type";
+        case LORA_SGMV_ERR_UNSUPPORTED: return "rank or variant not supported";
+        case LORA_SGMV_ERR_CUDA: return "CUDA runtime error";
+        case LORA_SGMV_ERR_WORKSPACE: return "workspace missing or too small";
+        case LORA_SGMV_ERR_RANGE: return "value out of range";
+    }
+    return "unknown status";
+}
+
+lora_sgmv_status lora_sgmv_group_segments(const int32_t* ids, int32_t T, int32_t num_adapters,
+                                          int32_t* seg_starts, int32_t* lora_idx, int32_t* perm,
+                                          int32_t* n_segments) {
+    if (!seg_starts || !lora_idx || !n_segments || (T > 0 && (!ids || !perm))) return LORA_SGMV_ERR_NULL;
+    if (T < 0 || num_adapters < 1) return LORA_SGMV_ERR_DIM;
+    for (int32_t t = 0; t < T; ++t)
+        if (ids[t] < 0 || ids[t] >= num_adapters) return LORA_SGMV_ERR_RANGE;
+    // counting sort: histogram, exclusive scan, stable scatter
+    std::vector<int32_t> count(static_cast<size_t>(num_adapters) + 1, 0);
+    for (int32_t t = 0; t < T; ++t) ++count[ids[t] + 1];
+    int32_t n = 0;
+    seg_starts[0] = 0;
+    for (int32_t a = 0; a < num_adapters; ++a) {
+        const int32_t c = count[a + 1];
+        count[a + 1] += count[a];  // count[a] becomes the first row of adapter a
+        if (c > 0) {
+            lora_idx[n] = a;
+            seg_starts[++n] = count[a + 1];
+        }
+    }
+    for (int32_t t = 0; t < T; ++t) perm[count[ids[t]]++] = t;
+    *n_segments = n;
+    return LORA_SGMV_OK;
+}
+
+size_t lora_sgmv_workspace_bytes(int32_t T, int32_t r) {
+    if (T <= 0 || r <= 0) return 0;
+    const size_t v = static_cast<size_t>(T) * static_cast<size_t>(r) * sizeof(float);
+    return (v + 255) / 256 * 256;
+}
+
+lora_sgmv_status lora_sgmv_shrink(float* V, const void* X, const void* const* A_ptrs,
+                                  const int32_t* seg_starts, const int32_t* lora_idx,
+                                  int32_t n_segments, int32_t num_adapters, int32_t T, int32_t H1,
+                                  int32_t r, lora_sgmv_dtype dtype, uint32_t* dev_status, void* stream) {
+    lora_sgmv_status st = check_common(n_segments, num_adapters, T, dtype);
+    if (st != LORA_SGMV_OK) return st;
+    if (H1 <= 0 || r <= 0) return LORA_SGMV_ERR_DIM;
+    if (!split_rank(r)) return LORA_SGMV_ERR_UNSUPPORTED;
+    if (n_segments == 0 || T == 0) return LORA_SGMV_OK;
+    if (!V || !X || !A_ptrs || !seg_starts || !lora_idx) return LORA_SGMV_ERR_NULL;
+    if (num_adapters < 1) return LORA_SGMV_ERR_DIM;
+    if (!aligned16(V) || !aligned16(X) || H1 % 8) return LORA_SGMV_ERR_ALIGN;
+    ShrinkParams p = {};
+    p.V = V;
+    p.X = X;
+    p.A_ptrs = A_ptrs;
+    p.B_check = nullptr;
+    p.seg_starts = seg_starts;
+    p.lora_idx = lora_idx;
+    p.dev_status = dev_status;
+    p.n_segments = n_segments;
+    p.num_adapters = num_adapters;
+    p.T = T;
+    p.H1 = H1;
+    const int max_len = estimate_max_len(0, T, n_segments);
+    return shrink_dispatch(p, r, dtype, max_len, static_cast<cudaStream_t>(stream));
+}
+
+lora_sgmv_status lora_sgmv_expand(void* Y, const float* V, const void* const* B_ptrs,
+                                  const int32_t* seg_starts, const int32_t* lora_idx,
+                                  int32_t n_segments, int32_t num_adapters, int32_t T, int32_t r,
+                                  int32_t H2, float scale, lora_sgmv_dtype dtype, uint32_t* dev_status,
+                                  void* stream) {
+    lora_sgmv_status st = check_common(n_segments, num_adapters, T, dtype);
+    if (st != LORA_SGMV_OK) return st;
+    if (H2 <= 0 || r <= 0) return LORA_SGMV_ERR_DIM;
+    if (!split_rank(r)) return LORA_SGMV_ERR_UNSUPPORTED;
+    if (n_segments == 0 || T == 0) return LORA_SGMV_OK;
+    if (!Y || !V || !B_ptrs || !seg_starts || !lora_idx) return LORA_SGMV_ERR_NULL;
+    if (num_adapters < 1) return LORA_SGMV_ERR_DIM;
+    if (!aligned16(Y) || !aligned16(V) || H2 % 8) return LORA_SGMV_ERR_ALIGN;
+    ExpandParams p = {};
+    p.Y = Y;
+    p.V = V;
+    p.B_ptrs = B_ptrs;
+    p.A_check = nullptr;
+    p.seg_starts = seg_starts;
+    p.lora_idx = lora_idx;
+    p.dev_status = dev_status;
+    p.n_segments = n_segments;
+    p.num_adapters = num_adapters;
+    p.T = T;
+    p.H2 = H2;
+    p.scale = scale;
+    const int max_len = estimate_max_len(0, T, n_segments);
+    return expand_dispatch(p, r, dtype, max_len, false, static_cast<cudaStream_t>(stream));
+}
+
+lora_sgmv_status lora_sgmv_apply_ex(void* Y, const void* X, const void* const* A_ptrs,
+                                    const void* const* B_ptrs, const int32_t* seg_starts,
+                                    const int32_t* lora_idx, int32_t n_segments, int32_t num_adapters,
+                                    int32_t T, int32_t H1, int32_t r, int32_t H2, float scale,
+                                    lora_sgmv_dtype dtype, int32_t max_seg_len, void* workspace,
+                                    size_t workspace_bytes, uint32_t* dev_status, lora_sgmv_variant variant,
+                                    void* stream) {
+    lora_sgmv_status st = check_common(n_segments, num_adapters, T, dtype);
+    if (st != LORA_SGMV_OK) return st;
+    if (H1 <= 0 || H2 <= 0 || r <= 0) return LORA_SGMV_ERR_DIM;
+    if (variant != LORA_SGMV_VARIANT_AUTO && variant != LORA_SGMV_VARIANT_SPLIT &&
+        variant != LORA_SGMV_VARIANT_GROUPED_TC)
+        return LORA_SGMV_ERR_UNSUPPORTED;
+    if (!lora_sgmv_rank_supported(r, variant)) return LORA_SGMV_ERR_UNSUPPORTED;
+    if (n_segments == 0 || T == 0) return LORA_SGMV_OK;
+    if (!Y || !X || !A_ptrs || !B_ptrs || !seg_starts || !lora_idx) return LORA_SGMV_ERR_NULL;
+    if (num_adapters < 1) return LORA_SGMV_ERR_DIM;
+    if (!aligned16(Y) || !aligned16(X) || H1 % 8 || H2 % 8) return LORA_SGMV_ERR_ALIGN;
+    const size_t need = lora_sgmv_workspace_bytes(T, r);
+    if (!workspace || workspace_bytes < need) return LORA_SGMV_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return LORA_SGMV_ERR_ALIGN;
+    const int max_len = estimate_max_len(max_seg_len, T, n_segments);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+    lora_sgmv_variant v = variant;
+    if (v == LORA_SGMV_VARIANT_AUTO)
+        v = (max_len >= sgmv::kGroupedMinSegment && sgmv::grouped_tc_supported(r, H1, H2, dtype))
+                ? LORA_SGMV_VARIANT_GROUPED_TC
+                : LORA_SGMV_VARIANT_SPLIT;
+
+    if (v == LORA_SGMV_VARIANT_GROUPED_TC) {
+        if (!sgmv::grouped_tc_supported(r, H1, H2, dtype)) return LORA_SGMV_ERR_UNSUPPORTED;
+        return sgmv::launch_grouped_tc(Y, X, A_ptrs, B_ptrs, seg_starts, lora_idx, n_segments, num_adapters,
+                                       T, H1, r, H2, scale, dtype, dev_status, s);
+    }
+
+    float* V = static_cast<float*>(workspace);
+
+    ShrinkParams sp = {};
+    sp.V = V;
+    sp.X = X;
+    sp.A_ptrs = A_ptrs;
+    sp.B_check = B_ptrs;
+    sp.seg_starts = seg_starts;
+    sp.lora_idx = lora_idx;
+    sp.dev_status = dev_status;
+    sp.n_segments = n_segments;
+    sp.num_adapters = num_adapters;
+    sp.T = T;
+    sp.H1 = H1;
+    st = shrink_dispatch(sp, r, dtype, max_len, s);
+    if (st != LORA_SGMV_OK) return st;
+
+    ExpandParams ep = {};
+    ep.Y = Y;
+    ep.V = V;
+    ep.B_ptrs = B_ptrs;
+    ep.A_check = A_ptrs;
+    ep.seg_starts = seg_starts;
+    ep.lora_idx = lora_idx;
+    ep.dev_status = nullptr;  // the shrink already reported this call's bad segments
+    ep.n_segments = n_segments;
+    ep.num_adapters = num_adapters;
+    ep.T = T;
+    ep.H2 = H2;
+    ep.scale = scale;
+    return expand_dispatch(ep, r, dtype, max_len, true, s);
+}
+
+lora_sgmv_status lora_sgmv_apply(void* Y, const void* X, const void* const* A_ptrs,
+                                 const void* const* B_ptrs, const int32_t* seg_starts,
+                                 const int32_t* lora_idx, int32_t n_segments, int32_t num_adapters,
+                                 int32_t T, int32_t H1, int32_t r, int32_t H2, float scale,
+                                 lora_sgmv_dtype dtype, int32_t max_seg_len, void* workspace,
+                                 size_t workspace_bytes, uint32_t* dev_status, void* stream) {
+    return lora_sgmv_apply_ex(Y, X, A_ptrs, B_ptrs, seg_starts, lora_idx, n_segments, num_adapters, T, H1, r,
+                              H2, scale, dtype, max_seg_len, workspace, workspace_bytes, dev_status,
+                              LORA_SGMV_VARIANT_AUTO, stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,289 @@
+// sgmv_split.cuh -- the split SGMV path: a split-K shrink kernel (H1 -> r) and a
+// streaming expand kernel (r -> H2) with the add onto Y fused in its epilogue.
+//
+// Shapes follow the Punica README's LoRA paragraph: A_i is [H1, r], B_i is
+// [r, H2], rows are tokens; the batch form (multi-LoRA paragraph) maps each
+// segment of rows to its own adapter.
+//
+// Shrink. One thread-block cluster of C CTAs per (segment, token-chunk slot).
+// CTA c of the cluster owns rows [c*KS, (c+1)*KS) of A_i; that slice of A_i
+// is one contiguous run of KS*r*2 bytes, read once with 128-bit coalesced
+// loads. Each CTA stages its slice of the chunk's X rows in shared memory,
+// accumulates fp32 partial sums per thread, reduces them with warp shuffles
+// and then across warps in shared memory. The C partial V tiles are summed in
+// a fixed order through distributed shared memory (DSMEM), and each CTA
+// stores its share of the reduced V with plain stores: no atomics, no
+// zero-fill of V, bit-reproducible.
+//
+// Expand. One CTA per (column block of 8*NT columns, segment, token-chunk
+// slot). Each thread owns 8 consecutive columns: it streams B_i[j, cols] for
+// j = 0..r-1 with 128-bit loads (each B_i byte is read once per token chunk),
+// multiplies by V rows held in shared memory, and performs the read-add-round-
+// write of Y in place. With programmatic dependent launch the expand grid is
+// scheduled while the shrink grid drains; everything it does before
+// griddepcontrol.wait (segment metadata, the first block of B_i) does not
+// depend on V.
+#pragma once
+
+#include <cooperative_groups.h>
+
+#include "sgmv_common.cuh"
+
+namespace sgmv {
+
+namespace cg = cooperative_groups;
+
+struct ShrinkParams {
+    float* V;
+    const void* X;
+    const void* const* A_ptrs;
+    const void* const* B_check;  // non-null in apply: a segment whose B_i is bad is skipped here too
+    const int32_t* seg_starts;
+    const int32_t* lora_idx;
+    uint32_t* dev_status;
+    int n_segments;
+    int num_adapters;
+    int T;
+    int H1;
+    int ks;  // rows of A_i per CTA, multiple of 8
+};
+
+struct ExpandParams {
+    void* Y;
+    const float* V;
+    const void* const* B_ptrs;
+    const void* const* A_check;  // non-null in apply: a segment whose A_i is bad is skipped here too
+    const int32_t* seg_starts;
+    const int32_t* lora_idx;
+    uint32_t* dev_status;
+    int n_segments;
+    int num_adapters;
+    int T;
+    int H2;
+    float scale;
+};
+
+constexpr int kShrinkThreads = 256;
+constexpr int kShrinkTokens = 8;   // tokens per chunk
+constexpr int kShrinkUnroll = 8;   // 16-byte loads in flight per thread
+constexpr int kExpandThreads = 128;
+constexpr int kExpandTokens = 8;
+
+__host__ __device__ constexpr size_t shrink_smem_bytes(int ks, int R) {
+    // X slice [TC][ks] (16-bit) + per-warp partials [NW][TC*R] + CTA partial [TC*R]
+    return size_t(kShrinkTokens) * ks * 2 + size_t(kShrinkThreads / 32) * kShrinkTokens * R * 4 +
+           size_t(kShrinkTokens) * R * 4;
+}
+
+// grid: x = C (one cluster along x), y = segment slots, z = token-chunk slots.
+template <typename T, int R>
+__global__ void __launch_bounds__(kShrinkThreads) sgmv_shrink_cluster_kernel(const ShrinkParams p) {
+    constexpr int NT = kShrinkThreads;
+    constexpr int TC = kShrinkTokens;
+    constexpr int G = R / 8;     // 16-byte vectors per row of A_i
+    constexpr int RL = NT / G;   // row lanes
+    constexpr int NW = NT / 32;
+    static_assert(R % 8 == 0 && G <= 32 && (32 % G) == 0, "rank must be 8..256, power of two");
+
+    cg::cluster_group cluster = cg::this_cluster();
+    const int c = static_cast<int>(cluster.block_rank());
+    const int C = static_cast<int>(cluster.num_blocks());
+    const int tid = threadIdx.x;
+    const int lane = tid & 31;
+    const int warp = tid >> 5;
+
+    extern __shared__ __align__(16) unsigned char smem[];
+    T* xs = reinterpret_cast<T*>(smem);
+    float* red = reinterpret_cast<float*>(smem + size_t(TC) * p.ks * 2);
+    float* part = red + NW * TC * R;
+
+    // The expand kernel may be scheduled as soon as every shrink CTA is running.
+    pdl_launch_dependents();
+
+    const int KS = p.ks;
+    const int k0 = c * KS;
+    const int nk = max(0, min(k0 + KS, p.H1) - k0);
+    const int cgi = tid % G;
+    const int rl = tid / G;
+    const T* __restrict__ X = static_cast<const T*>(p.X);
+
+    for (int s = blockIdx.y; s < p.n_segments; s += gridDim.y) {
+        Segment seg;
+        const uint32_t bad = load_segment(p.seg_starts, p.lora_idx, p.A_ptrs, p.B_check, s, p.T,
+                                          p.num_adapters, seg);
+        if (bad) {  // uniform over the cluster: every CTA read the same words
+            if (c == 0 && blockIdx.z == 0 && tid == 0) report(p.dev_status, bad);
+            continue;
+        }
+        const T* __restrict__ A = static_cast<const T*>(seg.a);
+        const int L = seg.end - seg.begin;
+        const int nchunks = (L + TC - 1) / TC;
+        for (int q = blockIdx.z; q < nchunks; q += gridDim.z) {
+            const int t0 = seg.begin + q * TC;
+            const int nt = min(TC, seg.end - t0);
+            // stage X[t0 .. t0+TC, k0 .. k0+nk) (rows past the chunk are zero)
+            const int vpr = nk / 8;
+            for (int v = tid; v < TC * vpr; v += NT) {
+                const int row = v / vpr;
+                const int col = (v - row * vpr) * 8;
+                uint4 val = make_uint4(0, 0, 0, 0);
+                if (row < nt) val = ld_vec(X + size_t(t0 + row) * p.H1 + k0 + col);
+                st_vec(xs + size_t(row) * KS + col, val);
+            }
+            __syncthreads();
+
+            float acc[TC][8];
+#pragma unroll
+            for (int t = 0; t < TC; ++t)
+#pragma unroll
+                for (int i = 0; i < 8; ++i) acc[t][i] = 0.f;
+
+            for (int kb = rl; kb < nk; kb += RL * kShrinkUnroll) {
+                uint4 av[kShrinkUnroll];
+#pragma unroll
+                for (int u = 0; u < kShrinkUnroll; ++u) {
+                    const int kr = kb + u * RL;
+                    av[u] = kr < nk ? ld_stream(A + size_t(k0 + kr) * R + cgi * 8) : make_uint4(0, 0, 0, 0);
+                }
+#pragma unroll
+                for (int u = 0; u < kShrinkUnroll; ++u) {
+                    const int kr = kb + u * RL;
+                    if (kr < nk) {
+                        float a[8];
+                        unpack8<T>(av[u], a);
+#pragma unroll
+                        for (int t = 0; t < TC; ++t) {
+                            const float x = Storage<T>::to1(xs[size_t(t) * KS + kr]);
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) acc[t][i] = fmaf(x, a[i], acc[t][i]);
+                        }
+                    }
+                }
+            }
+            // reduce over the row lanes of this warp (lanes sharing cgi)
+#pragma unroll
+            for (int off = G; off < 32; off <<= 1)
+#pragma unroll
+                for (int t = 0; t < TC; ++t)
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) acc[t][i] += __shfl_xor_sync(0xffffffffu, acc[t][i], off);
+            if (lane < G) {
+#pragma unroll
+                for (int t = 0; t < TC; ++t)
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) red[(warp * TC + t) * R + cgi * 8 + i] = acc[t][i];
+            }
+            __syncthreads();
+            for (int e = tid; e < TC * R; e += NT) {
+                float sum = 0.f;
+#pragma unroll
+                for (int w = 0; w < NW; ++w) sum += red[w * TC * R + e];
+                part[e] = sum;
+            }
+            // sum the C partial tiles across the cluster in rank order
+            cluster.sync();
+            const int per = (TC * R + C - 1) / C;
+            const int e0 = c * per;
+            const int e1 = min(e0 + per, TC * R);
+            for (int e = e0 + tid; e < e1; e += NT) {
+                float sum = 0.f;
+                for (int qr = 0; qr < C; ++qr) sum += cluster.map_shared_rank(part, qr)[e];
+                const int t = e / R;
+                const int j = e - t * R;
+                if (t < nt) p.V[size_t(t0 + t) * R + j] = sum;
+            }
+            cluster.sync();  // partial tiles may be overwritten / freed only after every read
+        }
+    }
+}
+
+// grid: x = column blocks of 8*NT columns, y = segment slots, z = token-chunk slots.
+template <typename T, int R>
+__global__ void __launch_bounds__(kExpandThreads) sgmv_expand_kernel(const ExpandParams p) {
+    constexpr int NT = kExpandThreads;
+    constexpr int TC = kExpandTokens;
+    constexpr int JB = R >= 128 ? 8 : (R < 16 ? R : 16);  // rows of B_i loaded per batch
+    __shared__ float vs[TC][R];
+
+    const int tid = threadIdx.x;
+    const int col = (blockIdx.x * NT + tid) * 8;
+    const bool active = col < p.H2;
+    T* __restrict__ Y = static_cast<T*>(p.Y);
+    bool waited = false;
+
+    for (int s = blockIdx.y; s < p.n_segments; s += gridDim.y) {
+        Segment seg;
+        const uint32_t bad = load_segment(p.seg_starts, p.lora_idx, p.A_check, p.B_ptrs, s, p.T,
+                                          p.num_adapters, seg);
+        if (bad) {
+            if (blockIdx.x == 0 && blockIdx.z == 0 && tid == 0) report(p.dev_status, bad);
+            continue;
+        }
+        const T* __restrict__ B = static_cast<const T*>(seg.b);
+        const int L = seg.end - seg.begin;
+        const int nchunks = (L + TC - 1) / TC;
+        for (int q = blockIdx.z; q < nchunks; q += gridDim.z) {
+            const int t0 = seg.begin + q * TC;
+            const int nt = min(TC, seg.end - t0);
+            // first batch of B_i rows does not depend on V: issue it before the wait
+            uint4 bv[JB];
+#pragma unroll
+            for (int u = 0; u < JB; ++u)
+                bv[u] = active ? ld_stream(B + size_t(u) * p.H2 + col) : make_uint4(0, 0, 0, 0);
+            if (!waited) {
+                pdl_wait();
+                waited = true;
+            }
+            for (int e = tid; e < TC * R; e += NT) {
+                const int t = e / R;
+                const int j = e - t * R;
+                vs[t][j] = t < nt ? p.V[size_t(t0 + t) * R + j] : 0.f;
+            }
+            __syncthreads();
+
+            float acc[TC][8];
+#pragma unroll
+            for (int t = 0; t < TC; ++t)
+#pragma unroll
+                for (int i = 0; i < 8; ++i) acc[t][i] = 0.f;
+#pragma unroll 1
+            for (int jb = 0; jb < R; jb += JB) {
+                if (jb > 0) {
+#pragma unroll
+                    for (int u = 0; u < JB; ++u)
+                        bv[u] = active ? ld_stream(B + size_t(jb + u) * p.H2 + col) : make_uint4(0, 0, 0, 0);
+                }
+#pragma unroll
+                for (int u = 0; u < JB; ++u) {
+                    float b[8];
+                    unpack8<T>(bv[u], b);
+#pragma unroll
+                    for (int t = 0; t < TC; ++t) {
+                        if (t < nt) {
+                            const float v = vs[t][jb + u];
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) acc[t][i] = fmaf(v, b[i], acc[t][i]);
+                        }
+                    }
+                }
+            }
+            if (active) {
+#pragma unroll
+                for (int t = 0; t < TC; ++t) {
+                    if (t < nt) {
+                        T* yp = Y + size_t(t0 + t) * p.H2 + col;
+                        float y[8];
+                        unpack8<T>(ld_vec(yp), y);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) y[i] = __fadd_rn(y[i], __fmul_rn(p.scale, acc[t][i]));
+                        st_vec(yp, pack8<T>(y));
+                    }
+                }
+            }
+            __syncthreads();  // vs is rewritten by the next chunk
+        }
+    }
+    if (!waited) pdl_wait();  // keep the dependency even when this CTA had no work
+}
+
+}  // namespace sgmv

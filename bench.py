@@ -1,0 +1,473 @@
+#!/usr/bin/env python
+"""SGMV benchmark: LoRA-delta tokens/s and achieved HBM bandwidth on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+
+Default workload ("distinct"): Llama-7B-shaped decode with the Distinct
+adapter distribution of the Punica README's throughput benchmark: 32 tokens,
+each on its own rank-16 adapter, H1 = H2 = 4096, fp16. One step is one decoder
+layer's LoRA work: four SGMV calls (q, k, v, o projections), each with its
+own adapters, input and output. Steps rotate over 32 layers, each with its own
+weights and activations (1.1 GiB in all, far above the 126 MB L2), so every
+step reads cold data, as a model's layers would.
+
+The timed region replays one CUDA graph per layer (the graph holds that
+layer's four lora_sgmv_apply calls) so host launch latency does not stand in
+for kernel time. ``e2e`` repeats the measurement through the public call with
+host buffers: each step copies its inputs from pinned host memory, groups the
+token batch on the host, runs the four calls, and reads the outputs back.
+
+Multi-GPU (torchrun): every rank runs its own replica of the workload (the
+path has no cross-GPU data exchange); value = all ranks' tokens / max time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from adapter_matmul_b200 import inputs  # noqa: E402
+
+METRIC = "LoRA-delta tokens/s (SGMV)"
+UNIT = "tokens/s"
+L2_BYTES = 126 * 1024 * 1024
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, "fallback"
+
+
+# ---------------------------------------------------------------------------------------------
+# workloads
+# ---------------------------------------------------------------------------------------------
+
+class Spec:
+    def __init__(self, name, workload, projections, layers, desc):
+        self.name, self.w, self.P, self.L, self.desc = name, workload, projections, layers, desc
+
+
+def make_spec(name: str) -> Spec:
+    if name == "distinct":
+        w = inputs.distinct()
+        return Spec(name, w, 4, 32, "Distinct decode, Llama-7B shape: H1=H2=4096, r=16, fp16, 32 tokens each on "
+                                    "its own adapter; step = one layer = 4 SGMV calls (q,k,v,o)")
+    w = inputs.make(name)
+    per_call = w.algorithmic_bytes()
+    layers = max(1, min(64, math.ceil(3 * L2_BYTES / per_call)))
+    return Spec(name, w, 1, layers, f"{name}: H1={w.H1}, H2={w.H2}, r={w.r}, {w.dtype}, T={w.T}, "
+                                    f"{len(w.touched_adapters())} adapters touched; step = 1 SGMV call")
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+# ---------------------------------------------------------------------------------------------
+# clocks (NVML, sampled during the timed region)
+# ---------------------------------------------------------------------------------------------
+
+_REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+            0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+            0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+
+class ClockSampler:
+    def __init__(self, index: int, period_s: float = 0.005):
+        self.samples, self.reasons, self.max_mhz = [], 0, None
+        self._stop = threading.Event()
+        self._period = period_s
+        try:
+            import pynvml
+            import torch
+
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            pr = torch.cuda.get_device_properties(index)
+            bus = f"{pr.pci_domain_id:08X}:{pr.pci_bus_id:02X}:{pr.pci_device_id:02X}.0"
+            try:
+                self._h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            except Exception:
+                self._h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._nv = None
+
+    def _sample(self):
+        nv = self._nv
+        self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+        try:
+            self.reasons |= int(nv.nvmlDeviceGetCurrentClocksEventReasons(self._h))
+        except Exception:
+            self.reasons |= int(nv.nvmlDeviceGetCurrentClocksThrottleReasons(self._h))
+
+    def _run(self):
+        while not self._stop.is_set():
+            self._sample()
+            time.sleep(self._period)
+
+    def __enter__(self):
+        if self._nv:
+            self._sample()
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self._nv:
+            self._stop.set()
+            self._t.join()
+            self._sample()
+
+    def summary(self):
+        if not self._nv or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        names = [n for bit, n in _REASONS.items() if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz, "reasons": names,
+                "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------------------------
+# the CPU oracle as a baseline (host cores)
+# ---------------------------------------------------------------------------------------------
+
+def oracle_baseline(spec: Spec, seconds: float):
+    """Time the oracle (single-threaded C, as it stands) on a bounded sample of the workload."""
+    import oracle
+
+    w = spec.w
+    seg, idx, _ = oracle.group_segments(w.ids, w.num_adapters)
+    # one call's host inputs; the sample repeats it, bounded in time
+    touched = w.touched_adapters()
+    Am = {i: w.adapter_a(i) for i in touched}
+    Bm = {i: w.adapter_b(i) for i in touched}
+    zA, zB = np.zeros((1, 1), np.uint16), np.zeros((1, 1), np.uint16)
+    A = [Am.get(i, zA) for i in range(w.num_adapters)]
+    B = [Bm.get(i, zB) for i in range(w.num_adapters)]
+    X, Y = w.x(), w.y0()
+    # rows per call: the whole batch unless a call alone exceeds the budget
+    t0 = time.perf_counter()
+    rows = min(w.T, max(1, int(seg[1] - seg[0])))
+    sub_seg = np.array([0, rows], np.int32)
+    sub_idx = idx[:1]
+    oracle.apply_f32(Y[:rows], X[:rows], A, B, sub_seg, sub_idx, w.scale, w.dtype)
+    per_row = (time.perf_counter() - t0) / rows
+    calls, tokens, t_start = 0, 0, time.perf_counter()
+    full_call_s = per_row * w.T
+    if full_call_s <= seconds / 2:
+        sample = f"whole SGMV calls of the workload ({w.T} tokens each), repeated for ~{seconds:.0f} s"
+        while time.perf_counter() - t_start < seconds:
+            oracle.apply_f32(Y, X, A, B, seg, idx, w.scale, w.dtype)
+            calls += 1
+            tokens += w.T
+    else:
+        n_rows = max(1, int(seconds / per_row))
+        sample = f"first {n_rows} of {w.T} token rows of one call (segment order)"
+        # take whole segments from the start until n_rows
+        take = int(np.searchsorted(seg, n_rows, side="right")) - 1
+        take = max(1, take)
+        oracle.apply_f32(Y[: seg[take]], X[: seg[take]], A, B, seg[: take + 1], idx[:take], w.scale, w.dtype)
+        calls, tokens = 1, int(seg[take])
+    elapsed = time.perf_counter() - t_start
+    # tokens/s of whole steps: a step holds spec.P calls over the same T tokens
+    value = tokens / spec.P / elapsed
+    return {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample,
+            "seconds": round(elapsed, 3), "calls": calls}
+
+
+# ---------------------------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------------------------
+
+def run_ours(args, spec: Spec, rank: int, world: int, local: int):
+    import torch
+    import torch.distributed as dist
+
+    from adapter_matmul_b200 import sgmv
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    w = spec.w
+    dt = sgmv.F16 if w.dtype == "f16" else sgmv.BF16
+    tdt = torch.float16 if w.dtype == "f16" else torch.bfloat16
+    seg, idx, _ = sgmv.lora_sgmv_group_segments(w.ids, w.num_adapters)
+    n = len(idx)
+    max_len = int(np.max(np.diff(seg)))
+    touched = w.touched_adapters()
+
+    def dev_bits(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(tdt).to(dev)
+
+    # per (layer, projection): adapters (pool), X, Y; adapters drawn from the seeded generator
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(1234 + rank)
+    calls = []
+    keep = []
+    for l in range(spec.L):
+        for p in range(spec.P):
+            proj = l * spec.P + p
+            A_pool = torch.empty((w.num_adapters, w.H1, w.r), dtype=tdt, device=dev)
+            B_pool = torch.empty((w.num_adapters, w.r, w.H2), dtype=tdt, device=dev)
+            if len(touched) < w.num_adapters:  # resident but unused by this batch
+                A_pool.normal_(0.0, 1.0 / math.sqrt(w.H1), generator=gen)
+                B_pool.normal_(0.0, 1.0 / math.sqrt(w.r), generator=gen)
+            for i in touched:
+                A_pool[i] = dev_bits(w.adapter_a(i, proj))
+                B_pool[i] = dev_bits(w.adapter_b(i, proj))
+            A_ptrs = torch.tensor([A_pool[i].data_ptr() for i in range(w.num_adapters)], dtype=torch.int64, device=dev)
+            B_ptrs = torch.tensor([B_pool[i].data_ptr() for i in range(w.num_adapters)], dtype=torch.int64, device=dev)
+            X = dev_bits(w.x(proj))
+            Y = torch.zeros((w.T, w.H2), dtype=tdt, device=dev)
+            keep += [A_pool, B_pool]
+            calls.append((l, p, X, Y, A_ptrs, B_ptrs))
+    d_seg = torch.from_numpy(seg).to(dev)
+    d_idx = torch.from_numpy(idx).to(dev)
+    ws_bytes = sgmv.lora_sgmv_workspace_bytes(w.T, w.r)
+    ws = torch.empty(ws_bytes // 4, dtype=torch.float32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    stream = torch.cuda.Stream(device=dev)
+    sh = stream.cuda_stream
+
+    def enqueue_layer(l):
+        for (ll, p, X, Y, A_ptrs, B_ptrs) in calls[l * spec.P:(l + 1) * spec.P]:
+            sgmv.lora_sgmv_apply(Y, X, A_ptrs, B_ptrs, d_seg, d_idx, n, w.num_adapters, w.T, w.H1, w.r, w.H2,
+                                 w.scale, dt, max_len, ws, ws_bytes, status, sh)
+
+    # one CUDA graph per layer
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        for l in range(spec.L):  # eager warm-up (attributes, first-touch)
+            enqueue_layer(l)
+    stream.synchronize()
+    graphs = []
+    for l in range(spec.L):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            enqueue_layer(l)
+        graphs.append(g)
+    launches_per_step = None
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            graphs[i % spec.L].replay()
+    stream.synchronize()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    # ---- timed region: K steps ----
+    barrier()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clocks:
+        with torch.cuda.stream(stream):
+            ev0.record(stream)
+            for i in range(args.steps):
+                graphs[i % spec.L].replay()
+            ev1.record(stream)
+        stream.synchronize()
+    torch.cuda.synchronize()
+    barrier()
+    ms = ev0.elapsed_time(ev1)
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_per_step = ms / args.steps
+
+    # kernels per step: count the launches of one eager layer
+    c0 = sgmv.lora_sgmv_launch_count()
+    with torch.cuda.stream(stream):
+        enqueue_layer(0)
+    stream.synchronize()
+    launches_per_step = sgmv.lora_sgmv_launch_count() - c0
+    gpu_launches = launches_per_step * args.steps
+
+    st = int(status.item())
+    if st != 0:
+        raise RuntimeError(f"device status {st:#x}: a segment was rejected")
+
+    # ---- roofline: one SGMV call = the unit (its kernels run back to back) ----
+    hbm, tc, which = peaks()
+    bytes_call = w.algorithmic_bytes()
+    call_s = ms_per_step / 1e3 / spec.P
+    achieved = bytes_call / call_s / 1e9
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
+                "frac": round(achieved / hbm, 4), "traffic": None,
+                "kernel": "one lora_sgmv_apply call (split shrink + expand kernels, chained by PDL)",
+                "peak_source": f"{which} (MEASURED_PEAKS.json hbm_gbs)" if which == "measured" else which,
+                "algorithmic_bytes_per_launch": bytes_call, "tflops": round(w.flops() / call_s / 1e12, 3)}
+
+    # ---- e2e through the public call with host buffers ----
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, spec, torch, sgmv, dev, stream, calls, dt, tdt)
+
+    result = None
+    if rank == 0:
+        tokens = w.T * args.steps * world
+        value = tokens / (ms / 1e3)
+        result = {
+            "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+            "config": {"workload": spec.desc, "name": spec.name, "T": w.T, "H1": w.H1, "H2": w.H2, "r": w.r,
+                       "adapters_touched": len(touched), "segments": n, "sgmv_calls_per_step": spec.P,
+                       "layers_rotated": spec.L,
+                       "l2": f"inputs larger than L2: {spec.L} layers rotated, "
+                             f"{spec.L * spec.P * bytes_call / 2**30:.2f} GiB of algorithmic bytes per rotation",
+                       "timing": "CUDA events on the launching stream around K graph replays",
+                       "parallelism": f"replicas x{world}"},
+            "roofline": roofline,
+            "gpu_launches": int(gpu_launches),
+            "clocks": clocks.summary(),
+        }
+        if e2e:
+            result["e2e"] = e2e
+    if world > 1:
+        dist.barrier()
+        del graphs
+        dist.destroy_process_group()
+    return result
+
+
+def run_e2e(args, spec, torch, sgmv, dev, stream, calls, dt, tdt):
+    """Same metric through lora_sgmv_group_segments + lora_sgmv_apply with host buffers."""
+    w = spec.w
+    steps = max(3, min(args.steps, 200))
+    # pinned host copies of every (layer, projection)'s inputs and outputs
+    hX = [torch.empty((w.T, w.H1), dtype=tdt, pin_memory=True) for _ in range(spec.P)]
+    hY = [torch.empty((w.T, w.H2), dtype=tdt, pin_memory=True) for _ in range(spec.P)]
+    for p in range(spec.P):
+        hX[p].copy_(calls[p][2].cpu())
+        hY[p].copy_(calls[p][3].cpu())
+    ids = np.ascontiguousarray(w.ids, dtype=np.int32)
+    h_seg = torch.empty(w.num_adapters + 1, dtype=torch.int32, pin_memory=True)
+    h_idx = torch.empty(w.num_adapters, dtype=torch.int32, pin_memory=True)
+    d_seg = torch.empty(w.num_adapters + 1, dtype=torch.int32, device=dev)
+    d_idx = torch.empty(w.num_adapters, dtype=torch.int32, device=dev)
+    dX = [torch.empty((w.T, w.H1), dtype=tdt, device=dev) for _ in range(spec.P)]
+    dY = [torch.empty((w.T, w.H2), dtype=tdt, device=dev) for _ in range(spec.P)]
+    outY = [torch.empty((w.T, w.H2), dtype=tdt, pin_memory=True) for _ in range(spec.P)]
+    ws_bytes = sgmv.lora_sgmv_workspace_bytes(w.T, w.r)
+    ws = torch.empty(ws_bytes // 4, dtype=torch.float32, device=dev)
+    sh = stream.cuda_stream
+    h2d = d2h = 0
+
+    def one(i):
+        nonlocal h2d, d2h
+        l = i % spec.L
+        seg, idx, _ = sgmv.lora_sgmv_group_segments(ids, w.num_adapters)
+        n = len(idx)
+        h_seg[: n + 1].copy_(torch.from_numpy(seg))
+        h_idx[:n].copy_(torch.from_numpy(idx))
+        max_len = int(np.max(np.diff(seg)))
+        with torch.cuda.stream(stream):
+            d_seg[: n + 1].copy_(h_seg[: n + 1], non_blocking=True)
+            d_idx[:n].copy_(h_idx[:n], non_blocking=True)
+            b_in = (n + 1 + n) * 4
+            b_out = 0
+            for p in range(spec.P):
+                _, _, _, _, A_ptrs, B_ptrs = calls[l * spec.P + p]
+                dX[p].copy_(hX[p], non_blocking=True)
+                dY[p].copy_(hY[p], non_blocking=True)
+                sgmv.lora_sgmv_apply(dY[p], dX[p], A_ptrs, B_ptrs, d_seg, d_idx, n, w.num_adapters, w.T, w.H1, w.r,
+                                     w.H2, w.scale, dt, max_len, ws, ws_bytes, None, sh)
+                outY[p].copy_(dY[p], non_blocking=True)
+                b_in += hX[p].numel() * 2 + hY[p].numel() * 2
+                b_out += outY[p].numel() * 2
+        stream.synchronize()
+        h2d, d2h = b_in, b_out
+
+    for i in range(3):
+        one(i)
+    t0 = time.perf_counter()
+    for i in range(steps):
+        one(i)
+    el = time.perf_counter() - t0
+    return {"value": round(w.T * steps / el, 1), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(d2h), "steps": steps,
+            "note": "wall clock; per step: host grouping, pinned H2D of X, Y and segments, "
+                    f"{spec.P} lora_sgmv_apply calls, D2H of Y, stream sync"}
+
+
+# ---------------------------------------------------------------------------------------------
+# reference arm: the oracle on the host cores
+# ---------------------------------------------------------------------------------------------
+
+def run_reference(args, spec: Spec, rank: int):
+    if rank != 0:
+        return None
+    per_step = max(1.0, min(10.0, 120.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_baseline(spec, per_step / 4)
+    t0 = time.perf_counter()
+    runs = [oracle_baseline(spec, per_step) for _ in range(args.steps)]
+    el = time.perf_counter() - t0
+    value = statistics.median(r["value"] for r in runs)
+    return {
+        "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": 0, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(el * 1e3 / max(1, args.steps), 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": spec.w.dtype, "data": "synthetic",
+        "config": {"workload": spec.desc, "name": spec.name, "T": spec.w.T},
+        "impl": "reference",
+        "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": runs[0]["sample"]},
+        "e2e": {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="distinct", choices=["distinct"] + list(inputs.CONFIGS))
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    rank, world, local = dist_env()
+    spec = make_spec(args.workload)
+    if args.impl == "reference":
+        out = run_reference(args, spec, rank)
+        if out:
+            print(json.dumps(out), flush=True)
+        return
+    result = run_ours(args, spec, rank, world, local)
+    if rank == 0 and result is not None:
+        if world == 1 and not args.no_cpu_baseline:
+            result["cpu_baseline"] = oracle_baseline(spec, args.cpu_seconds)
+        print(json.dumps(result), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,208 @@
+/*
+ * lora_sgmv.h -- C ABI of the SGMV library for NVIDIA B200 (sm_100a).
+ *
+ * SGMV ("Segmented Gather Matrix-Vector multiplication", Punica README,
+ * "Punica: Serving multiple LoRA finetuned LLM as one", the paragraph that
+ * names the kernel) computes the LoRA term of a batch in which each token
+ * uses its own adapter. The README's LoRA paragraph fixes the shapes: a
+ * frozen weight W is [H1, H2]; an adapter adds A [H1, r] and B [r, H2];
+ * y = x@(W + A@B) = x@W + x@A@B. Its multi-LoRA paragraph fixes the batch
+ * form: Y = X@W + (x1@A1@B1, ..., xn@An@Bn). This library adds the second
+ * term onto a Y that already holds X@W:
+ *
+ *     for every segment s, i = lora_idx[s], every row t in
+ *     [seg_starts[s], seg_starts[s+1]):
+ *         Y[t, :] += scale * (X[t, :] @ A_i) @ B_i
+ *
+ * computed as a shrink V = X@A_i (H1 -> r, fp32 result) and an expand
+ * Y += scale * V@B_i (r -> H2) with the add fused in.
+ *
+ * Conventions shared by every entry point
+ *   - Layout: all matrices row-major and dense. X is [T, H1], Y is [T, H2],
+ *     V is [T, r] fp32, A_i is [H1, r], B_i is [r, H2]. Rows are tokens.
+ *   - Storage type: fp16 or bf16 for X, Y, A_i, B_i (one type per call);
+ *     products are accumulated in fp32; V is fp32 and never rounded; Y is
+ *     rounded once, to nearest even, after the add.
+ *   - Pointers marked "device" are CUDA device pointers on the current
+ *     device; "host" pointers are ordinary CPU memory. The caller owns all
+ *     memory. Nothing is retained after a call returns and the library never
+ *     allocates device memory on the path of a call.
+ *   - Adapter tables: A_ptrs and B_ptrs are device arrays of num_adapters
+ *     device pointers; entry i points at A_i (resp. B_i). Adapters stay
+ *     resident in device memory between calls; only the table is passed.
+ *   - Segments: seg_starts is a device int32 array of n_segments+1 entries,
+ *     lora_idx a device int32 array of n_segments entries. Segments may come
+ *     in any order, may repeat an adapter, and may be empty (a no-op). Rows
+ *     outside every segment are never written.
+ *   - Asynchrony: every call only enqueues work on `stream` (a cudaStream_t
+ *     passed as void*; NULL is the legacy default stream) and returns. The
+ *     return value reports host-side validation and launch errors only; on
+ *     any error nothing is launched.
+ *   - Device-side checks: the segment arrays and pointer tables live on the
+ *     device and are checked by the kernels, per segment. A segment with
+ *     bounds outside 0 <= seg_starts[s] <= seg_starts[s+1] <= T, an adapter
+ *     id outside [0, num_adapters), or a null or non-16-byte-aligned table
+ *     entry is skipped and the matching LORA_SGMV_DEV_* bit is OR-ed into
+ *     *dev_status (a device uint32; may be NULL). No kernel traps.
+ *   - Alignment: X, Y, V and workspace must be 16-byte aligned; H1 and H2
+ *     must be multiples of 8.
+ *   - Thread safety: calls on different streams may run concurrently. The
+ *     library keeps no mutable global state other than a lazily filled,
+ *     mutex-guarded cache of device facts and kernel attributes, and an
+ *     atomic count of kernel launches.
+ */
+#ifndef LORA_SGMV_H
+#define LORA_SGMV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    LORA_SGMV_F16 = 0,
+    LORA_SGMV_BF16 = 1
+} lora_sgmv_dtype;
+
+typedef enum {
+    LORA_SGMV_OK = 0,
+    LORA_SGMV_ERR_NULL = 1,        /* a required pointer is NULL */
+    LORA_SGMV_ERR_DIM = 2,         /* a size is negative, zero where it must not be, or too large */
+    LORA_SGMV_ERR_ALIGN = 3,       /* a pointer or a row pitch is not 16-byte aligned */
+    LORA_SGMV_ERR_DTYPE = 4,       /* unknown storage type */
+    LORA_SGMV_ERR_UNSUPPORTED = 5, /* rank r or variant not built into this library */
+    LORA_SGMV_ERR_CUDA = 6,        /* a CUDA runtime call or kernel launch failed */
+    LORA_SGMV_ERR_WORKSPACE = 7,   /* workspace missing or smaller than lora_sgmv_workspace_bytes() */
+    LORA_SGMV_ERR_RANGE = 8        /* a host-side value is out of range (e.g. an adapter id) */
+} lora_sgmv_status;
+
+/* Bits OR-ed into *dev_status by the kernels. */
+#define LORA_SGMV_DEV_BAD_SEGMENT 0x1u  /* segment bounds invalid: segment skipped */
+#define LORA_SGMV_DEV_BAD_ADAPTER 0x2u  /* lora_idx[s] outside [0, num_adapters): skipped */
+#define LORA_SGMV_DEV_BAD_POINTER 0x4u  /* table entry NULL or not 16-byte aligned: skipped */
+
+/* Which kernels lora_sgmv_apply_ex runs. AUTO lets the dispatcher choose. */
+typedef enum {
+    LORA_SGMV_VARIANT_AUTO = 0,
+    LORA_SGMV_VARIANT_SPLIT = 1,      /* split-K shrink kernel, then streaming expand kernel */
+    LORA_SGMV_VARIANT_GROUPED_TC = 2  /* tcgen05/TMEM grouped kernel for long segments */
+} lora_sgmv_variant;
+
+/* Ranks r built into this library: 8, 16, 32, 64 and 128 for the split
+ * kernels; 16, 32 and 64 for the grouped tensor-core kernel. */
+int32_t lora_sgmv_rank_supported(int32_t r, lora_sgmv_variant variant);
+
+/* Human-readable name of a status code. Never NULL. */
+const char* lora_sgmv_status_string(lora_sgmv_status status);
+
+/* Library version as major*10000 + minor*100 + patch. */
+int32_t lora_sgmv_version(void);
+
+/* Number of kernels the library has launched successfully in this process
+ * (all devices, all streams). For instrumentation: benchmarks read it before
+ * and after a timed region. */
+uint64_t lora_sgmv_launch_count(void);
+
+/*
+ * lora_sgmv_group_segments -- segment bookkeeping, on the host.
+ *
+ * Groups a batch of per-token adapter ids into contiguous segments (the
+ * "segmented" part of SGMV): one segment per adapter that has tokens, in
+ * ascending adapter id; tokens of one adapter keep their batch order.
+ *
+ *   ids          host, int32[T]: adapter id of each token, in batch order.
+ *   T            number of tokens, >= 0.
+ *   num_adapters ids must lie in [0, num_adapters); num_adapters >= 1.
+ *   seg_starts   host, int32[num_adapters + 1] out: seg_starts[0] = 0,
+ *                seg_starts[n] = T, strictly increasing.
+ *   lora_idx     host, int32[num_adapters] out: adapter of each segment.
+ *   perm         host, int32[T] out: perm[p] = batch index of the token that
+ *                goes to row p of the grouped batch.
+ *   n_segments   host, int32 out: n, the number of segments written.
+ *
+ * Returns LORA_SGMV_ERR_NULL, _DIM or _RANGE (an id out of range) without
+ * writing the outputs, else LORA_SGMV_OK. Runs in O(T + num_adapters).
+ */
+lora_sgmv_status lora_sgmv_group_segments(const int32_t* ids, int32_t T, int32_t num_adapters,
+                                          int32_t* seg_starts, int32_t* lora_idx, int32_t* perm,
+                                          int32_t* n_segments);
+
+/*
+ * lora_sgmv_shrink -- V[t, :] = X[t, :] @ A_{lora_idx[s]} for rows t of each segment.
+ *
+ * The H1 -> r half of x@A@B (README LoRA paragraph), fp32 accumulation.
+ *   V            device, fp32[T, r] out: rows of valid segments are
+ *                overwritten; other rows are untouched.
+ *   X            device, [T, H1] fp16/bf16.
+ *   A_ptrs       device table of num_adapters device pointers to A_i [H1, r].
+ *   seg_starts, lora_idx, n_segments, num_adapters: as in the conventions.
+ *   T, H1, r     sizes; r must satisfy lora_sgmv_rank_supported(r, SPLIT).
+ *   dtype        storage type of X and A_i.
+ *   dev_status   device uint32 or NULL.
+ *   stream       cudaStream_t as void*.
+ */
+lora_sgmv_status lora_sgmv_shrink(float* V, const void* X, const void* const* A_ptrs,
+                                  const int32_t* seg_starts, const int32_t* lora_idx,
+                                  int32_t n_segments, int32_t num_adapters, int32_t T, int32_t H1,
+                                  int32_t r, lora_sgmv_dtype dtype, uint32_t* dev_status,
+                                  void* stream);
+
+/*
+ * lora_sgmv_expand -- Y[t, :] = round(Y[t, :] + scale * V[t, :] @ B_{lora_idx[s]}).
+ *
+ * The r -> H2 half, with the add onto the base output fused in; one rounding
+ * to the storage type per element.
+ *   Y            device, [T, H2] fp16/bf16, in/out.
+ *   V            device, fp32[T, r] (e.g. from lora_sgmv_shrink).
+ *   B_ptrs       device table of num_adapters device pointers to B_i [r, H2].
+ *   scale        multiplies the fp32 sum once, before the add.
+ *   other arguments as for lora_sgmv_shrink.
+ */
+lora_sgmv_status lora_sgmv_expand(void* Y, const float* V, const void* const* B_ptrs,
+                                  const int32_t* seg_starts, const int32_t* lora_idx,
+                                  int32_t n_segments, int32_t num_adapters, int32_t T, int32_t r,
+                                  int32_t H2, float scale, lora_sgmv_dtype dtype,
+                                  uint32_t* dev_status, void* stream);
+
+/* Bytes of workspace lora_sgmv_apply needs for T tokens at rank r (fp32 V,
+ * padded to 256 bytes). 0 if T or r is not positive. */
+size_t lora_sgmv_workspace_bytes(int32_t T, int32_t r);
+
+/*
+ * lora_sgmv_apply -- Y[t, :] += scale * (X[t, :] @ A_i) @ B_i, the whole SGMV.
+ *
+ *   Y, X, A_ptrs, B_ptrs, seg_starts, lora_idx, n_segments, num_adapters,
+ *   T, H1, r, H2, scale, dtype, dev_status, stream: as above.
+ *   max_seg_len  host hint: an upper bound on any segment's length, used only
+ *                to choose kernels and grid shapes; <= 0 means unknown (the
+ *                dispatcher then assumes ceil(T / n_segments)). Results do
+ *                not depend on it: a wrong hint costs speed, not correctness.
+ *   workspace    device scratch of at least lora_sgmv_workspace_bytes(T, r)
+ *                bytes, 16-byte aligned, owned by the caller; its contents
+ *                on entry do not matter. Calls that share a workspace must be
+ *                ordered on one stream.
+ */
+lora_sgmv_status lora_sgmv_apply(void* Y, const void* X, const void* const* A_ptrs,
+                                 const void* const* B_ptrs, const int32_t* seg_starts,
+                                 const int32_t* lora_idx, int32_t n_segments, int32_t num_adapters,
+                                 int32_t T, int32_t H1, int32_t r, int32_t H2, float scale,
+                                 lora_sgmv_dtype dtype, int32_t max_seg_len, void* workspace,
+                                 size_t workspace_bytes, uint32_t* dev_status, void* stream);
+
+/* lora_sgmv_apply with the kernels chosen by the caller. GROUPED_TC returns
+ * LORA_SGMV_ERR_UNSUPPORTED for ranks or types it does not cover. */
+lora_sgmv_status lora_sgmv_apply_ex(void* Y, const void* X, const void* const* A_ptrs,
+                                    const void* const* B_ptrs, const int32_t* seg_starts,
+                                    const int32_t* lora_idx, int32_t n_segments,
+                                    int32_t num_adapters, int32_t T, int32_t H1, int32_t r,
+                                    int32_t H2, float scale, lora_sgmv_dtype dtype,
+                                    int32_t max_seg_len, void* workspace, size_t workspace_bytes,
+                                    uint32_t* dev_status, lora_sgmv_variant variant, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LORA_SGMV_H */

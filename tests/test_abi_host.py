@@ -1,0 +1,135 @@
+"""Host-side checks of the C-ABI library; no GPU needed and no kernel is launched.
+
+- the library loads and exports every function include/lora_sgmv.h declares;
+- segment bookkeeping (host C++) is bit-exact against the oracle's grouping;
+- every host-side validation error returns its code before any CUDA call.
+"""
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+from adapter_matmul_b200 import inputs, sgmv
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "lora_sgmv.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(lora_sgmv_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_the_binding_exports():
+    assert declared_functions() == sorted(sgmv.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol():
+    lib = sgmv.load()
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_version_and_ranks():
+    assert sgmv.lora_sgmv_version() >= 100
+    for r in (8, 16, 32, 64, 128):
+        assert sgmv.lora_sgmv_rank_supported(r, sgmv.VARIANT_SPLIT)
+    for r in (0, 4, 24, 256):
+        assert not sgmv.lora_sgmv_rank_supported(r, sgmv.VARIANT_SPLIT)
+    assert sgmv.lora_sgmv_workspace_bytes(32, 16) == 2048
+    assert sgmv.lora_sgmv_workspace_bytes(3, 8) == 256
+    assert sgmv.lora_sgmv_workspace_bytes(0, 8) == 0
+    for st in range(9):
+        assert sgmv.status_string(st)
+
+
+# ---- bookkeeping: bit-exact against the oracle ---------------------------------------------
+
+@pytest.mark.parametrize("name", ["tiny", "distinct", "uniform_h4096", "skewed_h4096", "identical_h4096",
+                                  "prefill", "llama70b_decode_h28672"])
+def test_group_segments_bit_exact_on_configs(name):
+    w = inputs.make(name)
+    got = sgmv.lora_sgmv_group_segments(w.ids, w.num_adapters)
+    ref = oracle.group_segments(w.ids, w.num_adapters)
+    for g, o in zip(got, ref):
+        assert g.dtype == np.int32 and np.array_equal(g, o)
+
+
+def test_group_segments_bit_exact_random_and_edges():
+    rng = np.random.default_rng(0)
+    cases = [np.zeros(0, np.int32), np.array([5], np.int32), np.full(100, 3, np.int32),
+             np.arange(50, dtype=np.int32)[::-1].copy()]
+    for _ in range(200):
+        T = int(rng.integers(1, 300))
+        A = int(rng.integers(1, 70))
+        cases.append(rng.integers(0, A, T).astype(np.int32))
+    for ids in cases:
+        A = int(ids.max()) + 1 if ids.size else 1
+        A += int(rng.integers(0, 3))
+        got = sgmv.lora_sgmv_group_segments(ids, A)
+        ref = oracle.group_segments(ids, A)
+        for g, o in zip(got, ref):
+            assert np.array_equal(g, o)
+
+
+def test_group_segments_errors():
+    with pytest.raises(sgmv.SGMVError) as e:
+        sgmv.lora_sgmv_group_segments(np.array([0, 4], np.int32), 4)
+    assert e.value.status == 8
+    with pytest.raises(sgmv.SGMVError) as e:
+        sgmv.lora_sgmv_group_segments(np.array([0, -1], np.int32), 4)
+    assert e.value.status == 8
+    with pytest.raises(sgmv.SGMVError) as e:
+        sgmv.lora_sgmv_group_segments(np.array([0], np.int32), 0)
+    assert e.value.status == 2
+    lib = sgmv.load()
+    assert lib.lora_sgmv_group_segments(None, 3, 4, None, None, None, None) == 1
+
+
+# ---- host validation: every error path returns before touching the GPU ------------------------
+
+FAKE = 1 << 20  # a 16-byte-aligned non-null value; never dereferenced on these paths
+MIS = FAKE + 2  # misaligned
+
+
+def apply(**kw):
+    a = dict(Y=FAKE, X=FAKE, A=FAKE, B=FAKE, seg=FAKE, idx=FAKE, n=2, na=4, T=8, H1=256, r=16, H2=256,
+             scale=1.0, dt=0, mx=0, ws=FAKE, wsb=1 << 20, st=None, var=0)
+    a.update(kw)
+    return sgmv.load().lora_sgmv_apply_ex(a["Y"], a["X"], a["A"], a["B"], a["seg"], a["idx"], a["n"], a["na"],
+                                          a["T"], a["H1"], a["r"], a["H2"], a["scale"], a["dt"], a["mx"], a["ws"],
+                                          a["wsb"], a["st"], a["var"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(dt=7), 4), (dict(n=-1), 2), (dict(T=-1), 2), (dict(H1=0), 2), (dict(H2=-8), 2), (dict(r=0), 2),
+    (dict(r=24), 5), (dict(r=256), 5), (dict(var=9), 5),
+    (dict(Y=None), 1), (dict(X=None), 1), (dict(A=None), 1), (dict(B=None), 1), (dict(seg=None), 1),
+    (dict(idx=None), 1), (dict(na=0), 2),
+    (dict(Y=MIS), 3), (dict(X=MIS), 3), (dict(H1=260), 3), (dict(H2=100), 3),
+    (dict(ws=None), 7), (dict(wsb=100), 7), (dict(ws=MIS), 3),
+])
+def test_apply_validation_codes(kw, code):
+    assert apply(**kw) == code
+
+
+def test_empty_problems_are_noops_without_gpu():
+    # n_segments == 0 or T == 0 returns OK before any CUDA call, even with NULL pointers
+    assert apply(n=0, Y=None, X=None) == 0
+    assert apply(T=0, Y=None) == 0
+    lib = sgmv.load()
+    assert lib.lora_sgmv_shrink(None, None, None, None, None, 0, 1, 5, 64, 16, 0, None, None) == 0
+    assert lib.lora_sgmv_expand(None, None, None, None, None, 3, 1, 0, 16, 64, 1.0, 0, None, None) == 0
+
+
+def test_shrink_expand_validation_codes():
+    lib = sgmv.load()
+    sh = lambda **k: lib.lora_sgmv_shrink(k.get("V", FAKE), k.get("X", FAKE), FAKE, FAKE, FAKE, 2, 4, 8,
+                                          k.get("H1", 256), k.get("r", 16), k.get("dt", 0), None, None)
+    ex = lambda **k: lib.lora_sgmv_expand(k.get("Y", FAKE), k.get("V", FAKE), FAKE, FAKE, FAKE, 2, 4, 8,
+                                          k.get("r", 16), k.get("H2", 256), 1.0, k.get("dt", 0), None, None)
+    assert sh(V=None) == 1 and sh(X=MIS) == 3 and sh(H1=12) == 3 and sh(r=12) == 5 and sh(dt=3) == 4
+    assert ex(Y=None) == 1 and ex(V=MIS) == 3 and ex(H2=12) == 3 and ex(r=7) == 5 and ex(dt=-1) == 4

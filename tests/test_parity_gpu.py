@@ -1,0 +1,195 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle, element by element.
+
+Tolerance (written here, from the method's stated bar for fp16/bf16 outputs):
+|gpu - oracle| <= 2e-2 + 1e-2 * |oracle| per element. The oracle accumulates in
+fp32 in ascending order; the kernels accumulate in fp32 in another order, so
+results differ by rounding only. Bookkeeping and untouched rows are bit-exact.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from adapter_matmul_b200 import inputs, sgmv
+from gpu_helpers import DeviceProblem, assert_close, decode, dt_code, from_dev, to_dev
+
+pytestmark = pytest.mark.gpu
+
+SMALL_CONFIGS = ["tiny", "distinct", "uniform_h4096", "uniform_h11008", "skewed_h4096", "skewed_h11008",
+                 "identical_h4096", "identical_h11008"]
+
+
+@pytest.mark.parametrize("name", SMALL_CONFIGS)
+@pytest.mark.parametrize("y_random", [False, True])
+def test_config_full_oracle(name, y_random):
+    w = inputs.make(name)
+    p = DeviceProblem(w, y_random=y_random)
+    got = p.apply()
+    ref = p.oracle_apply()
+    assert_close(got, ref, w.dtype, name)
+    assert int(p.status.item()) == 0
+
+
+@pytest.mark.parametrize("name", ["distinct", "skewed_h11008"])
+def test_config_bf16_variant(name):
+    w = inputs.make(name)
+    w.dtype = "bf16"
+    p = DeviceProblem(w, y_random=True)
+    assert_close(p.apply(), p.oracle_apply(), "bf16", name + "/bf16")
+
+
+@pytest.mark.parametrize("r", [8, 16, 32, 64, 128])
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+@pytest.mark.parametrize("T", [1, 37, 130])
+def test_ragged_random_shapes(r, dtype, T):
+    # H1, H2 not multiples of the tile sizes; segments of every length
+    w = inputs.small_random(T, 7, 264, 136, r, dtype, seed=T * 1000 + r)
+    p = DeviceProblem(w, y_random=True)
+    assert_close(p.apply(variant=sgmv.VARIANT_SPLIT), p.oracle_apply(), dtype, w.name)
+
+
+def _sampled_check(p: DeviceProblem, got: np.ndarray, n_samples: int, seed: int):
+    w = p.w
+    rng = np.random.default_rng(seed)
+    seg, idx = p.seg, p.idx
+    owner = np.full(w.T, -1)
+    for s in range(len(idx)):
+        owner[seg[s]:seg[s + 1]] = idx[s]
+    rows = rng.integers(0, w.T, n_samples)
+    # always include the first and last row of every segment (ragged tile edges)
+    rows = np.concatenate([rows, seg[:-1], seg[1:] - 1])
+    cols = rng.integers(0, w.H2, rows.shape[0])
+    cols[: len(seg) - 1] = w.H2 - 1
+    worst = 0.0
+    for t, c in zip(rows, cols):
+        i = int(owner[t])
+        exp = oracle.apply_f32_element(p.x_bits[t], p.A[i], p.B[i], int(p.y_bits[t, c]), int(c), w.scale, w.dtype)
+        g, o = decode(np.array([got[t, c]], np.uint16), w.dtype)[0], decode(np.array([exp], np.uint16), w.dtype)[0]
+        assert abs(g - o) <= 2e-2 + 1e-2 * abs(o), (t, c, g, o)
+        worst = max(worst, abs(g - o))
+    assert np.all(np.isfinite(decode(got, w.dtype)))
+    return worst
+
+
+@pytest.mark.parametrize("name", ["prefill", "llama70b_decode_h28672", "llama70b_decode_h8192"])
+def test_full_size_sampled(name):
+    """Full-size configurations in the launch configuration the benchmark uses (AUTO)."""
+    w = inputs.make(name)
+    p = DeviceProblem(w, y_random=True)
+    got = p.apply()
+    _sampled_check(p, got, 400, 1)
+    assert int(p.status.item()) == 0
+
+
+def test_prefill_split_variant_sampled():
+    w = inputs.make("prefill")
+    p = DeviceProblem(w, y_random=True)
+    got = p.apply(variant=sgmv.VARIANT_SPLIT)
+    _sampled_check(p, got, 300, 2)
+
+
+# ---- shrink and expand entry points on their own ----------------------------------------------
+
+@pytest.mark.parametrize("name", ["skewed_h4096", "tiny"])
+def test_shrink_and_expand_entry_points(name):
+    w = inputs.make(name)
+    p = DeviceProblem(w, y_random=True)
+    A = [p.A.get(i, np.zeros((w.H1, w.r), np.uint16)) for i in range(w.num_adapters)]
+    B = [p.B.get(i, np.zeros((w.r, w.H2), np.uint16)) for i in range(w.num_adapters)]
+    V = torch.full((w.T, w.r), float("nan"), dtype=torch.float32, device="cuda")
+    sgmv.lora_sgmv_shrink(V, p.X, p.A_ptrs, p.d_seg, p.d_idx, p.n, w.num_adapters, w.T, w.H1, w.r,
+                          dt_code(w.dtype), p.status)
+    torch.cuda.synchronize()
+    Vo, _ = oracle.shrink_f32(p.x_bits, A, p.seg, p.idx, w.r, w.dtype)
+    np.testing.assert_allclose(V.cpu().numpy(), Vo, rtol=1e-4, atol=1e-4)
+    # expand from the oracle's V (uploaded): isolates the expand kernel
+    Vd = torch.from_numpy(Vo).cuda()
+    sgmv.lora_sgmv_expand(p.Y, Vd, p.B_ptrs, p.d_seg, p.d_idx, p.n, w.num_adapters, w.T, w.r, w.H2, 0.5,
+                          dt_code(w.dtype), p.status)
+    torch.cuda.synchronize()
+    ref, _ = oracle.expand_f32(p.y_bits, Vo, B, p.seg, p.idx, 0.5, w.dtype)
+    assert_close(from_dev(p.Y), ref, w.dtype, name + " expand")
+    assert int(p.status.item()) == 0
+
+
+# ---- segment semantics and edge cases --------------------------------------------------------
+
+def _custom(seg, idx, T=24, H1=512, H2=264, r=16, dtype="f16", na=5, seed=3):
+    w = inputs.small_random(T, na, H1, H2, r, dtype, seed=seed)
+    return DeviceProblem(w, y_random=True, adapters=list(range(na)), seg_starts=seg, lora_idx=idx)
+
+
+def test_no_segments_is_noop():
+    p = _custom([0], [])
+    before = from_dev(p.Y)
+    got = p.apply()
+    assert np.array_equal(got, before)
+
+
+def test_empty_repeated_unsorted_segments_and_uncovered_rows():
+    # rows 0..1 and 22..23 uncovered; empty segments; adapter 3 twice; unsorted ids
+    seg = [2, 2, 7, 7, 15, 16, 22]
+    idx = [4, 3, 0, 3, 1, 2]
+    p = _custom(seg, idx)
+    before = from_dev(p.Y)
+    got = p.apply()
+    ref = p.oracle_apply()
+    assert_close(got, ref, "f16", "custom segments")
+    for t in (0, 1, 22, 23):
+        assert np.array_equal(got[t], before[t])
+    assert int(p.status.item()) == 0
+
+
+def test_bad_segments_are_skipped_and_reported():
+    # [4,2) reversed; adapter 9 out of range; adapter 2 has a null table entry; [20,30) past T
+    seg = np.array([0, 4, 2, 8, 12, 16, 20, 30], np.int32)
+    idx = np.array([0, 1, 9, 3, 2, 4, 1], np.int32)
+    p = _custom(seg, idx)
+    p.A_ptrs[2] = 0
+    before = from_dev(p.Y)
+    got = p.apply()
+    st = int(p.status.item())
+    assert st & sgmv.DEV_BAD_SEGMENT and st & sgmv.DEV_BAD_ADAPTER and st & sgmv.DEV_BAD_POINTER
+    # valid segments: [0,4) adapter 0, [8,12) adapter 3, [16,20) adapter 4
+    ref = DeviceProblem(p.w, y_random=True, adapters=list(range(5)), seg_starts=[0, 4, 8, 12, 16, 20],
+                        lora_idx=[0, 0, 3, 3, 4]).oracle_apply()
+    for t in list(range(0, 4)) + list(range(8, 12)) + list(range(16, 20)):
+        assert_close(got[t:t + 1], ref[t:t + 1], "f16", f"row {t}")
+    for t in list(range(4, 8)) + list(range(12, 16)) + list(range(20, 24)):
+        assert np.array_equal(got[t], before[t]), t
+
+
+@pytest.mark.parametrize("scale", [0.0, -0.75, 2.0])
+def test_scale(scale):
+    p = _custom([0, 10, 24], [1, 3])
+    before = from_dev(p.Y)
+    got = p.apply(scale=scale)
+    assert_close(got, p.oracle_apply(scale=scale), "f16", f"scale {scale}")
+    if scale == 0.0:
+        assert np.array_equal(got, before)
+
+
+def test_deterministic_bits():
+    w = inputs.make("skewed_h11008")
+    p1 = DeviceProblem(w, y_random=True)
+    p2 = DeviceProblem(w, y_random=True)
+    assert np.array_equal(p1.apply(), p2.apply())
+
+
+def test_wrong_length_hint_still_correct():
+    w = inputs.make("skewed_h4096")
+    for hint in (1, 1000, 0):
+        p = DeviceProblem(w, y_random=True)
+        assert_close(p.apply(max_seg_len=hint), p.oracle_apply(), w.dtype, f"hint {hint}")
+
+
+def test_large_h1_and_many_segments():
+    # H1 = 16384 (largest shrink slice), 300 segments of mixed length
+    rng = np.random.default_rng(4)
+    lens = rng.integers(0, 5, 300)
+    seg = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    T = int(seg[-1])
+    idx = rng.integers(0, 6, 300).astype(np.int32)
+    w = inputs.small_random(T, 6, 16384, 520, 32, "bf16", seed=8)
+    p = DeviceProblem(w, y_random=True, adapters=list(range(6)), seg_starts=seg, lora_idx=idx)
+    assert_close(p.apply(), p.oracle_apply(), "bf16", "H1=16384")
