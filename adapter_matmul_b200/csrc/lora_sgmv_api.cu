@@ -387,3 +387,62 @@ lora_sgmv_status lora_sgmv_apply(void* Y, const void* X, const void* const* A_pt
 }
 
 }  // extern "C"
+
+// ---- apply for callers that cannot allocate device memory -----------------------------------
+//
+// Some callers cannot call cudaMalloc or any other allocator when they run
+// SGMV: code that runs inside a region where allocation is forbidden (a
+// real-time serving loop whose memory is fixed at start-up, a plugin whose
+// host framework owns all device memory), or code with no allocator handle at
+// all. lora_sgmv_apply_noalloc serves them: it runs the split kernels with
+// their fp32 V scratch in the fixed array below instead of a caller workspace.
+
+namespace {
+constexpr size_t kNoAllocMaxFloats = size_t(1) << 20;  // T * r <= 1,048,576 (4 MiB of fp32 V)
+constexpr int kNoAllocMaxDevices = 64;
+}  // namespace
+
+// Held on every device that loads this library, until the process exits.
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocMaxFloats];
+
+namespace {
+std::mutex g_noalloc_mu;
+float* g_noalloc_addr[kNoAllocMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on the current device. The name of a
+// __device__ array in host code is only a host-side stand-in; the address a
+// kernel may use comes from cudaGetSymbolAddress, once per device, with that
+// device current.
+lora_sgmv_status noalloc_scratch(float** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return LORA_SGMV_ERR_CUDA;
+    if (dev < 0 || dev >= kNoAllocMaxDevices) return LORA_SGMV_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (g_noalloc_addr[dev] == nullptr) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return LORA_SGMV_ERR_CUDA;
+        g_noalloc_addr[dev] = static_cast<float*>(p);
+    }
+    *out = g_noalloc_addr[dev];
+    return LORA_SGMV_OK;
+}
+}  // namespace
+
+extern "C" lora_sgmv_status lora_sgmv_apply_noalloc(void* Y, const void* X, const void* const* A_ptrs,
+                                                    const void* const* B_ptrs, const int32_t* seg_starts,
+                                                    const int32_t* lora_idx, int32_t n_segments,
+                                                    int32_t num_adapters, int32_t T, int32_t H1, int32_t r,
+                                                    int32_t H2, float scale, lora_sgmv_dtype dtype,
+                                                    int32_t max_seg_len, uint32_t* dev_status, void* stream) {
+    if (T > 0 && r > 0 && static_cast<size_t>(T) * static_cast<size_t>(r) > kNoAllocMaxFloats)
+        return LORA_SGMV_ERR_WORKSPACE;
+    lora_sgmv_status st = check_common(n_segments, num_adapters, T, dtype);
+    if (st != LORA_SGMV_OK) return st;
+    if (n_segments == 0 || T == 0) return LORA_SGMV_OK;
+    float* scratch = nullptr;
+    st = noalloc_scratch(&scratch);
+    if (st != LORA_SGMV_OK) return st;
+    return lora_sgmv_apply_ex(Y, X, A_ptrs, B_ptrs, seg_starts, lora_idx, n_segments, num_adapters, T, H1, r, H2,
+                              scale, dtype, max_seg_len, scratch, kNoAllocMaxFloats * sizeof(float), dev_status,
+                              LORA_SGMV_VARIANT_SPLIT, stream);
+}

@@ -36,7 +36,7 @@ STATUS_NAMES = {0: "OK", 1: "ERR_NULL", 2: "ERR_DIM", 3: "ERR_ALIGN", 4: "ERR_DT
 EXPORTS = [
     "lora_sgmv_rank_supported", "lora_sgmv_status_string", "lora_sgmv_version", "lora_sgmv_launch_count",
     "lora_sgmv_group_segments", "lora_sgmv_shrink", "lora_sgmv_expand", "lora_sgmv_workspace_bytes",
-    "lora_sgmv_apply", "lora_sgmv_apply_ex",
+    "lora_sgmv_apply", "lora_sgmv_apply_ex", "lora_sgmv_apply_noalloc",
 ]
 
 _lock = threading.Lock()
@@ -86,6 +86,9 @@ def load(path: Optional[str] = None):
         lib.lora_sgmv_apply_ex.restype = ctypes.c_int
         lib.lora_sgmv_apply_ex.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, ctypes.c_float,
                                            ctypes.c_int, i32, P, u64, P, ctypes.c_int, P]
+        lib.lora_sgmv_apply_noalloc.restype = ctypes.c_int
+        lib.lora_sgmv_apply_noalloc.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, ctypes.c_float,
+                                                ctypes.c_int, i32, P, P]
         if path is None:
             _lib = lib
         return lib
@@ -184,6 +187,16 @@ def lora_sgmv_apply_ex(Y, X, A_ptrs, B_ptrs, seg_starts, lora_idx, n_segments: i
                                      n_segments, num_adapters, T, H1, r, H2, float(scale), dtype, max_seg_len,
                                      _p(workspace), workspace_bytes, _p(dev_status), variant, _stream(stream)),
            "lora_sgmv_apply_ex")
+
+
+def lora_sgmv_apply_noalloc(Y, X, A_ptrs, B_ptrs, seg_starts, lora_idx, n_segments: int, num_adapters: int,
+                            T: int, H1: int, r: int, H2: int, scale: float, dtype: int, max_seg_len: int,
+                            dev_status=None, stream=None) -> None:
+    """lora_sgmv_apply without a workspace: for callers that cannot allocate device memory."""
+    _check(load().lora_sgmv_apply_noalloc(_p(Y), _p(X), _p(A_ptrs), _p(B_ptrs), _p(seg_starts), _p(lora_idx),
+                                          n_segments, num_adapters, T, H1, r, H2, float(scale), dtype, max_seg_len,
+                                          _p(dev_status), _stream(stream)),
+           "lora_sgmv_apply_noalloc")
 
 
 def pointer_table(tensors: Sequence, device=None):

@@ -201,6 +201,37 @@ lora_sgmv_status lora_sgmv_apply_ex(void* Y, const void* X, const void* const* A
                                     int32_t max_seg_len, void* workspace, size_t workspace_bytes,
                                     uint32_t* dev_status, lora_sgmv_variant variant, void* stream);
 
+/*
+ * lora_sgmv_apply_noalloc -- lora_sgmv_apply for callers that cannot allocate.
+ *
+ * The Punica README has no counterpart to this entry point; it exists for
+ * callers that may not call cudaMalloc (or any allocator) where they run
+ * SGMV -- for example a serving loop whose device memory is fixed at
+ * start-up, or a plugin whose host framework owns all device memory -- and
+ * so cannot supply the workspace lora_sgmv_apply needs.
+ *
+ * It runs the split kernels (LORA_SGMV_VARIANT_SPLIT) with their fp32 V
+ * scratch in a fixed array inside the library: 1,048,576 floats (4 MiB),
+ * which every GPU that loads the library holds until the process exits. It
+ * allocates nothing. Arguments are those of lora_sgmv_apply without the
+ * workspace; T * r above 1,048,576 is rejected with LORA_SGMV_ERR_WORKSPACE
+ * before anything is launched.
+ *
+ * The first call on each device looks up the array's device address (once
+ * per device, with that device current); make that first call before any
+ * stream capture. Every call on a device shares the one array and leaves
+ * its last contents there (nothing in it needs to start at zero: each call
+ * writes every V row it reads). Calls whose kernels overlap on the GPU --
+ * on different streams, or from different threads -- race on the array and
+ * give wrong results: order them on one stream.
+ */
+lora_sgmv_status lora_sgmv_apply_noalloc(void* Y, const void* X, const void* const* A_ptrs,
+                                         const void* const* B_ptrs, const int32_t* seg_starts,
+                                         const int32_t* lora_idx, int32_t n_segments,
+                                         int32_t num_adapters, int32_t T, int32_t H1, int32_t r,
+                                         int32_t H2, float scale, lora_sgmv_dtype dtype,
+                                         int32_t max_seg_len, uint32_t* dev_status, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
