@@ -13,6 +13,7 @@
 #include <vector>
 
 #include "../../include/lora_sgmv.h"
+#include "sgmv_fused.cuh"
 #include "sgmv_grouped_tc.cuh"
 #include "sgmv_split.cuh"
 
@@ -179,6 +180,99 @@ int estimate_max_len(int max_seg_len, int T, int n) {
     return n > 0 ? (T + n - 1) / n : T;
 }
 
+// ---- fused path ---------------------------------------------------------------------------
+
+int round8(int v) { return (v + 7) / 8 * 8; }
+
+// Largest number of clusters of the fused kernel that can be resident at once, per device.
+template <typename K>
+lora_sgmv_status fused_max_clusters(K kernel, size_t smem, int* out, int* cache) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return LORA_SGMV_ERR_CUDA;
+    if (dev < 0 || dev >= 64) return LORA_SGMV_ERR_UNSUPPORTED;
+    {
+        std::lock_guard<std::mutex> lock(g_mu);
+        if (cache[dev] > 0) {
+            *out = cache[dev];
+            return LORA_SGMV_OK;
+        }
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(sgmv::kFusedCluster, 1, 1);
+    cfg.blockDim = dim3(sgmv::kFusedThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = sgmv::kFusedCluster;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess || n <= 0) return LORA_SGMV_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_mu);
+    cache[dev] = n;
+    *out = n;
+    return LORA_SGMV_OK;
+}
+
+template <typename T, int R>
+lora_sgmv_status launch_fused(sgmv::FusedParams P, int max_len, cudaStream_t stream) {
+    static int smem_done = 0;
+    static int clusters_cache[64] = {};
+    using G = sgmv::FusedGeom<R>;
+    const int C = sgmv::kFusedCluster;
+    for (int i = 0; i < P.n_problems; ++i) {
+        P.prob[i].ks = round8((P.prob[i].H1 + C - 1) / C);
+        P.prob[i].ns = round8((P.prob[i].H2 + C - 1) / C);
+    }
+    P.chunk_slots = chunk_slots(max_len, sgmv::kFusedTokens, 64);
+    const size_t smem = G::SMEM;
+    auto kernel = sgmv::sgmv_fused_kernel<T, R>;
+    if (ensure_smem(kernel, smem, smem_done) != LORA_SGMV_OK) return LORA_SGMV_ERR_CUDA;
+    int max_clusters = 0;
+    lora_sgmv_status st = fused_max_clusters(kernel, smem, &max_clusters, clusters_cache);
+    if (st != LORA_SGMV_OK) return st;
+    const long long jobs = static_cast<long long>(P.n_problems) * P.n_segments * P.chunk_slots;
+    if (jobs > (1ll << 30)) return LORA_SGMV_ERR_DIM;
+    int clusters = static_cast<int>(std::min<long long>(jobs, max_clusters));
+    // balance rounds: the same number of jobs per cluster where possible
+    const long long rounds = (jobs + clusters - 1) / clusters;
+    clusters = static_cast<int>((jobs + rounds - 1) / rounds);
+
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(clusters * C, 1, 1);
+    cfg.blockDim = dim3(sgmv::kFusedThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = C;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return counted(cudaLaunchKernelEx(&cfg, kernel, P));
+}
+
+template <typename T>
+lora_sgmv_status fused_dispatch_r(const sgmv::FusedParams& P, int r, int max_len, cudaStream_t s) {
+    switch (r) {
+        case 8: return launch_fused<T, 8>(P, max_len, s);
+        case 16: return launch_fused<T, 16>(P, max_len, s);
+        case 32: return launch_fused<T, 32>(P, max_len, s);
+        case 64: return launch_fused<T, 64>(P, max_len, s);
+        case 128: return launch_fused<T, 128>(P, max_len, s);
+    }
+    return LORA_SGMV_ERR_UNSUPPORTED;
+}
+
+lora_sgmv_status fused_dispatch(const sgmv::FusedParams& P, int r, lora_sgmv_dtype dt, int max_len,
+                                cudaStream_t s) {
+    return dt == LORA_SGMV_F16 ? fused_dispatch_r<__half>(P, r, max_len, s)
+                               : fused_dispatch_r<__nv_bfloat16>(P, r, max_len, s);
+}
+
 lora_sgmv_status check_common(int32_t n_segments, int32_t num_adapters, int32_t T, lora_sgmv_dtype dtype) {
     if (dtype != LORA_SGMV_F16 && dtype != LORA_SGMV_BF16) return LORA_SGMV_ERR_DTYPE;
     if (n_segments < 0 || T < 0 || num_adapters < 0) return LORA_SGMV_ERR_DIM;
@@ -198,6 +292,7 @@ int32_t lora_sgmv_rank_supported(int32_t r, lora_sgmv_variant variant) {
         case LORA_SGMV_VARIANT_AUTO:
         case LORA_SGMV_VARIANT_SPLIT: return split_rank(r) ? 1 : 0;
         case LORA_SGMV_VARIANT_GROUPED_TC: return sgmv::grouped_tc_rank(r) ? 1 : 0;
+        case LORA_SGMV_VARIANT_FUSED: return split_rank(r) ? 1 : 0;
     }
     return 0;
 }
@@ -317,7 +412,7 @@ lora_sgmv_status lora_sgmv_apply_ex(void* Y, const void* X, const void* const* A
     if (st != LORA_SGMV_OK) return st;
     if (H1 <= 0 || H2 <= 0 || r <= 0) return LORA_SGMV_ERR_DIM;
     if (variant != LORA_SGMV_VARIANT_AUTO && variant != LORA_SGMV_VARIANT_SPLIT &&
-        variant != LORA_SGMV_VARIANT_GROUPED_TC)
+        variant != LORA_SGMV_VARIANT_GROUPED_TC && variant != LORA_SGMV_VARIANT_FUSED)
         return LORA_SGMV_ERR_UNSUPPORTED;
     if (!lora_sgmv_rank_supported(r, variant)) return LORA_SGMV_ERR_UNSUPPORTED;
     if (n_segments == 0 || T == 0) return LORA_SGMV_OK;
@@ -334,7 +429,26 @@ lora_sgmv_status lora_sgmv_apply_ex(void* Y, const void* X, const void* const* A
     if (v == LORA_SGMV_VARIANT_AUTO)
         v = (max_len >= sgmv::kGroupedMinSegment && sgmv::grouped_tc_supported(r, H1, H2, dtype))
                 ? LORA_SGMV_VARIANT_GROUPED_TC
-                : LORA_SGMV_VARIANT_SPLIT;
+                : LORA_SGMV_VARIANT_FUSED;
+
+    if (v == LORA_SGMV_VARIANT_FUSED) {
+        sgmv::FusedParams P = {};
+        P.prob[0].Y = Y;
+        P.prob[0].X = X;
+        P.prob[0].A_ptrs = A_ptrs;
+        P.prob[0].B_ptrs = B_ptrs;
+        P.prob[0].num_adapters = num_adapters;
+        P.prob[0].H1 = H1;
+        P.prob[0].H2 = H2;
+        P.prob[0].scale = scale;
+        P.seg_starts = seg_starts;
+        P.lora_idx = lora_idx;
+        P.dev_status = dev_status;
+        P.n_problems = 1;
+        P.n_segments = n_segments;
+        P.T = T;
+        return fused_dispatch(P, r, dtype, max_len, s);
+    }
 
     if (v == LORA_SGMV_VARIANT_GROUPED_TC) {
         if (!sgmv::grouped_tc_supported(r, H1, H2, dtype)) return LORA_SGMV_ERR_UNSUPPORTED;
@@ -387,6 +501,45 @@ lora_sgmv_status lora_sgmv_apply(void* Y, const void* X, const void* const* A_pt
 }
 
 }  // extern "C"
+
+extern "C" lora_sgmv_status lora_sgmv_apply_batched(const lora_sgmv_problem* problems, int32_t n_problems,
+                                                    const int32_t* seg_starts, const int32_t* lora_idx,
+                                                    int32_t n_segments, int32_t T, int32_t r, lora_sgmv_dtype dtype,
+                                                    int32_t max_seg_len, uint32_t* dev_status, void* stream) {
+    if (dtype != LORA_SGMV_F16 && dtype != LORA_SGMV_BF16) return LORA_SGMV_ERR_DTYPE;
+    if (!problems) return LORA_SGMV_ERR_NULL;
+    if (n_problems < 1 || n_problems > LORA_SGMV_MAX_PROBLEMS || n_segments < 0 || T < 0 || r <= 0)
+        return LORA_SGMV_ERR_DIM;
+    if (!split_rank(r)) return LORA_SGMV_ERR_UNSUPPORTED;
+    sgmv::FusedParams P = {};
+    for (int i = 0; i < n_problems; ++i) {
+        const lora_sgmv_problem& q = problems[i];
+        if (q.H1 <= 0 || q.H2 <= 0 || q.num_adapters < 0) return LORA_SGMV_ERR_DIM;
+        if (n_segments > 0 && T > 0) {
+            if (!q.Y || !q.X || !q.A_ptrs || !q.B_ptrs) return LORA_SGMV_ERR_NULL;
+            if (q.num_adapters < 1) return LORA_SGMV_ERR_DIM;
+            if (!aligned16(q.Y) || !aligned16(q.X) || q.H1 % 8 || q.H2 % 8) return LORA_SGMV_ERR_ALIGN;
+        }
+        P.prob[i].Y = q.Y;
+        P.prob[i].X = q.X;
+        P.prob[i].A_ptrs = q.A_ptrs;
+        P.prob[i].B_ptrs = q.B_ptrs;
+        P.prob[i].num_adapters = q.num_adapters;
+        P.prob[i].H1 = q.H1;
+        P.prob[i].H2 = q.H2;
+        P.prob[i].scale = q.scale;
+    }
+    if (n_segments == 0 || T == 0) return LORA_SGMV_OK;
+    if (!seg_starts || !lora_idx) return LORA_SGMV_ERR_NULL;
+    P.seg_starts = seg_starts;
+    P.lora_idx = lora_idx;
+    P.dev_status = dev_status;
+    P.n_problems = n_problems;
+    P.n_segments = n_segments;
+    P.T = T;
+    return fused_dispatch(P, r, dtype, estimate_max_len(max_seg_len, T, n_segments),
+                          static_cast<cudaStream_t>(stream));
+}
 
 // ---- apply for callers that cannot allocate device memory -----------------------------------
 //

@@ -92,7 +92,7 @@ __global__ void __launch_bounds__(kShrinkThreads) sgmv_shrink_cluster_kernel(con
     const int lane = tid & 31;
     const int warp = tid >> 5;
 
-    extern __shared__ __align__(16) unsigned char smem[];
+    extern __shared__ __align__(128) unsigned char smem[];
     T* xs = reinterpret_cast<T*>(smem);
     float* red = reinterpret_cast<float*>(smem + size_t(TC) * p.ks * 2);
     float* part = red + NW * TC * R;

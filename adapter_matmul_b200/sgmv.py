@@ -25,10 +25,13 @@ BF16 = 1
 VARIANT_AUTO = 0
 VARIANT_SPLIT = 1
 VARIANT_GROUPED_TC = 2
+VARIANT_FUSED = 3
+MAX_PROBLEMS = 8
 
 DEV_BAD_SEGMENT = 0x1
 DEV_BAD_ADAPTER = 0x2
 DEV_BAD_POINTER = 0x4
+DEV_TIMEOUT = 0x8
 
 STATUS_NAMES = {0: "OK", 1: "ERR_NULL", 2: "ERR_DIM", 3: "ERR_ALIGN", 4: "ERR_DTYPE", 5: "ERR_UNSUPPORTED",
                 6: "ERR_CUDA", 7: "ERR_WORKSPACE", 8: "ERR_RANGE"}
@@ -36,8 +39,15 @@ STATUS_NAMES = {0: "OK", 1: "ERR_NULL", 2: "ERR_DIM", 3: "ERR_ALIGN", 4: "ERR_DT
 EXPORTS = [
     "lora_sgmv_rank_supported", "lora_sgmv_status_string", "lora_sgmv_version", "lora_sgmv_launch_count",
     "lora_sgmv_group_segments", "lora_sgmv_shrink", "lora_sgmv_expand", "lora_sgmv_workspace_bytes",
-    "lora_sgmv_apply", "lora_sgmv_apply_ex", "lora_sgmv_apply_noalloc",
+    "lora_sgmv_apply", "lora_sgmv_apply_ex", "lora_sgmv_apply_batched", "lora_sgmv_apply_noalloc",
 ]
+
+
+class Problem(ctypes.Structure):
+    """Mirror of lora_sgmv_problem."""
+    _fields_ = [("Y", ctypes.c_void_p), ("X", ctypes.c_void_p), ("A_ptrs", ctypes.c_void_p),
+                ("B_ptrs", ctypes.c_void_p), ("num_adapters", ctypes.c_int32), ("H1", ctypes.c_int32),
+                ("H2", ctypes.c_int32), ("scale", ctypes.c_float)]
 
 _lock = threading.Lock()
 _lib = None
@@ -86,6 +96,8 @@ def load(path: Optional[str] = None):
         lib.lora_sgmv_apply_ex.restype = ctypes.c_int
         lib.lora_sgmv_apply_ex.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, ctypes.c_float,
                                            ctypes.c_int, i32, P, u64, P, ctypes.c_int, P]
+        lib.lora_sgmv_apply_batched.restype = ctypes.c_int
+        lib.lora_sgmv_apply_batched.argtypes = [P, i32, P, P, i32, i32, i32, ctypes.c_int, i32, P, P]
         lib.lora_sgmv_apply_noalloc.restype = ctypes.c_int
         lib.lora_sgmv_apply_noalloc.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, ctypes.c_float,
                                                 ctypes.c_int, i32, P, P]
@@ -187,6 +199,21 @@ def lora_sgmv_apply_ex(Y, X, A_ptrs, B_ptrs, seg_starts, lora_idx, n_segments: i
                                      n_segments, num_adapters, T, H1, r, H2, float(scale), dtype, max_seg_len,
                                      _p(workspace), workspace_bytes, _p(dev_status), variant, _stream(stream)),
            "lora_sgmv_apply_ex")
+
+
+def lora_sgmv_apply_batched(problems, seg_starts, lora_idx, n_segments: int, T: int, r: int, dtype: int,
+                            max_seg_len: int, dev_status=None, stream=None) -> None:
+    """problems: sequence of dicts (Y, X, A_ptrs, B_ptrs, num_adapters, H1, H2, scale) or Problem structs."""
+    arr = (Problem * max(1, len(problems)))()
+    for i, q in enumerate(problems):
+        if isinstance(q, Problem):
+            arr[i] = q
+        else:
+            arr[i] = Problem(_p(q["Y"]), _p(q["X"]), _p(q["A_ptrs"]), _p(q["B_ptrs"]), int(q["num_adapters"]),
+                             int(q["H1"]), int(q["H2"]), float(q.get("scale", 1.0)))
+    _check(load().lora_sgmv_apply_batched(ctypes.addressof(arr), len(problems), _p(seg_starts), _p(lora_idx),
+                                          n_segments, T, r, dtype, max_seg_len, _p(dev_status), _stream(stream)),
+           "lora_sgmv_apply_batched")
 
 
 def lora_sgmv_apply_noalloc(Y, X, A_ptrs, B_ptrs, seg_starts, lora_idx, n_segments: int, num_adapters: int,

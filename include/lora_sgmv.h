@@ -33,7 +33,9 @@
  *   - Segments: seg_starts is a device int32 array of n_segments+1 entries,
  *     lora_idx a device int32 array of n_segments entries. Segments may come
  *     in any order, may repeat an adapter, and may be empty (a no-op). Rows
- *     outside every segment are never written.
+ *     outside every segment are never written. Segments must not overlap
+ *     (each row in at most one segment); overlapping rows give undefined
+ *     results.
  *   - Asynchrony: every call only enqueues work on `stream` (a cudaStream_t
  *     passed as void*; NULL is the legacy default stream) and returns. The
  *     return value reports host-side validation and launch errors only; on
@@ -82,16 +84,18 @@ typedef enum {
 #define LORA_SGMV_DEV_BAD_SEGMENT 0x1u  /* segment bounds invalid: segment skipped */
 #define LORA_SGMV_DEV_BAD_ADAPTER 0x2u  /* lora_idx[s] outside [0, num_adapters): skipped */
 #define LORA_SGMV_DEV_BAD_POINTER 0x4u  /* table entry NULL or not 16-byte aligned: skipped */
+#define LORA_SGMV_DEV_TIMEOUT 0x8u      /* a bounded wait inside a kernel gave up: results invalid */
 
 /* Which kernels lora_sgmv_apply_ex runs. AUTO lets the dispatcher choose. */
 typedef enum {
     LORA_SGMV_VARIANT_AUTO = 0,
     LORA_SGMV_VARIANT_SPLIT = 1,      /* split-K shrink kernel, then streaming expand kernel */
-    LORA_SGMV_VARIANT_GROUPED_TC = 2  /* tcgen05/TMEM grouped kernel for long segments */
+    LORA_SGMV_VARIANT_GROUPED_TC = 2, /* tcgen05/TMEM grouped kernel for long segments */
+    LORA_SGMV_VARIANT_FUSED = 3       /* one kernel: cluster shrink, DSMEM V reduction, expand */
 } lora_sgmv_variant;
 
-/* Ranks r built into this library: 8, 16, 32, 64 and 128 for the split
- * kernels; 16, 32 and 64 for the grouped tensor-core kernel. */
+/* Ranks r built into this library: 8, 16, 32, 64 and 128 for the split and
+ * fused kernels; 16, 32 and 64 for the grouped tensor-core kernel. */
 int32_t lora_sgmv_rank_supported(int32_t r, lora_sgmv_variant variant);
 
 /* Human-readable name of a status code. Never NULL. */
@@ -200,6 +204,42 @@ lora_sgmv_status lora_sgmv_apply_ex(void* Y, const void* X, const void* const* A
                                     int32_t H2, float scale, lora_sgmv_dtype dtype,
                                     int32_t max_seg_len, void* workspace, size_t workspace_bytes,
                                     uint32_t* dev_status, lora_sgmv_variant variant, void* stream);
+
+/* One projection of a batched call (see lora_sgmv_apply_batched). */
+typedef struct {
+    void* Y;                      /* device, [T, H2], in/out */
+    const void* X;                /* device, [T, H1] */
+    const void* const* A_ptrs;    /* device table of num_adapters pointers to A_i [H1, r] */
+    const void* const* B_ptrs;    /* device table of num_adapters pointers to B_i [r, H2] */
+    int32_t num_adapters;
+    int32_t H1;
+    int32_t H2;
+    float scale;
+} lora_sgmv_problem;
+
+/* Most problems lora_sgmv_apply_batched takes in one call. */
+#define LORA_SGMV_MAX_PROBLEMS 8
+
+/*
+ * lora_sgmv_apply_batched -- several SGMV problems that share one token
+ * grouping (e.g. the q, k, v and o projections of a decoder layer, whose
+ * tokens map to the same adapters) in a single kernel launch.
+ *
+ * For every problem p and segment s, rows t of the segment:
+ *     problems[p].Y[t, :] += problems[p].scale * (problems[p].X[t, :] @ A_i) @ B_i
+ * with i = lora_idx[s] and A_i, B_i taken from problem p's tables. Each
+ * problem may have its own H1, H2, tables and adapter count; r and dtype are
+ * shared. Runs the fused kernel (LORA_SGMV_VARIANT_FUSED), which keeps V on
+ * chip and needs no workspace.
+ *   problems     host array of n_problems entries, 1 <= n_problems <= 8.
+ *   other arguments as for lora_sgmv_apply.
+ * Validation errors of any problem are returned before anything is launched.
+ */
+lora_sgmv_status lora_sgmv_apply_batched(const lora_sgmv_problem* problems, int32_t n_problems,
+                                         const int32_t* seg_starts, const int32_t* lora_idx,
+                                         int32_t n_segments, int32_t T, int32_t r,
+                                         lora_sgmv_dtype dtype, int32_t max_seg_len,
+                                         uint32_t* dev_status, void* stream);
 
 /*
  * lora_sgmv_apply_noalloc -- lora_sgmv_apply for callers that cannot allocate.

@@ -37,6 +37,7 @@ def test_version_and_ranks():
     assert sgmv.lora_sgmv_version() >= 100
     for r in (8, 16, 32, 64, 128):
         assert sgmv.lora_sgmv_rank_supported(r, sgmv.VARIANT_SPLIT)
+        assert sgmv.lora_sgmv_rank_supported(r, sgmv.VARIANT_FUSED)
     for r in (0, 4, 24, 256):
         assert not sgmv.lora_sgmv_rank_supported(r, sgmv.VARIANT_SPLIT)
     assert sgmv.lora_sgmv_workspace_bytes(32, 16) == 2048
@@ -133,3 +134,25 @@ def test_shrink_expand_validation_codes():
                                           k.get("r", 16), k.get("H2", 256), 1.0, k.get("dt", 0), None, None)
     assert sh(V=None) == 1 and sh(X=MIS) == 3 and sh(H1=12) == 3 and sh(r=12) == 5 and sh(dt=3) == 4
     assert ex(Y=None) == 1 and ex(V=MIS) == 3 and ex(H2=12) == 3 and ex(r=7) == 5 and ex(dt=-1) == 4
+
+
+def test_batched_validation_codes():
+    lib = sgmv.load()
+
+    def call(n_problems=2, T=8, r=16, dt=0, n=2, **pk):
+        arr = (sgmv.Problem * 8)()
+        for i in range(8):
+            q = dict(Y=FAKE, X=FAKE, A=FAKE, B=FAKE, na=4, H1=256, H2=512, scale=1.0)
+            q.update(pk)
+            arr[i] = sgmv.Problem(q["Y"], q["X"], q["A"], q["B"], q["na"], q["H1"], q["H2"], q["scale"])
+        return lib.lora_sgmv_apply_batched(ctypes.addressof(arr), n_problems, FAKE, FAKE, n, T, r, dt, 0, None, None)
+
+    import ctypes
+    assert call(dt=5) == 4
+    assert call(n_problems=0) == 2 and call(n_problems=9) == 2
+    assert call(r=12) == 5
+    assert call(Y=None) == 1 and call(A=None) == 1
+    assert call(X=MIS) == 3 and call(H2=100) == 3
+    assert call(na=0) == 2 and call(H1=0) == 2
+    assert call(n=0, Y=None) == 0  # empty: OK before any CUDA call
+    assert lib.lora_sgmv_apply_batched(None, 1, FAKE, FAKE, 1, 1, 16, 0, 0, None, None) == 1

@@ -21,10 +21,11 @@ SMALL_CONFIGS = ["tiny", "distinct", "uniform_h4096", "uniform_h11008", "skewed_
 
 @pytest.mark.parametrize("name", SMALL_CONFIGS)
 @pytest.mark.parametrize("y_random", [False, True])
-def test_config_full_oracle(name, y_random):
+@pytest.mark.parametrize("variant", [sgmv.VARIANT_AUTO, sgmv.VARIANT_SPLIT])
+def test_config_full_oracle(name, y_random, variant):
     w = inputs.make(name)
     p = DeviceProblem(w, y_random=y_random)
-    got = p.apply()
+    got = p.apply(variant=variant)
     ref = p.oracle_apply()
     assert_close(got, ref, w.dtype, name)
     assert int(p.status.item()) == 0
@@ -41,11 +42,41 @@ def test_config_bf16_variant(name):
 @pytest.mark.parametrize("r", [8, 16, 32, 64, 128])
 @pytest.mark.parametrize("dtype", ["f16", "bf16"])
 @pytest.mark.parametrize("T", [1, 37, 130])
-def test_ragged_random_shapes(r, dtype, T):
-    # H1, H2 not multiples of the tile sizes; segments of every length
+@pytest.mark.parametrize("variant", [sgmv.VARIANT_SPLIT, sgmv.VARIANT_FUSED])
+def test_ragged_random_shapes(r, dtype, T, variant):
+    # H1, H2 not multiples of the tile sizes; segments of every length (several token chunks)
     w = inputs.small_random(T, 7, 264, 136, r, dtype, seed=T * 1000 + r)
     p = DeviceProblem(w, y_random=True)
-    assert_close(p.apply(variant=sgmv.VARIANT_SPLIT), p.oracle_apply(), dtype, w.name)
+    assert_close(p.apply(variant=variant), p.oracle_apply(), dtype, w.name)
+
+
+@pytest.mark.parametrize("r", [16, 64])
+def test_fused_long_rows_many_tiles(r):
+    # H1 and H2 span many stages per CTA (several A and B tiles) with ragged ends
+    w = inputs.small_random(40, 5, 8200, 11000, r, "bf16", seed=r)
+    p = DeviceProblem(w, y_random=True)
+    assert_close(p.apply(variant=sgmv.VARIANT_FUSED), p.oracle_apply(), "bf16", "long rows")
+
+
+def test_batched_projections_with_different_shapes():
+    # q/k/v/o-like problems sharing one token grouping, in one launch
+    ids = inputs.skewed(4096).ids
+    shapes = [(4096, 4096), (4096, 1024), (4096, 1024), (2048, 4096)]
+    probs, refs = [], []
+    for k, (H1, H2) in enumerate(shapes):
+        w = inputs.Workload(f"proj{k}", H1, H2, 16, "f16", ids, 64, 0.5 + 0.25 * k, seed=k)
+        p = DeviceProblem(w, y_random=True)
+        probs.append(p)
+        refs.append(p.oracle_apply())
+    p0 = probs[0]
+    sgmv.lora_sgmv_apply_batched(
+        [dict(Y=p.Y, X=p.X, A_ptrs=p.A_ptrs, B_ptrs=p.B_ptrs, num_adapters=p.w.num_adapters, H1=p.w.H1,
+              H2=p.w.H2, scale=p.w.scale) for p in probs],
+        p0.d_seg, p0.d_idx, p0.n, p0.w.T, 16, sgmv.F16, p0.max_len(), p0.status)
+    torch.cuda.synchronize()
+    for p, ref in zip(probs, refs):
+        assert_close(from_dev(p.Y), ref, "f16", p.w.name)
+    assert int(p0.status.item()) == 0
 
 
 def _sampled_check(p: DeviceProblem, got: np.ndarray, n_samples: int, seed: int):
@@ -140,14 +171,15 @@ def test_empty_repeated_unsorted_segments_and_uncovered_rows():
     assert int(p.status.item()) == 0
 
 
-def test_bad_segments_are_skipped_and_reported():
+@pytest.mark.parametrize("variant", [sgmv.VARIANT_SPLIT, sgmv.VARIANT_FUSED])
+def test_bad_segments_are_skipped_and_reported(variant):
     # [4,2) reversed; adapter 9 out of range; adapter 2 has a null table entry; [20,30) past T
     seg = np.array([0, 4, 2, 8, 12, 16, 20, 30], np.int32)
     idx = np.array([0, 1, 9, 3, 2, 4, 1], np.int32)
     p = _custom(seg, idx)
     p.A_ptrs[2] = 0
     before = from_dev(p.Y)
-    got = p.apply()
+    got = p.apply(variant=variant)
     st = int(p.status.item())
     assert st & sgmv.DEV_BAD_SEGMENT and st & sgmv.DEV_BAD_ADAPTER and st & sgmv.DEV_BAD_POINTER
     # valid segments: [0,4) adapter 0, [8,12) adapter 3, [16,20) adapter 4
