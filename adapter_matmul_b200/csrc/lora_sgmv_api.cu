@@ -27,8 +27,16 @@ constexpr int kVersion = 100;  // 0.1.0
 // Number of kernels this library has launched successfully in this process.
 std::atomic<uint64_t> g_launches{0};
 
+// Last CUDA error a call of this thread ran into (cudaSuccess if none).
+thread_local cudaError_t t_last_error = cudaSuccess;
+
+cudaError_t record(cudaError_t e) {
+    if (e != cudaSuccess) t_last_error = e;
+    return e;
+}
+
 lora_sgmv_status counted(cudaError_t e) {
-    if (e != cudaSuccess) return LORA_SGMV_ERR_CUDA;
+    if (record(e) != cudaSuccess) return LORA_SGMV_ERR_CUDA;
     g_launches.fetch_add(1, std::memory_order_relaxed);
     return LORA_SGMV_OK;
 }
@@ -47,7 +55,7 @@ std::vector<DeviceFacts> g_devices;
 
 lora_sgmv_status device_facts(DeviceFacts& out) {
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return LORA_SGMV_ERR_CUDA;
+    if (record(cudaGetDevice(&dev)) != cudaSuccess) return LORA_SGMV_ERR_CUDA;
     std::lock_guard<std::mutex> lock(g_mu);
     if (dev >= static_cast<int>(g_devices.size())) g_devices.resize(dev + 1);
     DeviceFacts& f = g_devices[dev];
@@ -63,18 +71,20 @@ lora_sgmv_status device_facts(DeviceFacts& out) {
     return LORA_SGMV_OK;
 }
 
-// Opt a kernel into more than 48 KB of dynamic shared memory, once per device.
+// Opt a kernel into the dynamic shared memory a launch needs (above 48 KB), per device.
+// `granted` holds, per device, the largest size already granted to this kernel.
 template <typename K>
-lora_sgmv_status ensure_smem(K kernel, size_t bytes, int& done_mask) {
+lora_sgmv_status ensure_smem(K kernel, size_t bytes, int* granted) {
     if (bytes <= 48 * 1024) return LORA_SGMV_OK;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return LORA_SGMV_ERR_CUDA;
+    if (dev < 0 || dev >= 64) return LORA_SGMV_ERR_UNSUPPORTED;
     std::lock_guard<std::mutex> lock(g_mu);
-    const int bit = 1 << (dev & 31);
-    if (done_mask & bit) return LORA_SGMV_OK;
-    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess)
+    if (static_cast<size_t>(granted[dev]) >= bytes) return LORA_SGMV_OK;
+    if (record(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes))) !=
+        cudaSuccess)
         return LORA_SGMV_ERR_CUDA;
-    done_mask |= bit;
+    granted[dev] = static_cast<int>(bytes);
     return LORA_SGMV_OK;
 }
 
@@ -97,7 +107,7 @@ int cluster_size_for(int H1) {
 
 template <typename T, int R>
 lora_sgmv_status launch_shrink(const ShrinkParams& p0, int max_len, cudaStream_t stream) {
-    static int smem_done = 0;
+    static int smem_granted[64] = {};
     ShrinkParams p = p0;
     const int C = cluster_size_for(p.H1);
     p.ks = ((p.H1 + C - 1) / C + 7) / 8 * 8;
@@ -106,7 +116,7 @@ lora_sgmv_status launch_shrink(const ShrinkParams& p0, int max_len, cudaStream_t
     if (device_facts(f) != LORA_SGMV_OK) return LORA_SGMV_ERR_CUDA;
     if (smem > static_cast<size_t>(f.max_smem_optin)) return LORA_SGMV_ERR_DIM;
     auto kernel = sgmv::sgmv_shrink_cluster_kernel<T, R>;
-    if (ensure_smem(kernel, smem, smem_done) != LORA_SGMV_OK) return LORA_SGMV_ERR_CUDA;
+    if (ensure_smem(kernel, smem, smem_granted) != LORA_SGMV_OK) return LORA_SGMV_ERR_CUDA;
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(C, clamp_grid_y(p.n_segments), chunk_slots(max_len, sgmv::kShrinkTokens, 8));
@@ -184,60 +194,77 @@ int estimate_max_len(int max_seg_len, int T, int n) {
 
 int round8(int v) { return (v + 7) / 8 * 8; }
 
-// Largest number of clusters of the fused kernel that can be resident at once, per device.
+// Largest number of clusters of `cluster` CTAs with `smem` bytes each that can be resident at once.
 template <typename K>
-lora_sgmv_status fused_max_clusters(K kernel, size_t smem, int* out, int* cache) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return LORA_SGMV_ERR_CUDA;
-    if (dev < 0 || dev >= 64) return LORA_SGMV_ERR_UNSUPPORTED;
-    {
-        std::lock_guard<std::mutex> lock(g_mu);
-        if (cache[dev] > 0) {
-            *out = cache[dev];
-            return LORA_SGMV_OK;
-        }
-    }
+lora_sgmv_status max_active_clusters(K kernel, int cluster, size_t smem, int* out) {
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(sgmv::kFusedCluster, 1, 1);
+    cfg.gridDim = dim3(cluster, 1, 1);
     cfg.blockDim = dim3(sgmv::kFusedThreads, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = sgmv::kFusedCluster;
+    attr[0].val.clusterDim.x = cluster;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess || n <= 0) return LORA_SGMV_ERR_CUDA;
-    std::lock_guard<std::mutex> lock(g_mu);
-    cache[dev] = n;
+    if (record(cudaOccupancyMaxActiveClusters(&n, kernel, &cfg)) != cudaSuccess || n <= 0) return LORA_SGMV_ERR_CUDA;
     *out = n;
     return LORA_SGMV_OK;
 }
 
 template <typename T, int R>
 lora_sgmv_status launch_fused(sgmv::FusedParams P, int max_len, cudaStream_t stream) {
-    static int smem_done = 0;
-    static int clusters_cache[64] = {};
+    (void)max_len;
+    static int smem_granted[64] = {};
+    // resident clusters per (device, log2 cluster size, job-prefix size bucket)
+    static int resident[64][4][9] = {};
     using G = sgmv::FusedGeom<R>;
-    const int C = sgmv::kFusedCluster;
+    if (P.n_segments > sgmv::kFusedMaxSegments) return LORA_SGMV_ERR_DIM;
+    const int bucket = (P.n_segments + 1 + 1023) / 1024;  // 1..9
+    const size_t smem = G::BASE + size_t(bucket) * 1024 * 4;
+    auto kernel = sgmv::sgmv_fused_kernel<T, R>;
+    if (ensure_smem(kernel, smem, smem_granted) != LORA_SGMV_OK) return LORA_SGMV_ERR_CUDA;
+    int dev = 0;
+    if (record(cudaGetDevice(&dev)) != cudaSuccess) return LORA_SGMV_ERR_CUDA;
+    if (dev < 0 || dev >= 64) return LORA_SGMV_ERR_UNSUPPORTED;
+    auto resident_for = [&](int lc, int* out) -> lora_sgmv_status {
+        {
+            std::lock_guard<std::mutex> lock(g_mu);
+            if (resident[dev][lc][bucket - 1] > 0) {
+                *out = resident[dev][lc][bucket - 1];
+                return LORA_SGMV_OK;
+            }
+        }
+        int n = 0;
+        lora_sgmv_status st = max_active_clusters(kernel, 1 << lc, smem, &n);
+        if (st != LORA_SGMV_OK) return st;
+        std::lock_guard<std::mutex> lock(g_mu);
+        resident[dev][lc][bucket - 1] = n;
+        *out = n;
+        return LORA_SGMV_OK;
+    };
+    // jobs: token chunks of <= 8 over all segments and problems (upper bound from T and n)
+    const long long chunks = std::min<long long>(P.n_segments + (P.T + sgmv::kFusedTokens - 1) / sgmv::kFusedTokens,
+                                                 std::max(P.T, 1));
+    const long long jobs = std::max<long long>(1, chunks * P.n_problems);
+    int ctas = 0;
+    lora_sgmv_status st = resident_for(0, &ctas);
+    if (st != LORA_SGMV_OK) return st;
+    // cluster size: the largest C whose jobs*C CTAs are all resident at once; 1 if even that is too many
+    int lc = 3;
+    while (lc > 0 && jobs * (1ll << lc) > ctas) --lc;
+    int clusters_max = 0;
+    st = resident_for(lc, &clusters_max);
+    if (st != LORA_SGMV_OK) return st;
+    const int C = 1 << lc;
     for (int i = 0; i < P.n_problems; ++i) {
         P.prob[i].ks = round8((P.prob[i].H1 + C - 1) / C);
         P.prob[i].ns = round8((P.prob[i].H2 + C - 1) / C);
     }
-    P.chunk_slots = chunk_slots(max_len, sgmv::kFusedTokens, 64);
-    const size_t smem = G::SMEM;
-    auto kernel = sgmv::sgmv_fused_kernel<T, R>;
-    if (ensure_smem(kernel, smem, smem_done) != LORA_SGMV_OK) return LORA_SGMV_ERR_CUDA;
-    int max_clusters = 0;
-    lora_sgmv_status st = fused_max_clusters(kernel, smem, &max_clusters, clusters_cache);
-    if (st != LORA_SGMV_OK) return st;
-    const long long jobs = static_cast<long long>(P.n_problems) * P.n_segments * P.chunk_slots;
-    if (jobs > (1ll << 30)) return LORA_SGMV_ERR_DIM;
-    int clusters = static_cast<int>(std::min<long long>(jobs, max_clusters));
-    // balance rounds: the same number of jobs per cluster where possible
-    const long long rounds = (jobs + clusters - 1) / clusters;
+    int clusters = static_cast<int>(std::min<long long>(jobs, clusters_max));
+    const long long rounds = (jobs + clusters - 1) / clusters;  // balance jobs per cluster
     clusters = static_cast<int>((jobs + rounds - 1) / rounds);
 
     cudaLaunchConfig_t cfg = {};
@@ -286,6 +313,10 @@ extern "C" {
 int32_t lora_sgmv_version(void) { return kVersion; }
 
 uint64_t lora_sgmv_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+const char* lora_sgmv_last_error(void) {
+    return t_last_error == cudaSuccess ? "no CUDA error" : cudaGetErrorString(t_last_error);
+}
 
 int32_t lora_sgmv_rank_supported(int32_t r, lora_sgmv_variant variant) {
     switch (variant) {
@@ -429,7 +460,7 @@ lora_sgmv_status lora_sgmv_apply_ex(void* Y, const void* X, const void* const* A
     if (v == LORA_SGMV_VARIANT_AUTO)
         v = (max_len >= sgmv::kGroupedMinSegment && sgmv::grouped_tc_supported(r, H1, H2, dtype))
                 ? LORA_SGMV_VARIANT_GROUPED_TC
-                : LORA_SGMV_VARIANT_FUSED;
+                : (n_segments <= sgmv::kFusedMaxSegments ? LORA_SGMV_VARIANT_FUSED : LORA_SGMV_VARIANT_SPLIT);
 
     if (v == LORA_SGMV_VARIANT_FUSED) {
         sgmv::FusedParams P = {};

@@ -5,53 +5,57 @@
 // with adapter i and each row t of it, Y[t,:] += scale * (X[t,:] @ A_i) @ B_i,
 // A_i [H1, r], B_i [r, H2], row-major.
 //
-// Work decomposition. A job is (problem p, segment s, chunk of <= 8 tokens).
-// One thread-block cluster of C CTAs runs a job; CTA c owns rows
-// [c*KS, (c+1)*KS) of A_i for the shrink and columns [c*NS, (c+1)*NS) of B_i
-// for the expand, so every adapter byte is read once per job by one CTA.
-// Clusters are persistent (as many as fit on the GPU at once) and take jobs
-// round-robin.
+// Jobs. A job is (problem p, segment s, chunk of <= 8 tokens of s). At start
+// every CTA reads seg_starts once and builds the exact job list (a prefix sum
+// of the segments' chunk counts in shared memory), so long segments split
+// into as many jobs as they have chunks and no slot is empty. Clusters are
+// persistent (as many as are resident at once) and take jobs round-robin.
+//
+// Split of one job over a cluster of C CTAs (C = 1, 2, 4 or 8, chosen by the
+// host so that all jobs run in one resident wave when they can): CTA c owns
+// rows [c*KS, (c+1)*KS) of A_i for the shrink and columns [c*NS, (c+1)*NS) of
+// B_i for the expand, so each adapter byte is read once per job.
 //
 // Data movement. Warp 0 of each CTA is a producer: it streams the CTA's
 // operands through a ring of shared-memory stages with TMA bulk copies
-// (cp.async.bulk, completion counted on the stage's mbarrier). A shrink stage
-// holds up to KT rows of A_i (one contiguous copy) and the same KT columns of
-// the chunk's X rows; an expand stage holds the r rows of a column tile of
-// B_i (one copy per row, rows padded by 16 bytes so that the
-// consumers' 16-byte reads spread over all banks). B does not depend on V,
-// so the producer runs ahead into the expand stages while the consumers wait
-// for the cluster's reduction of V.
+// (cp.async.bulk; completion counted on the stage's mbarrier). A shrink stage
+// holds KT rows of A_i (one contiguous copy) and the same KT columns of the
+// chunk's X rows (KT shrinks as the chunk's token count grows). An expand
+// stage holds r rows of a column tile of B_i (one copy per row, rows padded
+// by 16 bytes so that 16-byte reads spread over the banks) and the matching
+// tile of the chunk's Y rows. Nothing in an expand stage depends on V, so the
+// producer streams ahead while the consumers reduce V.
 //
-// Compute. Warps 1..4 consume. Shrink: fp32 FMA over the stage, specialised
-// for 1, 2, 4 or 8 tokens; partial sums reduced across lanes by shuffles and
-// across warps in shared memory. The C partial V tiles are exchanged through
-// distributed shared memory: each CTA publishes its tile in its own shared
-// memory and signals every CTA's "ready" mbarrier remotely; each CTA then
-// sums all C tiles in rank order (so every CTA holds bit-identical V) and
-// signals every owner's "free" mbarrier. Expand: each thread covers 8 columns
-// and 8 of the r rows of a stage; lanes reduce over row groups by shuffles, and one
-// lane per column group adds scale * acc to Y (read before waiting on the
-// stage) and rounds once.
+// Compute. Warps 1..4 consume. Shrink: fp32 FMA over each stage, specialised
+// for 1, 2, 4 or 8 tokens; partial sums reduced over lanes by shuffles and
+// over warps in shared memory. Reduction of V over the cluster: each CTA
+// pushes its partial tile into every CTA's receive buffer with st.async,
+// whose completion is counted on the receiver's mbarrier; each CTA sums the
+// C tiles in rank order (so all hold identical V) and then tells every sender
+// that its slot may be reused. Expand: each thread covers 8 columns and 8 of
+// the r rows of a stage; lanes reduce over row groups by shuffles, and one
+// lane per column group adds scale * acc to the staged Y, rounds once and
+// stores to global memory.
 //
-// Every mbarrier wait is bounded; a wait that gives up sets
-// LORA_SGMV_DEV_TIMEOUT in the status word and the kernel runs to its end
-// (results are then invalid, but nothing hangs). The kernel never traps.
+// Every mbarrier wait is bounded in time; a wait that gives up sets
+// LORA_SGMV_DEV_TIMEOUT in the status word and the thread's later waits
+// return at once, so the kernel always ends. The kernel never traps.
 #pragma once
-
-#include <cooperative_groups.h>
 
 #include "sgmv_common.cuh"
 
 namespace sgmv {
 
 constexpr int kFusedMaxProblems = 8;
-constexpr int kFusedTokens = 8;       // tokens per job (chunk)
-constexpr int kFusedStages = 4;       // ring depth
-constexpr int kFusedStageData = 16384;  // payload bytes per stage
+constexpr int kFusedTokens = 8;  // tokens per job (chunk)
+constexpr int kFusedStages = 4;  // ring depth
 constexpr int kFusedConsumerWarps = 4;
-constexpr int kFusedThreads = 32 * (1 + kFusedConsumerWarps);
-constexpr int kFusedCluster = 8;
-constexpr uint32_t kSpinLimit = 1u << 22;
+constexpr int kFusedConsumers = 32 * kFusedConsumerWarps;
+constexpr int kFusedThreads = 32 + kFusedConsumers;
+constexpr int kFusedMaxCluster = 8;
+constexpr int kFusedMaxSegments = 8192;  // job list held in shared memory
+constexpr uint32_t kSpinLimit = 1u << 24;
+constexpr uint64_t kWaitLimitNs = 200ull * 1000 * 1000;
 
 struct FusedProblem {
     void* Y;
@@ -74,31 +78,39 @@ struct FusedParams {
     int n_problems;
     int n_segments;
     int T;
-    int chunk_slots;  // TY: token-chunk slots per segment
 };
 
 // compile-time geometry per rank
 template <int R>
 struct FusedGeom {
-    static constexpr int KT = (kFusedStageData / (2 * (R + kFusedTokens))) / 8 * 8;  // A rows per stage
-    static constexpr int NTC = kFusedStageData / (2 * R);                            // B columns per stage
-    static constexpr int BPITCH = NTC * 2 + 16;                                      // bytes per B row in smem
-    static constexpr int STAGE = (R * BPITCH > kFusedStageData ? R * BPITCH : kFusedStageData);
-    static constexpr int CG = R / 8;                                                 // 8-column groups of A
-    static constexpr int RLN = 128 / CG;                                             // shrink row lanes
-    static constexpr int RG = R / 8;                                                 // expand row groups
-    static constexpr int GC = 128 / RG;                                              // expand column groups
-    static_assert(NTC == 8 * GC, "expand tile must give every consumer thread 8 columns");
+    static constexpr int RG = R / 8;                                   // expand row groups (8 rows each)
+    static constexpr int NTC = (1024 / RG) < 512 ? (1024 / RG) : 512;  // B columns per stage
+    static constexpr int GC = NTC / 8;                                 // expand column groups
+    static_assert(RG * GC <= kFusedConsumers, "expand tile too wide");
+    static constexpr int BPITCH = NTC * 2 + 16;                        // bytes per staged B row
+    static constexpr int BSTAGE = R * BPITCH + kFusedTokens * NTC * 2;  // B rows + Y rows
+    static constexpr int STAGE = (BSTAGE > 16384 ? BSTAGE : 16384);
+    static constexpr int CG = R / 8;                                   // 8-column groups of A
+    static constexpr int RLN = kFusedConsumers / CG;                   // shrink row lanes
     static constexpr size_t RING = size_t(kFusedStages) * STAGE;
     static constexpr size_t RED = size_t(kFusedConsumerWarps) * kFusedTokens * R * 4;
-    static constexpr size_t SLOT = size_t(kFusedTokens) * R * 4;
-    static constexpr size_t SMEM = RING + RED + 2 * SLOT + SLOT /* vs */;
+    static constexpr size_t TILE = size_t(kFusedTokens) * R * 4;  // one partial V tile
+    static constexpr size_t RECV = kFusedMaxCluster * TILE;
+    static constexpr size_t BASE = RING + RED + RECV + TILE;      // + the job prefix (n+1 ints)
+    // A rows per shrink stage for a chunk of nt tokens (A rows plus X columns fill a stage)
+    static __host__ __device__ constexpr int kt_for(int nt) { return (STAGE / (2 * (R + nt))) / 8 * 8; }
 };
 
 // ---- PTX wrappers ------------------------------------------------------------------------
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint32_t map_rank(uint32_t local_addr, uint32_t rank) {
+    uint32_t remote;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local_addr), "r"(rank));
+    return remote;
 }
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
@@ -114,10 +126,9 @@ __device__ __forceinline__ void mbar_arrive_local(uint64_t* bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
-// Arrive on the mbarrier at the same offset in CTA `rank` of this cluster (release at cluster scope).
+// Arrive on the mbarrier at the same offset in CTA `rank` of this cluster (release, cluster scope).
 __device__ __forceinline__ void mbar_arrive_remote(uint64_t* bar, uint32_t rank) {
-    uint32_t remote;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(bar)), "r"(rank));
+    const uint32_t remote = map_rank(smem_u32(bar), rank);
     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote) : "memory");
 }
 
@@ -151,13 +162,11 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
     return t;
 }
 
-// Bounded waits. A wait gives up after kWaitLimitNs (or kSpinLimit polls), records
-// LORA_SGMV_DEV_TIMEOUT and marks the thread dead: every later wait of that thread
-// returns at once, so a broken protocol ends the kernel quickly instead of hanging it.
-constexpr uint64_t kWaitLimitNs = 200ull * 1000 * 1000;
-
+// Bounded wait: gives up after kWaitLimitNs (or kSpinLimit polls), records
+// LORA_SGMV_DEV_TIMEOUT and marks the thread dead; a dead thread's later
+// waits return at once, so a broken protocol ends the kernel quickly.
 template <bool kCluster>
-__device__ __forceinline__ void mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint32_t* status, bool& dead) {
+__device__ __forceinline__ void mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* status, bool& dead) {
     if (dead) return;
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t i = 0; i < kSpinLimit; ++i) {
@@ -166,14 +175,6 @@ __device__ __forceinline__ void mbar_wait_bounded(uint64_t* bar, uint32_t parity
     }
     dead = true;
     report(status, LORA_SGMV_DEV_TIMEOUT);
-}
-
-__device__ __forceinline__ void mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* status, bool& dead) {
-    mbar_wait_bounded<false>(bar, parity, status, dead);
-}
-
-__device__ __forceinline__ void mbar_wait_cluster(uint64_t* bar, uint32_t parity, uint32_t* status, bool& dead) {
-    mbar_wait_bounded<true>(bar, parity, status, dead);
 }
 
 // 1-D TMA bulk copy global -> this CTA's shared memory, completion on `bar`.
@@ -185,10 +186,19 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
         : "memory");
 }
 
-__device__ __forceinline__ void fence_cluster() { asm volatile("fence.acq_rel.cluster;" ::: "memory"); }
+// 16-byte asynchronous store into CTA `rank`'s shared memory; completion counted on
+// that CTA's mbarrier at the same offset as `bar`.
+__device__ __forceinline__ void st_async_v4(float* dst_local, float4 v, uint64_t* bar, uint32_t rank) {
+    const uint32_t dst = map_rank(smem_u32(dst_local), rank);
+    const uint32_t mb = map_rank(smem_u32(bar), rank);
+    asm volatile(
+        "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(dst),
+        "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w), "r"(mb)
+        : "memory");
+}
 
-__device__ __forceinline__ void consumer_sync() {  // named barrier 1 over the 4 consumer warps
-    asm volatile("bar.sync 1, %0;" ::"n"(32 * kFusedConsumerWarps) : "memory");
+__device__ __forceinline__ void consumer_sync() {  // named barrier 1 over the consumer warps
+    asm volatile("bar.sync 1, %0;" ::"n"(kFusedConsumers) : "memory");
 }
 
 __device__ __forceinline__ void cluster_sync_all() {
@@ -201,34 +211,83 @@ __device__ __forceinline__ uint32_t cluster_rank() {
     return r;
 }
 
-// ---- job enumeration (identical in producer and consumers) ------------------------------
+__device__ __forceinline__ uint32_t cluster_size() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+    return r;
+}
+
+// ---- job list --------------------------------------------------------------------------
+
+// Number of 8-token chunks of segment s, or 0 if the segment is empty or invalid.
+__device__ __forceinline__ int segment_chunks(const FusedParams& P, int s) {
+    const int b = __ldg(P.seg_starts + s), e = __ldg(P.seg_starts + s + 1);
+    if (b < 0 || b > e || e > P.T) return 0;
+    return (e - b + kFusedTokens - 1) / kFusedTokens;
+}
+
+// pref[s] = chunks of segments 0..s-1 (pref[0] = 0, pref[n] = chunks per problem), built by all threads.
+__device__ void build_job_prefix(const FusedParams& P, int* pref) {
+    __shared__ int warp_tot[kFusedThreads / 32];
+    const int n = P.n_segments;
+    const int nthreads = blockDim.x;
+    const int per = (n + nthreads - 1) / nthreads;
+    const int s0 = threadIdx.x * per;
+    const int s1 = min(n, s0 + per);
+    int local = 0;
+    for (int s = s0; s < s1; ++s) local += segment_chunks(P, s);
+    // inclusive scan of `local` over the block
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int v = local;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, v, off);
+        if (lane >= off) v += y;
+    }
+    if (lane == 31) warp_tot[warp] = v;
+    __syncthreads();
+    int before = 0;
+    for (int w = 0; w < warp; ++w) before += warp_tot[w];
+    int run = before + v - local;  // exclusive prefix of this thread's first segment
+    if (threadIdx.x == 0) pref[0] = 0;
+    for (int s = s0; s < s1; ++s) {
+        run += segment_chunks(P, s);
+        pref[s + 1] = run;
+    }
+    __syncthreads();
+}
 
 struct Job {
-    int p;      // problem
-    int t0;     // first token
-    int nt;     // tokens (1..8)
+    int p;   // problem
+    int t0;  // first token
+    int nt;  // tokens (1..8)
     const void* a;
     const void* b;
     int k0, nk;  // this CTA's rows of A_i
     int c0, nc;  // this CTA's columns of B_i
 };
 
-// Returns false when job slot j holds no work; otherwise fills `job` (uniform over the cluster).
-__device__ __forceinline__ bool job_at(const FusedParams& P, int j, int sub, int c, Job& job, uint32_t& bad) {
-    const int TY = P.chunk_slots;
-    const int qs = j % TY;
-    const int s = (j / TY) % P.n_segments;
-    const int p = j / (TY * P.n_segments);
+// Job j of the list: returns false if its segment fails the device-side checks.
+__device__ __forceinline__ bool job_at(const FusedParams& P, const int* pref, int j, int c, Job& job) {
+    const int per_problem = pref[P.n_segments];
+    const int p = j / per_problem;
+    const int r = j - p * per_problem;
+    int lo = 0, hi = P.n_segments;  // largest s with pref[s] <= r
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (pref[mid] <= r)
+            lo = mid;
+        else
+            hi = mid;
+    }
+    const int s = lo;
     const FusedProblem& pr = P.prob[p];
     Segment seg;
-    bad = load_segment(P.seg_starts, P.lora_idx, pr.A_ptrs, pr.B_ptrs, s, P.T, pr.num_adapters, seg);
-    if (bad) return false;
-    const int q = qs + sub * TY;
-    const int t0 = seg.begin + q * kFusedTokens;
-    if (t0 >= seg.end) return false;
+    if (load_segment(P.seg_starts, P.lora_idx, pr.A_ptrs, pr.B_ptrs, s, P.T, pr.num_adapters, seg)) return false;
+    const int q = r - pref[s];
     job.p = p;
-    job.t0 = t0;
-    job.nt = min(kFusedTokens, seg.end - t0);
+    job.t0 = seg.begin + q * kFusedTokens;
+    job.nt = min(kFusedTokens, seg.end - job.t0);
     job.a = seg.a;
     job.b = seg.b;
     job.k0 = c * pr.ks;
@@ -238,27 +297,25 @@ __device__ __forceinline__ bool job_at(const FusedParams& P, int j, int sub, int
     return true;
 }
 
-// Number of token chunks a job slot covers at most (sub-jobs); sub-job `sub` of slot j is chunk qs + sub*TY.
-__device__ __forceinline__ int slot_subjobs(const FusedParams& P, int j) {
-    const int TY = P.chunk_slots;
-    const int qs = j % TY;
-    const int s = (j / TY) % P.n_segments;
-    const int b = __ldg(P.seg_starts + s), e = __ldg(P.seg_starts + s + 1);
-    const int L = (b >= 0 && e >= b) ? e - b : 0;
-    const int chunks = (L + kFusedTokens - 1) / kFusedTokens;
-    return chunks > qs ? (chunks - qs + TY - 1) / TY : 0;
-}
+// ---- consumer body ----------------------------------------------------------------------
 
-// ---- consumer bodies ---------------------------------------------------------------------
+struct FusedSmem {
+    unsigned char* ring;
+    uint64_t* full;
+    uint64_t* empty;
+    uint64_t* vready;
+    uint64_t* vfree;
+    float* red;
+    float* recv;
+    float* vs;
+};
 
 template <typename T, int R, int NTOK>
-__device__ __forceinline__ void consume_job(const FusedParams& P, const Job& job, unsigned char* ring,
-                                            uint64_t* full, uint64_t* empty, float* red, float* slot,
-                                            float* vs, uint64_t* vready, uint64_t* vfree, uint32_t& it,
-                                            uint32_t u, int C, int ct, bool& dead) {
+__device__ __forceinline__ void consume_job(const FusedParams& P, const Job& job, const FusedSmem& S, uint32_t& it,
+                                            uint32_t u, int C, int c, int ct, bool& dead) {
     using G = FusedGeom<R>;
     const int lane = ct & 31;
-    const int cw = ct >> 5;  // consumer warp 0..3
+    const int cw = ct >> 5;
     const int nt = job.nt;
     const FusedProblem& pr = P.prob[job.p];
 
@@ -270,29 +327,29 @@ __device__ __forceinline__ void consume_job(const FusedParams& P, const Job& job
         for (int i = 0; i < 8; ++i) acc[t][i] = 0.f;
     const int cg = ct % G::CG;
     const int rl = ct / G::CG;
-    const int nA = (job.nk + G::KT - 1) / G::KT;
+    const int KT = G::kt_for(nt);
+    const int nA = (job.nk + KT - 1) / KT;
     for (int ta = 0; ta < nA; ++ta, ++it) {
         const uint32_t stage = it % kFusedStages;
-        mbar_wait(&full[stage], (it / kFusedStages) & 1u, P.dev_status, dead);
-        const unsigned char* st = ring + size_t(stage) * G::STAGE;
-        const T* xs = reinterpret_cast<const T*>(st + size_t(G::KT) * R * 2);
-        const int kt = min(G::KT, job.nk - ta * G::KT);
+        mbar_wait<false>(&S.full[stage], (it / kFusedStages) & 1u, P.dev_status, dead);
+        const unsigned char* st = S.ring + size_t(stage) * G::STAGE;
+        const T* xs = reinterpret_cast<const T*>(st + size_t(KT) * R * 2);
+        const int kt = min(KT, job.nk - ta * KT);
         for (int k = rl; k < kt; k += G::RLN) {
             float a[8];
             unpack8<T>(*reinterpret_cast<const uint4*>(st + (size_t(k) * R + cg * 8) * 2), a);
 #pragma unroll
             for (int t = 0; t < NTOK; ++t) {
                 if (t < nt) {
-                    const float x = Storage<T>::to1(xs[size_t(t) * G::KT + k]);
+                    const float x = Storage<T>::to1(xs[size_t(t) * KT + k]);
 #pragma unroll
                     for (int i = 0; i < 8; ++i) acc[t][i] = fmaf(x, a[i], acc[t][i]);
                 }
             }
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive_local(&empty[stage]);
+        if (lane == 0) mbar_arrive_local(&S.empty[stage]);
     }
-    // reduce over the row lanes of each warp (lanes sharing cg), then across the 4 warps
 #pragma unroll
     for (int off = G::CG; off < 32; off <<= 1)
 #pragma unroll
@@ -304,36 +361,36 @@ __device__ __forceinline__ void consume_job(const FusedParams& P, const Job& job
         for (int t = 0; t < NTOK; ++t)
             if (t < nt) {
 #pragma unroll
-                for (int i = 0; i < 8; ++i) red[(cw * kFusedTokens + t) * R + cg * 8 + i] = acc[t][i];
+                for (int i = 0; i < 8; ++i) S.red[(cw * kFusedTokens + t) * R + cg * 8 + i] = acc[t][i];
             }
     }
-    const uint32_t ph = u & 1u;
-    float* my_slot = slot + size_t(ph) * kFusedTokens * R;
-    // the slot may still be read by the cluster for job u-2
-    if (u >= 2) mbar_wait_cluster(&vfree[ph], ((u - 2) >> 1) & 1u, P.dev_status, dead);
     consumer_sync();
-    for (int e = ct; e < nt * R; e += 128) {
-        float sum = 0.f;
+
+    // ---------------- V: push this CTA's tile to every CTA of the cluster ----------------
+    const uint32_t tile_bytes = uint32_t(nt) * R * 4;
+    if (ct == 0) mbar_arrive_expect_tx(S.vready, tile_bytes * C);
+    // every receiver must have consumed this CTA's previous tile
+    if (u >= 1) mbar_wait<true>(S.vfree, (u - 1) & 1u, P.dev_status, dead);
+    for (int e4 = ct; e4 < nt * R / 4; e4 += kFusedConsumers) {
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-        for (int w = 0; w < kFusedConsumerWarps; ++w) sum += red[w * kFusedTokens * R + e];
-        my_slot[e] = sum;
-    }
-    fence_cluster();
-    consumer_sync();
-    if (ct < C) mbar_arrive_remote(&vready[ph], static_cast<uint32_t>(ct));
-    // every CTA's tile of this job is published once vready completes
-    mbar_wait_cluster(&vready[ph], (u >> 1) & 1u, P.dev_status, dead);
-    {
-        cooperative_groups::cluster_group cluster = cooperative_groups::this_cluster();
-        for (int e = ct; e < nt * R; e += 128) {
-            float sum = 0.f;
-            for (int q = 0; q < C; ++q) sum += cluster.map_shared_rank(my_slot, q)[e];
-            vs[e] = sum;
+        for (int w = 0; w < kFusedConsumerWarps; ++w) {
+            const float4 q = *reinterpret_cast<const float4*>(S.red + w * kFusedTokens * R + e4 * 4);
+            v.x += q.x;
+            v.y += q.y;
+            v.z += q.z;
+            v.w += q.w;
         }
+        for (int q = 0; q < C; ++q) st_async_v4(S.recv + size_t(c) * kFusedTokens * R + e4 * 4, v, S.vready, q);
     }
-    fence_cluster();
+    mbar_wait<true>(S.vready, u & 1u, P.dev_status, dead);
+    for (int e = ct; e < nt * R; e += kFusedConsumers) {
+        float sum = 0.f;
+        for (int q = 0; q < C; ++q) sum += S.recv[size_t(q) * kFusedTokens * R + e];
+        S.vs[e] = sum;
+    }
     consumer_sync();
-    if (ct < C) mbar_arrive_remote(&vfree[ph], static_cast<uint32_t>(ct));
+    if (ct < C) mbar_arrive_remote(S.vfree, static_cast<uint32_t>(ct));  // sender ct may reuse my slot
 
     // ---------------- expand: Y[t, cols] += scale * V[t,:] @ B_i[:, cols] ----------------
     const int rg = ct % G::RG;
@@ -343,23 +400,16 @@ __device__ __forceinline__ void consume_job(const FusedParams& P, const Job& job
     for (int tb = 0; tb < nB; ++tb, ++it) {
         const int col_in_tile = gc * 8;
         const int nct = min(G::NTC, job.nc - tb * G::NTC);
-        const bool writer = (rg == 0) && (col_in_tile < nct);
-        const int col = job.c0 + tb * G::NTC + col_in_tile;
-        uint4 yv[NTOK];
-        if (writer) {
-#pragma unroll
-            for (int t = 0; t < NTOK; ++t)
-                if (t < nt) yv[t] = ld_vec(Y + size_t(job.t0 + t) * pr.H2 + col);
-        }
+        const bool active = gc < G::GC && col_in_tile < nct;
         const uint32_t stage = it % kFusedStages;
-        mbar_wait(&full[stage], (it / kFusedStages) & 1u, P.dev_status, dead);
-        const unsigned char* st = ring + size_t(stage) * G::STAGE;
+        mbar_wait<false>(&S.full[stage], (it / kFusedStages) & 1u, P.dev_status, dead);
+        const unsigned char* st = S.ring + size_t(stage) * G::STAGE;
         float o[NTOK][8];
 #pragma unroll
         for (int t = 0; t < NTOK; ++t)
 #pragma unroll
             for (int i = 0; i < 8; ++i) o[t][i] = 0.f;
-        if (col_in_tile < nct) {
+        if (active) {
 #pragma unroll
             for (int jj = 0; jj < 8; ++jj) {
                 const int j = rg + G::RG * jj;
@@ -368,54 +418,62 @@ __device__ __forceinline__ void consume_job(const FusedParams& P, const Job& job
 #pragma unroll
                 for (int t = 0; t < NTOK; ++t) {
                     if (t < nt) {
-                        const float v = vs[t * R + j];
+                        const float v = S.vs[t * R + j];
 #pragma unroll
                         for (int i = 0; i < 8; ++i) o[t][i] = fmaf(v, b[i], o[t][i]);
                     }
                 }
             }
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive_local(&empty[stage]);
 #pragma unroll
         for (int off = 1; off < G::RG; off <<= 1)
 #pragma unroll
             for (int t = 0; t < NTOK; ++t)
 #pragma unroll
                 for (int i = 0; i < 8; ++i) o[t][i] += __shfl_xor_sync(0xffffffffu, o[t][i], off);
-        if (writer) {
+        if (active && rg == 0) {
+            const T* ys = reinterpret_cast<const T*>(st + size_t(R) * G::BPITCH);
+            const int col = job.c0 + tb * G::NTC + col_in_tile;
 #pragma unroll
             for (int t = 0; t < NTOK; ++t) {
                 if (t < nt) {
                     float y[8];
-                    unpack8<T>(yv[t], y);
+                    unpack8<T>(*reinterpret_cast<const uint4*>(ys + size_t(t) * G::NTC + col_in_tile), y);
 #pragma unroll
                     for (int i = 0; i < 8; ++i) y[i] = __fadd_rn(y[i], __fmul_rn(pr.scale, o[t][i]));
                     st_vec(Y + size_t(job.t0 + t) * pr.H2 + col, pack8<T>(y));
                 }
             }
         }
+        __syncwarp();
+        if (lane == 0) mbar_arrive_local(&S.empty[stage]);
     }
 }
 
 // ---- the kernel ----------------------------------------------------------------------------
 
-// grid.x = C * clusters, cluster (C,1,1). Block: warp 0 producer, warps 1..4 consumers.
+// grid.x = C * clusters, cluster (C,1,1), C in {1,2,4,8}. Warp 0 produces, warps 1..4 consume.
 template <typename T, int R>
 __global__ void __launch_bounds__(kFusedThreads, 2) sgmv_fused_kernel(const FusedParams P) {
     using G = FusedGeom<R>;
     extern __shared__ __align__(128) unsigned char smem[];
     __shared__ __align__(8) uint64_t full[kFusedStages];
     __shared__ __align__(8) uint64_t empty[kFusedStages];
-    __shared__ __align__(8) uint64_t vready[2];
-    __shared__ __align__(8) uint64_t vfree[2];
+    __shared__ __align__(8) uint64_t vready[1];
+    __shared__ __align__(8) uint64_t vfree[1];
 
-    unsigned char* ring = smem;
-    float* red = reinterpret_cast<float*>(smem + G::RING);
-    float* slot = red + kFusedConsumerWarps * kFusedTokens * R;
-    float* vs = slot + 2 * kFusedTokens * R;
+    FusedSmem S;
+    S.ring = smem;
+    S.red = reinterpret_cast<float*>(smem + G::RING);
+    S.recv = reinterpret_cast<float*>(smem + G::RING + G::RED);
+    S.vs = reinterpret_cast<float*>(smem + G::RING + G::RED + G::RECV);
+    int* pref = reinterpret_cast<int*>(smem + G::BASE);
+    S.full = full;
+    S.empty = empty;
+    S.vready = vready;
+    S.vfree = vfree;
 
-    const int C = kFusedCluster;
+    const int C = static_cast<int>(cluster_size());
     const int c = static_cast<int>(cluster_rank());
     const int cluster_id = blockIdx.x / C;
     const int n_clusters = gridDim.x / C;
@@ -427,56 +485,60 @@ __global__ void __launch_bounds__(kFusedThreads, 2) sgmv_fused_kernel(const Fuse
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], kFusedConsumerWarps);
         }
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(&vready[s], C);
-            mbar_init(&vfree[s], C);
-        }
+        mbar_init(vready, 1);  // own expect_tx arrival; the C tiles arrive as transaction bytes
+        mbar_init(vfree, C);   // one arrival per receiver
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    // every CTA's barriers exist before any remote arrive
-    cluster_sync_all();
+    build_job_prefix(P, pref);
+    cluster_sync_all();  // every CTA's barriers exist before any remote operation
 
-    const int J = P.n_problems * P.n_segments * P.chunk_slots;
+    const int J = P.n_problems * pref[P.n_segments];
     bool dead = false;
     if (warp == 0) {
         // ------------------------------ producer ------------------------------
         uint32_t it = 0;
         for (int j = cluster_id; j < J; j += n_clusters) {
-            const int subs = slot_subjobs(P, j);
-            for (int sub = 0; sub < subs; ++sub) {
-                Job job;
-                uint32_t bad;
-                if (!job_at(P, j, sub, c, job, bad)) continue;
-                const FusedProblem& pr = P.prob[job.p];
-                const T* X = static_cast<const T*>(pr.X);
-                const T* A = static_cast<const T*>(job.a);
-                const T* B = static_cast<const T*>(job.b);
-                const int nA = (job.nk + G::KT - 1) / G::KT;
-                for (int ta = 0; ta < nA; ++ta, ++it) {
-                    const uint32_t stage = it % kFusedStages;
-                    if (it >= kFusedStages) mbar_wait(&empty[stage], ((it / kFusedStages) - 1) & 1u, P.dev_status, dead);
-                    unsigned char* st = ring + size_t(stage) * G::STAGE;
-                    const int k = job.k0 + ta * G::KT;
-                    const int kt = min(G::KT, job.nk - ta * G::KT);
-                    if (lane == 0) mbar_arrive_expect_tx(&full[stage], uint32_t(kt) * (R + job.nt) * 2);
-                    __syncwarp();
-                    if (lane == 0) bulk_g2s(st, A + size_t(k) * R, uint32_t(kt) * R * 2, &full[stage]);
-                    else if (lane <= job.nt)
-                        bulk_g2s(st + size_t(G::KT) * R * 2 + size_t(lane - 1) * G::KT * 2,
-                                 X + size_t(job.t0 + lane - 1) * pr.H1 + k, uint32_t(kt) * 2, &full[stage]);
-                }
-                const int nB = (job.nc + G::NTC - 1) / G::NTC;
-                for (int tb = 0; tb < nB; ++tb, ++it) {
-                    const uint32_t stage = it % kFusedStages;
-                    if (it >= kFusedStages) mbar_wait(&empty[stage], ((it / kFusedStages) - 1) & 1u, P.dev_status, dead);
-                    unsigned char* st = ring + size_t(stage) * G::STAGE;
-                    const int col = job.c0 + tb * G::NTC;
-                    const int nct = min(G::NTC, job.nc - tb * G::NTC);
-                    if (lane == 0) mbar_arrive_expect_tx(&full[stage], uint32_t(nct) * R * 2);
-                    __syncwarp();
-                    for (int row = lane; row < R; row += 32)
+            Job job;
+            if (!job_at(P, pref, j, c, job)) continue;
+            const FusedProblem& pr = P.prob[job.p];
+            const T* X = static_cast<const T*>(pr.X);
+            const T* Yg = static_cast<const T*>(pr.Y);
+            const T* A = static_cast<const T*>(job.a);
+            const T* B = static_cast<const T*>(job.b);
+            const int KT = G::kt_for(job.nt);
+            const int nA = (job.nk + KT - 1) / KT;
+            for (int ta = 0; ta < nA; ++ta, ++it) {
+                const uint32_t stage = it % kFusedStages;
+                if (it >= kFusedStages)
+                    mbar_wait<false>(&empty[stage], ((it / kFusedStages) - 1) & 1u, P.dev_status, dead);
+                unsigned char* st = smem + size_t(stage) * G::STAGE;
+                const int k = job.k0 + ta * KT;
+                const int kt = min(KT, job.nk - ta * KT);
+                if (lane == 0) mbar_arrive_expect_tx(&full[stage], uint32_t(kt) * (R + job.nt) * 2);
+                __syncwarp();
+                if (lane == 0)
+                    bulk_g2s(st, A + size_t(k) * R, uint32_t(kt) * R * 2, &full[stage]);
+                else if (lane <= job.nt)
+                    bulk_g2s(st + size_t(KT) * R * 2 + size_t(lane - 1) * KT * 2,
+                             X + size_t(job.t0 + lane - 1) * pr.H1 + k, uint32_t(kt) * 2, &full[stage]);
+            }
+            const int nB = (job.nc + G::NTC - 1) / G::NTC;
+            for (int tb = 0; tb < nB; ++tb, ++it) {
+                const uint32_t stage = it % kFusedStages;
+                if (it >= kFusedStages)
+                    mbar_wait<false>(&empty[stage], ((it / kFusedStages) - 1) & 1u, P.dev_status, dead);
+                unsigned char* st = smem + size_t(stage) * G::STAGE;
+                const int col = job.c0 + tb * G::NTC;
+                const int nct = min(G::NTC, job.nc - tb * G::NTC);
+                if (lane == 0) mbar_arrive_expect_tx(&full[stage], uint32_t(nct) * (R + job.nt) * 2);
+                __syncwarp();
+                for (int row = lane; row < R + job.nt; row += 32) {
+                    if (row < R)
                         bulk_g2s(st + size_t(row) * G::BPITCH, B + size_t(row) * pr.H2 + col, uint32_t(nct) * 2,
                                  &full[stage]);
+                    else
+                        bulk_g2s(st + size_t(R) * G::BPITCH + size_t(row - R) * G::NTC * 2,
+                                 Yg + size_t(job.t0 + row - R) * pr.H2 + col, uint32_t(nct) * 2, &full[stage]);
                 }
             }
         }
@@ -485,36 +547,29 @@ __global__ void __launch_bounds__(kFusedThreads, 2) sgmv_fused_kernel(const Fuse
         const int ct = threadIdx.x - 32;
         uint32_t it = 0, u = 0;
         for (int j = cluster_id; j < J; j += n_clusters) {
-            const int subs = slot_subjobs(P, j);
-            for (int sub = 0; sub < subs; ++sub) {
-                Job job;
-                uint32_t bad;
-                if (!job_at(P, j, sub, c, job, bad)) continue;  // reported below
-                if (job.nt == 1)
-                    consume_job<T, R, 1>(P, job, ring, full, empty, red, slot, vs, vready, vfree, it, u, C, ct, dead);
-                else if (job.nt <= 2)
-                    consume_job<T, R, 2>(P, job, ring, full, empty, red, slot, vs, vready, vfree, it, u, C, ct, dead);
-                else if (job.nt <= 4)
-                    consume_job<T, R, 4>(P, job, ring, full, empty, red, slot, vs, vready, vfree, it, u, C, ct, dead);
-                else
-                    consume_job<T, R, 8>(P, job, ring, full, empty, red, slot, vs, vready, vfree, it, u, C, ct, dead);
-                ++u;
-            }
+            Job job;
+            if (!job_at(P, pref, j, c, job)) continue;
+            if (job.nt == 1)
+                consume_job<T, R, 1>(P, job, S, it, u, C, c, ct, dead);
+            else if (job.nt <= 2)
+                consume_job<T, R, 2>(P, job, S, it, u, C, c, ct, dead);
+            else if (job.nt <= 4)
+                consume_job<T, R, 4>(P, job, S, it, u, C, c, ct, dead);
+            else
+                consume_job<T, R, 8>(P, job, S, it, u, C, c, ct, dead);
+            ++u;
         }
-        // the last two exchange slots may still be read by the cluster
-        for (uint32_t v = (u >= 2 ? u - 2 : 0); v < u; ++v)
-            mbar_wait_cluster(&vfree[v & 1u], (v >> 1) & 1u, P.dev_status, dead);
-    }
-    // report each rejected segment once (the job loops above skip them silently)
-    if (threadIdx.x == 32 && c == 0) {
-        for (int j = cluster_id; j < J; j += n_clusters) {
-            if (j % P.chunk_slots) continue;
-            const int s = (j / P.chunk_slots) % P.n_segments;
-            const int p = j / (P.chunk_slots * P.n_segments);
-            Segment seg;
-            const uint32_t bad = load_segment(P.seg_starts, P.lora_idx, P.prob[p].A_ptrs, P.prob[p].B_ptrs, s,
-                                              P.T, P.prob[p].num_adapters, seg);
-            if (bad) report(P.dev_status, bad);
+        // every receiver has consumed this CTA's last tile before its shared memory goes away
+        if (u >= 1) mbar_wait<true>(vfree, (u - 1) & 1u, P.dev_status, dead);
+        // report each rejected segment once
+        if (ct == 0 && c == 0) {
+            for (int j = cluster_id; j < P.n_problems * P.n_segments; j += n_clusters) {
+                const int p = j / P.n_segments, s = j - p * P.n_segments;
+                Segment seg;
+                const uint32_t bad = load_segment(P.seg_starts, P.lora_idx, P.prob[p].A_ptrs, P.prob[p].B_ptrs, s,
+                                                  P.T, P.prob[p].num_adapters, seg);
+                if (bad) report(P.dev_status, bad);
+            }
         }
     }
 }

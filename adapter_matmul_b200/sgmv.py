@@ -38,6 +38,7 @@ STATUS_NAMES = {0: "OK", 1: "ERR_NULL", 2: "ERR_DIM", 3: "ERR_ALIGN", 4: "ERR_DT
 
 EXPORTS = [
     "lora_sgmv_rank_supported", "lora_sgmv_status_string", "lora_sgmv_version", "lora_sgmv_launch_count",
+    "lora_sgmv_last_error",
     "lora_sgmv_group_segments", "lora_sgmv_shrink", "lora_sgmv_expand", "lora_sgmv_workspace_bytes",
     "lora_sgmv_apply", "lora_sgmv_apply_ex", "lora_sgmv_apply_batched", "lora_sgmv_apply_noalloc",
 ]
@@ -56,7 +57,10 @@ _lib = None
 class SGMVError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
-        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)} ({status_string(status)})")
+        detail = status_string(status)
+        if status == 6:
+            detail += ": " + load().lora_sgmv_last_error().decode()
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)} ({detail})")
 
 
 def load(path: Optional[str] = None):
@@ -80,6 +84,8 @@ def load(path: Optional[str] = None):
         lib.lora_sgmv_status_string.argtypes = [ctypes.c_int]
         lib.lora_sgmv_version.restype = i32
         lib.lora_sgmv_version.argtypes = []
+        lib.lora_sgmv_last_error.restype = ctypes.c_char_p
+        lib.lora_sgmv_last_error.argtypes = []
         lib.lora_sgmv_launch_count.restype = ctypes.c_uint64
         lib.lora_sgmv_launch_count.argtypes = []
         lib.lora_sgmv_group_segments.restype = ctypes.c_int

@@ -101,6 +101,10 @@ int32_t lora_sgmv_rank_supported(int32_t r, lora_sgmv_variant variant);
 /* Human-readable name of a status code. Never NULL. */
 const char* lora_sgmv_status_string(lora_sgmv_status status);
 
+/* Text of the last CUDA error that a call made from this thread ran into
+ * (the cause behind LORA_SGMV_ERR_CUDA), or "no CUDA error". Never NULL. */
+const char* lora_sgmv_last_error(void);
+
 /* Library version as major*10000 + minor*100 + patch. */
 int32_t lora_sgmv_version(void);
 
@@ -230,7 +234,8 @@ typedef struct {
  * with i = lora_idx[s] and A_i, B_i taken from problem p's tables. Each
  * problem may have its own H1, H2, tables and adapter count; r and dtype are
  * shared. Runs the fused kernel (LORA_SGMV_VARIANT_FUSED), which keeps V on
- * chip and needs no workspace.
+ * chip and needs no workspace; it takes at most 8192 segments
+ * (LORA_SGMV_ERR_DIM beyond).
  *   problems     host array of n_problems entries, 1 <= n_problems <= 8.
  *   other arguments as for lora_sgmv_apply.
  * Validation errors of any problem are returned before anything is launched.
