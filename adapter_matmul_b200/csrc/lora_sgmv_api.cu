@@ -216,7 +216,6 @@ lora_sgmv_status max_active_clusters(K kernel, int cluster, size_t smem, int* ou
 
 template <typename T, int R>
 lora_sgmv_status launch_fused(sgmv::FusedParams P, int max_len, cudaStream_t stream) {
-    (void)max_len;
     static int smem_granted[64] = {};
     // resident clusters per (device, log2 cluster size, job-prefix size bucket)
     static int resident[64][4][9] = {};
@@ -248,17 +247,22 @@ lora_sgmv_status launch_fused(sgmv::FusedParams P, int max_len, cudaStream_t str
     // jobs: token chunks of <= 8 over all segments and problems (upper bound from T and n)
     const long long chunks = std::min<long long>(P.n_segments + (P.T + sgmv::kFusedTokens - 1) / sgmv::kFusedTokens,
                                                  std::max(P.T, 1));
-    const long long jobs = std::max<long long>(1, chunks * P.n_problems);
+    const long long jobs = std::max<long long>(
+        1, (max_len <= sgmv::kFusedTokens ? static_cast<long long>(P.n_segments) : chunks) * P.n_problems);
     int ctas = 0;
     lora_sgmv_status st = resident_for(0, &ctas);
     if (st != LORA_SGMV_OK) return st;
     // cluster size: the largest C whose jobs*C CTAs are all resident at once; 1 if even that is too many
     int lc = 3;
     while (lc > 0 && jobs * (1ll << lc) > ctas) --lc;
+#ifdef SGMV_FORCE_CLUSTER_LOG2
+    lc = SGMV_FORCE_CLUSTER_LOG2;
+#endif
     int clusters_max = 0;
     st = resident_for(lc, &clusters_max);
     if (st != LORA_SGMV_OK) return st;
     const int C = 1 << lc;
+    P.one_chunk = max_len <= sgmv::kFusedTokens ? 1 : 0;
     for (int i = 0; i < P.n_problems; ++i) {
         P.prob[i].ks = round8((P.prob[i].H1 + C - 1) / C);
         P.prob[i].ns = round8((P.prob[i].H2 + C - 1) / C);
@@ -272,13 +276,15 @@ lora_sgmv_status launch_fused(sgmv::FusedParams P, int max_len, cudaStream_t str
     cfg.blockDim = dim3(sgmv::kFusedThreads, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = C;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     return counted(cudaLaunchKernelEx(&cfg, kernel, P));
 }
 

@@ -37,6 +37,12 @@
 // lane per column group adds scale * acc to the staged Y, rounds once and
 // stores to global memory.
 //
+// Programmatic dependent launch: the kernel lets the next kernel on the stream
+// launch at once, and reads X and Y only after griddepcontrol.wait (which
+// returns when the previous kernel has completed). Segment metadata, pointer
+// tables and adapter weights are read before it: they must not be written by
+// the kernel that immediately precedes the call on the stream.
+//
 // Every mbarrier wait is bounded in time; a wait that gives up sets
 // LORA_SGMV_DEV_TIMEOUT in the status word and the thread's later waits
 // return at once, so the kernel always ends. The kernel never traps.
@@ -47,8 +53,14 @@
 namespace sgmv {
 
 constexpr int kFusedMaxProblems = 8;
-constexpr int kFusedTokens = 8;  // tokens per job (chunk)
-constexpr int kFusedStages = 4;  // ring depth
+#ifndef SGMV_FUSED_STAGES
+#define SGMV_FUSED_STAGES 4
+#endif
+#ifndef SGMV_FUSED_MIN_BLOCKS
+#define SGMV_FUSED_MIN_BLOCKS 2
+#endif
+constexpr int kFusedTokens = 8;                  // tokens per job (chunk)
+constexpr int kFusedStages = SGMV_FUSED_STAGES;  // ring depth
 constexpr int kFusedConsumerWarps = 4;
 constexpr int kFusedConsumers = 32 * kFusedConsumerWarps;
 constexpr int kFusedThreads = 32 + kFusedConsumers;
@@ -78,6 +90,7 @@ struct FusedParams {
     int n_problems;
     int n_segments;
     int T;
+    int one_chunk;  // host hint: every segment fits one chunk (job j is segment j; correct either way)
 };
 
 // compile-time geometry per rank
@@ -201,8 +214,17 @@ __device__ __forceinline__ void consumer_sync() {  // named barrier 1 over the c
     asm volatile("bar.sync 1, %0;" ::"n"(kFusedConsumers) : "memory");
 }
 
-__device__ __forceinline__ void cluster_sync_all() {
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+__device__ __forceinline__ void cluster_arrive() {
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void cluster_wait() {
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Bulk prefetch of global memory into L2 (no shared memory, no completion to wait on).
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
 
 __device__ __forceinline__ uint32_t cluster_rank() {
@@ -235,7 +257,17 @@ __device__ void build_job_prefix(const FusedParams& P, int* pref) {
     const int s0 = threadIdx.x * per;
     const int s1 = min(n, s0 + per);
     int local = 0;
-    for (int s = s0; s < s1; ++s) local += segment_chunks(P, s);
+    for (int s = s0; s < s1; ++s) {
+        local += segment_chunks(P, s);
+        // warm L1 for the lookups job_at() makes next: adapter id, then its table entries
+        const int i = __ldg(P.lora_idx + s);
+        for (int p = 0; p < P.n_problems; ++p) {
+            if (i >= 0 && i < P.prob[p].num_adapters) {
+                asm volatile("prefetch.global.L1 [%0];" ::"l"(P.prob[p].A_ptrs + i));
+                asm volatile("prefetch.global.L1 [%0];" ::"l"(P.prob[p].B_ptrs + i));
+            }
+        }
+    }
     // inclusive scan of `local` over the block
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     int v = local;
@@ -267,10 +299,20 @@ struct Job {
     int c0, nc;  // this CTA's columns of B_i
 };
 
-// Job j of the list: returns false if its segment fails the device-side checks.
-__device__ __forceinline__ bool job_at(const FusedParams& P, const int* pref, int j, int c, Job& job) {
+// Jobs of list entry j: (problem, segment, first chunk, number of chunks). With the
+// prefix, an entry is one chunk; in one-chunk mode an entry is a whole segment, whose
+// chunks the cluster then runs one after another.
+__device__ __forceinline__ void entry_at(const FusedParams& P, const int* pref, int j, int& p, int& s, int& q0,
+                                         int& nq) {
+    if (P.one_chunk) {
+        p = j / P.n_segments;
+        s = j - p * P.n_segments;
+        q0 = 0;
+        nq = segment_chunks(P, s);
+        return;
+    }
     const int per_problem = pref[P.n_segments];
-    const int p = j / per_problem;
+    p = j / per_problem;
     const int r = j - p * per_problem;
     int lo = 0, hi = P.n_segments;  // largest s with pref[s] <= r
     while (hi - lo > 1) {
@@ -280,11 +322,16 @@ __device__ __forceinline__ bool job_at(const FusedParams& P, const int* pref, in
         else
             hi = mid;
     }
-    const int s = lo;
+    s = lo;
+    q0 = r - pref[s];
+    nq = 1;
+}
+
+// Chunk q of segment s of problem p: returns false if the segment fails the device-side checks.
+__device__ __forceinline__ bool job_at(const FusedParams& P, int p, int s, int q, int c, Job& job) {
     const FusedProblem& pr = P.prob[p];
     Segment seg;
     if (load_segment(P.seg_starts, P.lora_idx, pr.A_ptrs, pr.B_ptrs, s, P.T, pr.num_adapters, seg)) return false;
-    const int q = r - pref[s];
     job.p = p;
     job.t0 = seg.begin + q * kFusedTokens;
     job.nt = min(kFusedTokens, seg.end - job.t0);
@@ -450,11 +497,95 @@ __device__ __forceinline__ void consume_job(const FusedParams& P, const Job& job
     }
 }
 
+// X columns of the first job's shrink stages (stages 0 .. tiles-1), requested once the
+// previous kernel on the stream has completed.
+template <typename T, int R>
+__device__ __forceinline__ void issue_deferred_x(unsigned char* ring, uint64_t* full, const void* Xv, int H1, int t0,
+                                                 int nt, int k0, int KT, int nk, int tiles, int lane) {
+    using G = FusedGeom<R>;
+    const T* X = static_cast<const T*>(Xv);
+    for (int ta = 0; ta < tiles; ++ta) {
+        unsigned char* st = ring + size_t(ta) * G::STAGE;
+        const int k = k0 + ta * KT;
+        const int kt = min(KT, nk - ta * KT);
+        if (lane >= 1 && lane <= nt)
+            bulk_g2s(st + size_t(KT) * R * 2 + size_t(lane - 1) * KT * 2, X + size_t(t0 + lane - 1) * H1 + k,
+                     uint32_t(kt) * 2, &full[ta]);
+    }
+}
+
+// Producer side of one job: shrink stages (A rows + X columns), then expand stages (B rows + Y rows).
+template <typename T, int R>
+__device__ __forceinline__ void produce_job(const FusedParams& P, const Job& job, unsigned char* smem, uint64_t* full,
+                                            uint64_t* empty, uint32_t& it, bool& waited, int lane, bool& dead) {
+    using G = FusedGeom<R>;
+    const FusedProblem& pr = P.prob[job.p];
+    const T* X = static_cast<const T*>(pr.X);
+    const T* Yg = static_cast<const T*>(pr.Y);
+    const T* A = static_cast<const T*>(job.a);
+    const T* B = static_cast<const T*>(job.b);
+    const int KT = G::kt_for(job.nt);
+    const int nA = (job.nk + KT - 1) / KT;
+    int deferred = 0;  // shrink stages of the first job whose X waits for the previous kernel
+    for (int ta = 0; ta < nA; ++ta, ++it) {
+        const uint32_t stage = it % kFusedStages;
+        if (it >= kFusedStages) {
+            if (!waited) {  // the ring is full: the deferred X must come first
+                pdl_wait();
+                waited = true;
+                issue_deferred_x<T, R>(smem, full, X, pr.H1, job.t0, job.nt, job.k0, KT, job.nk, deferred, lane);
+            }
+            mbar_wait<false>(&empty[stage], ((it / kFusedStages) - 1) & 1u, P.dev_status, dead);
+        }
+        unsigned char* st = smem + size_t(stage) * G::STAGE;
+        const int k = job.k0 + ta * KT;
+        const int kt = min(KT, job.nk - ta * KT);
+        if (lane == 0) mbar_arrive_expect_tx(&full[stage], uint32_t(kt) * (R + job.nt) * 2);
+        __syncwarp();
+        if (lane == 0) bulk_g2s(st, A + size_t(k) * R, uint32_t(kt) * R * 2, &full[stage]);
+        if (waited) {
+            if (lane >= 1 && lane <= job.nt)
+                bulk_g2s(st + size_t(KT) * R * 2 + size_t(lane - 1) * KT * 2,
+                         X + size_t(job.t0 + lane - 1) * pr.H1 + k, uint32_t(kt) * 2, &full[stage]);
+        } else {
+            deferred = ta + 1;
+        }
+        if (ta == 0 && job.nc > 0) {
+            // start B on its way to L2 while the shrink runs; the expand stages then hit L2
+            for (int row = lane; row < R; row += 32)
+                bulk_prefetch_l2(B + size_t(row) * pr.H2 + job.c0, uint32_t(job.nc) * 2);
+        }
+    }
+    if (!waited) {
+        pdl_wait();
+        waited = true;
+        issue_deferred_x<T, R>(smem, full, X, pr.H1, job.t0, job.nt, job.k0, KT, job.nk, deferred, lane);
+    }
+    if (job.nc > 0 && lane < job.nt) bulk_prefetch_l2(Yg + size_t(job.t0 + lane) * pr.H2 + job.c0, uint32_t(job.nc) * 2);
+    const int nB = (job.nc + G::NTC - 1) / G::NTC;
+    for (int tb = 0; tb < nB; ++tb, ++it) {
+        const uint32_t stage = it % kFusedStages;
+        if (it >= kFusedStages) mbar_wait<false>(&empty[stage], ((it / kFusedStages) - 1) & 1u, P.dev_status, dead);
+        unsigned char* st = smem + size_t(stage) * G::STAGE;
+        const int col = job.c0 + tb * G::NTC;
+        const int nct = min(G::NTC, job.nc - tb * G::NTC);
+        if (lane == 0) mbar_arrive_expect_tx(&full[stage], uint32_t(nct) * (R + job.nt) * 2);
+        __syncwarp();
+        for (int row = lane; row < R + job.nt; row += 32) {
+            if (row < R)
+                bulk_g2s(st + size_t(row) * G::BPITCH, B + size_t(row) * pr.H2 + col, uint32_t(nct) * 2, &full[stage]);
+            else
+                bulk_g2s(st + size_t(R) * G::BPITCH + size_t(row - R) * G::NTC * 2,
+                         Yg + size_t(job.t0 + row - R) * pr.H2 + col, uint32_t(nct) * 2, &full[stage]);
+        }
+    }
+}
+
 // ---- the kernel ----------------------------------------------------------------------------
 
 // grid.x = C * clusters, cluster (C,1,1), C in {1,2,4,8}. Warp 0 produces, warps 1..4 consume.
 template <typename T, int R>
-__global__ void __launch_bounds__(kFusedThreads, 2) sgmv_fused_kernel(const FusedParams P) {
+__global__ void __launch_bounds__(kFusedThreads, SGMV_FUSED_MIN_BLOCKS) sgmv_fused_kernel(const FusedParams P) {
     using G = FusedGeom<R>;
     extern __shared__ __align__(128) unsigned char smem[];
     __shared__ __align__(8) uint64_t full[kFusedStages];
@@ -480,6 +611,8 @@ __global__ void __launch_bounds__(kFusedThreads, 2) sgmv_fused_kernel(const Fuse
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
+    // the next kernel on the stream may start its prologue now (programmatic dependent launch)
+    pdl_launch_dependents();
     if (threadIdx.x == 0) {
         for (int s = 0; s < kFusedStages; ++s) {
             mbar_init(&full[s], 1);
@@ -489,76 +622,61 @@ __global__ void __launch_bounds__(kFusedThreads, 2) sgmv_fused_kernel(const Fuse
         mbar_init(vfree, C);   // one arrival per receiver
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    build_job_prefix(P, pref);
-    cluster_sync_all();  // every CTA's barriers exist before any remote operation
+    int entries;
+    if (P.one_chunk) {
+        __syncthreads();
+        entries = P.n_problems * P.n_segments;
+    } else {
+        build_job_prefix(P, pref);  // ends with __syncthreads
+        entries = P.n_problems * pref[P.n_segments];
+    }
+    // Barriers of every CTA exist before any remote operation: each CTA arrives here and
+    // waits only before its first remote operation (consumers, below).
+    if (C > 1) cluster_arrive();
 
-    const int J = P.n_problems * pref[P.n_segments];
     bool dead = false;
     if (warp == 0) {
         // ------------------------------ producer ------------------------------
+        // Adapter weights and segment metadata are not written by the previous kernel on the
+        // stream, so the first job's A rows are requested before griddepcontrol.wait; X and Y
+        // (which the previous kernel may produce) only after it.
         uint32_t it = 0;
-        for (int j = cluster_id; j < J; j += n_clusters) {
-            Job job;
-            if (!job_at(P, pref, j, c, job)) continue;
-            const FusedProblem& pr = P.prob[job.p];
-            const T* X = static_cast<const T*>(pr.X);
-            const T* Yg = static_cast<const T*>(pr.Y);
-            const T* A = static_cast<const T*>(job.a);
-            const T* B = static_cast<const T*>(job.b);
-            const int KT = G::kt_for(job.nt);
-            const int nA = (job.nk + KT - 1) / KT;
-            for (int ta = 0; ta < nA; ++ta, ++it) {
-                const uint32_t stage = it % kFusedStages;
-                if (it >= kFusedStages)
-                    mbar_wait<false>(&empty[stage], ((it / kFusedStages) - 1) & 1u, P.dev_status, dead);
-                unsigned char* st = smem + size_t(stage) * G::STAGE;
-                const int k = job.k0 + ta * KT;
-                const int kt = min(KT, job.nk - ta * KT);
-                if (lane == 0) mbar_arrive_expect_tx(&full[stage], uint32_t(kt) * (R + job.nt) * 2);
-                __syncwarp();
-                if (lane == 0)
-                    bulk_g2s(st, A + size_t(k) * R, uint32_t(kt) * R * 2, &full[stage]);
-                else if (lane <= job.nt)
-                    bulk_g2s(st + size_t(KT) * R * 2 + size_t(lane - 1) * KT * 2,
-                             X + size_t(job.t0 + lane - 1) * pr.H1 + k, uint32_t(kt) * 2, &full[stage]);
-            }
-            const int nB = (job.nc + G::NTC - 1) / G::NTC;
-            for (int tb = 0; tb < nB; ++tb, ++it) {
-                const uint32_t stage = it % kFusedStages;
-                if (it >= kFusedStages)
-                    mbar_wait<false>(&empty[stage], ((it / kFusedStages) - 1) & 1u, P.dev_status, dead);
-                unsigned char* st = smem + size_t(stage) * G::STAGE;
-                const int col = job.c0 + tb * G::NTC;
-                const int nct = min(G::NTC, job.nc - tb * G::NTC);
-                if (lane == 0) mbar_arrive_expect_tx(&full[stage], uint32_t(nct) * (R + job.nt) * 2);
-                __syncwarp();
-                for (int row = lane; row < R + job.nt; row += 32) {
-                    if (row < R)
-                        bulk_g2s(st + size_t(row) * G::BPITCH, B + size_t(row) * pr.H2 + col, uint32_t(nct) * 2,
-                                 &full[stage]);
-                    else
-                        bulk_g2s(st + size_t(R) * G::BPITCH + size_t(row - R) * G::NTC * 2,
-                                 Yg + size_t(job.t0 + row - R) * pr.H2 + col, uint32_t(nct) * 2, &full[stage]);
-                }
+        bool waited = false;
+        for (int j = cluster_id; j < entries; j += n_clusters) {
+            int p, s, q0, nq;
+            entry_at(P, pref, j, p, s, q0, nq);
+            for (int q = q0; q < q0 + nq; ++q) {
+                Job job;
+                if (!job_at(P, p, s, q, c, job)) break;
+                produce_job<T, R>(P, job, smem, full, empty, it, waited, lane, dead);
             }
         }
+        if (!waited) pdl_wait();
+        if (C > 1) cluster_wait();
     } else {
         // ------------------------------ consumers ------------------------------
+        if (C > 1) cluster_wait();
         const int ct = threadIdx.x - 32;
         uint32_t it = 0, u = 0;
-        for (int j = cluster_id; j < J; j += n_clusters) {
-            Job job;
-            if (!job_at(P, pref, j, c, job)) continue;
-            if (job.nt == 1)
-                consume_job<T, R, 1>(P, job, S, it, u, C, c, ct, dead);
-            else if (job.nt <= 2)
-                consume_job<T, R, 2>(P, job, S, it, u, C, c, ct, dead);
-            else if (job.nt <= 4)
-                consume_job<T, R, 4>(P, job, S, it, u, C, c, ct, dead);
-            else
-                consume_job<T, R, 8>(P, job, S, it, u, C, c, ct, dead);
-            ++u;
+        for (int j = cluster_id; j < entries; j += n_clusters) {
+            int p, s, q0, nq;
+            entry_at(P, pref, j, p, s, q0, nq);
+            for (int q = q0; q < q0 + nq; ++q) {
+                Job job;
+                if (!job_at(P, p, s, q, c, job)) break;
+                if (job.nt == 1)
+                    consume_job<T, R, 1>(P, job, S, it, u, C, c, ct, dead);
+                else if (job.nt <= 2)
+                    consume_job<T, R, 2>(P, job, S, it, u, C, c, ct, dead);
+                else if (job.nt <= 4)
+                    consume_job<T, R, 4>(P, job, S, it, u, C, c, ct, dead);
+                else
+                    consume_job<T, R, 8>(P, job, S, it, u, C, c, ct, dead);
+                ++u;
+            }
         }
+        // keep this grid behind its predecessor even when it had no work
+        pdl_wait();
         // every receiver has consumed this CTA's last tile before its shared memory goes away
         if (u >= 1) mbar_wait<true>(vfree, (u - 1) & 1u, P.dev_status, dead);
         // report each rejected segment once

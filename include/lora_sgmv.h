@@ -48,6 +48,15 @@
  *     *dev_status (a device uint32; may be NULL). No kernel traps.
  *   - Alignment: X, Y, V and workspace must be 16-byte aligned; H1 and H2
  *     must be multiples of 8.
+ *   - Overlap with the previous kernel: the fused kernel (variant FUSED,
+ *     which AUTO picks for short segments, and lora_sgmv_apply_batched) is
+ *     launched with programmatic dependent launch. It reads segment arrays,
+ *     pointer tables and adapter weights while the kernel before it on the
+ *     stream may still run, and reads X and Y only after that kernel has
+ *     completed. So seg_starts, lora_idx, the tables and the adapters of a
+ *     call must not be written by the kernel launched immediately before it
+ *     on the same stream (copies and earlier kernels are fine); X and Y may
+ *     be. Use LORA_SGMV_VARIANT_SPLIT where that does not hold.
  *   - Thread safety: calls on different streams may run concurrently. The
  *     library keeps no mutable global state other than a lazily filled,
  *     mutex-guarded cache of device facts and kernel attributes, and an
