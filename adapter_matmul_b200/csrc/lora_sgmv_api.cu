@@ -185,6 +185,63 @@ lora_sgmv_status expand_dispatch(const ExpandParams& p, int r, lora_sgmv_dtype d
                                : expand_dispatch_r<__nv_bfloat16>(p, r, max_len, chained, s);
 }
 
+// ---- grouped tensor-core path ------------------------------------------------------------------
+
+lora_sgmv_status launch_grouped(void* Y, const void* X, const void* const* A_ptrs, const void* const* B_ptrs,
+                                const int32_t* seg_starts, const int32_t* lora_idx, int n_segments, int num_adapters,
+                                int T, int H1, int r, int H2, float scale, lora_sgmv_dtype dt, uint32_t* dev_status,
+                                cudaStream_t stream) {
+    DeviceFacts f;
+    if (device_facts(f) != LORA_SGMV_OK) return LORA_SGMV_ERR_CUDA;
+    CUtensorMap tmX, tmY;
+    if (!sgmv::make_tile_map(&tmX, X, T, H1, dt) || !sgmv::make_tile_map(&tmY, Y, T, H2, dt)) {
+        t_last_error = cudaErrorInvalidValue;
+        return LORA_SGMV_ERR_CUDA;
+    }
+    sgmv::GroupedParams P = {};
+    P.Y = Y;
+    P.A_ptrs = A_ptrs;
+    P.B_ptrs = B_ptrs;
+    P.seg_starts = seg_starts;
+    P.lora_idx = lora_idx;
+    P.dev_status = dev_status;
+    P.n_segments = n_segments;
+    P.num_adapters = num_adapters;
+    P.T = T;
+    P.H1 = H1;
+    P.H2 = H2;
+    P.scale = scale;
+    // M-tiles: at most ceil(T/128) + n (each segment adds at most one partial tile)
+    const long long tiles_ub = (static_cast<long long>(T) + sgmv::kGM - 1) / sgmv::kGM + n_segments;
+    const long long tiles_est = std::max<long long>(1, (static_cast<long long>(T) + sgmv::kGM - 1) / sgmv::kGM);
+    const int max_split = (H2 + sgmv::kGN - 1) / sgmv::kGN;
+    int nsplit = static_cast<int>(std::max<long long>(1, (f.sms + tiles_est - 1) / tiles_est));
+    nsplit = std::min(nsplit, max_split);
+    const int span_tiles = ((H2 + sgmv::kGN - 1) / sgmv::kGN + nsplit - 1) / nsplit;
+    P.nspan = span_tiles * sgmv::kGN;
+    P.nsplit = (H2 + P.nspan - 1) / P.nspan;
+    const long long blocks = tiles_ub * P.nsplit;
+    if (blocks > (1ll << 31) - 1) return LORA_SGMV_ERR_DIM;
+    cudaError_t e = cudaSuccess;
+    const bool bf = dt == LORA_SGMV_BF16;
+    switch (r) {
+        case 16:
+            e = bf ? sgmv::launch_grouped_tc_kernel<__nv_bfloat16, 16>(tmX, tmY, P, int(blocks), stream)
+                   : sgmv::launch_grouped_tc_kernel<__half, 16>(tmX, tmY, P, int(blocks), stream);
+            break;
+        case 32:
+            e = bf ? sgmv::launch_grouped_tc_kernel<__nv_bfloat16, 32>(tmX, tmY, P, int(blocks), stream)
+                   : sgmv::launch_grouped_tc_kernel<__half, 32>(tmX, tmY, P, int(blocks), stream);
+            break;
+        case 64:
+            e = bf ? sgmv::launch_grouped_tc_kernel<__nv_bfloat16, 64>(tmX, tmY, P, int(blocks), stream)
+                   : sgmv::launch_grouped_tc_kernel<__half, 64>(tmX, tmY, P, int(blocks), stream);
+            break;
+        default: return LORA_SGMV_ERR_UNSUPPORTED;
+    }
+    return counted(e);
+}
+
 int estimate_max_len(int max_seg_len, int T, int n) {
     if (max_seg_len > 0) return std::min(max_seg_len, std::max(T, 1));
     return n > 0 ? (T + n - 1) / n : T;
@@ -489,8 +546,8 @@ lora_sgmv_status lora_sgmv_apply_ex(void* Y, const void* X, const void* const* A
 
     if (v == LORA_SGMV_VARIANT_GROUPED_TC) {
         if (!sgmv::grouped_tc_supported(r, H1, H2, dtype)) return LORA_SGMV_ERR_UNSUPPORTED;
-        return sgmv::launch_grouped_tc(Y, X, A_ptrs, B_ptrs, seg_starts, lora_idx, n_segments, num_adapters,
-                                       T, H1, r, H2, scale, dtype, dev_status, s);
+        return launch_grouped(Y, X, A_ptrs, B_ptrs, seg_starts, lora_idx, n_segments, num_adapters, T, H1, r, H2,
+                              scale, dtype, dev_status, s);
     }
 
     float* V = static_cast<float*>(workspace);

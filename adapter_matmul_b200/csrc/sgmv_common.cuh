@@ -89,6 +89,8 @@ struct Storage<__half> {
         return *reinterpret_cast<uint32_t*>(&h);
     }
     static __device__ __forceinline__ float to1(__half v) { return __half2float(v); }
+    // x rounded to the nearest fp16 value, returned as fp32
+    static __device__ __forceinline__ float round(float x) { return __half2float(__float2half_rn(x)); }
 };
 
 template <>
@@ -102,6 +104,8 @@ struct Storage<__nv_bfloat16> {
         return *reinterpret_cast<uint32_t*>(&h);
     }
     static __device__ __forceinline__ float to1(__nv_bfloat16 v) { return __bfloat162float(v); }
+    // x rounded to the nearest bf16 value, returned as fp32
+    static __device__ __forceinline__ float round(float x) { return __bfloat162float(__float2bfloat16_rn(x)); }
 };
 
 template <typename T>

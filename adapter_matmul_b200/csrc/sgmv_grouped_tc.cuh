@@ -1,23 +1,517 @@
-// sgmv_grouped_tc.cuh -- grouped tensor-core SGMV for long segments (placeholder).
+// sgmv_grouped_tc.cuh -- grouped SGMV on the 5th-generation tensor cores (tcgen05, TMEM)
+// for long segments (prefill).
+//
+// Maths (Punica README, LoRA and multi-LoRA paragraphs): for each segment s with
+// adapter i and every row t of it, Y[t,:] += scale * (X[t,:] @ A_i) @ B_i, A_i [H1, r],
+// B_i [r, H2], row-major. With many rows per segment both halves are real matrix
+// products: a [L, H1] x [H1, r] shrink and a [L, r] x [r, H2] expand per segment.
+//
+// One CTA computes one M-tile (128 rows of one segment) against one N-slice of H2:
+//   shrink  D1[128 x r] (TMEM, fp32) = X[t0:t0+128, :] @ A_i, K-steps of 64;
+//   V       the epilogue warps read D1 from TMEM and split it into two 16-bit
+//           operands V_hi + V_lo (V_hi = round(D1), V_lo = round(D1 - V_hi)), so
+//           the expand sees V to about 16 significant bits (the MMA takes 16-bit
+//           operands; V itself is never rounded to one 16-bit value);
+//   expand  D2[128 x 128] (TMEM, fp32) = V_hi @ B_tile + V_lo @ B_tile per N-tile,
+//           double-buffered in TMEM; the epilogue adds scale * D2 to the Y tile,
+//           rounds once to the storage type and stores only rows inside the segment.
+// Rows of a tile past the segment's end belong to the next segment (or past T, where
+// TMA fills zeros); their results are discarded, so tiles never write across segments.
+//
+// Data movement. X and Y tiles are TMA loads (cp.async.bulk.tensor, 128-byte swizzle)
+// through tensor maps built per call. Adapter tiles come from a device table of
+// pointers, so they are copied with cp.async (16 bytes per lane) straight into the
+// swizzled canonical layouts the MMA descriptors describe. Warp roles: warp 0
+// producer, warp 1 allocates TMEM and issues tcgen05.mma (one thread), warps 2..5
+// epilogue (one TMEM lane quarter each).
+//
+// Every mbarrier wait is bounded in time; a wait that gives up sets
+// LORA_SGMV_DEV_TIMEOUT and the kernel runs to its end (TMEM is always freed).
 #pragma once
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+#include <type_traits>
+
 #include "sgmv_common.cuh"
+#include "sgmv_fused.cuh"  // PTX wrappers shared with the fused kernel (mbarriers, timers)
 
 namespace sgmv {
 
-constexpr int kGroupedMinSegment = 128;
+constexpr int kGroupedMinSegment = 128;  // dispatcher: longest segment at least one M-tile
+constexpr int kGM = 128;                 // rows per M-tile (UMMA M)
+constexpr int kGK = 64;                  // K per shrink stage (one 128-byte swizzle atom of 16-bit values)
+constexpr int kGN = 128;                 // columns per expand N-tile
+constexpr int kGShrinkStages = 3;
+constexpr int kGExpandStages = 2;
+constexpr int kGThreads = 192;           // 6 warps
+constexpr int kGTmemCols = 512;
 
-inline bool grouped_tc_rank(int r) { return false && r; }
+inline bool grouped_tc_rank(int r) { return r == 16 || r == 32 || r == 64; }
 
 inline bool grouped_tc_supported(int r, int H1, int H2, lora_sgmv_dtype dt) {
-    (void)H1; (void)H2; (void)dt;
-    return grouped_tc_rank(r);
+    (void)dt;
+    return grouped_tc_rank(r) && H1 >= 64 && H2 >= 64 && H1 % 8 == 0 && H2 % 8 == 0;
 }
 
-inline lora_sgmv_status launch_grouped_tc(void*, const void*, const void* const*, const void* const*,
-                                          const int32_t*, const int32_t*, int, int, int, int, int, int,
-                                          float, lora_sgmv_dtype, uint32_t*, cudaStream_t) {
-    return LORA_SGMV_ERR_UNSUPPORTED;
+struct GroupedParams {
+    void* Y;
+    const void* const* A_ptrs;
+    const void* const* B_ptrs;
+    const int32_t* seg_starts;
+    const int32_t* lora_idx;
+    uint32_t* dev_status;
+    int n_segments;
+    int num_adapters;
+    int T;
+    int H1;
+    int H2;
+    float scale;
+    int nsplit;  // N-slices of H2
+    int nspan;   // columns per N-slice (multiple of kGN)
+};
+
+template <int R>
+struct GroupedGeom {
+    // shrink stage: X tile [128 x 64] (TMA, 128B swizzle) + A_i tile [64 x R] (MN-major)
+    static constexpr int X_BYTES = kGM * kGK * 2;
+    static constexpr int A_BYTES = kGK * R * 2;
+    static constexpr int SSTAGE = X_BYTES + ((A_BYTES + 1023) / 1024) * 1024;
+    // expand stage: Y tile [128 x 128] as two 64-column TMA boxes + B_i tile [R x 128] (MN-major)
+    static constexpr int Y_BYTES = kGM * kGN * 2;
+    static constexpr int B_BYTES = R * kGN * 2;
+    static constexpr int ESTAGE = Y_BYTES + B_BYTES;
+    static constexpr int V_BYTES = kGM * R * 2;  // one of V_hi, V_lo
+    static constexpr size_t SMEM = size_t(kGShrinkStages) * SSTAGE + size_t(kGExpandStages) * ESTAGE +
+                                   2 * size_t(V_BYTES) + 1024 /* alignment slack */;
+    // swizzle of an MN-major A_i tile (rows of R 16-bit values) and of K-major V rows
+    static constexpr int SW_BITS = R == 64 ? 3 : (R == 32 ? 2 : 1);           // 128B, 64B, 32B
+    static constexpr uint64_t SW_TYPE = R == 64 ? 2 : (R == 32 ? 4 : 6);      // descriptor layout type
+    static constexpr int ROW_BYTES = R * 2;                                   // bytes per row of R values
+};
+
+// ---- PTX wrappers specific to this kernel ---------------------------------------------------
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int c0, int c1, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+        "[%4];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// 16-byte cp.async; src_bytes == 0 fills the 16 bytes with zeros (nothing is read).
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes)
+                 : "memory");
+}
+
+// The mbarrier counts one arrival when all of this thread's earlier cp.async copies are done.
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// Shared-memory matrix descriptor (tcgen05): start, leading and stride byte offsets, layout.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo, uint64_t layout) {
+    uint64_t d = 0;
+    d |= uint64_t((saddr >> 4) & 0x3fff);
+    d |= uint64_t((lbo >> 4) & 0x3fff) << 16;
+    d |= uint64_t((sbo >> 4) & 0x3fff) << 32;
+    d |= uint64_t(1) << 46;  // descriptor version for tcgen05
+    d |= layout << 61;
+    return d;
+}
+
+// Instruction descriptor, kind::f16: D fp32, A/B fp16 (0) or bf16 (1), majors, N, M.
+__host__ __device__ constexpr uint32_t instr_desc(uint32_t ab_format, uint32_t a_mn_major, uint32_t b_mn_major,
+                                                   uint32_t N, uint32_t M) {
+    return (1u << 4) | (ab_format << 7) | (ab_format << 10) | (a_mn_major << 15) | (b_mn_major << 16) |
+           ((N >> 3) << 17) | ((M >> 4) << 24);
+}
+
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                       uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// mbarrier arrives once every tcgen05 operation this thread issued so far has completed.
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+
+// 32 consecutive fp32 columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// byte offset of 16-byte chunk `chunk` of row `row` in a swizzled tile with rows of 16 << bits bytes
+__device__ __forceinline__ uint32_t swz(uint32_t row, uint32_t chunk, int bits) {
+    const uint32_t lin = row * (16u << bits) + chunk * 16u;
+    return lin ^ (((lin >> 7) & ((1u << bits) - 1u)) << 4);
+}
+
+// Tile t (over all segments, 128 rows each) -> (segment, M-tile); false if t is past the last tile.
+// Run by one whole warp.
+__device__ bool find_tile(const GroupedParams& P, int tile, int& seg_out, int& mt_out) {
+    const int lane = threadIdx.x & 31;
+    int base = 0;
+    for (int s0 = 0; s0 < P.n_segments; s0 += 32) {
+        const int s = s0 + lane;
+        int cnt = 0;
+        if (s < P.n_segments) {
+            const int b = __ldg(P.seg_starts + s), e = __ldg(P.seg_starts + s + 1);
+            if (b >= 0 && b <= e && e <= P.T) cnt = (e - b + kGM - 1) / kGM;
+        }
+        int incl = cnt;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += y;
+        }
+        const int excl = base + incl - cnt;
+        const unsigned hit = __ballot_sync(0xffffffffu, cnt > 0 && tile >= excl && tile < excl + cnt);
+        if (hit) {
+            const int src = __ffs(hit) - 1;
+            seg_out = s0 + src;
+            mt_out = tile - __shfl_sync(0xffffffffu, excl, src);
+            return true;
+        }
+        base += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    return false;
+}
+
+// grid.x = tiles (upper bound) * nsplit; block kGThreads.
+template <typename T, int R>
+__global__ void __launch_bounds__(kGThreads, 1)
+    sgmv_grouped_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmY,
+                           const GroupedParams P) {
+    using G = GroupedGeom<R>;
+    extern __shared__ __align__(1024) unsigned char gsmem_raw[];
+    // 1024-byte alignment for the swizzled tiles
+    unsigned char* gsmem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(gsmem_raw) + 1023) & ~uintptr_t(1023));
+    unsigned char* sstage = gsmem;
+    unsigned char* estage = sstage + kGShrinkStages * G::SSTAGE;
+    unsigned char* vhi = estage + kGExpandStages * G::ESTAGE;
+    unsigned char* vlo = vhi + G::V_BYTES;
+
+    __shared__ __align__(8) uint64_t s_full[kGShrinkStages], s_empty[kGShrinkStages];
+    __shared__ __align__(8) uint64_t e_full[kGExpandStages], e_empty[kGExpandStages];
+    __shared__ __align__(8) uint64_t d1_full, v_full, d2_full[2], d2_empty[2];
+    __shared__ uint32_t tmem_base_s;
+    __shared__ int job_s[3];
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int tile = blockIdx.x / P.nsplit;
+    const int nsl = blockIdx.x - tile * P.nsplit;
+
+    if (warp == 0) {
+        int s = -1, mt = 0;
+        const bool ok = find_tile(P, tile, s, mt);
+        if (lane == 0) {
+            job_s[0] = ok ? s : -1;
+            job_s[1] = mt;
+            Segment seg;
+            if (ok && load_segment(P.seg_starts, P.lora_idx, P.A_ptrs, P.B_ptrs, s, P.T, P.num_adapters, seg))
+                job_s[0] = -1;  // rejected segment: reported by CTA 0 below
+        }
+        if (blockIdx.x == 0) {  // report every rejected segment once
+            for (int s2 = lane; s2 < P.n_segments; s2 += 32) {
+                Segment seg;
+                report(P.dev_status,
+                       load_segment(P.seg_starts, P.lora_idx, P.A_ptrs, P.B_ptrs, s2, P.T, P.num_adapters, seg));
+            }
+        }
+    }
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kGShrinkStages; ++i) {
+            mbar_init(&s_full[i], 1 + 32);  // TMA expect_tx arrival + 32 cp.async arrivals
+            mbar_init(&s_empty[i], 1);      // MMA commit
+        }
+        for (int i = 0; i < kGExpandStages; ++i) {
+            mbar_init(&e_full[i], 1 + 32);
+            mbar_init(&e_empty[i], 1 + 4);  // MMA commit (B read) + 4 epilogue warps (Y read)
+        }
+        mbar_init(&d1_full, 1);
+        mbar_init(&v_full, 4);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&d2_full[i], 1);
+            mbar_init(&d2_empty[i], 4);
+        }
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    const int seg_id = job_s[0];
+    if (seg_id < 0) return;  // no tile here, or a rejected segment (reported once)
+    const int mt = job_s[1];
+
+    Segment seg;
+    load_segment(P.seg_starts, P.lora_idx, P.A_ptrs, P.B_ptrs, seg_id, P.T, P.num_adapters, seg);
+    const int t0 = seg.begin + mt * kGM;
+    const int rows = min(kGM, seg.end - t0);  // valid rows of this tile
+    const int n_lo = nsl * P.nspan;
+    const int n_hi = min(P.H2, n_lo + P.nspan);
+    const int n_tiles = n_lo < n_hi ? (n_hi - n_lo + kGN - 1) / kGN : 0;
+    const int k_steps = (P.H1 + kGK - 1) / kGK;
+
+    // TMEM: D1 at columns [0, R), D2 buffers at 128 and 256
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tmem_base_s)),
+                     "r"(kGTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_base_s;
+    bool dead = false;
+
+    if (warp == 0) {
+        // ---------------------------------- producer ----------------------------------
+        const T* A = static_cast<const T*>(seg.a);
+        const T* B = static_cast<const T*>(seg.b);
+        for (int ks = 0; ks < k_steps; ++ks) {
+            const int st = ks % kGShrinkStages;
+            if (ks >= kGShrinkStages) mbar_wait<false>(&s_empty[st], ((ks / kGShrinkStages) - 1) & 1u, P.dev_status, dead);
+            unsigned char* xs = sstage + st * G::SSTAGE;
+            unsigned char* as = xs + G::X_BYTES;
+            if (lane == 0) {
+                mbar_arrive_expect_tx(&s_full[st], G::X_BYTES);
+                tma_load_2d(xs, &tmX, ks * kGK, t0, &s_full[st]);
+            }
+            // A_i rows [ks*64, ks*64+64), R values each, MN-major swizzled
+            constexpr int CHUNKS = kGK * R / 8;
+            for (int q = lane; q < CHUNKS; q += 32) {
+                const int k = q / (R / 8), c = q % (R / 8);
+                const int gk = ks * kGK + k;
+                const bool in = gk < P.H1;
+                cp_async16(as + swz(k, c, G::SW_BITS), A + size_t(in ? gk : 0) * R + c * 8, in ? 16u : 0u);
+            }
+            cp_async_arrive_noinc(&s_full[st]);
+        }
+        for (int nt = 0; nt < n_tiles; ++nt) {
+            const int st = nt % kGExpandStages;
+            if (nt >= kGExpandStages) mbar_wait<false>(&e_empty[st], ((nt / kGExpandStages) - 1) & 1u, P.dev_status, dead);
+            unsigned char* ys = estage + st * G::ESTAGE;
+            unsigned char* bs = ys + G::Y_BYTES;
+            const int n0 = n_lo + nt * kGN;
+            if (lane == 0) {
+                mbar_arrive_expect_tx(&e_full[st], G::Y_BYTES);
+                tma_load_2d(ys, &tmY, n0, t0, &e_full[st]);
+                tma_load_2d(ys + G::Y_BYTES / 2, &tmY, n0 + 64, t0, &e_full[st]);
+            }
+            // B_i rows 0..R-1, columns n0..n0+127 as two 64-column MN-major blocks (128B swizzle)
+            constexpr int CHUNKS = R * kGN / 8;
+            for (int q = lane; q < CHUNKS; q += 32) {
+                const int k = q / (kGN / 8), cc = q % (kGN / 8);
+                const int blk = cc / 8, c = cc % 8;
+                const int gn = n0 + cc * 8;
+                const bool in = gn < n_hi;
+                cp_async16(bs + blk * (R * 128) + swz(k, c, 3), B + size_t(k) * P.H2 + (in ? gn : 0), in ? 16u : 0u);
+            }
+            cp_async_arrive_noinc(&e_full[st]);
+        }
+        asm volatile("cp.async.wait_all;" ::: "memory");
+    } else if (warp == 1) {
+        // ---------------------------------- MMA issuer ----------------------------------
+        const uint32_t fmt = std::is_same<T, __nv_bfloat16>::value ? 1u : 0u;
+        const uint32_t idesc_s = instr_desc(fmt, 0, 1, R, kGM);    // X K-major, A_i MN-major, N = r
+        const uint32_t idesc_e = instr_desc(fmt, 0, 1, kGN, kGM);  // V K-major, B_i MN-major, N = 128
+        for (int ks = 0; ks < k_steps; ++ks) {
+            const int st = ks % kGShrinkStages;
+            mbar_wait<false>(&s_full[st], (ks / kGShrinkStages) & 1u, P.dev_status, dead);
+            fence_proxy_async();  // cp.async (generic proxy) writes -> tensor-core reads
+            tc_fence_after();
+            if (lane == 0) {
+                const uint32_t xa = smem_u32(sstage + st * G::SSTAGE);
+                const uint32_t aa = xa + G::X_BYTES;
+#pragma unroll
+                for (int kk = 0; kk < kGK / 16; ++kk) {
+                    const uint64_t adesc = smem_desc(xa + kk * 32, 16, 1024, 2);
+                    const uint64_t bdesc = smem_desc(aa + kk * 16 * G::ROW_BYTES, 16 * G::ROW_BYTES, 8 * G::ROW_BYTES,
+                                                     G::SW_TYPE);
+                    tc_mma(tmem, adesc, bdesc, idesc_s, (ks | kk) ? 1u : 0u);
+                }
+                tc_commit(&s_empty[st]);
+            }
+            __syncwarp();
+        }
+        if (lane == 0) tc_commit(&d1_full);
+        __syncwarp();
+        mbar_wait<false>(&v_full, 0, P.dev_status, dead);
+        tc_fence_after();
+        for (int nt = 0; nt < n_tiles; ++nt) {
+            const int st = nt % kGExpandStages;
+            const int buf = nt & 1;
+            if (nt >= 2) mbar_wait<false>(&d2_empty[buf], ((nt >> 1) - 1) & 1u, P.dev_status, dead);
+            mbar_wait<false>(&e_full[st], (nt / kGExpandStages) & 1u, P.dev_status, dead);
+            fence_proxy_async();
+            tc_fence_after();
+            if (lane == 0) {
+                const uint32_t ba = smem_u32(estage + st * G::ESTAGE + G::Y_BYTES);
+                const uint32_t d2 = tmem + 128u + 128u * buf;
+#pragma unroll
+                for (int kk = 0; kk < R / 16; ++kk) {
+                    const uint64_t bdesc = smem_desc(ba + kk * 16 * 128, R * 128, 1024, 2);
+                    const uint64_t ahi = smem_desc(smem_u32(vhi) + kk * 32, 16, 8 * G::ROW_BYTES, G::SW_TYPE);
+                    const uint64_t alo = smem_desc(smem_u32(vlo) + kk * 32, 16, 8 * G::ROW_BYTES, G::SW_TYPE);
+                    tc_mma(d2, ahi, bdesc, idesc_e, kk ? 1u : 0u);
+                    tc_mma(d2, alo, bdesc, idesc_e, 1u);
+                }
+                tc_commit(&d2_full[buf]);
+                tc_commit(&e_empty[st]);
+            }
+            __syncwarp();
+        }
+    } else {
+        // ---------------------------------- epilogue ----------------------------------
+        const int quarter = warp & 3;  // TMEM lanes [32*quarter, 32*quarter + 32)
+        const int m = quarter * 32 + lane;
+        const uint32_t lane_addr = tmem + (uint32_t(quarter * 32) << 16);
+        // V = D1 -> V_hi + V_lo (K-major, swizzled rows of R values)
+        mbar_wait<false>(&d1_full, 0, P.dev_status, dead);
+        tc_fence_after();
+#pragma unroll
+        for (int c0 = 0; c0 < R; c0 += 32) {
+            float v[32];
+            tmem_ld32(lane_addr + c0, v);
+            const int nchunks = (R - c0) < 32 ? (R - c0) / 8 : 4;
+            for (int ch = 0; ch < nchunks; ++ch) {
+                float hi[8], lo[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const float x = v[ch * 8 + i];
+                    const float h = Storage<T>::round(x);
+                    hi[i] = h;
+                    lo[i] = x - h;
+                }
+                const uint32_t off = swz(m, c0 / 8 + ch, G::SW_BITS);
+                st_vec(vhi + off, pack8<T>(hi));
+                st_vec(vlo + off, pack8<T>(lo));
+            }
+        }
+        fence_proxy_async();  // generic-proxy writes of V -> tensor-core reads
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_local(&v_full);
+
+        T* __restrict__ Y = static_cast<T*>(P.Y);
+        const bool row_ok = m < rows;
+        for (int nt = 0; nt < n_tiles; ++nt) {
+            const int st = nt % kGExpandStages;
+            const int buf = nt & 1;
+            mbar_wait<false>(&e_full[st], (nt / kGExpandStages) & 1u, P.dev_status, dead);
+            mbar_wait<false>(&d2_full[buf], (nt >> 1) & 1u, P.dev_status, dead);
+            tc_fence_after();
+            const unsigned char* ys = estage + st * G::ESTAGE;
+            const int n0 = n_lo + nt * kGN;
+#pragma unroll 1
+            for (int c0 = 0; c0 < kGN; c0 += 32) {
+                float acc[32];
+                tmem_ld32(lane_addr + 128u + 128u * buf + c0, acc);
+                if (row_ok) {
+                    const unsigned char* yb = ys + (c0 / 64) * (G::Y_BYTES / 2);
+#pragma unroll
+                    for (int ch = 0; ch < 4; ++ch) {
+                        const int col = n0 + c0 + ch * 8;
+                        if (col < n_hi) {
+                            float y[8];
+                            unpack8<T>(*reinterpret_cast<const uint4*>(yb + swz(m, (c0 % 64) / 8 + ch, 3)), y);
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) y[i] = __fadd_rn(y[i], __fmul_rn(P.scale, acc[ch * 8 + i]));
+                            st_vec(Y + size_t(t0 + m) * P.H2 + col, pack8<T>(y));
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive_local(&d2_empty[buf]);
+                mbar_arrive_local(&e_empty[st]);
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kGTmemCols) : "memory");
+}
+
+// ---- host side ---------------------------------------------------------------------------
+
+using EncodeTiledFn = PFN_cuTensorMapEncodeTiled_v12000;
+
+// cuTensorMapEncodeTiled from the driver, looked up once (no link-time dependency on libcuda).
+inline EncodeTiledFn encode_tiled_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// Row-major [rows, cols] 16-bit matrix, boxes of 128 rows x 64 columns, 128-byte swizzle,
+// zero fill outside the matrix.
+inline bool make_tile_map(CUtensorMap* map, const void* base, int rows, int cols, lora_sgmv_dtype dt) {
+    EncodeTiledFn enc = encode_tiled_fn();
+    if (!enc) return false;
+    cuuint64_t gdim[2] = {cuuint64_t(cols), cuuint64_t(rows)};
+    cuuint64_t gstride[1] = {cuuint64_t(cols) * 2};
+    cuuint32_t box[2] = {64, 128};
+    cuuint32_t estride[2] = {1, 1};
+    const CUresult r = enc(map, dt == LORA_SGMV_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                           2, const_cast<void*>(base), gdim, gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <typename T, int R>
+inline cudaError_t launch_grouped_tc_kernel(const CUtensorMap& tmX, const CUtensorMap& tmY, const GroupedParams& P,
+                                            int blocks, cudaStream_t stream) {
+    using G = GroupedGeom<R>;
+    static std::once_flag once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(once, [] {
+        attr_err = cudaFuncSetAttribute(sgmv_grouped_tc_kernel<T, R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        static_cast<int>(G::SMEM));
+    });
+    if (attr_err != cudaSuccess) return attr_err;
+    sgmv_grouped_tc_kernel<T, R><<<blocks, kGThreads, G::SMEM, stream>>>(tmX, tmY, P);
+    return cudaGetLastError();
 }
 
 }  // namespace sgmv

@@ -225,3 +225,45 @@ def test_large_h1_and_many_segments():
     w = inputs.small_random(T, 6, 16384, 520, 32, "bf16", seed=8)
     p = DeviceProblem(w, y_random=True, adapters=list(range(6)), seg_starts=seg, lora_idx=idx)
     assert_close(p.apply(), p.oracle_apply(), "bf16", "H1=16384")
+
+
+# ---- grouped tensor-core kernel (prefill) ---------------------------------------------------
+
+@pytest.mark.parametrize("r", [16, 32, 64])
+@pytest.mark.parametrize("dtype", ["bf16", "f16"])
+def test_grouped_tc_ragged_tiles(r, dtype):
+    # segments shorter than, equal to and longer than the 128-row tile; H1 not a multiple of the
+    # 64-wide K step; H2 not a multiple of the 128-wide N tile; an empty segment; Y non-zero
+    lens = [5, 128, 300, 0, 1, 129]
+    seg = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    idx = np.array([2, 0, 1, 3, 2, 4], np.int32)
+    w = inputs.small_random(int(seg[-1]), 5, 328, 392, r, dtype, seed=r)
+    p = DeviceProblem(w, y_random=True, adapters=list(range(5)), seg_starts=seg, lora_idx=idx)
+    got = p.apply(variant=sgmv.VARIANT_GROUPED_TC)
+    assert int(p.status.item()) == 0
+    assert_close(got, p.oracle_apply(), dtype, f"grouped r={r}")
+
+
+def test_grouped_tc_prefill_sampled():
+    w = inputs.make("prefill")
+    p = DeviceProblem(w, y_random=True)
+    got = p.apply(variant=sgmv.VARIANT_GROUPED_TC)
+    _sampled_check(p, got, 400, 3)
+    assert int(p.status.item()) == 0
+
+
+def test_grouped_tc_bad_segments_skipped():
+    seg = np.array([0, 200, 150, 400, 450], np.int32)  # [200,150) reversed
+    idx = np.array([0, 1, 7, 2], np.int32)             # adapter 7 out of range
+    w = inputs.small_random(450, 4, 256, 256, 64, "bf16", seed=5)
+    p = DeviceProblem(w, y_random=True, adapters=list(range(4)), seg_starts=seg, lora_idx=idx)
+    before = from_dev(p.Y)
+    got = p.apply(variant=sgmv.VARIANT_GROUPED_TC)
+    st = int(p.status.item())
+    assert st & sgmv.DEV_BAD_SEGMENT and st & sgmv.DEV_BAD_ADAPTER
+    ref = DeviceProblem(w, y_random=True, adapters=list(range(4)), seg_starts=[0, 200, 400, 450],
+                        lora_idx=[0, 0, 2]).oracle_apply()
+    # valid: [0,200) on adapter 0 and [400,450) on adapter 2; rows 200..399 only in rejected segments
+    assert_close(got[:200], ref[:200], "bf16", "valid segment 0")
+    assert_close(got[400:], ref[400:], "bf16", "valid segment 3")
+    assert np.array_equal(got[200:400], before[200:400])
