@@ -1,7 +1,7 @@
 // sgmv_fused.cuh -- one-kernel SGMV for short segments (decode): shrink, V reduction
 // and expand with the fused add, for one or several projections in one launch.
 //
-// Maths (Punica README, LoRA and multi-LoRA paragraphs): for each segment s
+// Maths (page “Punica：多 LoRA 模型统一服务框架”, the Punica README, its LoRA and multi-LoRA paragraphs): for each segment s
 // with adapter i and each row t of it, Y[t,:] += scale * (X[t,:] @ A_i) @ B_i,
 // A_i [H1, r], B_i [r, H2], row-major.
 //

@@ -1,7 +1,7 @@
 // sgmv_grouped_tc.cuh -- grouped SGMV on the 5th-generation tensor cores (tcgen05, TMEM)
 // for long segments (prefill).
 //
-// Maths (Punica README, LoRA and multi-LoRA paragraphs): for each segment s with
+// Maths (page “Punica：多 LoRA 模型统一服务框架”, the Punica README, its LoRA and multi-LoRA paragraphs): for each segment s with
 // adapter i and every row t of it, Y[t,:] += scale * (X[t,:] @ A_i) @ B_i, A_i [H1, r],
 // B_i [r, H2], row-major. With many rows per segment both halves are real matrix
 // products: a [L, H1] x [H1, r] shrink and a [L, r] x [r, H2] expand per segment.

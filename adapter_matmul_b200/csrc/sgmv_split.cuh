@@ -1,7 +1,7 @@
 // sgmv_split.cuh -- the split SGMV path: a split-K shrink kernel (H1 -> r) and a
 // streaming expand kernel (r -> H2) with the add onto Y fused in its epilogue.
 //
-// Shapes follow the Punica README's LoRA paragraph: A_i is [H1, r], B_i is
+// Shapes follow the LoRA paragraph of page “Punica：多 LoRA 模型统一服务框架” (the Punica README): A_i is [H1, r], B_i is
 // [r, H2], rows are tokens; the batch form (multi-LoRA paragraph) maps each
 // segment of rows to its own adapter.
 //

@@ -6,8 +6,8 @@ storage cast of freshly drawn normals. Both the CUDA path (through the tests
 and ``bench.py``) and the CPU oracle take their inputs from here.
 
 Workloads follow the adapter-popularity distributions named in the Punica
-README ("Punica: Serving multiple LoRA finetuned LLM as one", text-generation
-benchmark paragraph): Distinct (every request its own adapter), Identical (all
+README page ("Punica：多 LoRA 模型统一服务框架", text-generation benchmark
+paragraph): Distinct (every request its own adapter), Identical (all
 requests on one adapter), Uniform and Skewed (in between). The shapes are the
 LoRA shapes of the README's LoRA paragraph: ``A`` is ``[H1, r]``, ``B`` is
 ``[r, H2]``, rows are tokens.

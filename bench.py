@@ -4,7 +4,8 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
 
 Default workload ("distinct"): Llama-7B-shaped decode with the Distinct
-adapter distribution of the Punica README's throughput benchmark: 32 tokens,
+adapter distribution of the throughput benchmark on page “Punica：多 LoRA 模型统一服务框架” (the Punica
+README): 32 tokens,
 each on its own rank-16 adapter, H1 = H2 = 4096, fp16. One step is one decoder
 layer's LoRA work: four SGMV calls (q, k, v, o projections), each with its
 own adapters, input and output. Steps rotate over 32 layers, each with its own

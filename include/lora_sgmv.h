@@ -1,9 +1,8 @@
 /*
  * lora_sgmv.h -- C ABI of the SGMV library for NVIDIA B200 (sm_100a).
  *
- * SGMV ("Segmented Gather Matrix-Vector multiplication", Punica README,
- * "Punica: Serving multiple LoRA finetuned LLM as one", the paragraph that
- * names the kernel) computes the LoRA term of a batch in which each token
+ * SGMV ("Segmented Gather Matrix-Vector multiplication", the Punica README
+ * page "Punica：多 LoRA 模型统一服务框架", the paragraph that names the kernel) computes the LoRA term of a batch in which each token
  * uses its own adapter. The README's LoRA paragraph fixes the shapes: a
  * frozen weight W is [H1, H2]; an adapter adds A [H1, r] and B [r, H2];
  * y = x@(W + A@B) = x@W + x@A@B. Its multi-LoRA paragraph fixes the batch

@@ -8,7 +8,7 @@ seeded input generator.
 The arithmetic lives in ``sgmv_oracle.c`` (plain C, no CUDA, no BLAS), built
 with gcc into ``liboracle.so`` beside it. This wrapper only marshals numpy
 arrays. See that file's header for what is computed and from which passage
-of the Punica README.
+of the Punica README page “Punica：多 LoRA 模型统一服务框架”.
 """
 from __future__ import annotations
 

@@ -9,8 +9,8 @@
  * own, written from the IEEE 754 binary16 definition and from bfloat16 being
  * the upper half of an IEEE binary32.
  *
- * What it computes (Punica README, "Punica: Serving multiple LoRA finetuned
- * LLM as one", LoRA paragraph and the multi-LoRA batch paragraph after it):
+ * What it computes (the Punica README page, "Punica：多 LoRA 模型统一服务框架",
+ * its LoRA paragraph and the multi-LoRA batch paragraph after it):
  *   - a frozen weight W of shape [H1, H2]; an adapter adds A of shape [H1, r]
  *     and B of shape [r, H2]; y = x @ (W + A@B) = x@W + x@A@B (row vectors);
  *   - with n adapters (A_1, B_1) ... (A_n, B_n) and a batch X whose input x_j

@@ -1,6 +1,6 @@
 """Pins for the CPU oracle: each test checks it against something other than itself.
 
-What the pages fix (Punica README, LoRA paragraph and multi-LoRA paragraph):
+What the pages fix (page “Punica：多 LoRA 模型统一服务框架”, the Punica README: LoRA paragraph and multi-LoRA paragraph):
 the shapes A [H1, r], B [r, H2]; the identity x@(W + A@B) = x@W + x@A@B; the
 batched definition in which each row uses its own adapter. The pins below are:
 library conversions (numpy float16, torch bfloat16), a hand-worked example,
