@@ -13,6 +13,7 @@
 #include <vector>
 
 #include "../../include/lora_sgmv.h"
+#include "sgmv_decode_tc.cuh"
 #include "sgmv_fused.cuh"
 #include "sgmv_grouped_tc.cuh"
 #include "sgmv_split.cuh"
@@ -253,10 +254,10 @@ int round8(int v) { return (v + 7) / 8 * 8; }
 
 // Largest number of clusters of `cluster` CTAs with `smem` bytes each that can be resident at once.
 template <typename K>
-lora_sgmv_status max_active_clusters(K kernel, int cluster, size_t smem, int* out) {
+lora_sgmv_status max_active_clusters(K kernel, int cluster, size_t smem, int* out, int threads = sgmv::kFusedThreads) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(cluster, 1, 1);
-    cfg.blockDim = dim3(sgmv::kFusedThreads, 1, 1);
+    cfg.blockDim = dim3(threads, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -345,6 +346,97 @@ lora_sgmv_status launch_fused(sgmv::FusedParams P, int max_len, cudaStream_t str
     return counted(cudaLaunchKernelEx(&cfg, kernel, P));
 }
 
+// ---- tensor-core decode path -------------------------------------------------------------------
+
+bool decode_tc_supported(int r, int H1, int H2) { return (r == 16 || r == 32 || r == 64) && H1 >= 64 && H2 >= 64; }
+
+template <typename T, int R>
+lora_sgmv_status launch_decode_tc(sgmv::FusedParams P, const sgmv::XMaps& maps, int max_len, cudaStream_t stream) {
+    static int smem_granted[64] = {};
+    static int resident[64][4][9] = {};
+    using G = sgmv::DecodeTCGeom<R>;
+    constexpr int CH = sgmv::kDTokens;
+    if (P.n_segments > sgmv::kFusedMaxSegments) return LORA_SGMV_ERR_DIM;
+    const int bucket = (P.n_segments + 1 + 1023) / 1024;  // 1..9
+    const size_t smem = G::BASE + size_t(bucket) * 1024 * 4 + 1024 /* alignment slack */;
+    auto kernel = sgmv::sgmv_decode_tc_kernel<T, R>;
+    if (ensure_smem(kernel, smem, smem_granted) != LORA_SGMV_OK) return LORA_SGMV_ERR_CUDA;
+    int dev = 0;
+    if (record(cudaGetDevice(&dev)) != cudaSuccess) return LORA_SGMV_ERR_CUDA;
+    if (dev < 0 || dev >= 64) return LORA_SGMV_ERR_UNSUPPORTED;
+    auto resident_for = [&](int lc, int* out) -> lora_sgmv_status {
+        {
+            std::lock_guard<std::mutex> lock(g_mu);
+            if (resident[dev][lc][bucket - 1] > 0) {
+                *out = resident[dev][lc][bucket - 1];
+                return LORA_SGMV_OK;
+            }
+        }
+        int n = 0;
+        lora_sgmv_status st = max_active_clusters(kernel, 1 << lc, smem, &n, sgmv::kDThreads);
+        if (st != LORA_SGMV_OK) return st;
+        std::lock_guard<std::mutex> lock(g_mu);
+        resident[dev][lc][bucket - 1] = n;
+        *out = n;
+        return LORA_SGMV_OK;
+    };
+    const bool one_chunk = max_len <= CH;
+    const long long chunks =
+        std::min<long long>(P.n_segments + (P.T + CH - 1) / CH, std::max(P.T, 1));
+    const long long jobs = std::max<long long>(1, (one_chunk ? static_cast<long long>(P.n_segments) : chunks) *
+                                                      P.n_problems);
+    int ctas = 0;
+    lora_sgmv_status st = resident_for(0, &ctas);
+    if (st != LORA_SGMV_OK) return st;
+    int lc = 3;
+    while (lc > 0 && jobs * (1ll << lc) > ctas) --lc;
+    int clusters_max = 0;
+    st = resident_for(lc, &clusters_max);
+    if (st != LORA_SGMV_OK) return st;
+    const int C = 1 << lc;
+    P.one_chunk = one_chunk ? 1 : 0;
+    for (int i = 0; i < P.n_problems; ++i) {
+        P.prob[i].ks = (P.prob[i].H1 + C * sgmv::kGK - 1) / (C * sgmv::kGK) * sgmv::kGK;
+        P.prob[i].ns = (P.prob[i].H2 + C * sgmv::kGN - 1) / (C * sgmv::kGN) * sgmv::kGN;
+    }
+    int clusters = static_cast<int>(std::min<long long>(jobs, clusters_max));
+    const long long rounds = (jobs + clusters - 1) / clusters;
+    clusters = static_cast<int>((jobs + rounds - 1) / rounds);
+
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(clusters * C, 1, 1);
+    cfg.blockDim = dim3(sgmv::kDThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = C;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    return counted(cudaLaunchKernelEx(&cfg, kernel, maps, P));
+}
+
+lora_sgmv_status decode_tc_dispatch(sgmv::FusedParams& P, int r, lora_sgmv_dtype dt, int max_len, cudaStream_t s) {
+    sgmv::XMaps maps;
+    std::memset(&maps, 0, sizeof(maps));
+    for (int i = 0; i < P.n_problems; ++i)
+        if (!sgmv::make_tile_map(&maps.m[i], P.prob[i].X, P.T, P.prob[i].H1, dt, sgmv::kDTokens)) {
+            t_last_error = cudaErrorInvalidValue;
+            return LORA_SGMV_ERR_CUDA;
+        }
+    const bool bf = dt == LORA_SGMV_BF16;
+    switch (r) {
+        case 16: return bf ? launch_decode_tc<__nv_bfloat16, 16>(P, maps, max_len, s) : launch_decode_tc<__half, 16>(P, maps, max_len, s);
+        case 32: return bf ? launch_decode_tc<__nv_bfloat16, 32>(P, maps, max_len, s) : launch_decode_tc<__half, 32>(P, maps, max_len, s);
+        case 64: return bf ? launch_decode_tc<__nv_bfloat16, 64>(P, maps, max_len, s) : launch_decode_tc<__half, 64>(P, maps, max_len, s);
+    }
+    return LORA_SGMV_ERR_UNSUPPORTED;
+}
+
 template <typename T>
 lora_sgmv_status fused_dispatch_r(const sgmv::FusedParams& P, int r, int max_len, cudaStream_t s) {
     switch (r) {
@@ -387,6 +479,7 @@ int32_t lora_sgmv_rank_supported(int32_t r, lora_sgmv_variant variant) {
         case LORA_SGMV_VARIANT_SPLIT: return split_rank(r) ? 1 : 0;
         case LORA_SGMV_VARIANT_GROUPED_TC: return sgmv::grouped_tc_rank(r) ? 1 : 0;
         case LORA_SGMV_VARIANT_FUSED: return split_rank(r) ? 1 : 0;
+        case LORA_SGMV_VARIANT_FUSED_TC: return (r == 16 || r == 32 || r == 64) ? 1 : 0;
     }
     return 0;
 }
@@ -506,7 +599,8 @@ lora_sgmv_status lora_sgmv_apply_ex(void* Y, const void* X, const void* const* A
     if (st != LORA_SGMV_OK) return st;
     if (H1 <= 0 || H2 <= 0 || r <= 0) return LORA_SGMV_ERR_DIM;
     if (variant != LORA_SGMV_VARIANT_AUTO && variant != LORA_SGMV_VARIANT_SPLIT &&
-        variant != LORA_SGMV_VARIANT_GROUPED_TC && variant != LORA_SGMV_VARIANT_FUSED)
+        variant != LORA_SGMV_VARIANT_GROUPED_TC && variant != LORA_SGMV_VARIANT_FUSED &&
+        variant != LORA_SGMV_VARIANT_FUSED_TC)
         return LORA_SGMV_ERR_UNSUPPORTED;
     if (!lora_sgmv_rank_supported(r, variant)) return LORA_SGMV_ERR_UNSUPPORTED;
     if (n_segments == 0 || T == 0) return LORA_SGMV_OK;
@@ -523,9 +617,13 @@ lora_sgmv_status lora_sgmv_apply_ex(void* Y, const void* X, const void* const* A
     if (v == LORA_SGMV_VARIANT_AUTO)
         v = (max_len >= sgmv::kGroupedMinSegment && sgmv::grouped_tc_supported(r, H1, H2, dtype))
                 ? LORA_SGMV_VARIANT_GROUPED_TC
-                : (n_segments <= sgmv::kFusedMaxSegments ? LORA_SGMV_VARIANT_FUSED : LORA_SGMV_VARIANT_SPLIT);
+                : (n_segments > sgmv::kFusedMaxSegments
+                       ? LORA_SGMV_VARIANT_SPLIT
+                       : (max_len > 2 && decode_tc_supported(r, H1, H2) ? LORA_SGMV_VARIANT_FUSED_TC
+                                                                        : LORA_SGMV_VARIANT_FUSED));
 
-    if (v == LORA_SGMV_VARIANT_FUSED) {
+    if (v == LORA_SGMV_VARIANT_FUSED || v == LORA_SGMV_VARIANT_FUSED_TC) {
+        if (v == LORA_SGMV_VARIANT_FUSED_TC && !decode_tc_supported(r, H1, H2)) return LORA_SGMV_ERR_UNSUPPORTED;
         sgmv::FusedParams P = {};
         P.prob[0].Y = Y;
         P.prob[0].X = X;
@@ -541,6 +639,7 @@ lora_sgmv_status lora_sgmv_apply_ex(void* Y, const void* X, const void* const* A
         P.n_problems = 1;
         P.n_segments = n_segments;
         P.T = T;
+        if (v == LORA_SGMV_VARIANT_FUSED_TC) return decode_tc_dispatch(P, r, dtype, max_len, s);
         return fused_dispatch(P, r, dtype, max_len, s);
     }
 
@@ -631,8 +730,11 @@ extern "C" lora_sgmv_status lora_sgmv_apply_batched(const lora_sgmv_problem* pro
     P.n_problems = n_problems;
     P.n_segments = n_segments;
     P.T = T;
-    return fused_dispatch(P, r, dtype, estimate_max_len(max_seg_len, T, n_segments),
-                          static_cast<cudaStream_t>(stream));
+    const int max_len = estimate_max_len(max_seg_len, T, n_segments);
+    bool tc = max_len > 2;
+    for (int i = 0; i < n_problems; ++i) tc = tc && decode_tc_supported(r, problems[i].H1, problems[i].H2);
+    if (tc) return decode_tc_dispatch(P, r, dtype, max_len, static_cast<cudaStream_t>(stream));
+    return fused_dispatch(P, r, dtype, max_len, static_cast<cudaStream_t>(stream));
 }
 
 // ---- apply for callers that cannot allocate device memory -----------------------------------

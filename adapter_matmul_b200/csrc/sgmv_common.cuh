@@ -91,6 +91,7 @@ struct Storage<__half> {
     static __device__ __forceinline__ float to1(__half v) { return __half2float(v); }
     // x rounded to the nearest fp16 value, returned as fp32
     static __device__ __forceinline__ float round(float x) { return __half2float(__float2half_rn(x)); }
+    static __device__ __forceinline__ __half from1(float x) { return __float2half_rn(x); }
 };
 
 template <>
@@ -106,6 +107,7 @@ struct Storage<__nv_bfloat16> {
     static __device__ __forceinline__ float to1(__nv_bfloat16 v) { return __bfloat162float(v); }
     // x rounded to the nearest bf16 value, returned as fp32
     static __device__ __forceinline__ float round(float x) { return __bfloat162float(__float2bfloat16_rn(x)); }
+    static __device__ __forceinline__ __nv_bfloat16 from1(float x) { return __float2bfloat16_rn(x); }
 };
 
 template <typename T>

@@ -241,16 +241,19 @@ __device__ __forceinline__ uint32_t cluster_size() {
 
 // ---- job list --------------------------------------------------------------------------
 
-// Number of 8-token chunks of segment s, or 0 if the segment is empty or invalid.
+// Number of CH-token chunks of segment s, or 0 if the segment is empty or invalid.
+template <int CH = kFusedTokens>
 __device__ __forceinline__ int segment_chunks(const FusedParams& P, int s) {
     const int b = __ldg(P.seg_starts + s), e = __ldg(P.seg_starts + s + 1);
     if (b < 0 || b > e || e > P.T) return 0;
-    return (e - b + kFusedTokens - 1) / kFusedTokens;
+    return (e - b + CH - 1) / CH;
 }
 
-// pref[s] = chunks of segments 0..s-1 (pref[0] = 0, pref[n] = chunks per problem), built by all threads.
+// pref[s] = chunks of segments 0..s-1 (pref[0] = 0, pref[n] = chunks per problem), built by all
+// threads of the block (at most 256).
+template <int CH = kFusedTokens>
 __device__ void build_job_prefix(const FusedParams& P, int* pref) {
-    __shared__ int warp_tot[kFusedThreads / 32];
+    __shared__ int warp_tot[8];
     const int n = P.n_segments;
     const int nthreads = blockDim.x;
     const int per = (n + nthreads - 1) / nthreads;
@@ -258,7 +261,7 @@ __device__ void build_job_prefix(const FusedParams& P, int* pref) {
     const int s1 = min(n, s0 + per);
     int local = 0;
     for (int s = s0; s < s1; ++s) {
-        local += segment_chunks(P, s);
+        local += segment_chunks<CH>(P, s);
         // warm L1 for the lookups job_at() makes next: adapter id, then its table entries
         const int i = __ldg(P.lora_idx + s);
         for (int p = 0; p < P.n_problems; ++p) {
@@ -283,7 +286,7 @@ __device__ void build_job_prefix(const FusedParams& P, int* pref) {
     int run = before + v - local;  // exclusive prefix of this thread's first segment
     if (threadIdx.x == 0) pref[0] = 0;
     for (int s = s0; s < s1; ++s) {
-        run += segment_chunks(P, s);
+        run += segment_chunks<CH>(P, s);
         pref[s + 1] = run;
     }
     __syncthreads();
@@ -302,13 +305,14 @@ struct Job {
 // Jobs of list entry j: (problem, segment, first chunk, number of chunks). With the
 // prefix, an entry is one chunk; in one-chunk mode an entry is a whole segment, whose
 // chunks the cluster then runs one after another.
+template <int CH = kFusedTokens>
 __device__ __forceinline__ void entry_at(const FusedParams& P, const int* pref, int j, int& p, int& s, int& q0,
                                          int& nq) {
     if (P.one_chunk) {
         p = j / P.n_segments;
         s = j - p * P.n_segments;
         q0 = 0;
-        nq = segment_chunks(P, s);
+        nq = segment_chunks<CH>(P, s);
         return;
     }
     const int per_problem = pref[P.n_segments];
@@ -327,14 +331,15 @@ __device__ __forceinline__ void entry_at(const FusedParams& P, const int* pref, 
     nq = 1;
 }
 
-// Chunk q of segment s of problem p: returns false if the segment fails the device-side checks.
+// Chunk q (of CH tokens) of segment s of problem p: false if the segment fails the device-side checks.
+template <int CH = kFusedTokens>
 __device__ __forceinline__ bool job_at(const FusedParams& P, int p, int s, int q, int c, Job& job) {
     const FusedProblem& pr = P.prob[p];
     Segment seg;
     if (load_segment(P.seg_starts, P.lora_idx, pr.A_ptrs, pr.B_ptrs, s, P.T, pr.num_adapters, seg)) return false;
     job.p = p;
-    job.t0 = seg.begin + q * kFusedTokens;
-    job.nt = min(kFusedTokens, seg.end - job.t0);
+    job.t0 = seg.begin + q * CH;
+    job.nt = min(CH, seg.end - job.t0);
     job.a = seg.a;
     job.b = seg.b;
     job.k0 = c * pr.ks;

@@ -483,14 +483,15 @@ inline EncodeTiledFn encode_tiled_fn() {
     return fn;
 }
 
-// Row-major [rows, cols] 16-bit matrix, boxes of 128 rows x 64 columns, 128-byte swizzle,
+// Row-major [rows, cols] 16-bit matrix, boxes of box_rows rows x 64 columns, 128-byte swizzle,
 // zero fill outside the matrix.
-inline bool make_tile_map(CUtensorMap* map, const void* base, int rows, int cols, lora_sgmv_dtype dt) {
+inline bool make_tile_map(CUtensorMap* map, const void* base, int rows, int cols, lora_sgmv_dtype dt,
+                          int box_rows = 128) {
     EncodeTiledFn enc = encode_tiled_fn();
     if (!enc) return false;
     cuuint64_t gdim[2] = {cuuint64_t(cols), cuuint64_t(rows)};
     cuuint64_t gstride[1] = {cuuint64_t(cols) * 2};
-    cuuint32_t box[2] = {64, 128};
+    cuuint32_t box[2] = {64, cuuint32_t(box_rows)};
     cuuint32_t estride[2] = {1, 1};
     const CUresult r = enc(map, dt == LORA_SGMV_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
                            2, const_cast<void*>(base), gdim, gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,

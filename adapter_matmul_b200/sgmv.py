@@ -26,6 +26,7 @@ VARIANT_AUTO = 0
 VARIANT_SPLIT = 1
 VARIANT_GROUPED_TC = 2
 VARIANT_FUSED = 3
+VARIANT_FUSED_TC = 4
 MAX_PROBLEMS = 8
 
 DEV_BAD_SEGMENT = 0x1

@@ -99,11 +99,13 @@ typedef enum {
     LORA_SGMV_VARIANT_AUTO = 0,
     LORA_SGMV_VARIANT_SPLIT = 1,      /* split-K shrink kernel, then streaming expand kernel */
     LORA_SGMV_VARIANT_GROUPED_TC = 2, /* tcgen05/TMEM grouped kernel for long segments */
-    LORA_SGMV_VARIANT_FUSED = 3       /* one kernel: cluster shrink, DSMEM V reduction, expand */
+    LORA_SGMV_VARIANT_FUSED = 3,      /* one kernel: cluster shrink, V reduction on chip, expand (fp32 FMA) */
+    LORA_SGMV_VARIANT_FUSED_TC = 4    /* the same split on tcgen05, for segments of several tokens */
 } lora_sgmv_variant;
 
 /* Ranks r built into this library: 8, 16, 32, 64 and 128 for the split and
- * fused kernels; 16, 32 and 64 for the grouped tensor-core kernel. */
+ * fused kernels; 16, 32 and 64 for the tensor-core kernels (GROUPED_TC,
+ * FUSED_TC), which also need H1 and H2 of at least 64. */
 int32_t lora_sgmv_rank_supported(int32_t r, lora_sgmv_variant variant);
 
 /* Human-readable name of a status code. Never NULL. */
@@ -241,9 +243,10 @@ typedef struct {
  *     problems[p].Y[t, :] += problems[p].scale * (problems[p].X[t, :] @ A_i) @ B_i
  * with i = lora_idx[s] and A_i, B_i taken from problem p's tables. Each
  * problem may have its own H1, H2, tables and adapter count; r and dtype are
- * shared. Runs the fused kernel (LORA_SGMV_VARIANT_FUSED), which keeps V on
- * chip and needs no workspace; it takes at most 8192 segments
- * (LORA_SGMV_ERR_DIM beyond).
+ * shared. Runs a fused kernel, which keeps V on chip and needs no
+ * workspace: LORA_SGMV_VARIANT_FUSED_TC when max_seg_len > 2 and every
+ * problem suits the tensor-core kernel, else LORA_SGMV_VARIANT_FUSED. It
+ * takes at most 8192 segments (LORA_SGMV_ERR_DIM beyond).
  *   problems     host array of n_problems entries, 1 <= n_problems <= 8.
  *   other arguments as for lora_sgmv_apply.
  * Validation errors of any problem are returned before anything is launched.

@@ -38,6 +38,8 @@ def test_version_and_ranks():
     for r in (8, 16, 32, 64, 128):
         assert sgmv.lora_sgmv_rank_supported(r, sgmv.VARIANT_SPLIT)
         assert sgmv.lora_sgmv_rank_supported(r, sgmv.VARIANT_FUSED)
+        assert sgmv.lora_sgmv_rank_supported(r, sgmv.VARIANT_FUSED_TC) == (r in (16, 32, 64))
+        assert sgmv.lora_sgmv_rank_supported(r, sgmv.VARIANT_GROUPED_TC) == (r in (16, 32, 64))
     for r in (0, 4, 24, 256):
         assert not sgmv.lora_sgmv_rank_supported(r, sgmv.VARIANT_SPLIT)
     assert sgmv.lora_sgmv_workspace_bytes(32, 16) == 2048

@@ -21,7 +21,7 @@ SMALL_CONFIGS = ["tiny", "distinct", "uniform_h4096", "uniform_h11008", "skewed_
 
 @pytest.mark.parametrize("name", SMALL_CONFIGS)
 @pytest.mark.parametrize("y_random", [False, True])
-@pytest.mark.parametrize("variant", [sgmv.VARIANT_AUTO, sgmv.VARIANT_SPLIT])
+@pytest.mark.parametrize("variant", [sgmv.VARIANT_AUTO, sgmv.VARIANT_SPLIT, sgmv.VARIANT_FUSED])
 def test_config_full_oracle(name, y_random, variant):
     w = inputs.make(name)
     p = DeviceProblem(w, y_random=y_random)
@@ -42,20 +42,23 @@ def test_config_bf16_variant(name):
 @pytest.mark.parametrize("r", [8, 16, 32, 64, 128])
 @pytest.mark.parametrize("dtype", ["f16", "bf16"])
 @pytest.mark.parametrize("T", [1, 37, 130])
-@pytest.mark.parametrize("variant", [sgmv.VARIANT_SPLIT, sgmv.VARIANT_FUSED])
+@pytest.mark.parametrize("variant", [sgmv.VARIANT_SPLIT, sgmv.VARIANT_FUSED, sgmv.VARIANT_FUSED_TC])
 def test_ragged_random_shapes(r, dtype, T, variant):
     # H1, H2 not multiples of the tile sizes; segments of every length (several token chunks)
+    if not sgmv.lora_sgmv_rank_supported(r, variant):
+        pytest.skip("rank not built for this variant")
     w = inputs.small_random(T, 7, 264, 136, r, dtype, seed=T * 1000 + r)
     p = DeviceProblem(w, y_random=True)
     assert_close(p.apply(variant=variant), p.oracle_apply(), dtype, w.name)
 
 
 @pytest.mark.parametrize("r", [16, 64])
-def test_fused_long_rows_many_tiles(r):
+@pytest.mark.parametrize("variant", [sgmv.VARIANT_FUSED, sgmv.VARIANT_FUSED_TC])
+def test_fused_long_rows_many_tiles(r, variant):
     # H1 and H2 span many stages per CTA (several A and B tiles) with ragged ends
     w = inputs.small_random(40, 5, 8200, 11000, r, "bf16", seed=r)
     p = DeviceProblem(w, y_random=True)
-    assert_close(p.apply(variant=sgmv.VARIANT_FUSED), p.oracle_apply(), "bf16", "long rows")
+    assert_close(p.apply(variant=variant), p.oracle_apply(), "bf16", "long rows")
 
 
 def test_batched_projections_with_different_shapes():
@@ -171,7 +174,7 @@ def test_empty_repeated_unsorted_segments_and_uncovered_rows():
     assert int(p.status.item()) == 0
 
 
-@pytest.mark.parametrize("variant", [sgmv.VARIANT_SPLIT, sgmv.VARIANT_FUSED])
+@pytest.mark.parametrize("variant", [sgmv.VARIANT_SPLIT, sgmv.VARIANT_FUSED, sgmv.VARIANT_FUSED_TC])
 def test_bad_segments_are_skipped_and_reported(variant):
     # [4,2) reversed; adapter 9 out of range; adapter 2 has a null table entry; [20,30) past T
     seg = np.array([0, 4, 2, 8, 12, 16, 20, 30], np.int32)
