@@ -348,35 +348,47 @@ lora_sgmv_status launch_fused(sgmv::FusedParams P, int max_len, cudaStream_t str
 
 // ---- tensor-core decode path -------------------------------------------------------------------
 
-bool decode_tc_supported(int r, int H1, int H2) { return (r == 16 || r == 32 || r == 64) && H1 >= 64 && H2 >= 64; }
+// Dispatch between the two fused decode kernels, from measurements on B200: the tensor-core
+// kernel wins once segments hold several tokens and r is large enough that its expand
+// (r x 16-token MMAs) replaces a long fp32 FMA loop; at r = 16 the CUDA-core kernel stays ahead.
+bool decode_tc_preferred(int r, int max_len) { return max_len > 2 && r >= 32; }
+
+bool decode_tc_supported(int r, int H1, int H2) {
+    return (r == 16 || r == 32 || r == 64) && H1 >= 64 && H2 >= 64 && H1 % 64 == 0 && H2 % 64 == 0;
+}
 
 template <typename T, int R>
-lora_sgmv_status launch_decode_tc(sgmv::FusedParams P, const sgmv::XMaps& maps, int max_len, cudaStream_t stream) {
+lora_sgmv_status launch_decode_tc(sgmv::FusedParams P, const sgmv::DecodeMaps& maps, int max_len, cudaStream_t stream) {
     static int smem_granted[64] = {};
-    static int resident[64][4][9] = {};
+    // resident clusters per (device, cluster size, job-prefix size bucket)
+    static int resident[64][sgmv::kFusedMaxCluster + 1][9] = {};
     using G = sgmv::DecodeTCGeom<R>;
     constexpr int CH = sgmv::kDTokens;
     if (P.n_segments > sgmv::kFusedMaxSegments) return LORA_SGMV_ERR_DIM;
     const int bucket = (P.n_segments + 1 + 1023) / 1024;  // 1..9
-    const size_t smem = G::BASE + size_t(bucket) * 1024 * 4 + 1024 /* alignment slack */;
+    auto smem_for = [&](int C) {
+        return G::BASE + size_t(C) * G::TILE + size_t(bucket) * 1024 * 4 + 1024 /* alignment slack */;
+    };
     auto kernel = sgmv::sgmv_decode_tc_kernel<T, R>;
-    if (ensure_smem(kernel, smem, smem_granted) != LORA_SGMV_OK) return LORA_SGMV_ERR_CUDA;
+    if (ensure_smem(kernel, smem_for(sgmv::kFusedMaxCluster), smem_granted) != LORA_SGMV_OK) return LORA_SGMV_ERR_CUDA;
+    DeviceFacts f;
+    if (device_facts(f) != LORA_SGMV_OK) return LORA_SGMV_ERR_CUDA;
     int dev = 0;
     if (record(cudaGetDevice(&dev)) != cudaSuccess) return LORA_SGMV_ERR_CUDA;
     if (dev < 0 || dev >= 64) return LORA_SGMV_ERR_UNSUPPORTED;
-    auto resident_for = [&](int lc, int* out) -> lora_sgmv_status {
+    auto resident_for = [&](int C, int* out) -> lora_sgmv_status {
         {
             std::lock_guard<std::mutex> lock(g_mu);
-            if (resident[dev][lc][bucket - 1] > 0) {
-                *out = resident[dev][lc][bucket - 1];
+            if (resident[dev][C][bucket - 1] > 0) {
+                *out = resident[dev][C][bucket - 1];
                 return LORA_SGMV_OK;
             }
         }
         int n = 0;
-        lora_sgmv_status st = max_active_clusters(kernel, 1 << lc, smem, &n, sgmv::kDThreads);
+        lora_sgmv_status st = max_active_clusters(kernel, C, smem_for(C), &n, sgmv::kDThreads);
         if (st != LORA_SGMV_OK) return st;
         std::lock_guard<std::mutex> lock(g_mu);
-        resident[dev][lc][bucket - 1] = n;
+        resident[dev][C][bucket - 1] = n;
         *out = n;
         return LORA_SGMV_OK;
     };
@@ -385,19 +397,42 @@ lora_sgmv_status launch_decode_tc(sgmv::FusedParams P, const sgmv::XMaps& maps, 
         std::min<long long>(P.n_segments + (P.T + CH - 1) / CH, std::max(P.T, 1));
     const long long jobs = std::max<long long>(1, (one_chunk ? static_cast<long long>(P.n_segments) : chunks) *
                                                       P.n_problems);
-    int ctas = 0;
-    lora_sgmv_status st = resident_for(0, &ctas);
-    if (st != LORA_SGMV_OK) return st;
-    int lc = 3;
-    while (lc > 0 && jobs * (1ll << lc) > ctas) --lc;
-    int clusters_max = 0;
-    st = resident_for(lc, &clusters_max);
-    if (st != LORA_SGMV_OK) return st;
-    const int C = 1 << lc;
+    // cluster size: a cluster runs its jobs one after another, each CTA streaming 1/C of the
+    // job's adapter bytes; estimated time = rounds * (bytes per CTA / per-CTA bandwidth + a fixed
+    // cost per job for metadata, map setup, pipeline fill and the V exchange). Every CTA keeps at
+    // least one stage of A_i and of B_i.
+    constexpr double kCtaBytesPerUs = 40e3;  // ~40 GB/s that one CTA streams with TMA
+    constexpr double kJobFixedUs = 4.0;
+    int c_cap = sgmv::kFusedMaxCluster;
+    double job_bytes = 0;
+    for (int i = 0; i < P.n_problems; ++i) {
+        c_cap = std::min(c_cap, (P.prob[i].H1 + G::KS - 1) / G::KS);
+        c_cap = std::min(c_cap, (P.prob[i].H2 + G::NW - 1) / G::NW);
+        job_bytes += (double(P.prob[i].H1) + double(P.prob[i].H2)) * R * 2;
+    }
+    job_bytes /= P.n_problems;
+    c_cap = std::max(c_cap, 1);
+    int C = 1, clusters_max = 0;
+    double best = 1e300;
+    for (int c = 1; c <= c_cap; ++c) {
+        int cm = 0;
+        lora_sgmv_status st = resident_for(c, &cm);
+        if (st != LORA_SGMV_OK) {
+            if (c == 1) return st;
+            continue;  // this cluster size cannot be scheduled here
+        }
+        const long long rounds = (jobs + cm - 1) / cm;
+        const double cost = double(rounds) * (job_bytes / c / kCtaBytesPerUs + kJobFixedUs);
+        if (cost < best - 1e-9) {
+            best = cost;
+            C = c;
+            clusters_max = cm;
+        }
+    }
     P.one_chunk = one_chunk ? 1 : 0;
     for (int i = 0; i < P.n_problems; ++i) {
-        P.prob[i].ks = (P.prob[i].H1 + C * sgmv::kGK - 1) / (C * sgmv::kGK) * sgmv::kGK;
-        P.prob[i].ns = (P.prob[i].H2 + C * sgmv::kGN - 1) / (C * sgmv::kGN) * sgmv::kGN;
+        P.prob[i].ks = (P.prob[i].H1 + C * G::KS - 1) / (C * G::KS) * G::KS;
+        P.prob[i].ns = (P.prob[i].H2 + C * G::NW - 1) / (C * G::NW) * G::NW;
     }
     int clusters = static_cast<int>(std::min<long long>(jobs, clusters_max));
     const long long rounds = (jobs + clusters - 1) / clusters;
@@ -406,7 +441,7 @@ lora_sgmv_status launch_decode_tc(sgmv::FusedParams P, const sgmv::XMaps& maps, 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(clusters * C, 1, 1);
     cfg.blockDim = dim3(sgmv::kDThreads, 1, 1);
-    cfg.dynamicSmemBytes = smem;
+    cfg.dynamicSmemBytes = smem_for(C);
     cfg.stream = stream;
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -420,19 +455,24 @@ lora_sgmv_status launch_decode_tc(sgmv::FusedParams P, const sgmv::XMaps& maps, 
     return counted(cudaLaunchKernelEx(&cfg, kernel, maps, P));
 }
 
-lora_sgmv_status decode_tc_dispatch(sgmv::FusedParams& P, int r, lora_sgmv_dtype dt, int max_len, cudaStream_t s) {
-    sgmv::XMaps maps;
+template <int R>
+lora_sgmv_status decode_tc_maps_and_launch(sgmv::FusedParams& P, lora_sgmv_dtype dt, int max_len, cudaStream_t s) {
+    sgmv::DecodeMaps maps;
     std::memset(&maps, 0, sizeof(maps));
     for (int i = 0; i < P.n_problems; ++i)
-        if (!sgmv::make_tile_map(&maps.m[i], P.prob[i].X, P.T, P.prob[i].H1, dt, sgmv::kDTokens)) {
+        if (!sgmv::make_decode_maps<R>(maps, i, P.prob[i].X, P.prob[i].Y, P.T, P.prob[i].H1, P.prob[i].H2, dt)) {
             t_last_error = cudaErrorInvalidValue;
             return LORA_SGMV_ERR_CUDA;
         }
-    const bool bf = dt == LORA_SGMV_BF16;
+    return dt == LORA_SGMV_BF16 ? launch_decode_tc<__nv_bfloat16, R>(P, maps, max_len, s)
+                                : launch_decode_tc<__half, R>(P, maps, max_len, s);
+}
+
+lora_sgmv_status decode_tc_dispatch(sgmv::FusedParams& P, int r, lora_sgmv_dtype dt, int max_len, cudaStream_t s) {
     switch (r) {
-        case 16: return bf ? launch_decode_tc<__nv_bfloat16, 16>(P, maps, max_len, s) : launch_decode_tc<__half, 16>(P, maps, max_len, s);
-        case 32: return bf ? launch_decode_tc<__nv_bfloat16, 32>(P, maps, max_len, s) : launch_decode_tc<__half, 32>(P, maps, max_len, s);
-        case 64: return bf ? launch_decode_tc<__nv_bfloat16, 64>(P, maps, max_len, s) : launch_decode_tc<__half, 64>(P, maps, max_len, s);
+        case 16: return decode_tc_maps_and_launch<16>(P, dt, max_len, s);
+        case 32: return decode_tc_maps_and_launch<32>(P, dt, max_len, s);
+        case 64: return decode_tc_maps_and_launch<64>(P, dt, max_len, s);
     }
     return LORA_SGMV_ERR_UNSUPPORTED;
 }
@@ -619,8 +659,9 @@ lora_sgmv_status lora_sgmv_apply_ex(void* Y, const void* X, const void* const* A
                 ? LORA_SGMV_VARIANT_GROUPED_TC
                 : (n_segments > sgmv::kFusedMaxSegments
                        ? LORA_SGMV_VARIANT_SPLIT
-                       : (max_len > 2 && decode_tc_supported(r, H1, H2) ? LORA_SGMV_VARIANT_FUSED_TC
-                                                                        : LORA_SGMV_VARIANT_FUSED));
+                       : (decode_tc_preferred(r, max_len) && decode_tc_supported(r, H1, H2)
+                              ? LORA_SGMV_VARIANT_FUSED_TC
+                              : LORA_SGMV_VARIANT_FUSED));
 
     if (v == LORA_SGMV_VARIANT_FUSED || v == LORA_SGMV_VARIANT_FUSED_TC) {
         if (v == LORA_SGMV_VARIANT_FUSED_TC && !decode_tc_supported(r, H1, H2)) return LORA_SGMV_ERR_UNSUPPORTED;
@@ -731,7 +772,7 @@ extern "C" lora_sgmv_status lora_sgmv_apply_batched(const lora_sgmv_problem* pro
     P.n_segments = n_segments;
     P.T = T;
     const int max_len = estimate_max_len(max_seg_len, T, n_segments);
-    bool tc = max_len > 2;
+    bool tc = decode_tc_preferred(r, max_len);
     for (int i = 0; i < n_problems; ++i) tc = tc && decode_tc_supported(r, problems[i].H1, problems[i].H2);
     if (tc) return decode_tc_dispatch(P, r, dtype, max_len, static_cast<cudaStream_t>(stream));
     return fused_dispatch(P, r, dtype, max_len, static_cast<cudaStream_t>(stream));

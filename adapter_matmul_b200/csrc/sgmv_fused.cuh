@@ -139,6 +139,13 @@ __device__ __forceinline__ void mbar_arrive_local(uint64_t* bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
+// Arrival without release semantics, for "this buffer has been read" signals: the reads it
+// stands for have returned their values before it issues, and a release here would also wait
+// for every global store still in flight from this thread (a round trip to L2 per stage).
+__device__ __forceinline__ void mbar_arrive_relaxed(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.relaxed.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
 // Arrive on the mbarrier at the same offset in CTA `rank` of this cluster (release, cluster scope).
 __device__ __forceinline__ void mbar_arrive_remote(uint64_t* bar, uint32_t rank) {
     const uint32_t remote = map_rank(smem_u32(bar), rank);
@@ -177,14 +184,22 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 
 // Bounded wait: gives up after kWaitLimitNs (or kSpinLimit polls), records
 // LORA_SGMV_DEV_TIMEOUT and marks the thread dead; a dead thread's later
-// waits return at once, so a broken protocol ends the kernel quickly.
+// waits return at once, so a broken protocol ends the kernel quickly. The
+// global timer is slow to read, so it is read only after 64 unsuccessful
+// polls, and then every 64 polls.
 template <bool kCluster>
 __device__ __forceinline__ void mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* status, bool& dead) {
     if (dead) return;
-    const uint64_t t0 = globaltimer_ns();
+    uint64_t t0 = 0;
     for (uint32_t i = 0; i < kSpinLimit; ++i) {
         if (kCluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity)) return;
-        if ((i & 63u) == 63u && globaltimer_ns() - t0 > kWaitLimitNs) break;
+        if ((i & 63u) == 63u) {
+            const uint64_t now = globaltimer_ns();
+            if (t0 == 0)
+                t0 = now;
+            else if (now - t0 > kWaitLimitNs)
+                break;
+        }
     }
     dead = true;
     report(status, LORA_SGMV_DEV_TIMEOUT);
@@ -400,7 +415,7 @@ __device__ __forceinline__ void consume_job(const FusedParams& P, const Job& job
             }
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive_local(&S.empty[stage]);
+        if (lane == 0) mbar_arrive_relaxed(&S.empty[stage]);
     }
 #pragma unroll
     for (int off = G::CG; off < 32; off <<= 1)
@@ -498,7 +513,7 @@ __device__ __forceinline__ void consume_job(const FusedParams& P, const Job& job
             }
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive_local(&S.empty[stage]);
+        if (lane == 0) mbar_arrive_relaxed(&S.empty[stage]);
     }
 }
 

@@ -37,6 +37,7 @@
 
 #include "sgmv_common.cuh"
 #include "sgmv_fused.cuh"  // PTX wrappers shared with the fused kernel (mbarriers, timers)
+#include "sgmv_tmap.cuh"
 
 namespace sgmv {
 
@@ -99,6 +100,14 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
         "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
         "[%4];" ::"r"(smem_u32(dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int c0, int c1, int c2, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+        "[%5];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
         : "memory");
 }
 
@@ -450,11 +459,12 @@ __global__ void __launch_bounds__(kGThreads, 1)
                     }
                 }
             }
-            tc_fence_before();
+            // the TMEM reads completed at tcgen05.wait::ld; no tcgen05 fence here (it would also
+            // wait for the Y stores just issued)
             __syncwarp();
             if (lane == 0) {
-                mbar_arrive_local(&d2_empty[buf]);
-                mbar_arrive_local(&e_empty[st]);
+                mbar_arrive_relaxed(&d2_empty[buf]);
+                mbar_arrive_relaxed(&e_empty[st]);
             }
         }
     }

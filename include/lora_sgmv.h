@@ -105,7 +105,9 @@ typedef enum {
 
 /* Ranks r built into this library: 8, 16, 32, 64 and 128 for the split and
  * fused kernels; 16, 32 and 64 for the tensor-core kernels (GROUPED_TC,
- * FUSED_TC), which also need H1 and H2 of at least 64. */
+ * FUSED_TC). GROUPED_TC also needs H1 and H2 of at least 64; FUSED_TC needs
+ * H1 and H2 to be multiples of 64 (at least 64), and returns
+ * LORA_SGMV_ERR_UNSUPPORTED otherwise. */
 int32_t lora_sgmv_rank_supported(int32_t r, lora_sgmv_variant variant);
 
 /* Human-readable name of a status code. Never NULL. */
@@ -244,8 +246,8 @@ typedef struct {
  * with i = lora_idx[s] and A_i, B_i taken from problem p's tables. Each
  * problem may have its own H1, H2, tables and adapter count; r and dtype are
  * shared. Runs a fused kernel, which keeps V on chip and needs no
- * workspace: LORA_SGMV_VARIANT_FUSED_TC when max_seg_len > 2 and every
- * problem suits the tensor-core kernel, else LORA_SGMV_VARIANT_FUSED. It
+ * workspace: LORA_SGMV_VARIANT_FUSED_TC when max_seg_len > 2, r >= 32 and
+ * every problem suits the tensor-core kernel, else LORA_SGMV_VARIANT_FUSED. It
  * takes at most 8192 segments (LORA_SGMV_ERR_DIM beyond).
  *   problems     host array of n_problems entries, 1 <= n_problems <= 8.
  *   other arguments as for lora_sgmv_apply.

@@ -114,6 +114,8 @@ def apply(**kw):
     (dict(idx=None), 1), (dict(na=0), 2),
     (dict(Y=MIS), 3), (dict(X=MIS), 3), (dict(H1=260), 3), (dict(H2=100), 3),
     (dict(ws=None), 7), (dict(wsb=100), 7), (dict(ws=MIS), 3),
+    # the tensor-core decode kernel takes H1 and H2 in multiples of 64 only
+    (dict(var=4, H1=264), 5), (dict(var=4, H2=136), 5), (dict(var=4, r=8), 5),
 ])
 def test_apply_validation_codes(kw, code):
     assert apply(**kw) == code

@@ -47,7 +47,9 @@ def test_ragged_random_shapes(r, dtype, T, variant):
     # H1, H2 not multiples of the tile sizes; segments of every length (several token chunks)
     if not sgmv.lora_sgmv_rank_supported(r, variant):
         pytest.skip("rank not built for this variant")
-    w = inputs.small_random(T, 7, 264, 136, r, dtype, seed=T * 1000 + r)
+    # the tensor-core decode kernel takes multiples of 64, still ragged against its stage sizes
+    H1, H2 = (320, 192) if variant == sgmv.VARIANT_FUSED_TC else (264, 136)
+    w = inputs.small_random(T, 7, H1, H2, r, dtype, seed=T * 1000 + r)
     p = DeviceProblem(w, y_random=True)
     assert_close(p.apply(variant=variant), p.oracle_apply(), dtype, w.name)
 
@@ -56,7 +58,8 @@ def test_ragged_random_shapes(r, dtype, T, variant):
 @pytest.mark.parametrize("variant", [sgmv.VARIANT_FUSED, sgmv.VARIANT_FUSED_TC])
 def test_fused_long_rows_many_tiles(r, variant):
     # H1 and H2 span many stages per CTA (several A and B tiles) with ragged ends
-    w = inputs.small_random(40, 5, 8200, 11000, r, "bf16", seed=r)
+    H1, H2 = (8256, 11008) if variant == sgmv.VARIANT_FUSED_TC else (8200, 11000)
+    w = inputs.small_random(40, 5, H1, H2, r, "bf16", seed=r)
     p = DeviceProblem(w, y_random=True)
     assert_close(p.apply(variant=variant), p.oracle_apply(), "bf16", "long rows")
 
@@ -79,6 +82,30 @@ def test_batched_projections_with_different_shapes():
     torch.cuda.synchronize()
     for p, ref in zip(probs, refs):
         assert_close(from_dev(p.Y), ref, "f16", p.w.name)
+    assert int(p0.status.item()) == 0
+
+
+@pytest.mark.parametrize("r,dtype", [(64, "bf16"), (32, "f16")])
+def test_batched_projections_tensor_core_decode(r, dtype):
+    # four problems with different shapes through the tensor-core decode kernel (segments of
+    # several tokens, r >= 32): one launch, per-problem tensor maps and device-built adapter maps
+    ids = inputs.llama70b_decode(8192).ids[:96]
+    shapes = [(1024, 1024), (1024, 256), (512, 2048), (2048, 640)]
+    probs, refs = [], []
+    for k, (H1, H2) in enumerate(shapes):
+        w = inputs.Workload(f"tcproj{k}", H1, H2, r, dtype, ids, 1024, 1.0 - 0.25 * k, seed=10 + k)
+        p = DeviceProblem(w, y_random=True)
+        probs.append(p)
+        refs.append(p.oracle_apply())
+    p0 = probs[0]
+    assert p0.max_len() > 2
+    sgmv.lora_sgmv_apply_batched(
+        [dict(Y=p.Y, X=p.X, A_ptrs=p.A_ptrs, B_ptrs=p.B_ptrs, num_adapters=p.w.num_adapters, H1=p.w.H1,
+              H2=p.w.H2, scale=p.w.scale) for p in probs],
+        p0.d_seg, p0.d_idx, p0.n, p0.w.T, r, dt_code(dtype), p0.max_len(), p0.status)
+    torch.cuda.synchronize()
+    for p, ref in zip(probs, refs):
+        assert_close(from_dev(p.Y), ref, dtype, p.w.name)
     assert int(p0.status.item()) == 0
 
 
@@ -179,7 +206,7 @@ def test_bad_segments_are_skipped_and_reported(variant):
     # [4,2) reversed; adapter 9 out of range; adapter 2 has a null table entry; [20,30) past T
     seg = np.array([0, 4, 2, 8, 12, 16, 20, 30], np.int32)
     idx = np.array([0, 1, 9, 3, 2, 4, 1], np.int32)
-    p = _custom(seg, idx)
+    p = _custom(seg, idx, H2=256 if variant == sgmv.VARIANT_FUSED_TC else 264)
     p.A_ptrs[2] = 0
     before = from_dev(p.Y)
     got = p.apply(variant=variant)
