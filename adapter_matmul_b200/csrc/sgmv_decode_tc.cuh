@@ -17,9 +17,10 @@
 //            CTA of the cluster with st.async and summed in rank order; V (fp32) is written
 //            as the two 16-bit operands V_hi + V_lo (about 16 significant bits of V);
 //   expand   transposed, so that the MMA's N is the token count: for each 128-column group
-//            of a stage, D2^T[128 cols x 16 tokens] = B_tile^T[128 x r] @ V^T[r x 16],
-//            M=128 N=16, the B tile as an MN-major operand; double-buffered in TMEM; the
-//            epilogue adds scale * D2 to the staged Y rows, rounds once and stores them.
+//            of a stage, D2^T[128 cols x 32] = B_tile^T[128 x r] @ [V_hi^T | V_lo^T][r x 32],
+//            M=128 N=32, the B tile as an MN-major operand, V_hi and V_lo side by side so one
+//            MMA covers both; up to four D2 buffers in TMEM; the epilogue adds the two halves,
+//            adds scale * D2 to the staged Y rows, rounds once and stores them.
 //
 // Copies. A TMA copy has a fixed cost per instruction that dominates until the copy is
 // several KB long, so every stage is one or two instructions:
@@ -45,10 +46,9 @@
 namespace sgmv {
 
 constexpr int kDTokens = 16;    // tokens per job = N of the expand MMA
-constexpr int kDStages = 6;     // main ring: X + A_i (shrink) or B_i (expand) stages, freed by the MMA
 constexpr int kDYStages = 4;    // Y ring, freed by the epilogue
 constexpr int kDThreads = 224;
-constexpr int kDTmemCols = 256;  // D1 at [0, r), D2 buffers from column 64
+constexpr int kDTmemCols = 512;  // D1 at [0, r), D2 buffers from column 64 (one CTA per SM)
 constexpr int kDYMaps = 5;       // Y boxes of 1, 2, 4, 8 and 16 rows
 constexpr int kDEpiBatch = 2;    // expand stages per epilogue pass
 
@@ -68,23 +68,29 @@ struct DecodeTCGeom {
     static constexpr int A_BYTES = KS * R * 2;            // 16, 8, 8 KB (r = 64, 32, 16)
     static constexpr int XB = KS / 64;                    // X column blocks per shrink stage
     static constexpr int X_BYTES = XB * kDTokens * 128;   // 16 rows per block
-    static constexpr int NB = 16384 / (R * 128);          // 64-column blocks of B_i per expand stage
-    static constexpr int NW = NB * 64;                    // columns per expand stage: 128, 256, 512
-    static constexpr int B_BYTES = R * NW * 2;            // 16 KB
+    // 64-column blocks of B_i per expand stage: a stage carries 32 KB of B_i at r = 64, 16 KB
+    // otherwise (the per-stage costs of the MMA and the epilogue are paid per stage)
+    static constexpr int NB = (R == 64 ? 32768 : 16384) / (R * 128);
+    static constexpr int NW = NB * 64;                    // columns per expand stage: 256, 256, 512
+    static constexpr int B_BYTES = R * NW * 2;            // 32, 16, 16 KB
+    static constexpr int STAGES = R == 64 ? 4 : 6;        // main ring depth
     static constexpr int YW = NW < 256 ? NW : 256;        // Y box width
     static constexpr int YBOXES = NW / YW;
     static constexpr int Y_BYTES = round1024(kDTokens * NW * 2);  // one Y stage: [YBOXES][16 rows][YW]
     static constexpr int STAGE = round1024(cmax(X_BYTES + A_BYTES, B_BYTES));
-    static constexpr int VT_BYTES = round1024(kDTokens * R * 2);  // one of V_hi^T, V_lo^T
+    static constexpr int VT_BYTES = round1024(2 * kDTokens * R * 2);  // V^T: 16 rows of V_hi, then 16 of V_lo
     static constexpr int TILE = kDTokens * R * 4;                 // one partial V tile (fp32)
     static constexpr size_t BASE =
-        size_t(kDStages) * STAGE + size_t(kDYStages) * Y_BYTES + 2 * size_t(VT_BYTES);  // + C tiles + prefix
+        size_t(STAGES) * STAGE + size_t(kDYStages) * Y_BYTES + size_t(VT_BYTES);  // + C tiles + prefix
     static constexpr int SW_BITS = R == 64 ? 3 : (R == 32 ? 2 : 1);
     static constexpr uint64_t SW_TYPE = R == 64 ? 2 : (R == 32 ? 4 : 6);
     static constexpr int ROW_BYTES = R * 2;
-    static constexpr int D2_COLS = NB * 8;  // (NB / 2) groups x 16 tokens
+    static constexpr int D2_COLS = NB * 16;  // (NB / 2) groups x (16 tokens x hi, lo)
     static constexpr int ND2 = (kDTmemCols - 64) / D2_COLS < 4 ? (kDTmemCols - 64) / D2_COLS : 4;  // D2 buffers
     static_assert(ND2 >= 2, "TMEM holds fewer than two D2 buffers");
+    // all 512 TMEM columns are allocated, so two CTAs must never share an SM: the shared
+    // memory of one CTA rules out a second (an SM has 228 KB)
+    static_assert(2 * BASE > 228 * 1024, "two CTAs could share an SM and wait on each other's TMEM");
     // the shrink MMA reads 128 rows (16 KB) from each X block (rows past the 16 loaded ones are
     // never used); from the last stage that span runs into the Y ring, still inside the allocation
     static_assert((XB - 1) * 2048 + 16384 <= STAGE + kDYStages * Y_BYTES, "X operand span leaves the allocation");
@@ -161,7 +167,7 @@ template <typename T, int R>
 __global__ void __launch_bounds__(kDThreads, 1)
     sgmv_decode_tc_kernel(const __grid_constant__ DecodeMaps maps, const FusedParams P) {
     using G = DecodeTCGeom<R>;
-    constexpr int S = kDStages;
+    constexpr int S = G::STAGES;
     constexpr int SY = kDYStages;
     constexpr int ND2 = G::ND2;
     extern __shared__ __align__(1024) unsigned char dsm_raw[];
@@ -170,9 +176,8 @@ __global__ void __launch_bounds__(kDThreads, 1)
     const int c = static_cast<int>(cluster_rank());
     unsigned char* ring = dsm;
     unsigned char* yring = ring + S * G::STAGE;
-    unsigned char* vhi = yring + SY * G::Y_BYTES;
-    unsigned char* vlo = vhi + G::VT_BYTES;
-    float* recv = reinterpret_cast<float*>(vlo + G::VT_BYTES);  // C partial V tiles
+    unsigned char* vt = yring + SY * G::Y_BYTES;                  // V^T operand: [V_hi rows | V_lo rows]
+    float* recv = reinterpret_cast<float*>(vt + G::VT_BYTES);  // C partial V tiles
     int* pref = reinterpret_cast<int*>(reinterpret_cast<unsigned char*>(recv) + size_t(C) * G::TILE);
 
     __shared__ __align__(8) uint64_t full[S], empty[S], yfull[SY], yempty[SY];
@@ -373,7 +378,8 @@ __global__ void __launch_bounds__(kDThreads, 1)
         // ---------------------------------- MMA issuer ----------------------------------
         const uint32_t fmt = std::is_same<T, __nv_bfloat16>::value ? 1u : 0u;
         const uint32_t idesc_s = instr_desc(fmt, 0, 1, R, kGM);         // X K-major, A_i MN-major, N = r
-        const uint32_t idesc_e = instr_desc(fmt, 1, 0, kDTokens, kGM);  // B tile MN-major, V^T K-major, N = 16
+        // B tile MN-major, V^T K-major with N = 32: columns 0..15 of D2 take V_hi, 16..31 V_lo
+        const uint32_t idesc_e = instr_desc(fmt, 1, 0, 2 * kDTokens, kGM);
         uint32_t it = 0, u = 0, g = 0;
         for (int j = cluster_id; j < entries; j += n_clusters) {
             int p, s, q0, nq;
@@ -423,12 +429,9 @@ __global__ void __launch_bounds__(kDThreads, 1)
 #pragma unroll
                             for (int kk = 0; kk < R / 16; ++kk) {
                                 const uint64_t adesc = smem_desc(ba + 2 * gi * R * 128 + kk * 16 * 128, R * 128, 1024, 2);
-                                const uint64_t bhi =
-                                    smem_desc(smem_u32(vhi) + kk * 32, 16, 8 * G::ROW_BYTES, G::SW_TYPE);
-                                const uint64_t blo =
-                                    smem_desc(smem_u32(vlo) + kk * 32, 16, 8 * G::ROW_BYTES, G::SW_TYPE);
-                                tc_mma(d2 + 16u * gi, adesc, bhi, idesc_e, kk ? 1u : 0u);
-                                tc_mma(d2 + 16u * gi, adesc, blo, idesc_e, 1u);
+                                const uint64_t bdesc =
+                                    smem_desc(smem_u32(vt) + kk * 32, 16, 8 * G::ROW_BYTES, G::SW_TYPE);
+                                tc_mma(d2 + 32u * gi, adesc, bdesc, idesc_e, kk ? 1u : 0u);
                             }
                         tc_commit(&d2_full[buf]);
                         tc_commit(&empty[st]);
@@ -495,8 +498,8 @@ __global__ void __launch_bounds__(kDThreads, 1)
                                 lo[i] = v[ch * 8 + i] - hi[i];
                             }
                             const uint32_t off = swz(lane, ch, G::SW_BITS);
-                            st_vec(vhi + off, pack8<T>(hi));
-                            st_vec(vlo + off, pack8<T>(lo));
+                            st_vec(vt + off, pack8<T>(hi));
+                            st_vec(vt + swz(kDTokens + lane, ch, G::SW_BITS), pack8<T>(lo));
                         }
                     }
                     fence_proxy_async();
@@ -523,8 +526,11 @@ __global__ void __launch_bounds__(kDThreads, 1)
                         const int n0 = job.c0 + (tb + e) * G::NW;
 #pragma unroll
                         for (int gi = 0; gi < G::NB / 2; ++gi) {
-                            float acc[16];
-                            tmem_ld16(d2 + 16u * gi, acc);
+                            float acc[16], acc_lo[16];
+                            tmem_ld16(d2 + 32u * gi, acc);
+                            tmem_ld16(d2 + 32u * gi + 16u, acc_lo);
+#pragma unroll
+                            for (int t = 0; t < kDTokens; ++t) acc[t] += acc_lo[t];
                             const int cw = gi * 128 + quarter * 32 + lane;  // column within the stage
                             const int col = n0 + cw;
                             if (col < n_hi) {
