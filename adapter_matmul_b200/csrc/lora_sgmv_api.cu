@@ -212,12 +212,44 @@ lora_sgmv_status launch_grouped(void* Y, const void* X, const void* const* A_ptr
     P.H1 = H1;
     P.H2 = H2;
     P.scale = scale;
+    // templates of the A_i and B_i maps; each CTA replaces the address with its adapter's
+    CUtensorMap tmA, tmB;
+    {
+        const uint64_t da[2] = {uint64_t(r), uint64_t(H1)};
+        const uint64_t sa[1] = {uint64_t(r) * 2};
+        const uint32_t ba[2] = {uint32_t(r), uint32_t(sgmv::kGK)};
+        const CUtensorMapSwizzle swa =
+            r == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : (r == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
+        const uint64_t db[2] = {uint64_t(H2), uint64_t(r)};
+        const uint64_t sb[1] = {uint64_t(H2) * 2};
+        const uint32_t bb[2] = {64, uint32_t(r)};
+        if (!sgmv::encode_map(&tmA, X, dt, 2, da, sa, ba, swa) ||
+            !sgmv::encode_map(&tmB, X, dt, 2, db, sb, bb, CU_TENSOR_MAP_SWIZZLE_128B)) {
+            t_last_error = cudaErrorInvalidValue;
+            return LORA_SGMV_ERR_CUDA;
+        }
+    }
     // M-tiles: at most ceil(T/128) + n (each segment adds at most one partial tile)
     const long long tiles_ub = (static_cast<long long>(T) + sgmv::kGM - 1) / sgmv::kGM + n_segments;
     const long long tiles_est = std::max<long long>(1, (static_cast<long long>(T) + sgmv::kGM - 1) / sgmv::kGM);
     const int max_split = (H2 + sgmv::kGN - 1) / sgmv::kGN;
-    int nsplit = static_cast<int>(std::max<long long>(1, (f.sms + tiles_est - 1) / tiles_est));
-    nsplit = std::min(nsplit, max_split);
+    // N-slices per M-tile: every CTA of a tile streams the tile's X rows and A_i again and its
+    // slice of Y and B_i, one CTA per SM at a time; pick the split with the least bytes on the
+    // busiest SM (the slices of a tile run on different SMs)
+    int nsplit = 1;
+    {
+        const double shrink = (double(sgmv::kGM) * H1 + double(H1) * r) * 2;
+        const double expand = (2.0 * sgmv::kGM * H2 + double(r) * H2) * 2;
+        const int sms = std::max(f.sms, 1);
+        double best = 1e300;
+        for (int ns = 1; ns <= std::min(max_split, 16); ++ns) {
+            const double per_sm = double((tiles_est * ns + sms - 1) / sms) * (shrink + expand / ns);
+            if (per_sm < best * (1 - 1e-9)) {
+                best = per_sm;
+                nsplit = ns;
+            }
+        }
+    }
     const int span_tiles = ((H2 + sgmv::kGN - 1) / sgmv::kGN + nsplit - 1) / nsplit;
     P.nspan = span_tiles * sgmv::kGN;
     P.nsplit = (H2 + P.nspan - 1) / P.nspan;
@@ -227,16 +259,16 @@ lora_sgmv_status launch_grouped(void* Y, const void* X, const void* const* A_ptr
     const bool bf = dt == LORA_SGMV_BF16;
     switch (r) {
         case 16:
-            e = bf ? sgmv::launch_grouped_tc_kernel<__nv_bfloat16, 16>(tmX, tmY, P, int(blocks), stream)
-                   : sgmv::launch_grouped_tc_kernel<__half, 16>(tmX, tmY, P, int(blocks), stream);
+            e = bf ? sgmv::launch_grouped_tc_kernel<__nv_bfloat16, 16>(tmX, tmY, tmA, tmB, P, int(blocks), stream)
+                   : sgmv::launch_grouped_tc_kernel<__half, 16>(tmX, tmY, tmA, tmB, P, int(blocks), stream);
             break;
         case 32:
-            e = bf ? sgmv::launch_grouped_tc_kernel<__nv_bfloat16, 32>(tmX, tmY, P, int(blocks), stream)
-                   : sgmv::launch_grouped_tc_kernel<__half, 32>(tmX, tmY, P, int(blocks), stream);
+            e = bf ? sgmv::launch_grouped_tc_kernel<__nv_bfloat16, 32>(tmX, tmY, tmA, tmB, P, int(blocks), stream)
+                   : sgmv::launch_grouped_tc_kernel<__half, 32>(tmX, tmY, tmA, tmB, P, int(blocks), stream);
             break;
         case 64:
-            e = bf ? sgmv::launch_grouped_tc_kernel<__nv_bfloat16, 64>(tmX, tmY, P, int(blocks), stream)
-                   : sgmv::launch_grouped_tc_kernel<__half, 64>(tmX, tmY, P, int(blocks), stream);
+            e = bf ? sgmv::launch_grouped_tc_kernel<__nv_bfloat16, 64>(tmX, tmY, tmA, tmB, P, int(blocks), stream)
+                   : sgmv::launch_grouped_tc_kernel<__half, 64>(tmX, tmY, tmA, tmB, P, int(blocks), stream);
             break;
         default: return LORA_SGMV_ERR_UNSUPPORTED;
     }

@@ -147,21 +147,6 @@ __device__ __forceinline__ void epilogue_bar() { asm volatile("bar.sync 1, 128;"
 // digits of nt), so Y rows of other segments are never read or written. Box m (rows 2^m) of
 // a chunk starts at row offset nt & ~(2^(m+1) - 1).
 
-// Wait for a barrier phase without regard to earlier timeouts (lets copies land before the
-// CTA exits); bounded like every other wait.
-__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
-    uint64_t t0 = 0;
-    for (uint32_t i = 0; i < kSpinLimit; ++i) {
-        if (mbar_try_wait(bar, parity)) return;
-        if ((i & 63u) == 63u) {
-            const uint64_t now = globaltimer_ns();
-            if (t0 == 0)
-                t0 = now;
-            else if (now - t0 > kWaitLimitNs)
-                return;
-        }
-    }
-}
 
 template <typename T, int R>
 __global__ void __launch_bounds__(kDThreads, 1)

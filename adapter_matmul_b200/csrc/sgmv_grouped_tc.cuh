@@ -18,12 +18,13 @@
 // Rows of a tile past the segment's end belong to the next segment (or past T, where
 // TMA fills zeros); their results are discarded, so tiles never write across segments.
 //
-// Data movement. X and Y tiles are TMA loads (cp.async.bulk.tensor, 128-byte swizzle)
-// through tensor maps built per call. Adapter tiles come from a device table of
-// pointers, so they are copied with cp.async (16 bytes per lane) straight into the
-// swizzled canonical layouts the MMA descriptors describe. Warp roles: warp 0
-// producer, warp 1 allocates TMEM and issues tcgen05.mma (one thread), warps 2..5
-// epilogue (one TMEM lane quarter each).
+// Data movement. Every tile is a TMA load (cp.async.bulk.tensor) into the swizzled
+// canonical layout the MMA descriptors describe: X and Y through tensor maps built per
+// call, A_i and B_i (reached through a device table of pointers) through maps each CTA
+// makes from a per-call template (sgmv_tmap.cuh). Warp roles: warp 0 producer, warp 1
+// allocates TMEM and issues tcgen05.mma (one thread), warps 2..5 epilogue (one TMEM lane
+// quarter each). The host picks the number of N-slices per M-tile from the bytes the
+// busiest SM streams (every slice re-reads its tile's X rows and A_i).
 //
 // Every mbarrier wait is bounded in time; a wait that gives up sets
 // LORA_SGMV_DEV_TIMEOUT and the kernel runs to its end (TMEM is always freed).
@@ -109,17 +110,6 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, i
         "[%5];" ::"r"(smem_u32(dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
         : "memory");
-}
-
-// 16-byte cp.async; src_bytes == 0 fills the 16 bytes with zeros (nothing is read).
-__device__ __forceinline__ void cp_async16(void* dst, const void* src, uint32_t src_bytes) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes)
-                 : "memory");
-}
-
-// The mbarrier counts one arrival when all of this thread's earlier cp.async copies are done.
-__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
-    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
 __device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
@@ -214,10 +204,28 @@ __device__ bool find_tile(const GroupedParams& P, int tile, int& seg_out, int& m
     return false;
 }
 
-// grid.x = tiles (upper bound) * nsplit; block kGThreads.
+// Wait for a barrier phase without regard to earlier timeouts (lets copies land before the
+// CTA exits); bounded like every other wait.
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
+    uint64_t t0 = 0;
+    for (uint32_t i = 0; i < kSpinLimit; ++i) {
+        if (mbar_try_wait(bar, parity)) return;
+        if ((i & 63u) == 63u) {
+            const uint64_t now = globaltimer_ns();
+            if (t0 == 0)
+                t0 = now;
+            else if (now - t0 > kWaitLimitNs)
+                return;
+        }
+    }
+}
+
+// grid.x = tiles (upper bound) * nsplit; block kGThreads. tmA and tmB are templates of the
+// A_i and B_i maps (shape, box, swizzle); each CTA makes its adapter's maps from them.
 template <typename T, int R>
 __global__ void __launch_bounds__(kGThreads, 1)
     sgmv_grouped_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmY,
+                           const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                            const GroupedParams P) {
     using G = GroupedGeom<R>;
     extern __shared__ __align__(1024) unsigned char gsmem_raw[];
@@ -231,8 +239,10 @@ __global__ void __launch_bounds__(kGThreads, 1)
     __shared__ __align__(8) uint64_t s_full[kGShrinkStages], s_empty[kGShrinkStages];
     __shared__ __align__(8) uint64_t e_full[kGExpandStages], e_empty[kGExpandStages];
     __shared__ __align__(8) uint64_t d1_full, v_full, d2_full[2], d2_empty[2];
+    __shared__ __align__(128) CUtensorMap map_build[2];
     __shared__ uint32_t tmem_base_s;
     __shared__ int job_s[3];
+    __shared__ int table_s;
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -259,11 +269,11 @@ __global__ void __launch_bounds__(kGThreads, 1)
     }
     if (threadIdx.x == 0) {
         for (int i = 0; i < kGShrinkStages; ++i) {
-            mbar_init(&s_full[i], 1 + 32);  // TMA expect_tx arrival + 32 cp.async arrivals
-            mbar_init(&s_empty[i], 1);      // MMA commit
+            mbar_init(&s_full[i], 1);   // producer expect_tx; the TMA copies complete the bytes
+            mbar_init(&s_empty[i], 1);  // MMA commit
         }
         for (int i = 0; i < kGExpandStages; ++i) {
-            mbar_init(&e_full[i], 1 + 32);
+            mbar_init(&e_full[i], 1);
             mbar_init(&e_empty[i], 1 + 4);  // MMA commit (B read) + 4 epilogue warps (Y read)
         }
         mbar_init(&d1_full, 1);
@@ -273,6 +283,14 @@ __global__ void __launch_bounds__(kGThreads, 1)
             mbar_init(&d2_empty[i], 4);
         }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        table_s = -1;
+        if (job_s[0] >= 0) {
+            table_s = claim_map_table();
+            if (table_s < 0) {
+                report(P.dev_status, LORA_SGMV_DEV_TIMEOUT);
+                job_s[0] = -1;
+            }
+        }
     }
     __syncthreads();
     const int seg_id = job_s[0];
@@ -303,26 +321,35 @@ __global__ void __launch_bounds__(kGThreads, 1)
 
     if (warp == 0) {
         // ---------------------------------- producer ----------------------------------
-        const T* A = static_cast<const T*>(seg.a);
-        const T* B = static_cast<const T*>(seg.b);
+        // this CTA's adapter maps, from the templates: A_i boxes of 64 rows x r, B_i boxes of
+        // r rows x 64 columns; columns of B_i past this CTA's slice are loaded but never stored
+        CUtensorMap* gA = &g_map_tables[table_s].m[0];
+        CUtensorMap* gB = &g_map_tables[table_s].m[1];
+        map_template_to_smem(&map_build[0], &tmA);
+        map_template_to_smem(&map_build[1], &tmB);
+        if (lane == 0) {
+            map_set_address(&map_build[0], seg.a);
+            map_set_address(&map_build[1], seg.b);
+        }
+        __syncwarp();
+        map_publish(gA, &map_build[0]);
+        map_publish(gB, &map_build[1]);
+        if (lane == 0) {
+            map_acquire(gA);
+            map_acquire(gB);
+        }
+        __syncwarp();
         for (int ks = 0; ks < k_steps; ++ks) {
             const int st = ks % kGShrinkStages;
             if (ks >= kGShrinkStages) mbar_wait<false>(&s_empty[st], ((ks / kGShrinkStages) - 1) & 1u, P.dev_status, dead);
             unsigned char* xs = sstage + st * G::SSTAGE;
             unsigned char* as = xs + G::X_BYTES;
             if (lane == 0) {
-                mbar_arrive_expect_tx(&s_full[st], G::X_BYTES);
+                mbar_arrive_expect_tx(&s_full[st], G::X_BYTES + G::A_BYTES);
                 tma_load_2d(xs, &tmX, ks * kGK, t0, &s_full[st]);
+                tma_load_2d(as, gA, 0, ks * kGK, &s_full[st]);
             }
-            // A_i rows [ks*64, ks*64+64), R values each, MN-major swizzled
-            constexpr int CHUNKS = kGK * R / 8;
-            for (int q = lane; q < CHUNKS; q += 32) {
-                const int k = q / (R / 8), c = q % (R / 8);
-                const int gk = ks * kGK + k;
-                const bool in = gk < P.H1;
-                cp_async16(as + swz(k, c, G::SW_BITS), A + size_t(in ? gk : 0) * R + c * 8, in ? 16u : 0u);
-            }
-            cp_async_arrive_noinc(&s_full[st]);
+            __syncwarp();
         }
         for (int nt = 0; nt < n_tiles; ++nt) {
             const int st = nt % kGExpandStages;
@@ -331,22 +358,22 @@ __global__ void __launch_bounds__(kGThreads, 1)
             unsigned char* bs = ys + G::Y_BYTES;
             const int n0 = n_lo + nt * kGN;
             if (lane == 0) {
-                mbar_arrive_expect_tx(&e_full[st], G::Y_BYTES);
+                mbar_arrive_expect_tx(&e_full[st], G::Y_BYTES + G::B_BYTES);
                 tma_load_2d(ys, &tmY, n0, t0, &e_full[st]);
                 tma_load_2d(ys + G::Y_BYTES / 2, &tmY, n0 + 64, t0, &e_full[st]);
+                tma_load_2d(bs, gB, n0, 0, &e_full[st]);
+                tma_load_2d(bs + R * 128, gB, n0 + 64, 0, &e_full[st]);
             }
-            // B_i rows 0..R-1, columns n0..n0+127 as two 64-column MN-major blocks (128B swizzle)
-            constexpr int CHUNKS = R * kGN / 8;
-            for (int q = lane; q < CHUNKS; q += 32) {
-                const int k = q / (kGN / 8), cc = q % (kGN / 8);
-                const int blk = cc / 8, c = cc % 8;
-                const int gn = n0 + cc * 8;
-                const bool in = gn < n_hi;
-                cp_async16(bs + blk * (R * 128) + swz(k, c, 3), B + size_t(k) * P.H2 + (in ? gn : 0), in ? 16u : 0u);
-            }
-            cp_async_arrive_noinc(&e_full[st]);
+            __syncwarp();
         }
-        asm volatile("cp.async.wait_all;" ::: "memory");
+        // every copy issued lands before the CTA may exit
+        if (lane == 0) {
+            for (int i = k_steps > kGShrinkStages ? k_steps - kGShrinkStages : 0; i < k_steps; ++i)
+                drain_wait(&s_full[i % kGShrinkStages], (uint32_t(i) / kGShrinkStages) & 1u);
+            for (int i = n_tiles > kGExpandStages ? n_tiles - kGExpandStages : 0; i < n_tiles; ++i)
+                drain_wait(&e_full[i % kGExpandStages], (uint32_t(i) / kGExpandStages) & 1u);
+        }
+        __syncwarp();
     } else if (warp == 1) {
         // ---------------------------------- MMA issuer ----------------------------------
         const uint32_t fmt = std::is_same<T, __nv_bfloat16>::value ? 1u : 0u;
@@ -355,7 +382,6 @@ __global__ void __launch_bounds__(kGThreads, 1)
         for (int ks = 0; ks < k_steps; ++ks) {
             const int st = ks % kGShrinkStages;
             mbar_wait<false>(&s_full[st], (ks / kGShrinkStages) & 1u, P.dev_status, dead);
-            fence_proxy_async();  // cp.async (generic proxy) writes -> tensor-core reads
             tc_fence_after();
             if (lane == 0) {
                 const uint32_t xa = smem_u32(sstage + st * G::SSTAGE);
@@ -380,7 +406,6 @@ __global__ void __launch_bounds__(kGThreads, 1)
             const int buf = nt & 1;
             if (nt >= 2) mbar_wait<false>(&d2_empty[buf], ((nt >> 1) - 1) & 1u, P.dev_status, dead);
             mbar_wait<false>(&e_full[st], (nt / kGExpandStages) & 1u, P.dev_status, dead);
-            fence_proxy_async();
             tc_fence_after();
             if (lane == 0) {
                 const uint32_t ba = smem_u32(estage + st * G::ESTAGE + G::Y_BYTES);
@@ -473,6 +498,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
     tc_fence_after();
     if (warp == 1)
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kGTmemCols) : "memory");
+    if (threadIdx.x == 0) release_map_table(table_s);
 }
 
 // ---- host side ---------------------------------------------------------------------------
@@ -511,8 +537,9 @@ inline bool make_tile_map(CUtensorMap* map, const void* base, int rows, int cols
 }
 
 template <typename T, int R>
-inline cudaError_t launch_grouped_tc_kernel(const CUtensorMap& tmX, const CUtensorMap& tmY, const GroupedParams& P,
-                                            int blocks, cudaStream_t stream) {
+inline cudaError_t launch_grouped_tc_kernel(const CUtensorMap& tmX, const CUtensorMap& tmY, const CUtensorMap& tmA,
+                                            const CUtensorMap& tmB, const GroupedParams& P, int blocks,
+                                            cudaStream_t stream) {
     using G = GroupedGeom<R>;
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
@@ -521,7 +548,7 @@ inline cudaError_t launch_grouped_tc_kernel(const CUtensorMap& tmX, const CUtens
                                         static_cast<int>(G::SMEM));
     });
     if (attr_err != cudaSuccess) return attr_err;
-    sgmv_grouped_tc_kernel<T, R><<<blocks, kGThreads, G::SMEM, stream>>>(tmX, tmY, P);
+    sgmv_grouped_tc_kernel<T, R><<<blocks, kGThreads, G::SMEM, stream>>>(tmX, tmY, tmA, tmB, P);
     return cudaGetLastError();
 }
 
