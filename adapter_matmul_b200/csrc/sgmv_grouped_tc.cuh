@@ -463,27 +463,42 @@ __global__ void __launch_bounds__(kGThreads, 1)
             mbar_wait<false>(&e_full[st], (nt / kGExpandStages) & 1u, P.dev_status, dead);
             mbar_wait<false>(&d2_full[buf], (nt >> 1) & 1u, P.dev_status, dead);
             tc_fence_after();
-            const unsigned char* ys = estage + st * G::ESTAGE;
+            unsigned char* ys = estage + st * G::ESTAGE;
             const int n0 = n_lo + nt * kGN;
+            // row m of the tile: y + scale * D2, written back over the staged Y row
 #pragma unroll 1
             for (int c0 = 0; c0 < kGN; c0 += 32) {
                 float acc[32];
                 tmem_ld32(lane_addr + 128u + 128u * buf + c0, acc);
                 if (row_ok) {
-                    const unsigned char* yb = ys + (c0 / 64) * (G::Y_BYTES / 2);
+                    unsigned char* yb = ys + (c0 / 64) * (G::Y_BYTES / 2);
 #pragma unroll
                     for (int ch = 0; ch < 4; ++ch) {
-                        const int col = n0 + c0 + ch * 8;
-                        if (col < n_hi) {
+                        if (n0 + c0 + ch * 8 < n_hi) {
+                            unsigned char* yp = yb + swz(m, (c0 % 64) / 8 + ch, 3);
                             float y[8];
-                            unpack8<T>(*reinterpret_cast<const uint4*>(yb + swz(m, (c0 % 64) / 8 + ch, 3)), y);
+                            unpack8<T>(*reinterpret_cast<const uint4*>(yp), y);
 #pragma unroll
                             for (int i = 0; i < 8; ++i) y[i] = __fadd_rn(y[i], __fmul_rn(P.scale, acc[ch * 8 + i]));
-                            st_vec(Y + size_t(t0 + m) * P.H2 + col, pack8<T>(y));
+                            st_vec(yp, pack8<T>(y));
                         }
                     }
                 }
             }
+            __syncwarp();
+            // this warp's 32 rows leave row by row: 8 lanes per 128-byte row segment, so each
+            // store instruction writes four whole segments
+#pragma unroll
+            for (int b = 0; b < 2; ++b)
+#pragma unroll
+                for (int rq = 0; rq < 32; rq += 4) {
+                    const int rr = quarter * 32 + rq + (lane >> 3);
+                    const int c = lane & 7;
+                    const int col = n0 + b * 64 + c * 8;
+                    if (rr < rows && col < n_hi)
+                        st_vec(Y + size_t(t0 + rr) * P.H2 + col,
+                               *reinterpret_cast<const uint4*>(ys + b * (G::Y_BYTES / 2) + swz(rr, c, 3)));
+                }
             // the TMEM reads completed at tcgen05.wait::ld; no tcgen05 fence here (it would also
             // wait for the Y stores just issued)
             __syncwarp();

@@ -12,11 +12,16 @@ own adapters, input and output. Steps rotate over 32 layers, each with its own
 weights and activations (1.1 GiB in all, far above the 126 MB L2), so every
 step reads cold data, as a model's layers would.
 
-The timed region replays one CUDA graph per layer (the graph holds that
-layer's four lora_sgmv_apply calls) so host launch latency does not stand in
-for kernel time. ``e2e`` repeats the measurement through the public call with
-host buffers: each step copies its inputs from pinned host memory, groups the
-token batch on the host, runs the four calls, and reads the outputs back.
+Each layer's four projections share one token grouping, so a step is one
+lora_sgmv_apply_batched launch. The timed region replays CUDA graphs: one
+graph holding a whole rotation of layers back to back (consecutive launches
+overlap through programmatic dependent launch, as a captured decode step
+would), plus single-layer graphs for a remainder, so host launch latency does
+not stand in for kernel time. ``e2e`` repeats the measurement through the
+public call with host buffers: each step copies its inputs from pinned host
+memory, groups the token batch on the host, runs the four lora_sgmv_apply
+calls, and reads the outputs back. Other workloads (--workload) run one
+lora_sgmv_apply per step, the dispatcher choosing the kernels.
 
 Multi-GPU (torchrun): every rank runs its own replica of the workload (the
 path has no cross-GPU data exchange); value = all ranks' tokens / max time.
@@ -43,6 +48,39 @@ from adapter_matmul_b200 import inputs  # noqa: E402
 METRIC = "LoRA-delta tokens/s (SGMV)"
 UNIT = "tokens/s"
 L2_BYTES = 126 * 1024 * 1024
+
+
+# DRAM bytes (read + write) of one launch of the dominant kernel, from one ncu capture of the
+# same launch (summaries under profiles/). A figure holds only while the kernel's sources are
+# those it was taken from: their SHA-256 is stored with it and checked here, else "traffic"
+# is null.
+TRAFFIC = {
+    "distinct": {"bytes": 35724800, "profile": "profiles/fused_kernel_distinct_decode.md",
+                 "sources": ["sgmv_common.cuh", "sgmv_fused.cuh"], "sha256": "abde291ab9d6714445fec73dd5573bbe6715a423558b54f83708bca522bf7776"},
+    "llama70b_decode_h28672": {"bytes": 467304448 + 14324736, "profile": "profiles/decode_tc_kernel_llama70b_decode.md",
+                               "sources": ["sgmv_common.cuh", "sgmv_fused.cuh", "sgmv_tmap.cuh", "sgmv_grouped_tc.cuh",
+                                           "sgmv_decode_tc.cuh"], "sha256": "8b17c61cdcf52e4636b5b57846372e39b9c482b897320799056c8cf9fff05f82"},
+    "prefill": {"bytes": 168567296 + 21483520, "profile": "profiles/grouped_kernel_prefill.md",
+                "sources": ["sgmv_common.cuh", "sgmv_fused.cuh", "sgmv_tmap.cuh", "sgmv_grouped_tc.cuh"],
+                "sha256": "b3e02057f98552391de61d78cf0a228ef962176795d90aa824537c0d3605518e"},
+}
+
+
+def kernel_sources_sha(files) -> str:
+    import hashlib
+
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "adapter_matmul_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def measured_traffic(name: str):
+    e = TRAFFIC.get(name)
+    if e is None or kernel_sources_sha(e["sources"]) != e["sha256"]:
+        return None
+    return e["bytes"]
 
 
 def peaks():
@@ -345,7 +383,7 @@ def run_ours(args, spec: Spec, rank: int, world: int, local: int):
     kernel_name = ("sgmv_fused_kernel (lora_sgmv_apply_batched: %d projections per launch)" % spec.P
                    if spec.P > 1 else "lora_sgmv_apply kernels (dispatcher's choice)")
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
-                "frac": round(achieved / hbm, 4), "traffic": None, "kernel": kernel_name,
+                "frac": round(achieved / hbm, 4), "traffic": measured_traffic(spec.name), "kernel": kernel_name,
                 "peak_source": "measured (MEASURED_PEAKS.json hbm_gbs)" if which == "measured" else which,
                 "algorithmic_bytes_per_launch": bytes_launch,
                 "launch_us": round(launch_s * 1e6, 3),
