@@ -194,8 +194,15 @@ lora_sgmv_status launch_grouped(void* Y, const void* X, const void* const* A_ptr
                                 cudaStream_t stream) {
     DeviceFacts f;
     if (device_facts(f) != LORA_SGMV_OK) return LORA_SGMV_ERR_CUDA;
+    // Rows per M-tile: the fewest that keep every tile in one wave (at most ceil(T/tm) + n tiles
+    // for the SMs), not under 64; with more rows than 128 SMs can take, full 128-row tiles.
+    // A CTA streams its tile's X and Y rows plus A_i and B_i, so smaller tiles spread the rows
+    // over more SMs at the cost of more (L2-resident) adapter reads.
+    const int sms_avail = std::max(1, f.sms - n_segments);
+    int tm = static_cast<int>(std::min<long long>(sgmv::kGM, ((static_cast<long long>(T) + sms_avail - 1) / sms_avail + 7) / 8 * 8));
+    tm = std::max(tm, 64);
     CUtensorMap tmX, tmY;
-    if (!sgmv::make_tile_map(&tmX, X, T, H1, dt) || !sgmv::make_tile_map(&tmY, Y, T, H2, dt)) {
+    if (!sgmv::make_tile_map(&tmX, X, T, H1, dt, tm) || !sgmv::make_tile_map(&tmY, Y, T, H2, dt, tm)) {
         t_last_error = cudaErrorInvalidValue;
         return LORA_SGMV_ERR_CUDA;
     }
@@ -230,16 +237,17 @@ lora_sgmv_status launch_grouped(void* Y, const void* X, const void* const* A_ptr
         }
     }
     // M-tiles: at most ceil(T/128) + n (each segment adds at most one partial tile)
-    const long long tiles_ub = (static_cast<long long>(T) + sgmv::kGM - 1) / sgmv::kGM + n_segments;
-    const long long tiles_est = std::max<long long>(1, (static_cast<long long>(T) + sgmv::kGM - 1) / sgmv::kGM);
+    P.tm = tm;
+    const long long tiles_ub = (static_cast<long long>(T) + tm - 1) / tm + n_segments;
+    const long long tiles_est = std::max<long long>(1, (static_cast<long long>(T) + tm - 1) / tm);
     const int max_split = (H2 + sgmv::kGN - 1) / sgmv::kGN;
     // N-slices per M-tile: every CTA of a tile streams the tile's X rows and A_i again and its
     // slice of Y and B_i, one CTA per SM at a time; pick the split with the least bytes on the
     // busiest SM (the slices of a tile run on different SMs)
     int nsplit = 1;
     {
-        const double shrink = (double(sgmv::kGM) * H1 + double(H1) * r) * 2;
-        const double expand = (2.0 * sgmv::kGM * H2 + double(r) * H2) * 2;
+        const double shrink = (double(tm) * H1 + double(H1) * r) * 2;
+        const double expand = (2.0 * tm * H2 + double(r) * H2) * 2;
         const int sms = std::max(f.sms, 1);
         double best = 1e300;
         for (int ns = 1; ns <= std::min(max_split, 16); ++ns) {

@@ -46,8 +46,7 @@ constexpr int kGroupedMinSegment = 128;  // dispatcher: longest segment at least
 constexpr int kGM = 128;                 // rows per M-tile (UMMA M)
 constexpr int kGK = 64;                  // K per shrink stage (one 128-byte swizzle atom of 16-bit values)
 constexpr int kGN = 128;                 // columns per expand N-tile
-constexpr int kGShrinkStages = 3;
-constexpr int kGExpandStages = 2;
+constexpr int kGStages = 4;              // one ring for both phases: 2 K-steps or 1 N-tile per stage
 constexpr int kGThreads = 192;           // 6 warps
 constexpr int kGTmemCols = 512;
 
@@ -73,21 +72,24 @@ struct GroupedParams {
     float scale;
     int nsplit;  // N-slices of H2
     int nspan;   // columns per N-slice (multiple of kGN)
+    int tm;      // rows per M-tile, 8..128 (the MMA's M stays 128; rows past tm are never used)
 };
 
 template <int R>
 struct GroupedGeom {
-    // shrink stage: X tile [128 x 64] (TMA, 128B swizzle) + A_i tile [64 x R] (MN-major)
+    // shrink stage: two K-steps, [X tile 0][X tile 1][A tile 0][A tile 1]: X tiles [128 x 64]
+    // (TMA, 128B swizzle; tm rows loaded), A_i tiles [64 x R] (MN-major)
     static constexpr int X_BYTES = kGM * kGK * 2;
     static constexpr int A_BYTES = kGK * R * 2;
-    static constexpr int SSTAGE = X_BYTES + ((A_BYTES + 1023) / 1024) * 1024;
+    static constexpr int A_SLOT = ((A_BYTES + 1023) / 1024) * 1024;
+    static constexpr int SSTAGE = 2 * X_BYTES + 2 * A_SLOT;
     // expand stage: Y tile [128 x 128] as two 64-column TMA boxes + B_i tile [R x 128] (MN-major)
     static constexpr int Y_BYTES = kGM * kGN * 2;
     static constexpr int B_BYTES = R * kGN * 2;
     static constexpr int ESTAGE = Y_BYTES + B_BYTES;
+    static constexpr int STAGE = SSTAGE > ESTAGE ? SSTAGE : ESTAGE;
     static constexpr int V_BYTES = kGM * R * 2;  // one of V_hi, V_lo
-    static constexpr size_t SMEM = size_t(kGShrinkStages) * SSTAGE + size_t(kGExpandStages) * ESTAGE +
-                                   2 * size_t(V_BYTES) + 1024 /* alignment slack */;
+    static constexpr size_t SMEM = size_t(kGStages) * STAGE + 2 * size_t(V_BYTES) + 1024 /* alignment slack */;
     // swizzle of an MN-major A_i tile (rows of R 16-bit values) and of K-major V rows
     static constexpr int SW_BITS = R == 64 ? 3 : (R == 32 ? 2 : 1);           // 128B, 64B, 32B
     static constexpr uint64_t SW_TYPE = R == 64 ? 2 : (R == 32 ? 4 : 6);      // descriptor layout type
@@ -183,7 +185,7 @@ __device__ bool find_tile(const GroupedParams& P, int tile, int& seg_out, int& m
         int cnt = 0;
         if (s < P.n_segments) {
             const int b = __ldg(P.seg_starts + s), e = __ldg(P.seg_starts + s + 1);
-            if (b >= 0 && b <= e && e <= P.T) cnt = (e - b + kGM - 1) / kGM;
+            if (b >= 0 && b <= e && e <= P.T) cnt = (e - b + P.tm - 1) / P.tm;
         }
         int incl = cnt;
 #pragma unroll
@@ -231,13 +233,11 @@ __global__ void __launch_bounds__(kGThreads, 1)
     extern __shared__ __align__(1024) unsigned char gsmem_raw[];
     // 1024-byte alignment for the swizzled tiles
     unsigned char* gsmem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(gsmem_raw) + 1023) & ~uintptr_t(1023));
-    unsigned char* sstage = gsmem;
-    unsigned char* estage = sstage + kGShrinkStages * G::SSTAGE;
-    unsigned char* vhi = estage + kGExpandStages * G::ESTAGE;
+    unsigned char* ring = gsmem;
+    unsigned char* vhi = ring + kGStages * G::STAGE;
     unsigned char* vlo = vhi + G::V_BYTES;
 
-    __shared__ __align__(8) uint64_t s_full[kGShrinkStages], s_empty[kGShrinkStages];
-    __shared__ __align__(8) uint64_t e_full[kGExpandStages], e_empty[kGExpandStages];
+    __shared__ __align__(8) uint64_t full[kGStages], empty[kGStages];
     __shared__ __align__(8) uint64_t d1_full, v_full, d2_full[2], d2_empty[2];
     __shared__ __align__(128) CUtensorMap map_build[2];
     __shared__ uint32_t tmem_base_s;
@@ -268,13 +268,10 @@ __global__ void __launch_bounds__(kGThreads, 1)
         }
     }
     if (threadIdx.x == 0) {
-        for (int i = 0; i < kGShrinkStages; ++i) {
-            mbar_init(&s_full[i], 1);   // producer expect_tx; the TMA copies complete the bytes
-            mbar_init(&s_empty[i], 1);  // MMA commit
-        }
-        for (int i = 0; i < kGExpandStages; ++i) {
-            mbar_init(&e_full[i], 1);
-            mbar_init(&e_empty[i], 1 + 4);  // MMA commit (B read) + 4 epilogue warps (Y read)
+        for (int i = 0; i < kGStages; ++i) {
+            mbar_init(&full[i], 1);       // producer expect_tx; the TMA copies complete the bytes
+            mbar_init(&empty[i], 1 + 4);  // MMA commit + 4 arrivals (the MMA thread for shrink
+                                          // stages, the epilogue warps for expand stages)
         }
         mbar_init(&d1_full, 1);
         mbar_init(&v_full, 4);
@@ -299,12 +296,13 @@ __global__ void __launch_bounds__(kGThreads, 1)
 
     Segment seg;
     load_segment(P.seg_starts, P.lora_idx, P.A_ptrs, P.B_ptrs, seg_id, P.T, P.num_adapters, seg);
-    const int t0 = seg.begin + mt * kGM;
-    const int rows = min(kGM, seg.end - t0);  // valid rows of this tile
+    const int t0 = seg.begin + mt * P.tm;
+    const int rows = min(P.tm, seg.end - t0);  // valid rows of this tile
     const int n_lo = nsl * P.nspan;
     const int n_hi = min(P.H2, n_lo + P.nspan);
     const int n_tiles = n_lo < n_hi ? (n_hi - n_lo + kGN - 1) / kGN : 0;
     const int k_steps = (P.H1 + kGK - 1) / kGK;
+    const int s_stages = (k_steps + 1) / 2;  // shrink stages of two K-steps (the last may hold one)
 
     // TMEM: D1 at columns [0, R), D2 buffers at 128 and 256
     if (warp == 1) {
@@ -339,61 +337,68 @@ __global__ void __launch_bounds__(kGThreads, 1)
             map_acquire(gB);
         }
         __syncwarp();
-        for (int ks = 0; ks < k_steps; ++ks) {
-            const int st = ks % kGShrinkStages;
-            if (ks >= kGShrinkStages) mbar_wait<false>(&s_empty[st], ((ks / kGShrinkStages) - 1) & 1u, P.dev_status, dead);
-            unsigned char* xs = sstage + st * G::SSTAGE;
-            unsigned char* as = xs + G::X_BYTES;
+        uint32_t it = 0;
+        for (int ss = 0; ss < s_stages; ++ss, ++it) {
+            const uint32_t st = it % kGStages;
+            if (it >= kGStages) mbar_wait<false>(&empty[st], ((it / kGStages) - 1) & 1u, P.dev_status, dead);
+            unsigned char* xs = ring + st * G::STAGE;
+            const int nks = min(2, k_steps - 2 * ss);
             if (lane == 0) {
-                mbar_arrive_expect_tx(&s_full[st], G::X_BYTES + G::A_BYTES);
-                tma_load_2d(xs, &tmX, ks * kGK, t0, &s_full[st]);
-                tma_load_2d(as, gA, 0, ks * kGK, &s_full[st]);
+                mbar_arrive_expect_tx(&full[st], uint32_t(nks) * (uint32_t(P.tm) * kGK * 2 + G::A_BYTES));
+                for (int h = 0; h < nks; ++h) {
+                    const int ks = 2 * ss + h;
+                    tma_load_2d(xs + h * G::X_BYTES, &tmX, ks * kGK, t0, &full[st]);
+                    tma_load_2d(xs + 2 * G::X_BYTES + h * G::A_SLOT, gA, 0, ks * kGK, &full[st]);
+                }
             }
             __syncwarp();
         }
-        for (int nt = 0; nt < n_tiles; ++nt) {
-            const int st = nt % kGExpandStages;
-            if (nt >= kGExpandStages) mbar_wait<false>(&e_empty[st], ((nt / kGExpandStages) - 1) & 1u, P.dev_status, dead);
-            unsigned char* ys = estage + st * G::ESTAGE;
+        for (int nt = 0; nt < n_tiles; ++nt, ++it) {
+            const uint32_t st = it % kGStages;
+            if (it >= kGStages) mbar_wait<false>(&empty[st], ((it / kGStages) - 1) & 1u, P.dev_status, dead);
+            unsigned char* ys = ring + st * G::STAGE;
             unsigned char* bs = ys + G::Y_BYTES;
             const int n0 = n_lo + nt * kGN;
             if (lane == 0) {
-                mbar_arrive_expect_tx(&e_full[st], G::Y_BYTES + G::B_BYTES);
-                tma_load_2d(ys, &tmY, n0, t0, &e_full[st]);
-                tma_load_2d(ys + G::Y_BYTES / 2, &tmY, n0 + 64, t0, &e_full[st]);
-                tma_load_2d(bs, gB, n0, 0, &e_full[st]);
-                tma_load_2d(bs + R * 128, gB, n0 + 64, 0, &e_full[st]);
+                mbar_arrive_expect_tx(&full[st], 2u * P.tm * 64 * 2 + G::B_BYTES);
+                tma_load_2d(ys, &tmY, n0, t0, &full[st]);
+                tma_load_2d(ys + G::Y_BYTES / 2, &tmY, n0 + 64, t0, &full[st]);
+                tma_load_2d(bs, gB, n0, 0, &full[st]);
+                tma_load_2d(bs + R * 128, gB, n0 + 64, 0, &full[st]);
             }
             __syncwarp();
         }
         // every copy issued lands before the CTA may exit
-        if (lane == 0) {
-            for (int i = k_steps > kGShrinkStages ? k_steps - kGShrinkStages : 0; i < k_steps; ++i)
-                drain_wait(&s_full[i % kGShrinkStages], (uint32_t(i) / kGShrinkStages) & 1u);
-            for (int i = n_tiles > kGExpandStages ? n_tiles - kGExpandStages : 0; i < n_tiles; ++i)
-                drain_wait(&e_full[i % kGExpandStages], (uint32_t(i) / kGExpandStages) & 1u);
-        }
+        if (lane == 0)
+            for (uint32_t i = it > uint32_t(kGStages) ? it - kGStages : 0u; i < it; ++i)
+                drain_wait(&full[i % kGStages], (i / kGStages) & 1u);
         __syncwarp();
     } else if (warp == 1) {
         // ---------------------------------- MMA issuer ----------------------------------
         const uint32_t fmt = std::is_same<T, __nv_bfloat16>::value ? 1u : 0u;
         const uint32_t idesc_s = instr_desc(fmt, 0, 1, R, kGM);    // X K-major, A_i MN-major, N = r
         const uint32_t idesc_e = instr_desc(fmt, 0, 1, kGN, kGM);  // V K-major, B_i MN-major, N = 128
-        for (int ks = 0; ks < k_steps; ++ks) {
-            const int st = ks % kGShrinkStages;
-            mbar_wait<false>(&s_full[st], (ks / kGShrinkStages) & 1u, P.dev_status, dead);
+        uint32_t it = 0;
+        for (int ss = 0; ss < s_stages; ++ss, ++it) {
+            const uint32_t st = it % kGStages;
+            mbar_wait<false>(&full[st], (it / kGStages) & 1u, P.dev_status, dead);
             tc_fence_after();
             if (lane == 0) {
-                const uint32_t xa = smem_u32(sstage + st * G::SSTAGE);
-                const uint32_t aa = xa + G::X_BYTES;
+                const int nks = min(2, k_steps - 2 * ss);
+                const uint32_t xa0 = smem_u32(ring + st * G::STAGE);
+                for (int h = 0; h < nks; ++h) {
+                    const uint32_t xa = xa0 + h * G::X_BYTES;
+                    const uint32_t aa = xa0 + 2 * G::X_BYTES + h * G::A_SLOT;
 #pragma unroll
-                for (int kk = 0; kk < kGK / 16; ++kk) {
-                    const uint64_t adesc = smem_desc(xa + kk * 32, 16, 1024, 2);
-                    const uint64_t bdesc = smem_desc(aa + kk * 16 * G::ROW_BYTES, 16 * G::ROW_BYTES, 8 * G::ROW_BYTES,
-                                                     G::SW_TYPE);
-                    tc_mma(tmem, adesc, bdesc, idesc_s, (ks | kk) ? 1u : 0u);
+                    for (int kk = 0; kk < kGK / 16; ++kk) {
+                        const uint64_t adesc = smem_desc(xa + kk * 32, 16, 1024, 2);
+                        const uint64_t bdesc = smem_desc(aa + kk * 16 * G::ROW_BYTES, 16 * G::ROW_BYTES,
+                                                         8 * G::ROW_BYTES, G::SW_TYPE);
+                        tc_mma(tmem, adesc, bdesc, idesc_s, (ss | h | kk) ? 1u : 0u);
+                    }
                 }
-                tc_commit(&s_empty[st]);
+                tc_commit(&empty[st]);
+                for (int i = 0; i < 4; ++i) mbar_arrive_local(&empty[st]);
             }
             __syncwarp();
         }
@@ -401,14 +406,14 @@ __global__ void __launch_bounds__(kGThreads, 1)
         __syncwarp();
         mbar_wait<false>(&v_full, 0, P.dev_status, dead);
         tc_fence_after();
-        for (int nt = 0; nt < n_tiles; ++nt) {
-            const int st = nt % kGExpandStages;
+        for (int nt = 0; nt < n_tiles; ++nt, ++it) {
+            const uint32_t st = it % kGStages;
             const int buf = nt & 1;
             if (nt >= 2) mbar_wait<false>(&d2_empty[buf], ((nt >> 1) - 1) & 1u, P.dev_status, dead);
-            mbar_wait<false>(&e_full[st], (nt / kGExpandStages) & 1u, P.dev_status, dead);
+            mbar_wait<false>(&full[st], (it / kGStages) & 1u, P.dev_status, dead);
             tc_fence_after();
             if (lane == 0) {
-                const uint32_t ba = smem_u32(estage + st * G::ESTAGE + G::Y_BYTES);
+                const uint32_t ba = smem_u32(ring + st * G::STAGE + G::Y_BYTES);
                 const uint32_t d2 = tmem + 128u + 128u * buf;
 #pragma unroll
                 for (int kk = 0; kk < R / 16; ++kk) {
@@ -419,7 +424,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
                     tc_mma(d2, alo, bdesc, idesc_e, 1u);
                 }
                 tc_commit(&d2_full[buf]);
-                tc_commit(&e_empty[st]);
+                tc_commit(&empty[st]);
             }
             __syncwarp();
         }
@@ -458,12 +463,13 @@ __global__ void __launch_bounds__(kGThreads, 1)
         T* __restrict__ Y = static_cast<T*>(P.Y);
         const bool row_ok = m < rows;
         for (int nt = 0; nt < n_tiles; ++nt) {
-            const int st = nt % kGExpandStages;
+            const uint32_t it = uint32_t(s_stages + nt);
+            const uint32_t st = it % kGStages;
             const int buf = nt & 1;
-            mbar_wait<false>(&e_full[st], (nt / kGExpandStages) & 1u, P.dev_status, dead);
+            mbar_wait<false>(&full[st], (it / kGStages) & 1u, P.dev_status, dead);
             mbar_wait<false>(&d2_full[buf], (nt >> 1) & 1u, P.dev_status, dead);
             tc_fence_after();
-            unsigned char* ys = estage + st * G::ESTAGE;
+            unsigned char* ys = ring + st * G::STAGE;
             const int n0 = n_lo + nt * kGN;
             // row m of the tile: y + scale * D2, written back over the staged Y row
 #pragma unroll 1
@@ -504,7 +510,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
             __syncwarp();
             if (lane == 0) {
                 mbar_arrive_relaxed(&d2_empty[buf]);
-                mbar_arrive_relaxed(&e_empty[st]);
+                mbar_arrive_relaxed(&empty[st]);
             }
         }
     }
