@@ -60,9 +60,9 @@ TRAFFIC = {
     "llama70b_decode_h28672": {"bytes": 467304448 + 14324736, "profile": "profiles/decode_tc_kernel_llama70b_decode.md",
                                "sources": ["sgmv_common.cuh", "sgmv_fused.cuh", "sgmv_tmap.cuh", "sgmv_grouped_tc.cuh",
                                            "sgmv_decode_tc.cuh"], "sha256": "8b17c61cdcf52e4636b5b57846372e39b9c482b897320799056c8cf9fff05f82"},
-    "prefill": {"bytes": 168567296 + 21483520, "profile": "profiles/grouped_kernel_prefill.md",
+    "prefill": {"bytes": 168582912 + 22138368, "profile": "profiles/grouped_kernel_prefill.md",
                 "sources": ["sgmv_common.cuh", "sgmv_fused.cuh", "sgmv_tmap.cuh", "sgmv_grouped_tc.cuh"],
-                "sha256": "b3e02057f98552391de61d78cf0a228ef962176795d90aa824537c0d3605518e"},
+                "sha256": "782c566516423019f1d8c3fca6699ce82bea18ad7839cba6d761bee229f7004f"},
 }
 
 

@@ -47,9 +47,10 @@
  *     *dev_status (a device uint32; may be NULL). No kernel traps.
  *   - Alignment: X, Y, V and workspace must be 16-byte aligned; H1 and H2
  *     must be multiples of 8.
- *   - Overlap with the previous kernel: the fused kernel (variant FUSED,
- *     which AUTO picks for short segments, and lora_sgmv_apply_batched) is
- *     launched with programmatic dependent launch. It reads segment arrays,
+ *   - Overlap with the previous kernel: the fused kernels (variants FUSED
+ *     and FUSED_TC, which AUTO picks for short segments, and
+ *     lora_sgmv_apply_batched) are launched with programmatic dependent
+ *     launch. It reads segment arrays,
  *     pointer tables and adapter weights while the kernel before it on the
  *     stream may still run, and reads X and Y only after that kernel has
  *     completed. So seg_starts, lora_idx, the tables and the adapters of a
@@ -58,8 +59,12 @@
  *     be. Use LORA_SGMV_VARIANT_SPLIT where that does not hold.
  *   - Thread safety: calls on different streams may run concurrently. The
  *     library keeps no mutable global state other than a lazily filled,
- *     mutex-guarded cache of device facts and kernel attributes, and an
- *     atomic count of kernel launches.
+ *     mutex-guarded cache of device facts and kernel attributes, an atomic
+ *     count of kernel launches, and, on every device that loads it, a fixed
+ *     1 MiB array of tensor-map slots: the tensor-core kernels (GROUPED_TC,
+ *     FUSED_TC) reach adapters through tensor maps they build on the device,
+ *     and each of their CTAs claims a slot table with an atomic operation for
+ *     its lifetime, so concurrent kernels never share a slot.
  */
 #ifndef LORA_SGMV_H
 #define LORA_SGMV_H
