@@ -570,8 +570,9 @@ __device__ __forceinline__ void produce_job(const FusedParams& P, const Job& job
         } else {
             deferred = ta + 1;
         }
-        if (ta == 0 && job.nc > 0) {
-            // start B on its way to L2 while the shrink runs; the expand stages then hit L2
+        if (ta == min(nA, kFusedStages) - 1 && job.nc > 0) {
+            // start B on its way to L2 while the shrink runs, once the ring's first round of A
+            // copies is queued ahead of the prefetches; the expand stages then hit L2
             for (int row = lane; row < R; row += 32)
                 bulk_prefetch_l2(B + size_t(row) * pr.H2 + job.c0, uint32_t(job.nc) * 2);
         }

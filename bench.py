@@ -18,10 +18,11 @@ graph holding a whole rotation of layers back to back (consecutive launches
 overlap through programmatic dependent launch, as a captured decode step
 would), plus single-layer graphs for a remainder, so host launch latency does
 not stand in for kernel time. ``e2e`` repeats the measurement through the
-public call with host buffers: each step copies its inputs from pinned host
-memory, groups the token batch on the host, runs the four lora_sgmv_apply
-calls, and reads the outputs back. Other workloads (--workload) run one
-lora_sgmv_apply per step, the dispatcher choosing the kernels.
+public calls with host buffers: each step groups the token batch on the host,
+copies the segment arrays and the four projections' X and Y from pinned host
+memory, runs one lora_sgmv_apply_batched launch, and reads Y back. Other
+workloads (--workload) run one lora_sgmv_apply per step, the dispatcher
+choosing the kernels.
 
 Multi-GPU (torchrun): every rank runs its own replica of the workload (the
 path has no cross-GPU data exchange); value = all ranks' tokens / max time.
@@ -436,25 +437,31 @@ def run_ours(args, spec: Spec, rank: int, world: int, local: int):
 
 
 def run_e2e(args, spec, torch, sgmv, dev, stream, calls, dt, tdt, world=1):
-    """Same metric through lora_sgmv_group_segments + lora_sgmv_apply with host buffers."""
+    """Same metric through the public calls with host buffers: lora_sgmv_group_segments on the
+    host, then one lora_sgmv_apply_batched launch for the step's projections (lora_sgmv_apply
+    for one projection). Per step the segment arrays, X and Y of every projection go host ->
+    device (one pinned copy each, the projections packed), and the step's Y comes back."""
     w = spec.w
+    P = spec.P
     steps = max(3, min(args.steps, 200))
-    # pinned host copies of every (layer, projection)'s inputs and outputs
-    hX = [torch.empty((w.T, w.H1), dtype=tdt, pin_memory=True) for _ in range(spec.P)]
-    hY = [torch.empty((w.T, w.H2), dtype=tdt, pin_memory=True) for _ in range(spec.P)]
-    for p in range(spec.P):
+    hX = torch.empty((P, w.T, w.H1), dtype=tdt, pin_memory=True)
+    hY = torch.empty((P, w.T, w.H2), dtype=tdt, pin_memory=True)
+    for p in range(P):
         hX[p].copy_(calls[p][2].cpu())
         hY[p].copy_(calls[p][3].cpu())
+    outY = torch.empty((P, w.T, w.H2), dtype=tdt, pin_memory=True)
     ids = np.ascontiguousarray(w.ids, dtype=np.int32)
-    h_seg = torch.empty(w.num_adapters + 1, dtype=torch.int32, pin_memory=True)
-    h_idx = torch.empty(w.num_adapters, dtype=torch.int32, pin_memory=True)
-    d_seg = torch.empty(w.num_adapters + 1, dtype=torch.int32, device=dev)
-    d_idx = torch.empty(w.num_adapters, dtype=torch.int32, device=dev)
-    dX = [torch.empty((w.T, w.H1), dtype=tdt, device=dev) for _ in range(spec.P)]
-    dY = [torch.empty((w.T, w.H2), dtype=tdt, device=dev) for _ in range(spec.P)]
-    outY = [torch.empty((w.T, w.H2), dtype=tdt, pin_memory=True) for _ in range(spec.P)]
+    meta_len = 2 * w.num_adapters + 1
+    h_meta = torch.empty(meta_len, dtype=torch.int32, pin_memory=True)  # seg_starts, then lora_idx
+    h_meta_np = h_meta.numpy()
+    d_meta = torch.empty(meta_len, dtype=torch.int32, device=dev)
+    dX = torch.empty((P, w.T, w.H1), dtype=tdt, device=dev)
+    dY = torch.empty((P, w.T, w.H2), dtype=tdt, device=dev)
     ws_bytes = sgmv.lora_sgmv_workspace_bytes(w.T, w.r)
     ws = torch.empty(ws_bytes // 4, dtype=torch.float32, device=dev)
+    problems = [[sgmv.Problem(dY[p].data_ptr(), dX[p].data_ptr(), calls[l * P + p][4].data_ptr(),
+                              calls[l * P + p][5].data_ptr(), w.num_adapters, w.H1, w.H2, w.scale)
+                 for p in range(P)] for l in range(spec.L)]
     sh = stream.cuda_stream
     h2d = d2h = 0
 
@@ -463,25 +470,24 @@ def run_e2e(args, spec, torch, sgmv, dev, stream, calls, dt, tdt, world=1):
         l = i % spec.L
         seg, idx, _ = sgmv.lora_sgmv_group_segments(ids, w.num_adapters)
         n = len(idx)
-        h_seg[: n + 1].copy_(torch.from_numpy(seg))
-        h_idx[:n].copy_(torch.from_numpy(idx))
+        h_meta_np[: n + 1] = seg
+        h_meta_np[n + 1: 2 * n + 1] = idx
         max_len = int(np.max(np.diff(seg)))
+        d_seg, d_idx = d_meta.data_ptr(), d_meta.data_ptr() + 4 * (n + 1)
         with torch.cuda.stream(stream):
-            d_seg[: n + 1].copy_(h_seg[: n + 1], non_blocking=True)
-            d_idx[:n].copy_(h_idx[:n], non_blocking=True)
-            b_in = (n + 1 + n) * 4
-            b_out = 0
-            for p in range(spec.P):
-                _, _, _, _, A_ptrs, B_ptrs = calls[l * spec.P + p]
-                dX[p].copy_(hX[p], non_blocking=True)
-                dY[p].copy_(hY[p], non_blocking=True)
-                sgmv.lora_sgmv_apply(dY[p], dX[p], A_ptrs, B_ptrs, d_seg, d_idx, n, w.num_adapters, w.T, w.H1, w.r,
+            d_meta[: 2 * n + 1].copy_(h_meta[: 2 * n + 1], non_blocking=True)
+            dX.copy_(hX, non_blocking=True)
+            dY.copy_(hY, non_blocking=True)
+            if P > 1:
+                sgmv.lora_sgmv_apply_batched(problems[l], d_seg, d_idx, n, w.T, w.r, dt, max_len, None, sh)
+            else:
+                q = problems[l][0]
+                sgmv.lora_sgmv_apply(q.Y, q.X, q.A_ptrs, q.B_ptrs, d_seg, d_idx, n, w.num_adapters, w.T, w.H1, w.r,
                                      w.H2, w.scale, dt, max_len, ws, ws_bytes, None, sh)
-                outY[p].copy_(dY[p], non_blocking=True)
-                b_in += hX[p].numel() * 2 + hY[p].numel() * 2
-                b_out += outY[p].numel() * 2
+            outY.copy_(dY, non_blocking=True)
         stream.synchronize()
-        h2d, d2h = b_in, b_out
+        h2d = (2 * n + 1) * 4 + hX.numel() * 2 + hY.numel() * 2
+        d2h = outY.numel() * 2
 
     for i in range(3):
         one(i)
@@ -493,11 +499,12 @@ def run_e2e(args, spec, torch, sgmv, dev, stream, calls, dt, tdt, world=1):
     for i in range(steps):
         one(i)
     el = max_over_ranks(time.perf_counter() - t0, world, dev)
+    call = "1 lora_sgmv_apply_batched launch" if P > 1 else "1 lora_sgmv_apply call"
     return {"value": round(job_tokens_per_s(w.T * steps, world, el), 1), "unit": UNIT,
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": steps,
             "note": "host wall clock (the host's grouping is part of the step), slowest rank; per step: host "
-                    f"grouping, pinned H2D of X, Y and segments, {spec.P} lora_sgmv_apply calls, D2H of Y, "
-                    "stream sync"}
+                    f"grouping, pinned H2D of the segment arrays and of X and Y ({P} projections), {call}, "
+                    "D2H of Y, stream sync"}
 
 
 # ---------------------------------------------------------------------------------------------
