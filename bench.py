@@ -56,11 +56,13 @@ L2_BYTES = 126 * 1024 * 1024
 # those it was taken from: their SHA-256 is stored with it and checked here, else "traffic"
 # is null.
 TRAFFIC = {
-    "distinct": {"bytes": 35724800, "profile": "profiles/fused_kernel_distinct_decode.md",
-                 "sources": ["sgmv_common.cuh", "sgmv_fused.cuh"], "sha256": "abde291ab9d6714445fec73dd5573bbe6715a423558b54f83708bca522bf7776"},
-    "llama70b_decode_h28672": {"bytes": 467304448 + 14324736, "profile": "profiles/decode_tc_kernel_llama70b_decode.md",
+    "distinct": {"bytes": 35724288 + 2048, "profile": "profiles/fused_kernel_distinct_decode.md",
+                 "sources": ["sgmv_common.cuh", "sgmv_fused.cuh"],
+                 "sha256": "e2d41ed385c1ba3b023529a9127f563df5317aa29af52d1bb8a4398c386b2c2b"},
+    "llama70b_decode_h28672": {"bytes": 467455488 + 14396416, "profile": "profiles/decode_tc_kernel_llama70b_decode.md",
                                "sources": ["sgmv_common.cuh", "sgmv_fused.cuh", "sgmv_tmap.cuh", "sgmv_grouped_tc.cuh",
-                                           "sgmv_decode_tc.cuh"], "sha256": "8b17c61cdcf52e4636b5b57846372e39b9c482b897320799056c8cf9fff05f82"},
+                                           "sgmv_decode_tc.cuh"],
+                               "sha256": "23c5a02c9a668903c76d25adb77b9d92cbd23959e96c572763906ada3125b25a"},
     "prefill": {"bytes": 168582912 + 22138368, "profile": "profiles/grouped_kernel_prefill.md",
                 "sources": ["sgmv_common.cuh", "sgmv_fused.cuh", "sgmv_tmap.cuh", "sgmv_grouped_tc.cuh"],
                 "sha256": "782c566516423019f1d8c3fca6699ce82bea18ad7839cba6d761bee229f7004f"},
