@@ -64,6 +64,19 @@ def test_fused_long_rows_many_tiles(r, variant):
     assert_close(p.apply(variant=variant), p.oracle_apply(), "bf16", "long rows")
 
 
+@pytest.mark.parametrize("H1,H2", [(512, 768), (640, 1280), (896, 1792)])
+def test_decode_tc_odd_cluster_sizes(H1, H2):
+    # few jobs and K/N extents of 3, 5 and 7 stages: the cost model picks clusters of 3, 5 or 7
+    # CTAs (non-power-of-two), each with its own K- and N-slice and a V exchange among them
+    seg = np.array([0, 5, 8, 8, 11], np.int32)
+    idx = np.array([1, 0, 2, 1], np.int32)
+    w = inputs.small_random(11, 3, H1, H2, 64, "bf16", seed=H1)
+    p = DeviceProblem(w, y_random=True, adapters=[0, 1, 2], seg_starts=seg, lora_idx=idx)
+    got = p.apply(variant=sgmv.VARIANT_FUSED_TC)
+    assert int(p.status.item()) == 0
+    assert_close(got, p.oracle_apply(), "bf16", f"decode tc {H1}x{H2}")
+
+
 def test_batched_projections_with_different_shapes():
     # q/k/v/o-like problems sharing one token grouping, in one launch
     ids = inputs.skewed(4096).ids
