@@ -410,9 +410,15 @@ lora_sgmv_status launch_decode_tc(sgmv::FusedParams P, const sgmv::DecodeMaps& m
         return G::BASE + size_t(C) * G::TILE + size_t(bucket) * 1024 * 4 + 1024 /* alignment slack */;
     };
     auto kernel = sgmv::sgmv_decode_tc_kernel<T, R>;
-    if (ensure_smem(kernel, smem_for(sgmv::kFusedMaxCluster), smem_granted) != LORA_SGMV_OK) return LORA_SGMV_ERR_CUDA;
     DeviceFacts f;
     if (device_facts(f) != LORA_SGMV_OK) return LORA_SGMV_ERR_CUDA;
+    // the largest cluster whose shared memory (ring + one partial V tile per CTA of the cluster
+    // + the job prefix) fits a CTA, leaving 4 KB for the kernel's static shared memory
+    const size_t smem_cap = f.max_smem_optin > 4096 ? size_t(f.max_smem_optin) - 4096 : 0;
+    int c_fit = sgmv::kFusedMaxCluster;
+    while (c_fit > 0 && smem_for(c_fit) > smem_cap) --c_fit;
+    if (c_fit == 0) return LORA_SGMV_ERR_DIM;
+    if (ensure_smem(kernel, smem_for(c_fit), smem_granted) != LORA_SGMV_OK) return LORA_SGMV_ERR_CUDA;
     int dev = 0;
     if (record(cudaGetDevice(&dev)) != cudaSuccess) return LORA_SGMV_ERR_CUDA;
     if (dev < 0 || dev >= 64) return LORA_SGMV_ERR_UNSUPPORTED;
@@ -443,7 +449,7 @@ lora_sgmv_status launch_decode_tc(sgmv::FusedParams P, const sgmv::DecodeMaps& m
     // least one stage of A_i and of B_i.
     constexpr double kCtaBytesPerUs = 40e3;  // ~40 GB/s that one CTA streams with TMA
     constexpr double kJobFixedUs = 4.0;
-    int c_cap = sgmv::kFusedMaxCluster;
+    int c_cap = c_fit;
     double job_bytes = 0;
     for (int i = 0; i < P.n_problems; ++i) {
         c_cap = std::min(c_cap, (P.prob[i].H1 + G::KS - 1) / G::KS);

@@ -77,6 +77,20 @@ def test_decode_tc_odd_cluster_sizes(H1, H2):
     assert_close(got, p.oracle_apply(), "bf16", f"decode tc {H1}x{H2}")
 
 
+def test_decode_tc_many_segments():
+    # ~8000 segments: the job prefix takes most of the shared memory the cluster's V tiles
+    # would use, so the host must fall back to smaller clusters
+    rng = np.random.default_rng(7)
+    lens = np.concatenate([np.ones(7990, np.int64), rng.integers(3, 20, size=10)])
+    seg = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    idx = (np.arange(len(lens)) % 64).astype(np.int32)
+    w = inputs.small_random(int(seg[-1]), 64, 128, 192, 64, "bf16", seed=11)
+    p = DeviceProblem(w, y_random=True, adapters=list(range(64)), seg_starts=seg, lora_idx=idx)
+    got = p.apply(variant=sgmv.VARIANT_FUSED_TC)
+    assert int(p.status.item()) == 0
+    assert_close(got, p.oracle_apply(), "bf16", "decode tc, 8000 segments")
+
+
 def test_batched_projections_with_different_shapes():
     # q/k/v/o-like problems sharing one token grouping, in one launch
     ids = inputs.skewed(4096).ids
