@@ -22,9 +22,10 @@
 // canonical layout the MMA descriptors describe: X and Y through tensor maps built per
 // call, A_i and B_i (reached through a device table of pointers) through maps each CTA
 // makes from a per-call template (sgmv_tmap.cuh). Warp roles: warp 0 producer, warp 1
-// allocates TMEM and issues tcgen05.mma (one thread), warps 2..5 epilogue (one TMEM lane
-// quarter each). The host picks the number of N-slices per M-tile from the bytes the
-// busiest SM streams (every slice re-reads its tile's X rows and A_i).
+// allocates TMEM and issues tcgen05.mma (one thread), warps 2..9 epilogue (one TMEM lane
+// quarter and one 64-column half of each N-tile each). The host picks the number of
+// N-slices per M-tile from the bytes the busiest SM streams (every slice re-reads its tile's
+// X rows and A_i).
 //
 // Every mbarrier wait is bounded in time; a wait that gives up sets
 // LORA_SGMV_DEV_TIMEOUT and the kernel runs to its end (TMEM is always freed).
@@ -47,7 +48,8 @@ constexpr int kGM = 128;                 // rows per M-tile (UMMA M)
 constexpr int kGK = 64;                  // K per shrink stage (one 128-byte swizzle atom of 16-bit values)
 constexpr int kGN = 128;                 // columns per expand N-tile
 constexpr int kGStages = 4;              // one ring for both phases: 2 K-steps or 1 N-tile per stage
-constexpr int kGThreads = 192;           // 6 warps
+constexpr int kGThreads = 320;           // 10 warps: producer, MMA issuer, 8 epilogue warps
+constexpr int kGEpiWarps = 8;            // two per TMEM lane quarter, one per 64-column half of a tile
 constexpr int kGTmemCols = 512;
 
 inline bool grouped_tc_rank(int r) { return r == 16 || r == 32 || r == 64; }
@@ -270,14 +272,14 @@ __global__ void __launch_bounds__(kGThreads, 1)
     if (threadIdx.x == 0) {
         for (int i = 0; i < kGStages; ++i) {
             mbar_init(&full[i], 1);       // producer expect_tx; the TMA copies complete the bytes
-            mbar_init(&empty[i], 1 + 4);  // MMA commit + 4 arrivals (the MMA thread for shrink
+            mbar_init(&empty[i], 1 + kGEpiWarps);  // MMA commit + 8 arrivals (the MMA thread for shrink
                                           // stages, the epilogue warps for expand stages)
         }
         mbar_init(&d1_full, 1);
-        mbar_init(&v_full, 4);
+        mbar_init(&v_full, kGEpiWarps);
         for (int i = 0; i < 2; ++i) {
             mbar_init(&d2_full[i], 1);
-            mbar_init(&d2_empty[i], 4);
+            mbar_init(&d2_empty[i], kGEpiWarps);
         }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         table_s = -1;
@@ -398,7 +400,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
                     }
                 }
                 tc_commit(&empty[st]);
-                for (int i = 0; i < 4; ++i) mbar_arrive_local(&empty[st]);
+                for (int i = 0; i < kGEpiWarps; ++i) mbar_arrive_local(&empty[st]);
             }
             __syncwarp();
         }
@@ -430,18 +432,19 @@ __global__ void __launch_bounds__(kGThreads, 1)
         }
     } else {
         // ---------------------------------- epilogue ----------------------------------
-        const int quarter = warp & 3;  // TMEM lanes [32*quarter, 32*quarter + 32)
+        const int quarter = warp & 3;       // TMEM lanes [32*quarter, 32*quarter + 32)
+        const int half = (warp - 2) >> 2;   // columns [64*half, 64*half + 64) of each N-tile
         const int m = quarter * 32 + lane;
         const uint32_t lane_addr = tmem + (uint32_t(quarter * 32) << 16);
         // V = D1 -> V_hi + V_lo (K-major, swizzled rows of R values)
         mbar_wait<false>(&d1_full, 0, P.dev_status, dead);
         tc_fence_after();
-#pragma unroll
-        for (int c0 = 0; c0 < R; c0 += 32) {
+        for (int c0 = 32 * half; c0 < R; c0 += 64) {  // the two halves share V's columns
             float v[32];
             tmem_ld32(lane_addr + c0, v);
-            const int nchunks = (R - c0) < 32 ? (R - c0) / 8 : 4;
-            for (int ch = 0; ch < nchunks; ++ch) {
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch) {
+                if (c0 + ch * 8 >= R) break;
                 float hi[8], lo[8];
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
@@ -473,7 +476,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
             const int n0 = n_lo + nt * kGN;
             // row m of the tile: y + scale * D2, written back over the staged Y row
 #pragma unroll 1
-            for (int c0 = 0; c0 < kGN; c0 += 32) {
+            for (int c0 = 64 * half; c0 < 64 * half + 64; c0 += 32) {
                 float acc[32];
                 tmem_ld32(lane_addr + 128u + 128u * buf + c0, acc);
                 if (row_ok) {
@@ -492,19 +495,17 @@ __global__ void __launch_bounds__(kGThreads, 1)
                 }
             }
             __syncwarp();
-            // this warp's 32 rows leave row by row: 8 lanes per 128-byte row segment, so each
-            // store instruction writes four whole segments
+            // this warp's 32 rows of its 64-column half leave row by row: 8 lanes per 128-byte
+            // row segment, so each store instruction writes four whole segments
 #pragma unroll
-            for (int b = 0; b < 2; ++b)
-#pragma unroll
-                for (int rq = 0; rq < 32; rq += 4) {
-                    const int rr = quarter * 32 + rq + (lane >> 3);
-                    const int c = lane & 7;
-                    const int col = n0 + b * 64 + c * 8;
-                    if (rr < rows && col < n_hi)
-                        st_vec(Y + size_t(t0 + rr) * P.H2 + col,
-                               *reinterpret_cast<const uint4*>(ys + b * (G::Y_BYTES / 2) + swz(rr, c, 3)));
-                }
+            for (int rq = 0; rq < 32; rq += 4) {
+                const int rr = quarter * 32 + rq + (lane >> 3);
+                const int c = lane & 7;
+                const int col = n0 + half * 64 + c * 8;
+                if (rr < rows && col < n_hi)
+                    st_vec(Y + size_t(t0 + rr) * P.H2 + col,
+                           *reinterpret_cast<const uint4*>(ys + half * (G::Y_BYTES / 2) + swz(rr, c, 3)));
+            }
             // the TMEM reads completed at tcgen05.wait::ld; no tcgen05 fence here (it would also
             // wait for the Y stores just issued)
             __syncwarp();
