@@ -36,8 +36,9 @@
 // as its reads are done; Y stages have their own ring, freed by the epilogue, so the stream of
 // adapter bytes never waits on the epilogue's latency. D2 has up to four TMEM buffers.
 //
-// Warps: 0 producer of X, A_i and B_i, 1 TMEM owner and MMA issuer, 2..5 exchange and
-// epilogue (one TMEM lane quarter each), 6 producer of Y. Programmatic dependent launch: X and Y are read only after
+// Warps: 0 producer of X, A_i and B_i, 1 TMEM owner and MMA issuer, 2..9 epilogue (two per
+// TMEM lane quarter, each taking every other 128-column group of a stage; one of them also
+// runs the V exchange), 10 producer of Y. Programmatic dependent launch: X and Y are read only after
 // griddepcontrol.wait. Every wait is bounded in time.
 #pragma once
 
@@ -47,7 +48,8 @@ namespace sgmv {
 
 constexpr int kDTokens = 16;    // tokens per job = N of the expand MMA
 constexpr int kDYStages = 4;    // Y ring, freed by the epilogue
-constexpr int kDThreads = 224;
+constexpr int kDThreads = 352;  // producer, MMA issuer, 8 epilogue warps, Y producer
+constexpr int kDEpiWarps = 8;   // two per TMEM lane quarter, splitting each stage's 128-column groups
 constexpr int kDTmemCols = 512;  // D1 at [0, r), D2 buffers from column 64 (one CTA per SM)
 constexpr int kDYMaps = 5;       // Y boxes of 1, 2, 4, 8 and 16 rows
 constexpr int kDEpiBatch = 2;    // expand stages per epilogue pass
@@ -184,13 +186,13 @@ __global__ void __launch_bounds__(kDThreads, 1)
         }
         for (int i = 0; i < SY; ++i) {
             mbar_init(&yfull[i], 1);
-            mbar_init(&yempty[i], 4);  // the 4 epilogue warps
+            mbar_init(&yempty[i], kDEpiWarps);
         }
         mbar_init(&d1_full, 1);
         mbar_init(&v_full, 1);
         for (int i = 0; i < ND2; ++i) {
             mbar_init(&d2_full[i], 1);
-            mbar_init(&d2_empty[i], 4);
+            mbar_init(&d2_empty[i], kDEpiWarps);
         }
         mbar_init(&vready, 1);  // own expect_tx; the C tiles arrive as transaction bytes
         mbar_init(&vfree, C);   // one arrival per receiver
@@ -322,7 +324,7 @@ __global__ void __launch_bounds__(kDThreads, 1)
             for (uint32_t i = it > uint32_t(S) ? it - S : 0u; i < it; ++i) drain_wait(&full[i % S], (i / S) & 1u);
         __syncwarp();
         if (C > 1) cluster_wait();
-    } else if (warp == 6) {
+    } else if (warp == 10) {
         // --------------------------------- Y producer ---------------------------------
         // Y rows of each expand stage, through their own ring, so that the adapter stream
         // above never waits for the epilogue
@@ -429,7 +431,8 @@ __global__ void __launch_bounds__(kDThreads, 1)
         if (C > 1) cluster_wait();
     } else {
         // ------------------------------ exchange and epilogue ------------------------------
-        const int quarter = warp & 3;  // TMEM lanes [32*quarter, 32*quarter + 32)
+        const int quarter = warp & 3;      // TMEM lanes [32*quarter, 32*quarter + 32)
+        const int half = (warp - 2) >> 2;  // 128-column groups half, half + 2, ... of each stage
         const uint32_t lane_base = tmem + (uint32_t(quarter * 32) << 16);
         if (C > 1) cluster_wait();
         uint32_t yit = 0, u = 0, g = 0;
@@ -442,7 +445,7 @@ __global__ void __launch_bounds__(kDThreads, 1)
                 const FusedProblem& pr = P.prob[job.p];
                 const int nA = (job.nk + G::KS - 1) / G::KS;
                 const int nB = (job.nc + G::NW - 1) / G::NW;
-                if (quarter == 0) {
+                if (quarter == 0 && half == 0) {
                     // partial V of this CTA: D1 rows 0..nt-1 (lanes 0..15 of quarter 0)
                     mbar_wait<false>(&d1_full, u & 1u, P.dev_status, dead);
                     tc_fence_after();
@@ -509,8 +512,7 @@ __global__ void __launch_bounds__(kDThreads, 1)
                         const unsigned char* ys = yring + ((yit + e) % SY) * G::Y_BYTES;
                         const uint32_t d2 = lane_base + 64u + uint32_t(G::D2_COLS) * ((g + e) % ND2);
                         const int n0 = job.c0 + (tb + e) * G::NW;
-#pragma unroll
-                        for (int gi = 0; gi < G::NB / 2; ++gi) {
+                        for (int gi = half; gi < G::NB / 2; gi += 2) {
                             float acc[16], acc_lo[16];
                             tmem_ld16(d2 + 32u * gi, acc);
                             tmem_ld16(d2 + 32u * gi + 16u, acc_lo);
@@ -546,7 +548,7 @@ __global__ void __launch_bounds__(kDThreads, 1)
                 ++u;
             }
         }
-        if (quarter == 0) {
+        if (quarter == 0 && half == 0) {
             pdl_wait();
             if (u >= 1) mbar_wait<true>(&vfree, (u - 1) & 1u, P.dev_status, dead);
             if (c == 0 && lane == 0) {  // report each rejected segment once
