@@ -59,13 +59,13 @@ TRAFFIC = {
     "distinct": {"bytes": 35724288 + 2048, "profile": "profiles/fused_kernel_distinct_decode.md",
                  "sources": ["sgmv_common.cuh", "sgmv_fused.cuh"],
                  "sha256": "e2d41ed385c1ba3b023529a9127f563df5317aa29af52d1bb8a4398c386b2c2b"},
-    "llama70b_decode_h28672": {"bytes": 467455488 + 14396416, "profile": "profiles/decode_tc_kernel_llama70b_decode.md",
+    "llama70b_decode_h28672": {"bytes": 467335424 + 14264320, "profile": "profiles/decode_tc_kernel_llama70b_decode.md",
                                "sources": ["sgmv_common.cuh", "sgmv_fused.cuh", "sgmv_tmap.cuh", "sgmv_grouped_tc.cuh",
                                            "sgmv_decode_tc.cuh"],
-                               "sha256": "23c5a02c9a668903c76d25adb77b9d92cbd23959e96c572763906ada3125b25a"},
-    "prefill": {"bytes": 168582912 + 22138368, "profile": "profiles/grouped_kernel_prefill.md",
+                               "sha256": "267fc74554376e0dce2e3f10499d73fab8d51fea0612dacb3445d99515dec955"},
+    "prefill": {"bytes": 168609024 + 21820416, "profile": "profiles/grouped_kernel_prefill.md",
                 "sources": ["sgmv_common.cuh", "sgmv_fused.cuh", "sgmv_tmap.cuh", "sgmv_grouped_tc.cuh"],
-                "sha256": "782c566516423019f1d8c3fca6699ce82bea18ad7839cba6d761bee229f7004f"},
+                "sha256": "ac9d51d05a761e2b4057b75a73f86a10c89895e1982478c529ca7b3a8ff7df66"},
 }
 
 
