@@ -112,7 +112,8 @@ lora_sgmv_status launch_shrink(const ShrinkParams& p0, int max_len, cudaStream_t
     ShrinkParams p = p0;
     const int C = cluster_size_for(p.H1);
     p.ks = ((p.H1 + C - 1) / C + 7) / 8 * 8;
-    const size_t smem = sgmv::shrink_smem_bytes(p.ks, R);
+    p.flat = p.n_segments <= sgmv::kShrinkFlatMaxSegments ? 1 : 0;
+    const size_t smem = sgmv::shrink_smem_bytes(p.ks, R, p.flat ? p.n_segments : 0);
     DeviceFacts f;
     if (device_facts(f) != LORA_SGMV_OK) return LORA_SGMV_ERR_CUDA;
     if (smem > static_cast<size_t>(f.max_smem_optin)) return LORA_SGMV_ERR_DIM;
@@ -120,7 +121,14 @@ lora_sgmv_status launch_shrink(const ShrinkParams& p0, int max_len, cudaStream_t
     if (ensure_smem(kernel, smem, smem_granted) != LORA_SGMV_OK) return LORA_SGMV_ERR_CUDA;
 
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(C, clamp_grid_y(p.n_segments), chunk_slots(max_len, sgmv::kShrinkTokens, 8));
+    if (p.flat) {
+        // at most one chunk per token, and at most one partial chunk per segment
+        const long long units = std::min<long long>(
+            static_cast<long long>(p.n_segments) + (p.T + sgmv::kShrinkTokens - 1) / sgmv::kShrinkTokens, p.T);
+        cfg.gridDim = dim3(C, static_cast<unsigned>(std::max<long long>(1, std::min<long long>(units, 65535))), 1);
+    } else {
+        cfg.gridDim = dim3(C, clamp_grid_y(p.n_segments), chunk_slots(max_len, sgmv::kShrinkTokens, 8));
+    }
     cfg.blockDim = dim3(sgmv::kShrinkThreads, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
@@ -393,13 +401,27 @@ lora_sgmv_status launch_fused(sgmv::FusedParams P, int max_len, cudaStream_t str
 // (r x 16-token MMAs) replaces a long fp32 FMA loop; at r = 16 the CUDA-core kernel stays ahead.
 bool decode_tc_preferred(int r, int max_len) { return max_len > 2 && r >= 32; }
 
+// The split form of the tensor-core decode (V by the split-K shrink kernel, then an expand that
+// spreads each job's N over independent CTAs) pays a second launch and a V round trip through
+// the workspace, and wins when the fused form would leave SMs idle: fewer jobs than SMs, each
+// with a large B_i (several MB) to stream.
+bool split_tc_preferred(int T, int n_segments, int max_len, int H1, int H2, int r) {
+    DeviceFacts f;
+    const int sms = device_facts(f) == LORA_SGMV_OK ? f.sms : 148;
+    const long long chunks = std::min<long long>(n_segments + (T + 15) / 16, std::max(T, 1));
+    const long long jobs = max_len <= 16 ? n_segments : chunks;
+    (void)H1;
+    return jobs < sms && double(H2) * r * 2 >= 2e6;
+}
+
 bool decode_tc_supported(int r, int H1, int H2) {
     return (r == 16 || r == 32 || r == 64) && H1 >= 64 && H2 >= 64 && H1 % 64 == 0 && H2 % 64 == 0;
 }
 
 template <typename T, int R>
-lora_sgmv_status launch_decode_tc(sgmv::FusedParams P, const sgmv::DecodeMaps& maps, int max_len, cudaStream_t stream) {
-    static int smem_granted[64] = {};
+lora_sgmv_status launch_decode_tc(sgmv::FusedParams P, const sgmv::DecodeMaps& maps, int max_len, cudaStream_t stream,
+                                  const float* v_in) {
+    static int smem_granted[2][64] = {};  // per kernel mode
     // resident clusters per (device, cluster size, job-prefix size bucket)
     static int resident[64][sgmv::kFusedMaxCluster + 1][9] = {};
     using G = sgmv::DecodeTCGeom<R>;
@@ -409,7 +431,8 @@ lora_sgmv_status launch_decode_tc(sgmv::FusedParams P, const sgmv::DecodeMaps& m
     auto smem_for = [&](int C) {
         return G::BASE + size_t(C) * G::TILE + size_t(bucket) * 1024 * 4 + 1024 /* alignment slack */;
     };
-    auto kernel = sgmv::sgmv_decode_tc_kernel<T, R>;
+    // one kernel per mode: with V from the workspace, or computed by the cluster
+    auto kernel = v_in ? sgmv::sgmv_decode_tc_kernel<T, R, true> : sgmv::sgmv_decode_tc_kernel<T, R, false>;
     DeviceFacts f;
     if (device_facts(f) != LORA_SGMV_OK) return LORA_SGMV_ERR_CUDA;
     // the largest cluster whose shared memory (ring + one partial V tile per CTA of the cluster
@@ -418,7 +441,7 @@ lora_sgmv_status launch_decode_tc(sgmv::FusedParams P, const sgmv::DecodeMaps& m
     int c_fit = sgmv::kFusedMaxCluster;
     while (c_fit > 0 && smem_for(c_fit) > smem_cap) --c_fit;
     if (c_fit == 0) return LORA_SGMV_ERR_DIM;
-    if (ensure_smem(kernel, smem_for(c_fit), smem_granted) != LORA_SGMV_OK) return LORA_SGMV_ERR_CUDA;
+    if (ensure_smem(kernel, smem_for(c_fit), smem_granted[v_in ? 1 : 0]) != LORA_SGMV_OK) return LORA_SGMV_ERR_CUDA;
     int dev = 0;
     if (record(cudaGetDevice(&dev)) != cudaSuccess) return LORA_SGMV_ERR_CUDA;
     if (dev < 0 || dev >= 64) return LORA_SGMV_ERR_UNSUPPORTED;
@@ -443,6 +466,55 @@ lora_sgmv_status launch_decode_tc(sgmv::FusedParams P, const sgmv::DecodeMaps& m
         std::min<long long>(P.n_segments + (P.T + CH - 1) / CH, std::max(P.T, 1));
     const long long jobs = std::max<long long>(1, (one_chunk ? static_cast<long long>(P.n_segments) : chunks) *
                                                       P.n_problems);
+    if (v_in) {
+        // V is precomputed: each job's N is cut into S slices and the jobs x S units are walked
+        // by independent CTAs, all resident at once. Estimated time = rounds x (slice bytes at
+        // the ~24 GB/s one CTA of this kernel streams + a fixed cost per unit).
+        constexpr double kCtaBytesPerUs = 24e3;
+        constexpr double kUnitFixedUs = 3.0;
+        int resident1 = 0;
+        lora_sgmv_status st1 = resident_for(1, &resident1);
+        if (st1 != LORA_SGMV_OK) return st1;
+        resident1 = std::max(resident1, 1);
+        int s_cap = 16;
+        double job_bytes = 0;
+        for (int i = 0; i < P.n_problems; ++i) {
+            s_cap = std::min(s_cap, (P.prob[i].H2 + G::NW - 1) / G::NW);
+            job_bytes += double(P.prob[i].H2) * R * 2;
+        }
+        job_bytes /= P.n_problems;
+        s_cap = std::max(s_cap, 1);
+        int S = 1;
+        long long rounds = 1;
+        double best = 1e300;
+        for (int sl = 1; sl <= s_cap; ++sl) {
+            const long long units = jobs * sl;
+            const long long rd = (units + resident1 - 1) / resident1;
+            const double cost = double(rd) * (job_bytes / sl / kCtaBytesPerUs + kUnitFixedUs);
+            if (cost < best - 1e-9) {
+                best = cost;
+                S = sl;
+                rounds = rd;
+            }
+        }
+        P.one_chunk = one_chunk ? 1 : 0;
+        for (int i = 0; i < P.n_problems; ++i) {
+            P.prob[i].ks = 0;  // no shrink
+            P.prob[i].ns = (P.prob[i].H2 + S * G::NW - 1) / (S * G::NW) * G::NW;
+        }
+        const long long ctas = (jobs * S + rounds - 1) / rounds;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>(ctas), 1, 1);
+        cfg.blockDim = dim3(sgmv::kDThreads, 1, 1);
+        cfg.dynamicSmemBytes = smem_for(1);
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        return counted(cudaLaunchKernelEx(&cfg, kernel, maps, P, v_in, S));
+    }
     // cluster size: a cluster runs its jobs one after another, each CTA streaming 1/C of the
     // job's adapter bytes; estimated time = rounds * (bytes per CTA / per-CTA bandwidth + a fixed
     // cost per job for metadata, map setup, pipeline fill and the V exchange). Every CTA keeps at
@@ -498,11 +570,12 @@ lora_sgmv_status launch_decode_tc(sgmv::FusedParams P, const sgmv::DecodeMaps& m
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    return counted(cudaLaunchKernelEx(&cfg, kernel, maps, P));
+    return counted(cudaLaunchKernelEx(&cfg, kernel, maps, P, static_cast<const float*>(nullptr), 1));
 }
 
 template <int R>
-lora_sgmv_status decode_tc_maps_and_launch(sgmv::FusedParams& P, lora_sgmv_dtype dt, int max_len, cudaStream_t s) {
+lora_sgmv_status decode_tc_maps_and_launch(sgmv::FusedParams& P, lora_sgmv_dtype dt, int max_len, cudaStream_t s,
+                                           const float* v_in) {
     sgmv::DecodeMaps maps;
     std::memset(&maps, 0, sizeof(maps));
     for (int i = 0; i < P.n_problems; ++i)
@@ -510,15 +583,16 @@ lora_sgmv_status decode_tc_maps_and_launch(sgmv::FusedParams& P, lora_sgmv_dtype
             t_last_error = cudaErrorInvalidValue;
             return LORA_SGMV_ERR_CUDA;
         }
-    return dt == LORA_SGMV_BF16 ? launch_decode_tc<__nv_bfloat16, R>(P, maps, max_len, s)
-                                : launch_decode_tc<__half, R>(P, maps, max_len, s);
+    return dt == LORA_SGMV_BF16 ? launch_decode_tc<__nv_bfloat16, R>(P, maps, max_len, s, v_in)
+                                : launch_decode_tc<__half, R>(P, maps, max_len, s, v_in);
 }
 
-lora_sgmv_status decode_tc_dispatch(sgmv::FusedParams& P, int r, lora_sgmv_dtype dt, int max_len, cudaStream_t s) {
+lora_sgmv_status decode_tc_dispatch(sgmv::FusedParams& P, int r, lora_sgmv_dtype dt, int max_len, cudaStream_t s,
+                                    const float* v_in = nullptr) {
     switch (r) {
-        case 16: return decode_tc_maps_and_launch<16>(P, dt, max_len, s);
-        case 32: return decode_tc_maps_and_launch<32>(P, dt, max_len, s);
-        case 64: return decode_tc_maps_and_launch<64>(P, dt, max_len, s);
+        case 16: return decode_tc_maps_and_launch<16>(P, dt, max_len, s, v_in);
+        case 32: return decode_tc_maps_and_launch<32>(P, dt, max_len, s, v_in);
+        case 64: return decode_tc_maps_and_launch<64>(P, dt, max_len, s, v_in);
     }
     return LORA_SGMV_ERR_UNSUPPORTED;
 }
@@ -565,7 +639,8 @@ int32_t lora_sgmv_rank_supported(int32_t r, lora_sgmv_variant variant) {
         case LORA_SGMV_VARIANT_SPLIT: return split_rank(r) ? 1 : 0;
         case LORA_SGMV_VARIANT_GROUPED_TC: return sgmv::grouped_tc_rank(r) ? 1 : 0;
         case LORA_SGMV_VARIANT_FUSED: return split_rank(r) ? 1 : 0;
-        case LORA_SGMV_VARIANT_FUSED_TC: return (r == 16 || r == 32 || r == 64) ? 1 : 0;
+        case LORA_SGMV_VARIANT_FUSED_TC:
+        case LORA_SGMV_VARIANT_SPLIT_TC: return (r == 16 || r == 32 || r == 64) ? 1 : 0;
     }
     return 0;
 }
@@ -686,7 +761,7 @@ lora_sgmv_status lora_sgmv_apply_ex(void* Y, const void* X, const void* const* A
     if (H1 <= 0 || H2 <= 0 || r <= 0) return LORA_SGMV_ERR_DIM;
     if (variant != LORA_SGMV_VARIANT_AUTO && variant != LORA_SGMV_VARIANT_SPLIT &&
         variant != LORA_SGMV_VARIANT_GROUPED_TC && variant != LORA_SGMV_VARIANT_FUSED &&
-        variant != LORA_SGMV_VARIANT_FUSED_TC)
+        variant != LORA_SGMV_VARIANT_FUSED_TC && variant != LORA_SGMV_VARIANT_SPLIT_TC)
         return LORA_SGMV_ERR_UNSUPPORTED;
     if (!lora_sgmv_rank_supported(r, variant)) return LORA_SGMV_ERR_UNSUPPORTED;
     if (n_segments == 0 || T == 0) return LORA_SGMV_OK;
@@ -706,11 +781,13 @@ lora_sgmv_status lora_sgmv_apply_ex(void* Y, const void* X, const void* const* A
                 : (n_segments > sgmv::kFusedMaxSegments
                        ? LORA_SGMV_VARIANT_SPLIT
                        : (decode_tc_preferred(r, max_len) && decode_tc_supported(r, H1, H2)
-                              ? LORA_SGMV_VARIANT_FUSED_TC
+                              ? (split_tc_preferred(T, n_segments, max_len, H1, H2, r) ? LORA_SGMV_VARIANT_SPLIT_TC
+                                                                                      : LORA_SGMV_VARIANT_FUSED_TC)
                               : LORA_SGMV_VARIANT_FUSED));
 
-    if (v == LORA_SGMV_VARIANT_FUSED || v == LORA_SGMV_VARIANT_FUSED_TC) {
-        if (v == LORA_SGMV_VARIANT_FUSED_TC && !decode_tc_supported(r, H1, H2)) return LORA_SGMV_ERR_UNSUPPORTED;
+    if (v == LORA_SGMV_VARIANT_FUSED || v == LORA_SGMV_VARIANT_FUSED_TC || v == LORA_SGMV_VARIANT_SPLIT_TC) {
+        if ((v == LORA_SGMV_VARIANT_FUSED_TC || v == LORA_SGMV_VARIANT_SPLIT_TC) && !decode_tc_supported(r, H1, H2))
+            return LORA_SGMV_ERR_UNSUPPORTED;
         sgmv::FusedParams P = {};
         P.prob[0].Y = Y;
         P.prob[0].X = X;
@@ -727,6 +804,26 @@ lora_sgmv_status lora_sgmv_apply_ex(void* Y, const void* X, const void* const* A
         P.n_segments = n_segments;
         P.T = T;
         if (v == LORA_SGMV_VARIANT_FUSED_TC) return decode_tc_dispatch(P, r, dtype, max_len, s);
+        if (v == LORA_SGMV_VARIANT_SPLIT_TC) {
+            // V first (split-K shrink kernel, fp32 into the workspace), then the expand spread
+            // over every SM, each job's N split among independent CTAs
+            float* V = static_cast<float*>(workspace);
+            ShrinkParams sp = {};
+            sp.V = V;
+            sp.X = X;
+            sp.A_ptrs = A_ptrs;
+            sp.B_check = B_ptrs;
+            sp.seg_starts = seg_starts;
+            sp.lora_idx = lora_idx;
+            sp.dev_status = dev_status;
+            sp.n_segments = n_segments;
+            sp.num_adapters = num_adapters;
+            sp.T = T;
+            sp.H1 = H1;
+            st = shrink_dispatch(sp, r, dtype, max_len, s);
+            if (st != LORA_SGMV_OK) return st;
+            return decode_tc_dispatch(P, r, dtype, max_len, s, V);
+        }
         return fused_dispatch(P, r, dtype, max_len, s);
     }
 

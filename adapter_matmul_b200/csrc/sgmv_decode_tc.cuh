@@ -150,17 +150,25 @@ __device__ __forceinline__ void epilogue_bar() { asm volatile("bar.sync 1, 128;"
 // a chunk starts at row offset nt & ~(2^(m+1) - 1).
 
 
-template <typename T, int R>
+template <typename T, int R, bool PRE_V>
 __global__ void __launch_bounds__(kDThreads, 1)
-    sgmv_decode_tc_kernel(const __grid_constant__ DecodeMaps maps, const FusedParams P) {
+    sgmv_decode_tc_kernel(const __grid_constant__ DecodeMaps maps, const FusedParams P, const float* v_in,
+                          int n_slices) {
     using G = DecodeTCGeom<R>;
     constexpr int S = G::STAGES;
     constexpr int SY = kDYStages;
     constexpr int ND2 = G::ND2;
     extern __shared__ __align__(1024) unsigned char dsm_raw[];
     unsigned char* dsm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
-    const int C = static_cast<int>(cluster_size());
-    const int c = static_cast<int>(cluster_rank());
+    // PRE_V false: a cluster of C CTAs splits each job's K (shrink, V exchanged on chip) and
+    // N, and the clusters walk the entries (v_in and n_slices unused). PRE_V true: V [T, r]
+    // (fp32, v_in) was computed by an earlier kernel and the shrink is skipped; each entry's N is
+    // cut into n_slices slices and every (entry, slice) pair is a unit of work, walked by
+    // independent CTAs (no cluster).
+    constexpr bool pre_v = PRE_V;
+    const int C = pre_v ? 1 : static_cast<int>(cluster_size());
+    const int c = pre_v ? 0 : static_cast<int>(cluster_rank());
+    const int n_sl = pre_v ? n_slices : 1;
     unsigned char* ring = dsm;
     unsigned char* yring = ring + S * G::STAGE;
     unsigned char* vt = yring + SY * G::Y_BYTES;                  // V^T operand: [V_hi rows | V_lo rows]
@@ -173,7 +181,7 @@ __global__ void __launch_bounds__(kDThreads, 1)
     __shared__ uint32_t tmem_base_s;
     __shared__ int table_s;
 
-    const int cluster_id = blockIdx.x / C;
+    const int cluster_id = blockIdx.x / C;  // in pre-V mode: the CTA
     const int n_clusters = gridDim.x / C;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -241,12 +249,14 @@ __global__ void __launch_bounds__(kDThreads, 1)
             deferred = 0;
             __syncwarp();
         };
-        for (int j = cluster_id; j < entries; j += n_clusters) {
+        for (int w = cluster_id; w < entries * n_sl; w += n_clusters) {
+            const int j = pre_v ? w / n_sl : w;
+            const int cw = pre_v ? w - j * n_sl : c;  // N slice (and K slice)
             int p, s, q0, nq;
             entry_at<kDTokens>(P, pref, j, p, s, q0, nq);
             for (int q = q0; q < q0 + nq; ++q) {
                 Job job;
-                if (!job_at<kDTokens>(P, p, s, q, c, job)) break;
+                if (!job_at<kDTokens>(P, p, s, q, cw, job)) break;
                 const int nA = (job.nk + G::KS - 1) / G::KS;
                 const int nB = (job.nc + G::NW - 1) / G::NW;
                 if (nA + nB == 0) continue;
@@ -330,12 +340,14 @@ __global__ void __launch_bounds__(kDThreads, 1)
         // above never waits for the epilogue
         pdl_wait();
         uint32_t yit = 0;
-        for (int j = cluster_id; j < entries; j += n_clusters) {
+        for (int w = cluster_id; w < entries * n_sl; w += n_clusters) {
+            const int j = pre_v ? w / n_sl : w;
+            const int cw = pre_v ? w - j * n_sl : c;  // N slice (and K slice)
             int p, s, q0, nq;
             entry_at<kDTokens>(P, pref, j, p, s, q0, nq);
             for (int q = q0; q < q0 + nq; ++q) {
                 Job job;
-                if (!job_at<kDTokens>(P, p, s, q, c, job)) break;
+                if (!job_at<kDTokens>(P, p, s, q, cw, job)) break;
                 const int nB = (job.nc + G::NW - 1) / G::NW;
                 for (int tb = 0; tb < nB; ++tb, ++yit) {
                     const uint32_t sy = yit % SY;
@@ -368,12 +380,14 @@ __global__ void __launch_bounds__(kDThreads, 1)
         // B tile MN-major, V^T K-major with N = 32: columns 0..15 of D2 take V_hi, 16..31 V_lo
         const uint32_t idesc_e = instr_desc(fmt, 1, 0, 2 * kDTokens, kGM);
         uint32_t it = 0, u = 0, g = 0;
-        for (int j = cluster_id; j < entries; j += n_clusters) {
+        for (int w = cluster_id; w < entries * n_sl; w += n_clusters) {
+            const int j = pre_v ? w / n_sl : w;
+            const int cw = pre_v ? w - j * n_sl : c;  // N slice (and K slice)
             int p, s, q0, nq;
             entry_at<kDTokens>(P, pref, j, p, s, q0, nq);
             for (int q = q0; q < q0 + nq; ++q) {
                 Job job;
-                if (!job_at<kDTokens>(P, p, s, q, c, job)) break;
+                if (!job_at<kDTokens>(P, p, s, q, cw, job)) break;
                 const int nA = (job.nk + G::KS - 1) / G::KS;
                 const int nB = (job.nc + G::NW - 1) / G::NW;
                 for (int ta = 0; ta < nA; ++ta, ++it) {
@@ -436,12 +450,14 @@ __global__ void __launch_bounds__(kDThreads, 1)
         const uint32_t lane_base = tmem + (uint32_t(quarter * 32) << 16);
         if (C > 1) cluster_wait();
         uint32_t yit = 0, u = 0, g = 0;
-        for (int j = cluster_id; j < entries; j += n_clusters) {
+        for (int w = cluster_id; w < entries * n_sl; w += n_clusters) {
+            const int j = pre_v ? w / n_sl : w;
+            const int cw = pre_v ? w - j * n_sl : c;  // N slice (and K slice)
             int p, s, q0, nq;
             entry_at<kDTokens>(P, pref, j, p, s, q0, nq);
             for (int q = q0; q < q0 + nq; ++q) {
                 Job job;
-                if (!job_at<kDTokens>(P, p, s, q, c, job)) break;
+                if (!job_at<kDTokens>(P, p, s, q, cw, job)) break;
                 const FusedProblem& pr = P.prob[job.p];
                 const int nA = (job.nk + G::KS - 1) / G::KS;
                 const int nB = (job.nc + G::NW - 1) / G::NW;
@@ -449,52 +465,80 @@ __global__ void __launch_bounds__(kDThreads, 1)
                     // partial V of this CTA: D1 rows 0..nt-1 (lanes 0..15 of quarter 0)
                     mbar_wait<false>(&d1_full, u & 1u, P.dev_status, dead);
                     tc_fence_after();
-                    float v[R];
-                    tmem_ld_row<R>(lane_base, v);
-                    if (nA == 0) {
+                    // V^T operand rows: token `lane`, 8 values of chunk ch, K-major swizzled; hi + lo
+                    auto put_v8 = [&](int ch, const float* x8) {
+                        float hi[8], lo[8];
 #pragma unroll
-                        for (int i = 0; i < R; ++i) v[i] = 0.f;
-                    }
-                    const uint32_t tile_bytes = uint32_t(job.nt) * R * 4;
-                    if (lane == 0) mbar_arrive_expect_tx(&vready, tile_bytes * C);
-                    if (u >= 1) mbar_wait<true>(&vfree, (u - 1) & 1u, P.dev_status, dead);
-                    if (lane < job.nt) {
-                        float* slot = recv + (size_t(c) * kDTokens + lane) * R;
-                        for (int qr = 0; qr < C; ++qr)
-#pragma unroll
-                            for (int i = 0; i < R; i += 4)
-                                st_async_v4(slot + i, make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]), &vready, qr);
-                    }
-                    mbar_wait<true>(&vready, u & 1u, P.dev_status, dead);
-#pragma unroll
-                    for (int i = 0; i < R; ++i) v[i] = 0.f;  // rows past the chunk: V^T columns of zeros
-                    if (lane < job.nt) {
-                        for (int qr = 0; qr < C; ++qr) {
-                            const float* src = recv + (size_t(qr) * kDTokens + lane) * R;
-#pragma unroll
-                            for (int i = 0; i < R; ++i) v[i] += src[i];
+                        for (int i = 0; i < 8; ++i) {
+                            hi[i] = Storage<T>::round(x8[i]);
+                            lo[i] = x8[i] - hi[i];
                         }
-                    }
-                    if (lane < kDTokens) {
-                        // V^T operand rows: token `lane`, R values, K-major swizzled; hi + lo
+                        st_vec(vt + swz(lane, ch, G::SW_BITS), pack8<T>(hi));
+                        st_vec(vt + swz(kDTokens + lane, ch, G::SW_BITS), pack8<T>(lo));
+                    };
+                    if (pre_v) {
+                        // V rows of the chunk from the earlier kernel (read once it has completed);
+                        // rows past the chunk are V^T columns of zeros
+                        pdl_wait();
+                        if (lane < kDTokens) {
+                            const float4* src = reinterpret_cast<const float4*>(v_in + size_t(job.t0 + lane) * R);
 #pragma unroll
-                        for (int ch = 0; ch < R / 8; ++ch) {
-                            float hi[8], lo[8];
-#pragma unroll
-                            for (int i = 0; i < 8; ++i) {
-                                hi[i] = Storage<T>::round(v[ch * 8 + i]);
-                                lo[i] = v[ch * 8 + i] - hi[i];
+                            for (int ch = 0; ch < R / 8; ++ch) {
+                                float x8[8];
+                                const float4 a = lane < job.nt ? src[2 * ch] : make_float4(0.f, 0.f, 0.f, 0.f);
+                                const float4 b = lane < job.nt ? src[2 * ch + 1] : make_float4(0.f, 0.f, 0.f, 0.f);
+                                x8[0] = a.x, x8[1] = a.y, x8[2] = a.z, x8[3] = a.w;
+                                x8[4] = b.x, x8[5] = b.y, x8[6] = b.z, x8[7] = b.w;
+                                put_v8(ch, x8);
                             }
-                            const uint32_t off = swz(lane, ch, G::SW_BITS);
-                            st_vec(vt + off, pack8<T>(hi));
-                            st_vec(vt + swz(kDTokens + lane, ch, G::SW_BITS), pack8<T>(lo));
+                        }
+                    } else {
+                        float v[R];
+                        tmem_ld_row<R>(lane_base, v);
+                        if (nA == 0) {
+#pragma unroll
+                            for (int i = 0; i < R; ++i) v[i] = 0.f;
+                        }
+                        const uint32_t tile_bytes = uint32_t(job.nt) * R * 4;
+                        if (lane == 0) mbar_arrive_expect_tx(&vready, tile_bytes * C);
+                        if (u >= 1) mbar_wait<true>(&vfree, (u - 1) & 1u, P.dev_status, dead);
+                        if (lane < job.nt) {
+                            float* slot = recv + (size_t(c) * kDTokens + lane) * R;
+                            for (int qr = 0; qr < C; ++qr)
+#pragma unroll
+                                for (int i = 0; i < R; i += 4)
+                                    st_async_v4(slot + i, make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]), &vready,
+                                                qr);
+                        }
+                        mbar_wait<true>(&vready, u & 1u, P.dev_status, dead);
+#pragma unroll
+                        for (int i = 0; i < R; ++i) v[i] = 0.f;  // rows past the chunk: V^T columns of zeros
+                        if (lane < job.nt) {
+                            for (int qr = 0; qr < C; ++qr) {
+                                const float* src = recv + (size_t(qr) * kDTokens + lane) * R;
+#pragma unroll
+                                for (int i = 0; i < R; ++i) v[i] += src[i];
+                            }
+                        }
+                        if (lane < kDTokens) {
+#pragma unroll
+                            for (int ch = 0; ch < R / 8; ++ch) {
+                                float hi[8], lo[8];
+#pragma unroll
+                                for (int i = 0; i < 8; ++i) {
+                                    hi[i] = Storage<T>::round(v[ch * 8 + i]);
+                                    lo[i] = v[ch * 8 + i] - hi[i];
+                                }
+                                st_vec(vt + swz(lane, ch, G::SW_BITS), pack8<T>(hi));
+                                st_vec(vt + swz(kDTokens + lane, ch, G::SW_BITS), pack8<T>(lo));
+                            }
                         }
                     }
                     fence_proxy_async();
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive_local(&v_full);
-                    if (lane < C) mbar_arrive_remote(&vfree, static_cast<uint32_t>(lane));
+                    if (!pre_v && lane < C) mbar_arrive_remote(&vfree, static_cast<uint32_t>(lane));
                 }
                 // expand epilogue: this warp's 32 columns of each 128-column group, all tokens,
                 // kDEpiBatch stages per pass: whatever a pass waits for after its Y stores is paid
@@ -550,7 +594,7 @@ __global__ void __launch_bounds__(kDThreads, 1)
         }
         if (quarter == 0 && half == 0) {
             pdl_wait();
-            if (u >= 1) mbar_wait<true>(&vfree, (u - 1) & 1u, P.dev_status, dead);
+            if (!pre_v && u >= 1) mbar_wait<true>(&vfree, (u - 1) & 1u, P.dev_status, dead);
             if (c == 0 && lane == 0) {  // report each rejected segment once
                 for (int j = cluster_id; j < P.n_problems * P.n_segments; j += n_clusters) {
                     const int p2 = j / P.n_segments, s2 = j - p2 * P.n_segments;

@@ -5,11 +5,14 @@
 // [r, H2], rows are tokens; the batch form (multi-LoRA paragraph) maps each
 // segment of rows to its own adapter.
 //
-// Shrink. One thread-block cluster of C CTAs per (segment, token-chunk slot).
+// Shrink. One thread-block cluster of C CTAs per token chunk (8 tokens of one segment;
+// the clusters walk a flat list of the chunks, or segment and chunk slots when there are
+// too many segments for the list's prefix to fit in shared memory).
 // CTA c of the cluster owns rows [c*KS, (c+1)*KS) of A_i; that slice of A_i
 // is one contiguous run of KS*r*2 bytes, read once with 128-bit coalesced
 // loads. Each CTA stages its slice of the chunk's X rows in shared memory,
-// accumulates fp32 partial sums per thread, reduces them with warp shuffles
+// accumulates fp32 partial sums per thread (one token row for a one-token chunk, with twice
+// the loads of A_i in flight, else eight), reduces them with warp shuffles
 // and then across warps in shared memory. The C partial V tiles are summed in
 // a fixed order through distributed shared memory (DSMEM), and each CTA
 // stores its share of the reduced V with plain stores: no atomics, no
@@ -45,7 +48,8 @@ struct ShrinkParams {
     int num_adapters;
     int T;
     int H1;
-    int ks;  // rows of A_i per CTA, multiple of 8
+    int ks;    // rows of A_i per CTA, multiple of 8
+    int flat;  // 1: grid over the flat (segment, chunk) list (shared memory holds its prefix)
 };
 
 struct ExpandParams {
@@ -69,28 +73,134 @@ constexpr int kShrinkUnroll = 8;   // 16-byte loads in flight per thread
 constexpr int kExpandThreads = 128;
 constexpr int kExpandTokens = 8;
 
-__host__ __device__ constexpr size_t shrink_smem_bytes(int ks, int R) {
+constexpr int kShrinkFlatMaxSegments = 8192;  // flat grid: the chunk prefix fits in shared memory
+
+__host__ __device__ constexpr size_t shrink_smem_bytes(int ks, int R, int flat_segments = 0) {
     // X slice [TC][ks] (16-bit) + per-warp partials [NW][TC*R] + CTA partial [TC*R]
+    // (+ flat grid: chunk prefix [n_segments + 1] and per-warp totals [NW])
     return size_t(kShrinkTokens) * ks * 2 + size_t(kShrinkThreads / 32) * kShrinkTokens * R * 4 +
-           size_t(kShrinkTokens) * R * 4;
+           size_t(kShrinkTokens) * R * 4 +
+           (flat_segments > 0 ? size_t(flat_segments + 1 + kShrinkThreads / 32) * 4 : 0);
 }
 
-// grid: x = C (one cluster along x), y = segment slots, z = token-chunk slots.
+// One token chunk [t0, t0 + nt) of a segment, this CTA's rows [k0, k0 + nk) of its A_i:
+// stage the chunk's X slice, accumulate TCN token rows (rows past nt are zero) with U
+// 16-byte loads of A_i in flight per thread, reduce over the CTA, sum the C partial tiles
+// across the cluster in rank order and store this CTA's share of V. Every CTA of the cluster
+// calls it for the same chunk.
+template <typename T, int R, int TCN, int U>
+__device__ __forceinline__ void shrink_chunk(const ShrinkParams& p, cg::cluster_group& cluster, const T* __restrict__ A,
+                                             int t0, int nt, int k0, int nk, T* xs, float* red, float* part) {
+    constexpr int NT = kShrinkThreads;
+    constexpr int G = R / 8;     // 16-byte vectors per row of A_i
+    constexpr int RL = NT / G;   // row lanes
+    constexpr int NW = NT / 32;
+    const int tid = threadIdx.x;
+    const int lane = tid & 31;
+    const int warp = tid >> 5;
+    const int cgi = tid % G;
+    const int rl = tid / G;
+    const int KS = p.ks;
+    const int c = static_cast<int>(cluster.block_rank());
+    const int C = static_cast<int>(cluster.num_blocks());
+    const T* __restrict__ X = static_cast<const T*>(p.X);
+
+    // stage X[t0 .. t0+TCN, k0 .. k0+nk) (rows past the chunk are zero)
+    const int vpr = nk / 8;
+    for (int v = tid; v < TCN * vpr; v += NT) {
+        const int row = v / vpr;
+        const int col = (v - row * vpr) * 8;
+        uint4 val = make_uint4(0, 0, 0, 0);
+        if (row < nt) val = ld_vec(X + size_t(t0 + row) * p.H1 + k0 + col);
+        st_vec(xs + size_t(row) * KS + col, val);
+    }
+    __syncthreads();
+
+    float acc[TCN][8];
+#pragma unroll
+    for (int t = 0; t < TCN; ++t)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[t][i] = 0.f;
+
+    for (int kb = rl; kb < nk; kb += RL * U) {
+        uint4 av[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int kr = kb + u * RL;
+            av[u] = kr < nk ? ld_stream(A + size_t(k0 + kr) * R + cgi * 8) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int kr = kb + u * RL;
+            if (kr < nk) {
+                float a[8];
+                unpack8<T>(av[u], a);
+#pragma unroll
+                for (int t = 0; t < TCN; ++t) {
+                    const float x = Storage<T>::to1(xs[size_t(t) * KS + kr]);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) acc[t][i] = fmaf(x, a[i], acc[t][i]);
+                }
+            }
+        }
+    }
+    // reduce over the row lanes of this warp (lanes sharing cgi)
+#pragma unroll
+    for (int off = G; off < 32; off <<= 1)
+#pragma unroll
+        for (int t = 0; t < TCN; ++t)
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc[t][i] += __shfl_xor_sync(0xffffffffu, acc[t][i], off);
+    if (lane < G) {
+#pragma unroll
+        for (int t = 0; t < TCN; ++t)
+#pragma unroll
+            for (int i = 0; i < 8; ++i) red[(warp * TCN + t) * R + cgi * 8 + i] = acc[t][i];
+    }
+    __syncthreads();
+    for (int e = tid; e < TCN * R; e += NT) {
+        float sum = 0.f;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) sum += red[w * TCN * R + e];
+        part[e] = sum;
+    }
+    // sum the C partial tiles across the cluster in rank order
+    cluster.sync();
+    const int per = (TCN * R + C - 1) / C;
+    const int e0 = c * per;
+    const int e1 = min(e0 + per, TCN * R);
+    for (int e = e0 + tid; e < e1; e += NT) {
+        float sum = 0.f;
+        for (int qr = 0; qr < C; ++qr) sum += cluster.map_shared_rank(part, qr)[e];
+        const int t = e / R;
+        const int j = e - t * R;
+        if (t < nt) p.V[size_t(t0 + t) * R + j] = sum;
+    }
+    cluster.sync();  // partial tiles and the X slice may be overwritten only after every read
+}
+
+// Token chunks of segment s (0 for a segment the checks reject).
+__device__ __forceinline__ int shrink_segment_chunks(const ShrinkParams& p, int s) {
+    Segment seg;
+    if (load_segment(p.seg_starts, p.lora_idx, p.A_ptrs, p.B_check, s, p.T, p.num_adapters, seg)) return 0;
+    return (seg.end - seg.begin + kShrinkTokens - 1) / kShrinkTokens;
+}
+
+// Two grids. p.flat == 0: x = C (one cluster along x), y = segment slots, z = token-chunk
+// slots. p.flat == 1: x = C, y = slots over the flat list of (segment, chunk) units, z = 1;
+// every CTA builds the list's prefix (chunks before each segment) in shared memory, so the
+// grid holds no CTA without a chunk.
 template <typename T, int R>
 __global__ void __launch_bounds__(kShrinkThreads) sgmv_shrink_cluster_kernel(const ShrinkParams p) {
     constexpr int NT = kShrinkThreads;
     constexpr int TC = kShrinkTokens;
-    constexpr int G = R / 8;     // 16-byte vectors per row of A_i
-    constexpr int RL = NT / G;   // row lanes
+    constexpr int G = R / 8;
     constexpr int NW = NT / 32;
     static_assert(R % 8 == 0 && G <= 32 && (32 % G) == 0, "rank must be 8..256, power of two");
 
     cg::cluster_group cluster = cg::this_cluster();
     const int c = static_cast<int>(cluster.block_rank());
-    const int C = static_cast<int>(cluster.num_blocks());
     const int tid = threadIdx.x;
-    const int lane = tid & 31;
-    const int warp = tid >> 5;
 
     extern __shared__ __align__(128) unsigned char smem[];
     T* xs = reinterpret_cast<T*>(smem);
@@ -100,12 +210,67 @@ __global__ void __launch_bounds__(kShrinkThreads) sgmv_shrink_cluster_kernel(con
     // The expand kernel may be scheduled as soon as every shrink CTA is running.
     pdl_launch_dependents();
 
-    const int KS = p.ks;
-    const int k0 = c * KS;
-    const int nk = max(0, min(k0 + KS, p.H1) - k0);
-    const int cgi = tid % G;
-    const int rl = tid / G;
-    const T* __restrict__ X = static_cast<const T*>(p.X);
+    const int k0 = c * p.ks;
+    const int nk = max(0, min(k0 + p.ks, p.H1) - k0);
+    auto run_chunk = [&](const T* A, int t0, int nt) {
+        if (nt == 1)
+            shrink_chunk<T, R, 1, 2 * kShrinkUnroll>(p, cluster, A, t0, nt, k0, nk, xs, red, part);
+        else
+            shrink_chunk<T, R, TC, kShrinkUnroll>(p, cluster, A, t0, nt, k0, nk, xs, red, part);
+    };
+
+    if (p.flat) {
+        int* pref = reinterpret_cast<int*>(part + TC * R);  // n_segments + 1 entries
+        int* wtot = pref + p.n_segments + 1;                // NW entries
+        const int n = p.n_segments;
+        const int per_thr = (n + NT - 1) / NT;
+        const int s0 = min(n, tid * per_thr), s1 = min(n, s0 + per_thr);
+        int local = 0;
+        for (int s = s0; s < s1; ++s) {  // chunk counts, parked in the prefix slots
+            const int k = shrink_segment_chunks(p, s);
+            pref[s + 1] = k;
+            local += k;
+        }
+        const int lane = tid & 31, warp = tid >> 5;
+        int v = local;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, v, off);
+            if (lane >= off) v += y;
+        }
+        if (lane == 31) wtot[warp] = v;
+        __syncthreads();
+        int run = v - local;
+        for (int w = 0; w < warp; ++w) run += wtot[w];
+        if (tid == 0) pref[0] = 0;
+        for (int s = s0; s < s1; ++s) {
+            run += pref[s + 1];
+            pref[s + 1] = run;
+        }
+        __syncthreads();
+        const int total = pref[n];
+        for (int u = blockIdx.y; u < total; u += gridDim.y) {
+            int lo = 0, hi = n;  // largest s with pref[s] <= u
+            while (hi - lo > 1) {
+                const int mid = (lo + hi) >> 1;
+                if (pref[mid] <= u)
+                    lo = mid;
+                else
+                    hi = mid;
+            }
+            Segment seg;
+            load_segment(p.seg_starts, p.lora_idx, p.A_ptrs, p.B_check, lo, p.T, p.num_adapters, seg);
+            const int t0 = seg.begin + (u - pref[lo]) * TC;
+            run_chunk(static_cast<const T*>(seg.a), t0, min(TC, seg.end - t0));
+        }
+        if (c == 0 && tid == 0)  // report each rejected segment once
+            for (int s = blockIdx.y; s < n; s += gridDim.y) {
+                Segment seg;
+                report(p.dev_status, load_segment(p.seg_starts, p.lora_idx, p.A_ptrs, p.B_check, s, p.T,
+                                                  p.num_adapters, seg));
+            }
+        return;
+    }
 
     for (int s = blockIdx.y; s < p.n_segments; s += gridDim.y) {
         Segment seg;
@@ -115,84 +280,10 @@ __global__ void __launch_bounds__(kShrinkThreads) sgmv_shrink_cluster_kernel(con
             if (c == 0 && blockIdx.z == 0 && tid == 0) report(p.dev_status, bad);
             continue;
         }
-        const T* __restrict__ A = static_cast<const T*>(seg.a);
-        const int L = seg.end - seg.begin;
-        const int nchunks = (L + TC - 1) / TC;
+        const int nchunks = (seg.end - seg.begin + TC - 1) / TC;
         for (int q = blockIdx.z; q < nchunks; q += gridDim.z) {
             const int t0 = seg.begin + q * TC;
-            const int nt = min(TC, seg.end - t0);
-            // stage X[t0 .. t0+TC, k0 .. k0+nk) (rows past the chunk are zero)
-            const int vpr = nk / 8;
-            for (int v = tid; v < TC * vpr; v += NT) {
-                const int row = v / vpr;
-                const int col = (v - row * vpr) * 8;
-                uint4 val = make_uint4(0, 0, 0, 0);
-                if (row < nt) val = ld_vec(X + size_t(t0 + row) * p.H1 + k0 + col);
-                st_vec(xs + size_t(row) * KS + col, val);
-            }
-            __syncthreads();
-
-            float acc[TC][8];
-#pragma unroll
-            for (int t = 0; t < TC; ++t)
-#pragma unroll
-                for (int i = 0; i < 8; ++i) acc[t][i] = 0.f;
-
-            for (int kb = rl; kb < nk; kb += RL * kShrinkUnroll) {
-                uint4 av[kShrinkUnroll];
-#pragma unroll
-                for (int u = 0; u < kShrinkUnroll; ++u) {
-                    const int kr = kb + u * RL;
-                    av[u] = kr < nk ? ld_stream(A + size_t(k0 + kr) * R + cgi * 8) : make_uint4(0, 0, 0, 0);
-                }
-#pragma unroll
-                for (int u = 0; u < kShrinkUnroll; ++u) {
-                    const int kr = kb + u * RL;
-                    if (kr < nk) {
-                        float a[8];
-                        unpack8<T>(av[u], a);
-#pragma unroll
-                        for (int t = 0; t < TC; ++t) {
-                            const float x = Storage<T>::to1(xs[size_t(t) * KS + kr]);
-#pragma unroll
-                            for (int i = 0; i < 8; ++i) acc[t][i] = fmaf(x, a[i], acc[t][i]);
-                        }
-                    }
-                }
-            }
-            // reduce over the row lanes of this warp (lanes sharing cgi)
-#pragma unroll
-            for (int off = G; off < 32; off <<= 1)
-#pragma unroll
-                for (int t = 0; t < TC; ++t)
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) acc[t][i] += __shfl_xor_sync(0xffffffffu, acc[t][i], off);
-            if (lane < G) {
-#pragma unroll
-                for (int t = 0; t < TC; ++t)
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) red[(warp * TC + t) * R + cgi * 8 + i] = acc[t][i];
-            }
-            __syncthreads();
-            for (int e = tid; e < TC * R; e += NT) {
-                float sum = 0.f;
-#pragma unroll
-                for (int w = 0; w < NW; ++w) sum += red[w * TC * R + e];
-                part[e] = sum;
-            }
-            // sum the C partial tiles across the cluster in rank order
-            cluster.sync();
-            const int per = (TC * R + C - 1) / C;
-            const int e0 = c * per;
-            const int e1 = min(e0 + per, TC * R);
-            for (int e = e0 + tid; e < e1; e += NT) {
-                float sum = 0.f;
-                for (int qr = 0; qr < C; ++qr) sum += cluster.map_shared_rank(part, qr)[e];
-                const int t = e / R;
-                const int j = e - t * R;
-                if (t < nt) p.V[size_t(t0 + t) * R + j] = sum;
-            }
-            cluster.sync();  // partial tiles may be overwritten / freed only after every read
+            run_chunk(static_cast<const T*>(seg.a), t0, min(TC, seg.end - t0));
         }
     }
 }

@@ -27,6 +27,7 @@ VARIANT_SPLIT = 1
 VARIANT_GROUPED_TC = 2
 VARIANT_FUSED = 3
 VARIANT_FUSED_TC = 4
+VARIANT_SPLIT_TC = 5
 MAX_PROBLEMS = 8
 
 DEV_BAD_SEGMENT = 0x1

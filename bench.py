@@ -390,20 +390,28 @@ def run_ours(args, spec: Spec, rank: int, world: int, local: int):
     if st != 0:
         raise RuntimeError(f"device status {st:#x}: a segment was rejected")
 
-    # ---- roofline of the dominant (here: only) kernel, per launch ----
+    # ---- roofline of the dominant kernel, per launch ----
+    # One launch per call: that kernel. Several launches per call (the split forms: a shrink
+    # kernel, then an expand kernel): the whole call, its algorithmic bytes over its duration.
     hbm, tc, which = peaks()
     bytes_call = w.algorithmic_bytes()
-    bytes_launch = bytes_call * spec.P // launches_per_step
-    launch_s = ms_per_step / 1e3 / launches_per_step
+    if launches_per_step > spec.P:
+        bytes_launch = bytes_call
+        launch_s = ms_per_step / 1e3 / spec.P
+        kernel_name = ("lora_sgmv_apply, dispatcher's choice: %d launches per call, roofline over the whole call"
+                       % (launches_per_step // spec.P))
+    else:
+        bytes_launch = bytes_call * spec.P // launches_per_step
+        launch_s = ms_per_step / 1e3 / launches_per_step
+        kernel_name = ("sgmv_fused_kernel (lora_sgmv_apply_batched: %d projections per launch)" % spec.P
+                       if spec.P > 1 else "lora_sgmv_apply kernels (dispatcher's choice)")
     achieved = bytes_launch / launch_s / 1e9
-    kernel_name = ("sgmv_fused_kernel (lora_sgmv_apply_batched: %d projections per launch)" % spec.P
-                   if spec.P > 1 else "lora_sgmv_apply kernels (dispatcher's choice)")
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
                 "frac": round(achieved / hbm, 4), "traffic": measured_traffic(spec.name), "kernel": kernel_name,
                 "peak_source": "measured (MEASURED_PEAKS.json hbm_gbs)" if which == "measured" else which,
                 "algorithmic_bytes_per_launch": bytes_launch,
                 "launch_us": round(launch_s * 1e6, 3),
-                "tflops": round(w.flops() * spec.P / launches_per_step / launch_s / 1e12, 3)}
+                "tflops": round(w.flops() * bytes_launch / bytes_call / launch_s / 1e12, 3)}
 
     # ---- e2e through the public call with host buffers ----
     e2e = None

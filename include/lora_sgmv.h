@@ -105,14 +105,18 @@ typedef enum {
     LORA_SGMV_VARIANT_SPLIT = 1,      /* split-K shrink kernel, then streaming expand kernel */
     LORA_SGMV_VARIANT_GROUPED_TC = 2, /* tcgen05/TMEM grouped kernel for long segments */
     LORA_SGMV_VARIANT_FUSED = 3,      /* one kernel: cluster shrink, V reduction on chip, expand (fp32 FMA) */
-    LORA_SGMV_VARIANT_FUSED_TC = 4    /* the same split on tcgen05, for segments of several tokens */
+    LORA_SGMV_VARIANT_FUSED_TC = 4,   /* the same split on tcgen05, for segments of several tokens */
+    LORA_SGMV_VARIANT_SPLIT_TC = 5    /* split-K shrink kernel (V into the workspace), then the
+                                         tcgen05 expand with each segment's H2 split over
+                                         independent CTAs: uses every SM when segments are few
+                                         and B_i is large */
 } lora_sgmv_variant;
 
 /* Ranks r built into this library: 8, 16, 32, 64 and 128 for the split and
  * fused kernels; 16, 32 and 64 for the tensor-core kernels (GROUPED_TC,
- * FUSED_TC). GROUPED_TC also needs H1 and H2 of at least 64; FUSED_TC needs
- * H1 and H2 to be multiples of 64 (at least 64), and returns
- * LORA_SGMV_ERR_UNSUPPORTED otherwise. */
+ * FUSED_TC, SPLIT_TC). GROUPED_TC also needs H1 and H2 of at least 64;
+ * FUSED_TC and SPLIT_TC need H1 and H2 to be multiples of 64 (at least 64),
+ * and return LORA_SGMV_ERR_UNSUPPORTED otherwise. */
 int32_t lora_sgmv_rank_supported(int32_t r, lora_sgmv_variant variant);
 
 /* Human-readable name of a status code. Never NULL. */

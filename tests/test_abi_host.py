@@ -39,6 +39,7 @@ def test_version_and_ranks():
         assert sgmv.lora_sgmv_rank_supported(r, sgmv.VARIANT_SPLIT)
         assert sgmv.lora_sgmv_rank_supported(r, sgmv.VARIANT_FUSED)
         assert sgmv.lora_sgmv_rank_supported(r, sgmv.VARIANT_FUSED_TC) == (r in (16, 32, 64))
+        assert sgmv.lora_sgmv_rank_supported(r, sgmv.VARIANT_SPLIT_TC) == (r in (16, 32, 64))
         assert sgmv.lora_sgmv_rank_supported(r, sgmv.VARIANT_GROUPED_TC) == (r in (16, 32, 64))
     for r in (0, 4, 24, 256):
         assert not sgmv.lora_sgmv_rank_supported(r, sgmv.VARIANT_SPLIT)
@@ -116,6 +117,7 @@ def apply(**kw):
     (dict(ws=None), 7), (dict(wsb=100), 7), (dict(ws=MIS), 3),
     # the tensor-core decode kernel takes H1 and H2 in multiples of 64 only
     (dict(var=4, H1=264), 5), (dict(var=4, H2=136), 5), (dict(var=4, r=8), 5),
+    (dict(var=5, H1=264), 5), (dict(var=5, H2=136), 5), (dict(var=5, r=128), 5), (dict(var=6), 5),
 ])
 def test_apply_validation_codes(kw, code):
     assert apply(**kw) == code

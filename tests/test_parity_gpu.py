@@ -42,23 +42,25 @@ def test_config_bf16_variant(name):
 @pytest.mark.parametrize("r", [8, 16, 32, 64, 128])
 @pytest.mark.parametrize("dtype", ["f16", "bf16"])
 @pytest.mark.parametrize("T", [1, 37, 130])
-@pytest.mark.parametrize("variant", [sgmv.VARIANT_SPLIT, sgmv.VARIANT_FUSED, sgmv.VARIANT_FUSED_TC])
+@pytest.mark.parametrize("variant", [sgmv.VARIANT_SPLIT, sgmv.VARIANT_FUSED, sgmv.VARIANT_FUSED_TC,
+                                     sgmv.VARIANT_SPLIT_TC])
 def test_ragged_random_shapes(r, dtype, T, variant):
     # H1, H2 not multiples of the tile sizes; segments of every length (several token chunks)
     if not sgmv.lora_sgmv_rank_supported(r, variant):
         pytest.skip("rank not built for this variant")
     # the tensor-core decode kernel takes multiples of 64, still ragged against its stage sizes
-    H1, H2 = (320, 192) if variant == sgmv.VARIANT_FUSED_TC else (264, 136)
+    tc = variant in (sgmv.VARIANT_FUSED_TC, sgmv.VARIANT_SPLIT_TC)
+    H1, H2 = (320, 192) if tc else (264, 136)
     w = inputs.small_random(T, 7, H1, H2, r, dtype, seed=T * 1000 + r)
     p = DeviceProblem(w, y_random=True)
     assert_close(p.apply(variant=variant), p.oracle_apply(), dtype, w.name)
 
 
 @pytest.mark.parametrize("r", [16, 64])
-@pytest.mark.parametrize("variant", [sgmv.VARIANT_FUSED, sgmv.VARIANT_FUSED_TC])
+@pytest.mark.parametrize("variant", [sgmv.VARIANT_FUSED, sgmv.VARIANT_FUSED_TC, sgmv.VARIANT_SPLIT_TC])
 def test_fused_long_rows_many_tiles(r, variant):
     # H1 and H2 span many stages per CTA (several A and B tiles) with ragged ends
-    H1, H2 = (8256, 11008) if variant == sgmv.VARIANT_FUSED_TC else (8200, 11000)
+    H1, H2 = (8200, 11000) if variant == sgmv.VARIANT_FUSED else (8256, 11008)
     w = inputs.small_random(40, 5, H1, H2, r, "bf16", seed=r)
     p = DeviceProblem(w, y_random=True)
     assert_close(p.apply(variant=variant), p.oracle_apply(), "bf16", "long rows")
@@ -75,6 +77,16 @@ def test_decode_tc_odd_cluster_sizes(H1, H2):
     got = p.apply(variant=sgmv.VARIANT_FUSED_TC)
     assert int(p.status.item()) == 0
     assert_close(got, p.oracle_apply(), "bf16", f"decode tc {H1}x{H2}")
+
+
+@pytest.mark.parametrize("name", ["llama70b_decode_h28672", "llama70b_decode_h8192"])
+def test_split_tc_full_size_sampled(name):
+    # the split tensor-core form on the 70B-shaped decode (V through the workspace)
+    w = inputs.make(name)
+    p = DeviceProblem(w, y_random=True)
+    got = p.apply(variant=sgmv.VARIANT_SPLIT_TC)
+    _sampled_check(p, got, 300, 9)
+    assert int(p.status.item()) == 0
 
 
 def test_decode_tc_many_segments():
@@ -228,12 +240,14 @@ def test_empty_repeated_unsorted_segments_and_uncovered_rows():
     assert int(p.status.item()) == 0
 
 
-@pytest.mark.parametrize("variant", [sgmv.VARIANT_SPLIT, sgmv.VARIANT_FUSED, sgmv.VARIANT_FUSED_TC])
+@pytest.mark.parametrize("variant", [sgmv.VARIANT_SPLIT, sgmv.VARIANT_FUSED, sgmv.VARIANT_FUSED_TC,
+                                     sgmv.VARIANT_SPLIT_TC])
 def test_bad_segments_are_skipped_and_reported(variant):
     # [4,2) reversed; adapter 9 out of range; adapter 2 has a null table entry; [20,30) past T
     seg = np.array([0, 4, 2, 8, 12, 16, 20, 30], np.int32)
     idx = np.array([0, 1, 9, 3, 2, 4, 1], np.int32)
-    p = _custom(seg, idx, H2=256 if variant == sgmv.VARIANT_FUSED_TC else 264)
+    tc = variant in (sgmv.VARIANT_FUSED_TC, sgmv.VARIANT_SPLIT_TC)
+    p = _custom(seg, idx, H2=256 if tc else 264)
     p.A_ptrs[2] = 0
     before = from_dev(p.Y)
     got = p.apply(variant=variant)
