@@ -206,48 +206,72 @@ class ClockSampler:
 # the CPU oracle as a baseline (host cores)
 # ---------------------------------------------------------------------------------------------
 
+class OracleSampler:
+    """The oracle (single-threaded C, as it stands) on bounded samples of one workload.
+
+    The host inputs (grouping, the touched adapters, X and Y) are made once; every sample
+    then runs for about the time it is given: whole SGMV calls repeated when a call fits in
+    half of it, else the first rows of one call in segment order (whole segments, then part
+    of the next, at least one row)."""
+
+    def __init__(self, spec: Spec):
+        import oracle
+
+        self.oracle, self.spec = oracle, spec
+        w = spec.w
+        self.seg, self.idx, _ = oracle.group_segments(w.ids, w.num_adapters)
+        touched = set(int(i) for i in w.touched_adapters())
+        zA = np.zeros((w.H1, w.r), np.uint16)  # shared by every untouched adapter
+        zB = np.zeros((w.r, w.H2), np.uint16)
+        self.A = [w.adapter_a(i) if i in touched else zA for i in range(w.num_adapters)]
+        self.B = [w.adapter_b(i) if i in touched else zB for i in range(w.num_adapters)]
+        self.X, self.Y = w.x(), w.y0()
+        # seconds per token row, from up to 4 rows of the first segment
+        rows = max(1, min(4, int(self.seg[1] - self.seg[0])))
+        t0 = time.perf_counter()
+        self._run_rows(rows)
+        self.per_row = (time.perf_counter() - t0) / rows
+
+    @staticmethod
+    def first_rows(seg, idx, n: int):
+        """Segment bounds and adapter ids of the first n rows (segment order) of a call: the
+        segments that end at or before row n, then the part of the next one below n."""
+        whole = int(np.searchsorted(seg, n, side="right")) - 1
+        cut = [int(v) for v in seg[: whole + 1]]
+        if cut[-1] < n:
+            cut.append(n)
+        return np.array(cut, np.int32), np.asarray(idx[: len(cut) - 1], np.int32)
+
+    def _run_rows(self, n: int) -> None:
+        """The first n rows (segment order) of one call."""
+        sub_seg, sub_idx = self.first_rows(self.seg, self.idx, n)
+        w = self.spec.w
+        self.oracle.apply_f32(self.Y[:n], self.X[:n], self.A, self.B, sub_seg, sub_idx, w.scale, w.dtype)
+
+    def sample(self, seconds: float) -> dict:
+        w = self.spec.w
+        t_start = time.perf_counter()
+        if self.per_row * w.T <= seconds / 2:
+            what = f"whole SGMV calls of the workload ({w.T} tokens each), repeated for ~{seconds:.3g} s"
+            calls, tokens = 0, 0
+            while calls == 0 or time.perf_counter() - t_start < seconds:
+                self.oracle.apply_f32(self.Y, self.X, self.A, self.B, self.seg, self.idx, w.scale, w.dtype)
+                calls += 1
+                tokens += w.T
+        else:
+            n = max(1, min(w.T, int(seconds / self.per_row)))
+            what = f"first {n} of {w.T} token rows of one call (segment order)"
+            self._run_rows(n)
+            calls, tokens = 1, n
+        elapsed = time.perf_counter() - t_start
+        # tokens/s of whole steps: a step holds spec.P calls over the same T tokens
+        return {"value": tokens / self.spec.P / elapsed, "unit": UNIT, "cores": 1, "kind": "oracle",
+                "sample": what, "seconds": round(elapsed, 6), "calls": calls}
+
+
 def oracle_baseline(spec: Spec, seconds: float):
     """Time the oracle (single-threaded C, as it stands) on a bounded sample of the workload."""
-    import oracle
-
-    w = spec.w
-    seg, idx, _ = oracle.group_segments(w.ids, w.num_adapters)
-    # one call's host inputs; the sample repeats it, bounded in time
-    touched = w.touched_adapters()
-    Am = {i: w.adapter_a(i) for i in touched}
-    Bm = {i: w.adapter_b(i) for i in touched}
-    zA, zB = np.zeros((1, 1), np.uint16), np.zeros((1, 1), np.uint16)
-    A = [Am.get(i, zA) for i in range(w.num_adapters)]
-    B = [Bm.get(i, zB) for i in range(w.num_adapters)]
-    X, Y = w.x(), w.y0()
-    # rows per call: the whole batch unless a call alone exceeds the budget
-    t0 = time.perf_counter()
-    rows = min(w.T, max(1, int(seg[1] - seg[0])))
-    sub_seg = np.array([0, rows], np.int32)
-    sub_idx = idx[:1]
-    oracle.apply_f32(Y[:rows], X[:rows], A, B, sub_seg, sub_idx, w.scale, w.dtype)
-    per_row = (time.perf_counter() - t0) / rows
-    calls, tokens, t_start = 0, 0, time.perf_counter()
-    full_call_s = per_row * w.T
-    if full_call_s <= seconds / 2:
-        sample = f"whole SGMV calls of the workload ({w.T} tokens each), repeated for ~{seconds:.0f} s"
-        while time.perf_counter() - t_start < seconds:
-            oracle.apply_f32(Y, X, A, B, seg, idx, w.scale, w.dtype)
-            calls += 1
-            tokens += w.T
-    else:
-        n_rows = max(1, int(seconds / per_row))
-        sample = f"first {n_rows} of {w.T} token rows of one call (segment order)"
-        # take whole segments from the start until n_rows
-        take = int(np.searchsorted(seg, n_rows, side="right")) - 1
-        take = max(1, take)
-        oracle.apply_f32(Y[: seg[take]], X[: seg[take]], A, B, seg[: take + 1], idx[:take], w.scale, w.dtype)
-        calls, tokens = 1, int(seg[take])
-    elapsed = time.perf_counter() - t_start
-    # tokens/s of whole steps: a step holds spec.P calls over the same T tokens
-    value = tokens / spec.P / elapsed
-    return {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample,
-            "seconds": round(elapsed, 3), "calls": calls}
+    return OracleSampler(spec).sample(seconds)
 
 
 # ---------------------------------------------------------------------------------------------
@@ -518,14 +542,20 @@ def run_e2e(args, spec, torch, sgmv, dev, stream, calls, dt, tdt, world=1):
 # reference arm: the oracle on the host cores
 # ---------------------------------------------------------------------------------------------
 
+REFERENCE_BUDGET_S = 120.0
+
+
 def run_reference(args, spec: Spec, rank: int):
     if rank != 0:
         return None
-    per_step = max(1.0, min(10.0, 120.0 / max(1, args.steps + args.warmup)))
+    # the timed steps share a budget of about two minutes of oracle time (at most 10 s a
+    # step); warm-up steps get a quarter of a step's share each
+    sampler = OracleSampler(spec)
+    per_step = min(10.0, REFERENCE_BUDGET_S / max(1, args.steps))
     for _ in range(args.warmup):
-        oracle_baseline(spec, per_step / 4)
+        sampler.sample(per_step / 4)
     t0 = time.perf_counter()
-    runs = [oracle_baseline(spec, per_step) for _ in range(args.steps)]
+    runs = [sampler.sample(per_step) for _ in range(args.steps)]
     el = time.perf_counter() - t0
     value = statistics.median(r["value"] for r in runs)
     return {
