@@ -16,6 +16,7 @@
 #include "sgmv_decode_tc.cuh"
 #include "sgmv_fused.cuh"
 #include "sgmv_grouped_tc.cuh"
+#include "sgmv_pad.cuh"
 #include "sgmv_split.cuh"
 
 namespace {
@@ -615,6 +616,24 @@ lora_sgmv_status fused_dispatch(const sgmv::FusedParams& P, int r, lora_sgmv_dty
                                : fused_dispatch_r<__nv_bfloat16>(P, r, max_len, s);
 }
 
+// One padding launch: dst [rows_dst, cols_dst] from src [rows_src, cols_src] (16-bit elements).
+lora_sgmv_status launch_pad(void* dst, const void* src, int64_t rows_dst, int64_t cols_dst, int64_t rows_src,
+                            int64_t cols_src, cudaStream_t stream) {
+    DeviceFacts f;
+    if (device_facts(f) != LORA_SGMV_OK) return LORA_SGMV_ERR_CUDA;
+    const int64_t n = rows_dst * cols_dst;
+    const int64_t blocks = std::max<int64_t>(
+        1, std::min<int64_t>((n + sgmv::kPadThreads - 1) / sgmv::kPadThreads, int64_t(f.sms) * 8));
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(blocks), 1, 1);
+    cfg.blockDim = dim3(sgmv::kPadThreads, 1, 1);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cfg.numAttrs = 0;
+    return counted(cudaLaunchKernelEx(&cfg, sgmv::sgmv_pad_kernel, static_cast<uint16_t*>(dst),
+                                      static_cast<const uint16_t*>(src), rows_dst, cols_dst, rows_src, cols_src));
+}
+
 lora_sgmv_status check_common(int32_t n_segments, int32_t num_adapters, int32_t T, lora_sgmv_dtype dtype) {
     if (dtype != LORA_SGMV_F16 && dtype != LORA_SGMV_BF16) return LORA_SGMV_ERR_DTYPE;
     if (n_segments < 0 || T < 0 || num_adapters < 0) return LORA_SGMV_ERR_DIM;
@@ -689,6 +708,23 @@ size_t lora_sgmv_workspace_bytes(int32_t T, int32_t r) {
     if (T <= 0 || r <= 0) return 0;
     const size_t v = static_cast<size_t>(T) * static_cast<size_t>(r) * sizeof(float);
     return (v + 255) / 256 * 256;
+}
+
+lora_sgmv_status lora_sgmv_pad_rank(void* A_dst, const void* A_src, void* B_dst, const void* B_src, int32_t H1,
+                                    int32_t H2, int32_t r_src, int32_t r, lora_sgmv_dtype dtype, void* stream) {
+    if (dtype != LORA_SGMV_F16 && dtype != LORA_SGMV_BF16) return LORA_SGMV_ERR_DTYPE;
+    const bool has_a = A_dst || A_src, has_b = B_dst || B_src;
+    if (!has_a && !has_b) return LORA_SGMV_ERR_NULL;
+    if ((has_a && (!A_dst || !A_src)) || (has_b && (!B_dst || !B_src))) return LORA_SGMV_ERR_NULL;
+    if (r_src < 1 || r < r_src) return LORA_SGMV_ERR_DIM;
+    if ((has_a && H1 < 1) || (has_b && H2 < 1)) return LORA_SGMV_ERR_DIM;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (has_a) {
+        lora_sgmv_status st = launch_pad(A_dst, A_src, H1, r, H1, r_src, s);
+        if (st != LORA_SGMV_OK) return st;
+    }
+    if (has_b) return launch_pad(B_dst, B_src, r, H2, r_src, H2, s);
+    return LORA_SGMV_OK;
 }
 
 lora_sgmv_status lora_sgmv_shrink(float* V, const void* X, const void* const* A_ptrs,

@@ -159,6 +159,35 @@ lora_sgmv_status lora_sgmv_group_segments(const int32_t* ids, int32_t T, int32_t
                                           int32_t* n_segments);
 
 /*
+ * lora_sgmv_pad_rank -- one adapter of rank r_src, padded with zeros to rank r.
+ *
+ * Adapters of different ranks share one call once all are padded to one rank:
+ * the authors' answer on different ranks (page "Punica: Serving multiple LoRA
+ * finetuned LLM as one", the Hacker News thread) is padding, as the kernels
+ * are bound by memory, not arithmetic. The padded adapter gives the original
+ * adapter's result: the extra entries of V are zero and the extra terms of
+ * each expand sum are zero (up to the sign of an exact zero sum).
+ *   A_dst        device, [H1, r] out: A_dst[k, j] = A_src[k, j] for j < r_src,
+ *                0 for r_src <= j < r.
+ *   A_src        device, [H1, r_src].
+ *   B_dst        device, [r, H2] out: B_dst[j, :] = B_src[j, :] for j < r_src,
+ *                0 for r_src <= j < r.
+ *   B_src        device, [r_src, H2].
+ *   Either pair may be (NULL, NULL) to pad only the other matrix; H1 (H2) is
+ *   then unused.
+ *   H1, H2       sizes (>= 1 for each matrix given).
+ *   r_src, r     1 <= r_src <= r; r_src == r copies.
+ *   dtype        16-bit storage type of the four matrices.
+ *   stream       cudaStream_t as void*; one kernel launch per matrix given.
+ * A destination must not overlap its source. Returns LORA_SGMV_ERR_DTYPE,
+ * _NULL (no pair given, or half a pair) or _DIM before any launch, _CUDA if a
+ * launch fails, else LORA_SGMV_OK. Runs at adapter load time, not per call.
+ */
+lora_sgmv_status lora_sgmv_pad_rank(void* A_dst, const void* A_src, void* B_dst, const void* B_src,
+                                    int32_t H1, int32_t H2, int32_t r_src, int32_t r,
+                                    lora_sgmv_dtype dtype, void* stream);
+
+/*
  * lora_sgmv_shrink -- V[t, :] = X[t, :] @ A_{lora_idx[s]} for rows t of each segment.
  *
  * The H1 -> r half of x@A@B (README LoRA paragraph), fp32 accumulation.

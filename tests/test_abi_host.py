@@ -142,6 +142,21 @@ def test_shrink_expand_validation_codes():
     assert ex(Y=None) == 1 and ex(V=MIS) == 3 and ex(H2=12) == 3 and ex(r=7) == 5 and ex(dt=-1) == 4
 
 
+def test_pad_rank_validation_codes():
+    lib = sgmv.load()
+
+    def pad(Ad=FAKE, As=FAKE + 4096, Bd=FAKE + 8192, Bs=FAKE + 12288, H1=64, H2=48, rs=8, r=16, dt=0):
+        return lib.lora_sgmv_pad_rank(Ad, As, Bd, Bs, H1, H2, rs, r, dt, None)
+
+    assert pad(dt=2) == 4 and pad(dt=-1) == 4
+    assert pad(Ad=None, As=None, Bd=None, Bs=None) == 1
+    assert pad(Ad=None) == 1 and pad(Bs=None) == 1
+    assert pad(rs=0) == 2 and pad(rs=17) == 2 and pad(r=4) == 2
+    assert pad(H1=0) == 2 and pad(H2=-1) == 2
+    # a pair left out makes its size unused
+    assert pad(Ad=None, As=None, H1=0, rs=17) == 2
+
+
 def test_batched_validation_codes():
     lib = sgmv.load()
 

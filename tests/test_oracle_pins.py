@@ -328,3 +328,51 @@ def test_group_segments_invariants_and_stable_argsort(maker):
 def test_group_segments_rejects_out_of_range_ids():
     with pytest.raises(ValueError):
         oracle.group_segments([0, 5, 1], 4)
+
+
+# ---------------------------------------------------------------------------------------------
+# mixed ranks by zero padding (the authors' answer on different ranks, page "Punica: Serving
+# multiple LoRA finetuned LLM as one", the Hacker News thread)
+# ---------------------------------------------------------------------------------------------
+
+def _mixed_rank_case(dt, seed):
+    rng = np.random.default_rng(seed)
+    T, H1, H2, r = 14, 24, 16, 8
+    ranks = [2, 8, 5, 3]  # adapter i has rank ranks[i]; all are padded to r
+    X = inputs.cast_f32_bits(rng.standard_normal((T, H1)).astype(np.float32), dt)
+    Y = inputs.cast_f32_bits(rng.standard_normal((T, H2)).astype(np.float32), dt)
+    A = [inputs.cast_f32_bits(rng.standard_normal((H1, k)).astype(np.float32) * 0.3, dt) for k in ranks]
+    B = [inputs.cast_f32_bits(rng.standard_normal((k, H2)).astype(np.float32) * 0.5, dt) for k in ranks]
+    Ap = [np.pad(a, ((0, 0), (0, r - a.shape[1]))) for a in A]  # zero columns
+    Bp = [np.pad(b, ((0, r - b.shape[0]), (0, 0))) for b in B]  # zero rows
+    seg, idx = [0, 3, 4, 9, 14], [2, 0, 3, 1]
+    return X, Y, A, B, Ap, Bp, seg, idx
+
+
+@pytest.mark.parametrize("dt", ["f16", "bf16"])
+def test_mixed_ranks_padded_equal_each_adapters_own_product(dt):
+    """Padded to one rank, every segment still gets x@A_i@B_i at adapter i's own rank
+    (numpy, fp64, with the unpadded matrices)."""
+    X, Y, A, B, Ap, Bp, seg, idx = _mixed_rank_case(dt, 23)
+    x, y = dec(X, dt), dec(Y, dt)
+    ref = y.copy()
+    for s in range(len(idx)):
+        i = idx[s]
+        ref[seg[s]:seg[s + 1]] += 0.75 * (x[seg[s]:seg[s + 1]] @ dec(A[i], dt)) @ dec(B[i], dt)
+    got, sk = oracle.apply_f64(y, X, Ap, Bp, seg, idx, 0.75, dt)
+    assert sk == 0
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("dt", ["f16", "bf16"])
+def test_zero_padding_leaves_fp32_results_bit_identical(dt):
+    """The fp32 oracle on padded adapters equals, bit for bit, one call per segment on the
+    adapter at its own rank: the extra terms are exact zeros."""
+    X, Y, A, B, Ap, Bp, seg, idx = _mixed_rank_case(dt, 29)
+    got, sk = oracle.apply_f32(Y, X, Ap, Bp, seg, idx, 1.25, dt)
+    assert sk == 0
+    for s in range(len(idx)):
+        b, e, i = seg[s], seg[s + 1], idx[s]
+        own, sk1 = oracle.apply_f32(Y[b:e], X[b:e], [A[i]], [B[i]], [0, e - b], [0], 1.25, dt)
+        assert sk1 == 0
+        assert np.array_equal(got[b:e], own), s
