@@ -83,6 +83,26 @@ def measured_traffic(name: str):
     return e["bytes"]
 
 
+NOMINAL_HBM_GBS = 8000.0  # B200 HBM3e, the vendor's figure
+
+
+def make_roofline(bytes_launch: float, flops_launch: float, launch_s: float, hbm_gbs: float, bf16_tflops: float,
+                  which: str, traffic, kernel_name: str) -> dict:
+    """The roofline object of the JSON line: algorithmic bytes (and FLOPs) of one launch over
+    its measured duration, against the measured copy peak (frac), the nominal HBM figure
+    (frac_nominal) and, for the tensor pipe, the measured dense bf16 peak (tensor_frac)."""
+    achieved = bytes_launch / launch_s / 1e9
+    tflops = flops_launch / launch_s / 1e12
+    return {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_gbs, "unit": "GB/s",
+            "frac": round(achieved / hbm_gbs, 4), "traffic": traffic, "kernel": kernel_name,
+            "peak_source": "measured (MEASURED_PEAKS.json hbm_gbs)" if which == "measured" else which,
+            "frac_nominal": round(achieved / NOMINAL_HBM_GBS, 4),
+            "algorithmic_bytes_per_launch": int(bytes_launch),
+            "launch_us": round(launch_s * 1e6, 3),
+            "tflops": round(tflops, 3),
+            "tensor_frac": round(tflops / bf16_tflops, 4)}
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -274,6 +294,91 @@ def oracle_baseline(spec: Spec, seconds: float):
     return OracleSampler(spec).sample(seconds)
 
 
+def rows_share(seg, idx, a: int, b: int):
+    """Segment bounds (relative to row a) and adapter ids of rows [a, b) of a call."""
+    seg = np.asarray(seg, np.int64)
+    cut, ids = [0], []
+    for s in range(len(seg) - 1):
+        lo, hi = max(int(seg[s]), a), min(int(seg[s + 1]), b)
+        if lo < hi:
+            cut.append(hi - a)
+            ids.append(int(idx[s]))
+    return np.array(cut, np.int32), np.array(ids, np.int32)
+
+
+def _all_cores_worker(name: str, a: int, b: int, seconds: float, barrier, queue) -> None:
+    """One process of the all-cores baseline: the oracle on rows [a, b) of one call."""
+    try:
+        import oracle
+
+        w = make_spec(name).w
+        seg, idx, _ = oracle.group_segments(w.ids, w.num_adapters)
+        sub_seg, sub_idx = rows_share(seg, idx, a, b)
+        need = set(int(i) for i in sub_idx)
+        zA, zB = np.zeros((w.H1, w.r), np.uint16), np.zeros((w.r, w.H2), np.uint16)
+        A = [w.adapter_a(i) if i in need else zA for i in range(w.num_adapters)]
+        B = [w.adapter_b(i) if i in need else zB for i in range(w.num_adapters)]
+        X, Y = w.x()[a:b], w.y0()[a:b]
+        n = b - a
+        t0 = time.perf_counter()
+        probe = min(n, 4)
+        ps, pi = rows_share(sub_seg, sub_idx, 0, probe)
+        oracle.apply_f32(Y[:probe], X[:probe], A, B, ps, pi, w.scale, w.dtype)
+        per_row = (time.perf_counter() - t0) / probe
+        barrier.wait(timeout=120)
+        t_start = time.perf_counter()
+        tokens = 0
+        if per_row * n <= seconds / 2:
+            while tokens == 0 or time.perf_counter() - t_start < seconds:
+                oracle.apply_f32(Y, X, A, B, sub_seg, sub_idx, w.scale, w.dtype)
+                tokens += n
+        else:
+            m = max(1, min(n, int(seconds / per_row)))
+            ps, pi = rows_share(sub_seg, sub_idx, 0, m)
+            oracle.apply_f32(Y[:m], X[:m], A, B, ps, pi, w.scale, w.dtype)
+            tokens = m
+        queue.put((tokens, time.perf_counter() - t_start, None))
+    except Exception as e:  # reported by the parent; the run goes on without this figure
+        queue.put((0, 0.0, f"{type(e).__name__}: {e}"))
+
+
+def oracle_all_cores(spec: Spec, seconds: float, max_procs: int = 64) -> dict:
+    """The same oracle, unchanged, on every host core: one process per core, each on its own
+    contiguous share of one call's rows (with only the adapters its rows use), started
+    together; throughput = all processes' tokens over the slowest one's time. Processes are
+    spawned (never forked: the parent may hold a CUDA context). On any failure the figure is
+    replaced by the reason and the run goes on."""
+    import multiprocessing as mp
+
+    try:
+        cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else (os.cpu_count() or 1)
+        w = spec.w
+        procs_n = max(1, min(cores, max_procs, w.T))
+        bounds = [round(k * w.T / procs_n) for k in range(procs_n + 1)]
+        ctx = mp.get_context("spawn")
+        barrier = ctx.Barrier(procs_n)
+        queue = ctx.Queue()
+        procs = [ctx.Process(target=_all_cores_worker,
+                             args=(spec.name, bounds[k], bounds[k + 1], seconds, barrier, queue), daemon=True)
+                 for k in range(procs_n)]
+        for p in procs:
+            p.start()
+        results = [queue.get(timeout=180 + 4 * seconds) for _ in procs]
+        for p in procs:
+            p.join(timeout=30)
+        errors = [e for _, _, e in results if e]
+        if errors:
+            return {"unavailable": errors[0]}
+        tokens = sum(t for t, _, _ in results)
+        slowest = max(el for _, el, _ in results)
+        return {"value": round(tokens / spec.P / slowest, 3), "unit": UNIT, "cores": procs_n, "kind": "oracle",
+                "sample": f"{procs_n} processes of the single-threaded oracle, each on its own share of the "
+                          f"rows of one call (about {w.T // procs_n} rows each), run for ~{seconds:.3g} s or "
+                          f"its first rows"}
+    except Exception as e:
+        return {"unavailable": f"{type(e).__name__}: {e}"}
+
+
 # ---------------------------------------------------------------------------------------------
 # our arm
 # ---------------------------------------------------------------------------------------------
@@ -426,13 +531,8 @@ def run_ours(args, spec: Spec, rank: int, world: int, local: int):
         launch_s = ms_per_step / 1e3 / launches_per_step
         kernel_name = ("sgmv_fused_kernel (lora_sgmv_apply_batched: %d projections per launch)" % spec.P
                        if spec.P > 1 else "lora_sgmv_apply kernels (dispatcher's choice)")
-    achieved = bytes_launch / launch_s / 1e9
-    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
-                "frac": round(achieved / hbm, 4), "traffic": measured_traffic(spec.name), "kernel": kernel_name,
-                "peak_source": "measured (MEASURED_PEAKS.json hbm_gbs)" if which == "measured" else which,
-                "algorithmic_bytes_per_launch": bytes_launch,
-                "launch_us": round(launch_s * 1e6, 3),
-                "tflops": round(w.flops() * bytes_launch / bytes_call / launch_s / 1e12, 3)}
+    roofline = make_roofline(bytes_launch, w.flops() * bytes_launch / bytes_call, launch_s, hbm, tc, which,
+                             measured_traffic(spec.name), kernel_name)
 
     # ---- e2e through the public call with host buffers ----
     e2e = None
@@ -594,6 +694,7 @@ def main():
     if rank == 0 and result is not None:
         if world == 1 and not args.no_cpu_baseline:
             result["cpu_baseline"] = oracle_baseline(spec, args.cpu_seconds)
+            result["cpu_baseline"]["all_cores"] = oracle_all_cores(spec, args.cpu_seconds)
         print(json.dumps(result), flush=True)
 
 

@@ -71,3 +71,51 @@ def test_reference_arm_partial_rows_on_a_large_workload(monkeypatch):
     out = bench.run_reference(SimpleNamespace(steps=50, warmup=3), spec, 0)
     assert out["cpu_baseline"]["sample"].startswith("first ")
     assert out["value"] > 0
+
+
+def test_make_roofline_arithmetic():
+    import bench
+
+    r = bench.make_roofline(36700160, 3.0e9, 10.975e-6, 6544.7, 1630.0, "measured", 35726336, "k")
+    assert r["achieved"] == round(36700160 / 10.975e-6 / 1e9, 1)
+    assert r["frac"] == round(36700160 / 10.975e-6 / 1e9 / 6544.7, 4)
+    assert r["frac_nominal"] == round(36700160 / 10.975e-6 / 1e9 / 8000.0, 4)
+    assert r["tflops"] == round(3.0e9 / 10.975e-6 / 1e12, 3)
+    assert r["tensor_frac"] == round(3.0e9 / 10.975e-6 / 1e12 / 1630.0, 4)
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s" and r["peak"] == 6544.7 and r["traffic"] == 35726336
+    assert r["launch_us"] == 10.975 and r["algorithmic_bytes_per_launch"] == 36700160
+
+
+def test_rows_share_partitions_a_call():
+    import bench
+    import oracle
+    from adapter_matmul_b200 import inputs
+
+    seg = np.array([0, 3, 5, 9], np.int32)
+    idx = np.array([7, 2, 4], np.int32)
+    s, i = bench.rows_share(seg, idx, 2, 7)
+    assert s.tolist() == [0, 1, 3, 5] and i.tolist() == [7, 2, 4]
+    s, i = bench.rows_share(seg, idx, 3, 5)
+    assert s.tolist() == [0, 2] and i.tolist() == [2]
+    # shares computed apart and put side by side equal the whole call, bit for bit
+    w = inputs.small_random(37, 4, 48, 40, 8, "bf16", seed=5)
+    seg, idx, _ = oracle.group_segments(w.ids, w.num_adapters)
+    X, Y = w.x(), w.y_random()
+    A = [w.adapter_a(k) for k in range(4)]
+    B = [w.adapter_b(k) for k in range(4)]
+    full, _ = oracle.apply_f32(Y, X, A, B, seg, idx, w.scale, w.dtype)
+    bounds = [0, 5, 6, 20, 37]
+    parts = []
+    for a, b in zip(bounds[:-1], bounds[1:]):
+        s, i = bench.rows_share(seg, idx, a, b)
+        part, _ = oracle.apply_f32(Y[a:b], X[a:b], A, B, s, i, w.scale, w.dtype)
+        parts.append(part)
+    assert np.array_equal(np.concatenate(parts), full)
+
+
+def test_all_cores_baseline_runs_in_spawned_processes():
+    import bench
+
+    out = bench.oracle_all_cores(bench.make_spec("tiny"), 0.3, max_procs=4)
+    assert "unavailable" not in out, out
+    assert out["kind"] == "oracle" and out["value"] > 0 and 1 <= out["cores"] <= 4
