@@ -406,9 +406,7 @@ bool decode_tc_preferred(int r, int max_len) { return max_len > 2 && r >= 32; }
 // spreads each job's N over independent CTAs) pays a second launch and a V round trip through
 // the workspace, and wins when the fused form would leave SMs idle: fewer jobs than SMs, each
 // with a large B_i (several MB) to stream.
-bool split_tc_preferred(int T, int n_segments, int max_len, int H1, int H2, int r) {
-    DeviceFacts f;
-    const int sms = device_facts(f) == LORA_SGMV_OK ? f.sms : 148;
+bool split_tc_preferred(int T, int n_segments, int max_len, int H1, int H2, int r, int sms) {
     const long long chunks = std::min<long long>(n_segments + (T + 15) / 16, std::max(T, 1));
     const long long jobs = max_len <= 16 ? n_segments : chunks;
     (void)H1;
@@ -417,6 +415,19 @@ bool split_tc_preferred(int T, int n_segments, int max_len, int H1, int H2, int 
 
 bool decode_tc_supported(int r, int H1, int H2) {
     return (r == 16 || r == 32 || r == 64) && H1 >= 64 && H2 >= 64 && H1 % 64 == 0 && H2 % 64 == 0;
+}
+
+// The kernels AUTO runs for a call (host arithmetic only). max_len: the longest segment, as
+// estimated by estimate_max_len; sms: the device's SM count.
+lora_sgmv_variant auto_variant(int T, int n_segments, int max_len, int H1, int H2, int r, lora_sgmv_dtype dtype,
+                               int sms) {
+    if (max_len >= sgmv::kGroupedMinSegment && sgmv::grouped_tc_supported(r, H1, H2, dtype))
+        return LORA_SGMV_VARIANT_GROUPED_TC;
+    if (n_segments > sgmv::kFusedMaxSegments) return LORA_SGMV_VARIANT_SPLIT;
+    if (decode_tc_preferred(r, max_len) && decode_tc_supported(r, H1, H2))
+        return split_tc_preferred(T, n_segments, max_len, H1, H2, r, sms) ? LORA_SGMV_VARIANT_SPLIT_TC
+                                                                          : LORA_SGMV_VARIANT_FUSED_TC;
+    return LORA_SGMV_VARIANT_FUSED;
 }
 
 template <typename T, int R>
@@ -646,6 +657,13 @@ extern "C" {
 
 int32_t lora_sgmv_version(void) { return kVersion; }
 
+lora_sgmv_variant lora_sgmv_auto_variant(int32_t T, int32_t n_segments, int32_t H1, int32_t r, int32_t H2,
+                                         lora_sgmv_dtype dtype, int32_t max_seg_len, int32_t sm_count) {
+    if (T <= 0 || n_segments <= 0 || H1 <= 0 || H2 <= 0 || r <= 0 || sm_count <= 0) return LORA_SGMV_VARIANT_AUTO;
+    if (dtype != LORA_SGMV_F16 && dtype != LORA_SGMV_BF16) return LORA_SGMV_VARIANT_AUTO;
+    return auto_variant(T, n_segments, estimate_max_len(max_seg_len, T, n_segments), H1, H2, r, dtype, sm_count);
+}
+
 uint64_t lora_sgmv_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 const char* lora_sgmv_last_error(void) {
@@ -811,15 +829,11 @@ lora_sgmv_status lora_sgmv_apply_ex(void* Y, const void* X, const void* const* A
     cudaStream_t s = static_cast<cudaStream_t>(stream);
 
     lora_sgmv_variant v = variant;
-    if (v == LORA_SGMV_VARIANT_AUTO)
-        v = (max_len >= sgmv::kGroupedMinSegment && sgmv::grouped_tc_supported(r, H1, H2, dtype))
-                ? LORA_SGMV_VARIANT_GROUPED_TC
-                : (n_segments > sgmv::kFusedMaxSegments
-                       ? LORA_SGMV_VARIANT_SPLIT
-                       : (decode_tc_preferred(r, max_len) && decode_tc_supported(r, H1, H2)
-                              ? (split_tc_preferred(T, n_segments, max_len, H1, H2, r) ? LORA_SGMV_VARIANT_SPLIT_TC
-                                                                                      : LORA_SGMV_VARIANT_FUSED_TC)
-                              : LORA_SGMV_VARIANT_FUSED));
+    if (v == LORA_SGMV_VARIANT_AUTO) {
+        DeviceFacts f;
+        if (device_facts(f) != LORA_SGMV_OK) return LORA_SGMV_ERR_CUDA;
+        v = auto_variant(T, n_segments, max_len, H1, H2, r, dtype, f.sms);
+    }
 
     if (v == LORA_SGMV_VARIANT_FUSED || v == LORA_SGMV_VARIANT_FUSED_TC || v == LORA_SGMV_VARIANT_SPLIT_TC) {
         if ((v == LORA_SGMV_VARIANT_FUSED_TC || v == LORA_SGMV_VARIANT_SPLIT_TC) && !decode_tc_supported(r, H1, H2))

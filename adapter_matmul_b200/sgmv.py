@@ -43,7 +43,7 @@ EXPORTS = [
     "lora_sgmv_last_error",
     "lora_sgmv_group_segments", "lora_sgmv_shrink", "lora_sgmv_expand", "lora_sgmv_workspace_bytes",
     "lora_sgmv_apply", "lora_sgmv_apply_ex", "lora_sgmv_apply_batched", "lora_sgmv_apply_noalloc",
-    "lora_sgmv_pad_rank",
+    "lora_sgmv_pad_rank", "lora_sgmv_auto_variant",
 ]
 
 
@@ -110,6 +110,8 @@ def load(path: Optional[str] = None):
         lib.lora_sgmv_apply_noalloc.restype = ctypes.c_int
         lib.lora_sgmv_apply_noalloc.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, ctypes.c_float,
                                                 ctypes.c_int, i32, P, P]
+        lib.lora_sgmv_auto_variant.restype = ctypes.c_int
+        lib.lora_sgmv_auto_variant.argtypes = [i32, i32, i32, i32, i32, ctypes.c_int, i32, i32]
         lib.lora_sgmv_pad_rank.restype = ctypes.c_int
         lib.lora_sgmv_pad_rank.argtypes = [P, P, P, P, i32, i32, i32, i32, ctypes.c_int, P]
         if path is None:
@@ -235,6 +237,12 @@ def lora_sgmv_apply_noalloc(Y, X, A_ptrs, B_ptrs, seg_starts, lora_idx, n_segmen
                                           n_segments, num_adapters, T, H1, r, H2, float(scale), dtype, max_seg_len,
                                           _p(dev_status), _stream(stream)),
            "lora_sgmv_apply_noalloc")
+
+
+def lora_sgmv_auto_variant(T: int, n_segments: int, H1: int, r: int, H2: int, dtype: int, max_seg_len: int = 0,
+                           sm_count: int = 148) -> int:
+    """The variant lora_sgmv_apply (AUTO) runs for a call of these sizes (host only)."""
+    return int(load().lora_sgmv_auto_variant(T, n_segments, H1, r, H2, dtype, max_seg_len, sm_count))
 
 
 def lora_sgmv_pad_rank(A_dst, A_src, B_dst, B_src, H1: int, H2: int, r_src: int, r: int, dtype: int,

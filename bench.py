@@ -134,6 +134,27 @@ def make_spec(name: str) -> Spec:
                                     f"{len(w.touched_adapters())} adapters touched; step = 1 SGMV call")
 
 
+VARIANT_NAMES = {1: "SPLIT", 2: "GROUPED_TC", 3: "FUSED", 4: "FUSED_TC", 5: "SPLIT_TC"}
+
+
+def dispatch_name(spec: Spec, n_segments: int, max_len: int, dt: int, device):
+    """The kernels of one step, as the library's dispatcher chooses them (None if unknown)."""
+    try:
+        import torch
+
+        from adapter_matmul_b200 import sgmv
+
+        w = spec.w
+        if spec.P > 1:  # one batched launch: the fused kernel, on tcgen05 where the rule allows
+            tc = max_len > 2 and w.r >= 32 and w.r <= 64 and w.H1 % 64 == 0 and w.H2 % 64 == 0
+            return f"batched {'FUSED_TC' if tc else 'FUSED'} ({spec.P} projections per launch)"
+        sms = torch.cuda.get_device_properties(device).multi_processor_count
+        v = sgmv.lora_sgmv_auto_variant(w.T, n_segments, w.H1, w.r, w.H2, dt, max_len, sms)
+        return VARIANT_NAMES.get(v)
+    except Exception:
+        return None
+
+
 def max_over_ranks(x: float, world: int, device=None) -> float:
     """The largest of every rank's x (the slowest replica sets a multi-GPU time)."""
     if world <= 1:
@@ -548,6 +569,7 @@ def run_ours(args, spec: Spec, rank: int, world: int, local: int):
             "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
             "config": {"workload": spec.desc, "name": spec.name, "T": w.T, "H1": w.H1, "H2": w.H2, "r": w.r,
                        "adapters_touched": len(touched), "segments": n, "sgmv_calls_per_step": spec.P,
+                       "dispatch": dispatch_name(spec, n, max_len, dt, dev),
                        "layers_rotated": spec.L,
                        "l2": f"inputs larger than L2: {spec.L} layers rotated, "
                              f"{spec.L * spec.P * bytes_call / 2**30:.2f} GiB of algorithmic bytes per rotation",

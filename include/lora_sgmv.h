@@ -249,6 +249,25 @@ lora_sgmv_status lora_sgmv_apply(void* Y, const void* X, const void* const* A_pt
                                  lora_sgmv_dtype dtype, int32_t max_seg_len, void* workspace,
                                  size_t workspace_bytes, uint32_t* dev_status, void* stream);
 
+/*
+ * lora_sgmv_auto_variant -- the kernels lora_sgmv_apply (variant AUTO) runs for
+ * a call of these sizes on a GPU with sm_count SMs. Host arithmetic only: no
+ * CUDA call, no device needed.
+ *   T, n_segments, H1, r, H2, dtype, max_seg_len: as for lora_sgmv_apply.
+ *   sm_count     the device's multiprocessor count (148 on a B200).
+ * The rule: the longest segment (max_seg_len, else ceil(T / n_segments)) of
+ * at least 128 rows with r in {16, 32, 64} -> GROUPED_TC; else more than
+ * 8192 segments -> SPLIT; else segments of more than 2 tokens, r >= 32 and
+ * H1, H2 multiples of 64 -> SPLIT_TC when there are fewer jobs (16-token
+ * chunks, or segments when none is longer than 16) than SMs and each B_i
+ * holds at least 2 MB, else FUSED_TC; else FUSED.
+ * Returns LORA_SGMV_VARIANT_AUTO when a size or sm_count is not positive or
+ * dtype is unknown.
+ */
+lora_sgmv_variant lora_sgmv_auto_variant(int32_t T, int32_t n_segments, int32_t H1, int32_t r,
+                                         int32_t H2, lora_sgmv_dtype dtype, int32_t max_seg_len,
+                                         int32_t sm_count);
+
 /* lora_sgmv_apply with the kernels chosen by the caller. GROUPED_TC returns
  * LORA_SGMV_ERR_UNSUPPORTED for ranks or types it does not cover. */
 lora_sgmv_status lora_sgmv_apply_ex(void* Y, const void* X, const void* const* A_ptrs,

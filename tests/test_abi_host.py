@@ -177,3 +177,43 @@ def test_batched_validation_codes():
     assert call(na=0) == 2 and call(H1=0) == 2
     assert call(n=0, Y=None) == 0  # empty: OK before any CUDA call
     assert lib.lora_sgmv_apply_batched(None, 1, FAKE, FAKE, 1, 1, 16, 0, 0, None, None) == 1
+
+
+@pytest.mark.parametrize("name,want", [
+    ("tiny", "FUSED"), ("distinct", "FUSED"), ("uniform_h4096", "FUSED"), ("uniform_h11008", "FUSED"),
+    ("skewed_h4096", "FUSED"), ("skewed_h11008", "FUSED"), ("identical_h4096", "FUSED"),
+    ("identical_h11008", "FUSED"), ("prefill", "GROUPED_TC"), ("llama70b_decode_h28672", "SPLIT_TC"),
+    ("llama70b_decode_h8192", "FUSED_TC")])
+def test_auto_variant_on_the_configurations(name, want):
+    # the dispatcher's choice for each benchmark configuration on a 148-SM B200 (host only)
+    w = inputs.make(name)
+    seg, idx, _ = sgmv.lora_sgmv_group_segments(w.ids, w.num_adapters)
+    dt = sgmv.F16 if w.dtype == "f16" else sgmv.BF16
+    got = sgmv.lora_sgmv_auto_variant(w.T, len(idx), w.H1, w.r, w.H2, dt, int(np.max(np.diff(seg))), 148)
+    assert got == getattr(sgmv, "VARIANT_" + want)
+
+
+def test_auto_variant_rule_edges():
+    V, F16, BF16 = sgmv, sgmv.F16, sgmv.BF16
+    auto = sgmv.lora_sgmv_auto_variant
+    # the grouped kernel from one M-tile of rows, for the ranks it has
+    assert auto(4096, 8, 4096, 64, 4096, BF16, 128) == V.VARIANT_GROUPED_TC
+    assert auto(4096, 8, 4096, 64, 4096, BF16, 127) != V.VARIANT_GROUPED_TC
+    assert auto(4096, 8, 4096, 128, 4096, BF16, 512) == V.VARIANT_FUSED  # no tensor-core kernel at r = 128
+    # unknown length: ceil(T / n)
+    assert auto(1024, 8, 4096, 64, 4096, BF16, 0) == V.VARIANT_GROUPED_TC
+    # more segments than the fused kernels hold
+    assert auto(9000, 8193, 4096, 16, 4096, F16, 1) == V.VARIANT_SPLIT
+    # tensor-core decode needs segments of 3+ tokens, r >= 32, H multiples of 64
+    assert auto(256, 95, 8192, 64, 28672, BF16, 2) == V.VARIANT_FUSED
+    assert auto(256, 95, 8192, 16, 28672, BF16, 56) == V.VARIANT_FUSED
+    assert auto(256, 95, 8192, 64, 28680, BF16, 56) == V.VARIANT_FUSED
+    # the split form: fewer jobs than SMs and B_i of 2 MB or more
+    assert auto(256, 95, 8192, 64, 28672, BF16, 56, 148) == V.VARIANT_SPLIT_TC
+    assert auto(256, 95, 8192, 64, 28672, BF16, 56, 100) == V.VARIANT_FUSED_TC   # 111 jobs, 100 SMs
+    assert auto(256, 95, 8192, 64, 16384, BF16, 56, 148) == V.VARIANT_SPLIT_TC   # 2.1 MB
+    assert auto(256, 95, 8192, 64, 8192, BF16, 56, 148) == V.VARIANT_FUSED_TC    # 1 MB
+    # invalid sizes
+    assert auto(0, 1, 64, 16, 64, F16, 1) == V.VARIANT_AUTO
+    assert auto(8, 1, 64, 16, 64, 7, 1) == V.VARIANT_AUTO
+    assert auto(8, 1, 64, 16, 64, F16, 1, 0) == V.VARIANT_AUTO

@@ -119,3 +119,13 @@ def test_all_cores_baseline_runs_in_spawned_processes():
     out = bench.oracle_all_cores(bench.make_spec("tiny"), 0.3, max_procs=4)
     assert "unavailable" not in out, out
     assert out["kind"] == "oracle" and out["value"] > 0 and 1 <= out["cores"] <= 4
+
+
+def test_dispatch_name_of_the_batched_default_line():
+    import bench
+    from adapter_matmul_b200 import sgmv
+
+    spec = bench.make_spec("distinct")
+    assert bench.dispatch_name(spec, 32, 1, sgmv.F16, 0) == "batched FUSED (4 projections per launch)"
+    assert set(bench.VARIANT_NAMES.values()) == {"SPLIT", "GROUPED_TC", "FUSED", "FUSED_TC", "SPLIT_TC"}
+    assert all(getattr(sgmv, "VARIANT_" + name) == v for v, name in bench.VARIANT_NAMES.items())
