@@ -338,3 +338,18 @@ def test_grouped_tc_bad_segments_skipped():
     assert_close(got[:200], ref[:200], "bf16", "valid segment 0")
     assert_close(got[400:], ref[400:], "bf16", "valid segment 3")
     assert np.array_equal(got[200:400], before[200:400])
+
+
+@pytest.mark.parametrize("variant", [sgmv.VARIANT_AUTO, sgmv.VARIANT_SPLIT])
+def test_more_segments_than_the_flat_chunk_list(variant):
+    # 9000 segments of 0..3 tokens: more than the shrink's flat chunk list holds (8192 segments),
+    # so its clusters walk segment and chunk slots instead; AUTO takes the split kernels here
+    rng = np.random.default_rng(12)
+    lens = rng.integers(0, 4, 9000)
+    seg = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    idx = rng.integers(0, 5, 9000).astype(np.int32)
+    w = inputs.small_random(int(seg[-1]), 5, 256, 136, 16, "f16", seed=12)
+    p = DeviceProblem(w, y_random=True, adapters=list(range(5)), seg_starts=seg, lora_idx=idx)
+    got = p.apply(variant=variant)
+    assert int(p.status.item()) == 0
+    assert_close(got, p.oracle_apply(), "f16", f"9000 segments, variant {variant}")
