@@ -28,7 +28,8 @@
 //   X    one 3-D box {64 columns, 16 rows, KS/64 column blocks} of a view of X whose third
 //        dimension steps 128 bytes, landing as KS/64 swizzled K-major blocks of 16 rows,
 //   B_i  one 3-D box {64 columns, r rows, NB column blocks}, landing as NB MN-major blocks,
-//   Y    one or two 2-D boxes of 1, 4 or 16 rows (the smallest that holds the chunk).
+//   Y    exact 2-D boxes of 16, 8, 4, 2 and 1 rows (the binary digits of the chunk length,
+//        so no row of another segment is read or written).
 // A_i and B_i come from a device table, so their tensor maps are made on the device from a
 // template per problem (sgmv_tmap.cuh); X and Y maps are made on the host per call.
 //
@@ -40,6 +41,13 @@
 // TMEM lane quarter, each taking every other 128-column group of a stage; one of them also
 // runs the V exchange), 10 producer of Y. Programmatic dependent launch: X and Y are read only after
 // griddepcontrol.wait. Every wait is bounded in time.
+//
+// Pre-V mode (template flag PRE_V, the split form): V [T, r] (fp32) comes from an earlier
+// kernel (the split-K shrink) through global memory. There is no shrink and no cluster: each
+// job's H2 is cut into n_slices slices, every (job, slice) pair is a unit of work, and the
+// CTAs (independent, one per SM) take the units round-robin, so that a few large adapters
+// still spread over every SM. A unit reads its chunk's V rows after griddepcontrol.wait and
+// runs the same expand pipeline over its slice.
 #pragma once
 
 #include "sgmv_grouped_tc.cuh"
