@@ -406,10 +406,9 @@ bool decode_tc_preferred(int r, int max_len) { return max_len > 2 && r >= 32; }
 // spreads each job's N over independent CTAs) pays a second launch and a V round trip through
 // the workspace, and wins when the fused form would leave SMs idle: fewer jobs than SMs, each
 // with a large B_i (several MB) to stream.
-bool split_tc_preferred(int T, int n_segments, int max_len, int H1, int H2, int r, int sms) {
+bool split_tc_preferred(int T, int n_segments, int max_len, int H2, int r, int sms) {
     const long long chunks = std::min<long long>(n_segments + (T + 15) / 16, std::max(T, 1));
     const long long jobs = max_len <= 16 ? n_segments : chunks;
-    (void)H1;
     return jobs < sms && double(H2) * r * 2 >= 2e6;
 }
 
@@ -425,7 +424,7 @@ lora_sgmv_variant auto_variant(int T, int n_segments, int max_len, int H1, int H
         return LORA_SGMV_VARIANT_GROUPED_TC;
     if (n_segments > sgmv::kFusedMaxSegments) return LORA_SGMV_VARIANT_SPLIT;
     if (decode_tc_preferred(r, max_len) && decode_tc_supported(r, H1, H2))
-        return split_tc_preferred(T, n_segments, max_len, H1, H2, r, sms) ? LORA_SGMV_VARIANT_SPLIT_TC
+        return split_tc_preferred(T, n_segments, max_len, H2, r, sms) ? LORA_SGMV_VARIANT_SPLIT_TC
                                                                           : LORA_SGMV_VARIANT_FUSED_TC;
     return LORA_SGMV_VARIANT_FUSED;
 }
