@@ -24,7 +24,7 @@ namespace {
 using sgmv::ExpandParams;
 using sgmv::ShrinkParams;
 
-constexpr int kVersion = 100;  // 0.1.0
+constexpr int kVersion = 200;  // 0.2.0: variant SPLIT_TC, lora_sgmv_pad_rank, lora_sgmv_auto_variant
 
 // Number of kernels this library has launched successfully in this process.
 std::atomic<uint64_t> g_launches{0};

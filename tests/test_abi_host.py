@@ -34,7 +34,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_version_and_ranks():
-    assert sgmv.lora_sgmv_version() >= 100
+    assert sgmv.lora_sgmv_version() >= 200  # 0.2.0 or later
     for r in (8, 16, 32, 64, 128):
         assert sgmv.lora_sgmv_rank_supported(r, sgmv.VARIANT_SPLIT)
         assert sgmv.lora_sgmv_rank_supported(r, sgmv.VARIANT_FUSED)
