@@ -256,7 +256,7 @@ lora_sgmv_status lora_sgmv_apply(void* Y, const void* X, const void* const* A_pt
  *   T, n_segments, H1, r, H2, dtype, max_seg_len: as for lora_sgmv_apply.
  *   sm_count     the device's multiprocessor count (148 on a B200).
  * The rule: the longest segment (max_seg_len, else ceil(T / n_segments)) of
- * at least 128 rows with r in {16, 32, 64} -> GROUPED_TC; else more than
+ * at least 128 rows with r in {16, 32, 64} and H1, H2 >= 64 -> GROUPED_TC; else more than
  * 8192 segments -> SPLIT; else segments of more than 2 tokens, r >= 32 and
  * H1, H2 multiples of 64 -> SPLIT_TC when there are fewer jobs (16-token
  * chunks, or segments when none is longer than 16) than SMs and each B_i
