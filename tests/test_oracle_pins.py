@@ -126,6 +126,28 @@ def test_hand_worked_example_golden():
     assert np.array_equal(Y64, np.array(g["Y"]))
 
 
+def bf16_bits(vals):
+    """Exact bfloat16 bits of values that bfloat16 holds (torch's conversion, not the oracle's)."""
+    t = torch.tensor(np.asarray(vals, dtype=np.float64)).to(torch.bfloat16)
+    assert torch.equal(t.to(torch.float64), torch.tensor(np.asarray(vals, dtype=np.float64)))
+    return t.view(torch.int16).numpy().view(np.uint16)
+
+
+def test_hand_worked_bf16_example_with_scale_and_ties_golden():
+    g = json.load(open(os.path.join(GOLDEN, "lora_worked_example_bf16_ties.json")))
+    X, Y0 = bf16_bits(g["X"]), bf16_bits(g["Y_base"])
+    A = [bf16_bits(a) for a in g["A"]]
+    B = [bf16_bits(b) for b in g["B"]]
+    seg, idx, scale = g["seg_starts"], g["lora_idx"], g["scale"]
+    V, sk = oracle.shrink_f32(X, A, seg, idx, g["r"], "bf16")
+    assert sk == 0
+    assert np.array_equal(V, np.array(g["V"], dtype=np.float32))
+    Y, _ = oracle.apply_f32(Y0, X, A, B, seg, idx, scale, "bf16")
+    assert np.array_equal(dec(Y, "bf16"), np.array(g["Y"]))  # the two ties went to the even neighbour
+    Y64, _ = oracle.apply_f64(dec(Y0, "bf16"), X, A, B, seg, idx, scale, "bf16")
+    assert np.array_equal(Y64, np.array(g["Y_unrounded"]))
+
+
 @pytest.mark.parametrize("dt", ["f16", "bf16"])
 def test_identity_against_materialised_weight(dt):
     """x@(W + A@B) == x@W + (x@A)@B, with W + A@B materialised in fp64 by numpy."""
