@@ -398,3 +398,54 @@ def test_zero_padding_leaves_fp32_results_bit_identical(dt):
         own, sk1 = oracle.apply_f32(Y[b:e], X[b:e], [A[i]], [B[i]], [0, e - b], [0], 1.25, dt)
         assert sk1 == 0
         assert np.array_equal(got[b:e], own), s
+
+
+# ---------------------------------------------------------------------------------------------
+# algebraic invariants of the definition on random shapes (binary64 twin; small integer-valued
+# operands are exact in fp16, so sums of them are exact too)
+# ---------------------------------------------------------------------------------------------
+
+from hypothesis import given, settings  # noqa: E402
+from hypothesis import strategies as st  # noqa: E402
+
+
+def _int_case(rng, T, H1, r, H2, nA, lo=-3, hi=4):
+    X = f16_bits(rng.integers(lo, hi, (T, H1)))
+    A = [f16_bits(rng.integers(lo, hi, (H1, r))) for _ in range(nA)]
+    B = [f16_bits(rng.integers(lo, hi, (r, H2))) for _ in range(nA)]
+    return X, A, B
+
+
+@settings(max_examples=40, deadline=None)
+@given(st.integers(1, 12), st.integers(1, 9), st.integers(1, 5), st.integers(1, 9), st.integers(0, 10 ** 6))
+def test_delta_is_linear_in_scale_and_additive_in_B(T, H1, r, H2, seed):
+    rng = np.random.default_rng(seed)
+    X, A, B = _int_case(rng, T, H1, r, H2, 2)
+    B2 = [f16_bits(rng.integers(-3, 4, (r, H2))) for _ in range(2)]
+    Bsum = [f16_bits(dec(b, "f16") + dec(c, "f16")) for b, c in zip(B, B2)]  # |values| <= 6: exact
+    cut = int(rng.integers(0, T + 1))
+    seg, idx = [0, cut, T], [1, 0]
+    zero = np.zeros((T, H2))
+    d1, _ = oracle.apply_f64(zero, X, A, B, seg, idx, 1.0, "f16")
+    d2, _ = oracle.apply_f64(zero, X, A, B2, seg, idx, 1.0, "f16")
+    ds, _ = oracle.apply_f64(zero, X, A, Bsum, seg, idx, 1.0, "f16")
+    assert np.array_equal(ds, d1 + d2)                       # additive in B_i (exact: integers)
+    d3, _ = oracle.apply_f64(zero, X, A, B, seg, idx, -2.5, "f16")
+    assert np.array_equal(d3, -2.5 * d1)                     # linear in scale (exact: dyadic)
+    # against numpy's products, row by row with each row's own adapter
+    x = dec(X, "f16")
+    for t in range(T):
+        i = idx[0] if t < cut else idx[1]
+        assert np.array_equal(d1[t], (x[t] @ dec(A[i], "f16")) @ dec(B[i], "f16"))
+
+
+@settings(max_examples=30, deadline=None)
+@given(st.integers(2, 12), st.integers(1, 9), st.integers(1, 5), st.integers(1, 9), st.integers(0, 10 ** 6))
+def test_zero_rows_of_x_leave_y_unchanged(T, H1, r, H2, seed):
+    rng = np.random.default_rng(seed)
+    X, A, B = _int_case(rng, T, H1, r, H2, 3)
+    zero_rows = rng.random(T) < 0.5
+    X[zero_rows] = 0
+    Y = f16_bits(rng.integers(-8, 9, (T, H2)))
+    got, _ = oracle.apply_f32(Y, X, A, B, [0, T], [int(rng.integers(0, 3))], 0.75, "f16")
+    assert np.array_equal(got[zero_rows], Y[zero_rows])
