@@ -449,3 +449,54 @@ def test_zero_rows_of_x_leave_y_unchanged(T, H1, r, H2, seed):
     Y = f16_bits(rng.integers(-8, 9, (T, H2)))
     got, _ = oracle.apply_f32(Y, X, A, B, [0, T], [int(rng.integers(0, 3))], 0.75, "f16")
     assert np.array_equal(got[zero_rows], Y[zero_rows])
+
+
+# ---------------------------------------------------------------------------------------------
+# the one-element function used for sampled checks at full size
+# ---------------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("dt", ["f16", "bf16"])
+@pytest.mark.parametrize("r", [8, 16, 64, 128])
+def test_element_function_equals_whole_batch_bit_for_bit(dt, r):
+    # every element of ragged random problems (non-zero base output, scale not a power of two,
+    # several adapters, empty segment): oracle_apply_f32_element must give the bits that
+    # oracle_apply_f32 (pinned by everything above) writes there. A slip such as B_i indexed
+    # as [c, j], a dropped base term or scale applied per term fails it.
+    rng = np.random.default_rng(1000 + r)
+    T, H1, H2, nA = 11, 72, 40, 3
+    X = inputs.cast_f32_bits(rng.standard_normal((T, H1)).astype(np.float32), dt)
+    A = [inputs.cast_f32_bits((rng.standard_normal((H1, r)) / np.sqrt(H1)).astype(np.float32), dt)
+         for _ in range(nA)]
+    B = [inputs.cast_f32_bits((rng.standard_normal((r, H2)) / np.sqrt(r)).astype(np.float32), dt)
+         for _ in range(nA)]
+    Y = inputs.cast_f32_bits(rng.standard_normal((T, H2)).astype(np.float32), dt)
+    seg, idx = [0, 4, 4, 9, 11], [2, 0, 1, 2]
+    for scale in (0.6180339887, -1.75):
+        full, _ = oracle.apply_f32(Y, X, A, B, seg, idx, scale, dt)
+        for s in range(len(idx)):
+            for t in range(seg[s], seg[s + 1]):
+                for c in range(H2):
+                    got = oracle.apply_f32_element(X[t], A[idx[s]], B[idx[s]], int(Y[t, c]), c, scale, dt)
+                    assert got == int(full[t, c]), (dt, r, scale, t, c)
+
+
+@pytest.mark.parametrize("dt", ["f16", "bf16"])
+def test_element_function_exact_on_integer_operands(dt):
+    # small integers: every product and sum is exact in fp32, so the element equals numpy's
+    # y + scale * (x @ A) @ B exactly (scale 0.5 keeps it dyadic), independently of the oracle
+    rng = np.random.default_rng(77)
+    H1, r, H2 = 24, 8, 16
+    enc = f16_bits if dt == "f16" else bf16_bits
+    x = enc(rng.integers(-3, 4, H1))
+    Ai = enc(rng.integers(-2, 3, (H1, r)))
+    Bi = enc(rng.integers(-2, 3, (r, H2)))
+    y = enc(rng.integers(-20, 21, H2))
+    exact = dec(y, dt) + 0.5 * ((dec(x, dt) @ dec(Ai, dt)) @ dec(Bi, dt))
+    # one rounding of the exact value to the storage type, by numpy / torch
+    if dt == "f16":
+        ref = exact.astype(np.float16).astype(np.float64)
+    else:
+        ref = torch.tensor(exact).to(torch.float32).to(torch.bfloat16).to(torch.float64).numpy()
+    for c in range(H2):
+        got = oracle.apply_f32_element(x, Ai, Bi, int(y[c]), c, 0.5, dt)
+        assert dec(np.array([got], np.uint16), dt)[0] == ref[c], c
