@@ -75,6 +75,9 @@ def _load():
             lib.oracle_expand_f64.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i32, ctypes.c_double, ctypes.c_int]
             lib.oracle_apply_f64.restype = ctypes.c_int
             lib.oracle_apply_f64.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, ctypes.c_double, ctypes.c_int]
+            lib.oracle_base_plus_delta_f32.restype = ctypes.c_int
+            lib.oracle_base_plus_delta_f32.argtypes = [P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32,
+                                                       ctypes.c_float, ctypes.c_int]
             lib.oracle_apply_f32_element.restype = ctypes.c_uint16
             lib.oracle_apply_f32_element.argtypes = [P, P, P, ctypes.c_uint16, i32, i32, i32, i32, ctypes.c_float, ctypes.c_int]
             _lib = lib
@@ -186,6 +189,22 @@ def apply_f32_element(x_row, Ai, Bi, y_in_bits: int, c: int, scale: float, dtype
     H2 = Bi.shape[1]
     return int(_load().oracle_apply_f32_element(_ptr(x_row), _ptr(Ai), _ptr(Bi), int(y_in_bits), H1, r, H2,
                                                 int(c), float(scale), _DT[dtype]))
+
+
+def base_plus_delta_f32(X, W, A: Sequence[np.ndarray], B: Sequence[np.ndarray], seg_starts, lora_idx,
+                        scale: float, dtype: str) -> Tuple[np.ndarray, int]:
+    """Y = round(X@W + scale * (X@A_i)@B_i) per row (round(X@W) for rows in no valid segment)."""
+    X, W = _u16(X), _u16(W)
+    T, H1 = X.shape
+    H2 = W.shape[1]
+    assert W.shape[0] == H1
+    r = A[0].shape[1] if len(A) else 0
+    Y = np.zeros((T, H2), dtype=np.uint16)
+    seg, idx = _i32(seg_starts), _i32(lora_idx)
+    ta, tb = _Table(A), _Table(B)
+    sk = _load().oracle_base_plus_delta_f32(_ptr(Y), _ptr(X), _ptr(W), ta.ptr, tb.ptr, _ptr(seg), _ptr(idx),
+                                            idx.shape[0], len(A), T, H1, r, H2, float(scale), _DT[dtype])
+    return Y, sk
 
 
 # -- binary64 twin ------------------------------------------------------------------

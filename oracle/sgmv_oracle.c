@@ -19,6 +19,9 @@
  *     segments, segment s (rows seg_starts[s] .. seg_starts[s+1]-1) using
  *     adapter lora_idx[s], and adds it onto the base output already in Y.
  *
+ * oracle_base_plus_delta_f32 computes the whole batch form, Y = X@W plus the
+ * delta, for the layer that fuses the delta into the base product.
+ *
  * The kernel contract adds a scale factor: Y[t,:] += scale * (X[t,:]@A_i)@B_i.
  * The product is taken as (x@A)@B -- shrink H1 -> r, then expand r -> H2 --
  * which is the association the README's identity writes.
@@ -347,4 +350,71 @@ uint16_t oracle_apply_f32_element(const uint16_t* x_row, const uint16_t* Ai, con
     const float delta = scale * acc;
     const float out = (float)decode(y_in, dtype) + delta;
     return encode((double)out, dtype);
+}
+
+/* ---------------------------------------------------------------------- */
+/* The whole layer: base product plus the delta                             */
+/* ---------------------------------------------------------------------- */
+
+/*
+ * Y = X@W + (x_t@A_i@B_i)_t, the multi-LoRA batch of the README's multi-LoRA
+ * paragraph with the kernel contract's scale: for every row t,
+ *   base[c] = sum_k X[t, k] * W[k, c]               (fp32, k ascending)
+ * and, when row t lies in a valid segment s with adapter i = lora_idx[s],
+ *   v[j]    = sum_k X[t, k] * A_i[k, j]             (fp32, k ascending)
+ *   acc[c]  = sum_j v[j] * B_i[j, c]                (fp32, j ascending)
+ *   Y[t, c] = round(base[c] + scale * acc[c])
+ * else Y[t, c] = round(base[c]). W is [H1, H2] row-major; Y is written, not
+ * read. A row covered by several segments gets the delta of the last one
+ * (segments must not overlap). Returns the number of skipped segments.
+ */
+int oracle_base_plus_delta_f32(uint16_t* Y, const uint16_t* X, const uint16_t* W,
+                               const uint16_t* const* A, const uint16_t* const* B,
+                               const int32_t* seg_starts, const int32_t* lora_idx,
+                               int32_t n_segments, int32_t num_adapters, int32_t T, int32_t H1,
+                               int32_t r, int32_t H2, float scale, int dtype)
+{
+    int skipped = 0;
+    int32_t* owner = (int32_t*)malloc(sizeof(int32_t) * ((size_t)T + 1));
+    float* base = (float*)malloc(sizeof(float) * ((size_t)H2 + 1));
+    float* xrow = (float*)malloc(sizeof(float) * ((size_t)H1 + 1));
+    float* v = (float*)malloc(sizeof(float) * ((size_t)r + 1));
+    for (int32_t t = 0; t < T; ++t) owner[t] = -1;
+    for (int32_t s = 0; s < n_segments; ++s) {
+        if (!segment_valid(seg_starts, lora_idx, s, T, num_adapters)) { ++skipped; continue; }
+        for (int32_t t = seg_starts[s]; t < seg_starts[s + 1]; ++t) owner[t] = lora_idx[s];
+    }
+    for (int32_t t = 0; t < T; ++t) {
+        for (int32_t k = 0; k < H1; ++k) xrow[k] = (float)decode(X[(size_t)t * H1 + k], dtype);
+        for (int32_t c = 0; c < H2; ++c) base[c] = 0.0f;
+        for (int32_t k = 0; k < H1; ++k) {
+            const float xk = xrow[k];
+            const uint16_t* wrow = W + (size_t)k * H2;
+            for (int32_t c = 0; c < H2; ++c) base[c] += xk * (float)decode(wrow[c], dtype);
+        }
+        uint16_t* y = Y + (size_t)t * H2;
+        if (owner[t] < 0) {
+            for (int32_t c = 0; c < H2; ++c) y[c] = encode((double)base[c], dtype);
+            continue;
+        }
+        const uint16_t* Ai = A[owner[t]];
+        const uint16_t* Bi = B[owner[t]];
+        for (int32_t j = 0; j < r; ++j) v[j] = 0.0f;
+        for (int32_t k = 0; k < H1; ++k) {
+            const float xk = xrow[k];
+            const uint16_t* arow = Ai + (size_t)k * r;
+            for (int32_t j = 0; j < r; ++j) v[j] += xk * (float)decode(arow[j], dtype);
+        }
+        for (int32_t c = 0; c < H2; ++c) {
+            float acc = 0.0f;
+            for (int32_t j = 0; j < r; ++j) acc += v[j] * (float)decode(Bi[(size_t)j * H2 + c], dtype);
+            const float delta = scale * acc;
+            y[c] = encode((double)(base[c] + delta), dtype);
+        }
+    }
+    free(owner);
+    free(base);
+    free(xrow);
+    free(v);
+    return skipped;
 }

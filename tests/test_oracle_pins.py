@@ -500,3 +500,102 @@ def test_element_function_exact_on_integer_operands(dt):
     for c in range(H2):
         got = oracle.apply_f32_element(x, Ai, Bi, int(y[c]), c, 0.5, dt)
         assert dec(np.array([got], np.uint16), dt)[0] == ref[c], c
+
+
+# ---------------------------------------------------------------------------------------------
+# the whole layer, Y = X@W + the delta (README multi-LoRA paragraph): base_plus_delta_f32
+# ---------------------------------------------------------------------------------------------
+
+def _layer_int_case(rng, dt, T=13, H1=24, H2=20, r=4, nA=3):
+    enc = f16_bits if dt == "f16" else bf16_bits
+    X = enc(rng.integers(-3, 4, (T, H1)))
+    W = enc(rng.integers(-3, 4, (H1, H2)))
+    A = [enc(rng.integers(-2, 3, (H1, r))) for _ in range(nA)]
+    B = [enc(rng.integers(-2, 3, (r, H2))) for _ in range(nA)]
+    return X, W, A, B
+
+
+def _round_to(values, dt):
+    """One round-to-nearest-even of exact values to the storage type (numpy / torch)."""
+    if dt == "f16":
+        return values.astype(np.float16).astype(np.float64)
+    return torch.tensor(values).to(torch.float32).to(torch.bfloat16).to(torch.float64).numpy()
+
+
+@pytest.mark.parametrize("dt", ["f16", "bf16"])
+def test_layer_identity_with_materialised_weight(dt):
+    # integer operands: every product and partial sum is exact in fp32, so the layer must equal,
+    # bit for bit, x @ (W + scale * A_i @ B_i) with the merged weight built in fp64 by numpy --
+    # the README identity x@(W + A@B) = x@W + x@A@B, row by row with each row's own adapter;
+    # rows in no segment (0, 1 and 12) and the rejected segment's rows get x@W alone
+    rng = np.random.default_rng(31)
+    X, W, A, B = _layer_int_case(rng, dt)
+    seg = [2, 5, 5, 9, 11, 12]
+    idx = [2, 0, 1, 7, 0]  # [5,5) empty; adapter 7 does not exist: [9,11) rejected
+    got, skipped = oracle.base_plus_delta_f32(X, W, A, B, seg, idx, 0.5, dt)
+    assert skipped == 1
+    x, w = dec(X, dt), dec(W, dt)
+    owner = {t: i for s, i in enumerate(idx) if i < 3 for t in range(seg[s], seg[s + 1])}
+    for t in range(X.shape[0]):
+        merged = w if t not in owner else w + 0.5 * (dec(A[owner[t]], dt) @ dec(B[owner[t]], dt))
+        assert np.array_equal(dec(got[t], dt), _round_to(x[t] @ merged, dt)), t
+
+
+@pytest.mark.parametrize("dt", ["f16", "bf16"])
+def test_layer_with_zero_weight_is_the_delta_alone(dt):
+    # W = 0: base is +0 everywhere, so each row equals what the SGMV oracle (pinned above) adds
+    # onto a zero base, bit for bit
+    rng = np.random.default_rng(5)
+    T, H1, H2, r = 10, 40, 24, 8
+    X = inputs.cast_f32_bits(rng.standard_normal((T, H1)).astype(np.float32), dt)
+    A = [inputs.cast_f32_bits((rng.standard_normal((H1, r)) / 6).astype(np.float32), dt) for _ in range(2)]
+    B = [inputs.cast_f32_bits((rng.standard_normal((r, H2)) / 3).astype(np.float32), dt) for _ in range(2)]
+    W = np.zeros((H1, H2), np.uint16)
+    seg, idx = [0, 4, 10], [1, 0]
+    got, _ = oracle.base_plus_delta_f32(X, W, A, B, seg, idx, 0.7, dt)
+    ref, _ = oracle.apply_f32(np.zeros((T, H2), np.uint16), X, A, B, seg, idx, 0.7, dt)
+    assert np.array_equal(got, ref)
+
+
+@pytest.mark.parametrize("dt", ["f16", "bf16"])
+def test_layer_without_segments_is_the_base_product(dt):
+    # no segments: Y = round(X@W); against numpy's fp64 product within the fp32 summation bound
+    # plus one rounding of the storage type
+    rng = np.random.default_rng(6)
+    T, H1, H2 = 9, 96, 33
+    X = inputs.cast_f32_bits(rng.standard_normal((T, H1)).astype(np.float32), dt)
+    W = inputs.cast_f32_bits((rng.standard_normal((H1, H2)) / np.sqrt(H1)).astype(np.float32), dt)
+    A = [np.zeros((H1, 4), np.uint16)]
+    B = [np.zeros((4, H2), np.uint16)]
+    got, _ = oracle.base_plus_delta_f32(X, W, A, B, [0], [], 1.0, dt)
+    x, w = dec(X, dt), dec(W, dt)
+    exact = x @ w
+    bound = H1 * 2.0 ** -24 * (np.abs(x) @ np.abs(w))
+    ulp = 2.0 ** (-10 if dt == "f16" else -7) * np.maximum(np.abs(exact), 2.0 ** -14)
+    assert np.all(np.abs(dec(got, dt) - exact) <= ulp + bound)
+
+
+@pytest.mark.parametrize("dt", ["f16", "bf16"])
+def test_layer_random_operands_against_fp64_merged_weight(dt):
+    # random normal operands, several adapters and a non-dyadic scale: within the fp32 bound of
+    # the merged-weight product in fp64, plus one storage rounding
+    rng = np.random.default_rng(8)
+    T, H1, H2, r = 16, 64, 40, 8
+    X = inputs.cast_f32_bits(rng.standard_normal((T, H1)).astype(np.float32), dt)
+    W = inputs.cast_f32_bits((rng.standard_normal((H1, H2)) / np.sqrt(H1)).astype(np.float32), dt)
+    A = [inputs.cast_f32_bits((rng.standard_normal((H1, r)) / np.sqrt(H1)).astype(np.float32), dt)
+         for _ in range(3)]
+    B = [inputs.cast_f32_bits((rng.standard_normal((r, H2)) / np.sqrt(r)).astype(np.float32), dt)
+         for _ in range(3)]
+    seg, idx = [0, 5, 11, 16], [2, 0, 1]
+    scale = 0.37
+    got, _ = oracle.base_plus_delta_f32(X, W, A, B, seg, idx, scale, dt)
+    x, w = dec(X, dt), dec(W, dt)
+    for s in range(3):
+        a, b = dec(A[idx[s]], dt), dec(B[idx[s]], dt)
+        rows = slice(seg[s], seg[s + 1])
+        exact = x[rows] @ (w + scale * (a @ b))
+        terms = np.abs(x[rows]) @ np.abs(w) + abs(scale) * ((np.abs(x[rows]) @ np.abs(a)) @ np.abs(b))
+        bound = (H1 + r + 2) * 2.0 ** -24 * terms
+        ulp = 2.0 ** (-10 if dt == "f16" else -7) * np.maximum(np.abs(exact), 2.0 ** -14)
+        assert np.all(np.abs(dec(got[rows], dt) - exact) <= ulp + bound), s
