@@ -15,8 +15,10 @@
 #include "../../include/lora_sgmv.h"
 #include "sgmv_decode_tc.cuh"
 #include "sgmv_fused.cuh"
+#include "sgmv_gemm_tc.cuh"
 #include "sgmv_grouped_tc.cuh"
 #include "sgmv_pad.cuh"
+#include "sgmv_shrink_tma.cuh"
 #include "sgmv_split.cuh"
 
 namespace {
@@ -24,7 +26,7 @@ namespace {
 using sgmv::ExpandParams;
 using sgmv::ShrinkParams;
 
-constexpr int kVersion = 200;  // 0.2.0: variant SPLIT_TC, lora_sgmv_pad_rank, lora_sgmv_auto_variant
+constexpr int kVersion = 300;  // 0.3.0: early reads before the PDL wait only on request (flags)
 
 // Number of kernels this library has launched successfully in this process.
 std::atomic<uint64_t> g_launches{0};
@@ -107,8 +109,123 @@ int cluster_size_for(int H1) {
     return c;
 }
 
+// Largest number of clusters of `cluster` CTAs with `smem` bytes each that can be resident at once.
+template <typename K>
+lora_sgmv_status max_active_clusters(K kernel, int cluster, size_t smem, int* out, int threads = sgmv::kFusedThreads) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(cluster, 1, 1);
+    cfg.blockDim = dim3(threads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = cluster;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (record(cudaOccupancyMaxActiveClusters(&n, kernel, &cfg)) != cudaSuccess || n <= 0) return LORA_SGMV_ERR_CUDA;
+    *out = n;
+    return LORA_SGMV_OK;
+}
+
+// Cluster size of the TMA shrink: slices of A_i of at least 512 rows, at most 8 CTAs.
+int shrink_tma_cluster(int H1) {
+    int C = 1;
+    while (C < 8 && H1 / (C * 2) >= 512) C *= 2;
+    return C;
+}
+
+// The shrink with every operand staged by TMA (sgmv_shrink_tma.cuh).
+template <typename T, int R>
+lora_sgmv_status launch_shrink_tma(const ShrinkParams& p0, cudaStream_t stream) {
+    using G = sgmv::ShrinkTmaGeom<R>;
+    static int smem_granted[64] = {};
+    static int resident[64][4][9] = {};  // (device, log2 cluster size, prefix bucket)
+    const int C = shrink_tma_cluster(p0.H1);
+    sgmv::ShrinkTmaParams p = {};
+    p.V = p0.V;
+    p.A_ptrs = p0.A_ptrs;
+    p.B_check = p0.B_check;
+    p.seg_starts = p0.seg_starts;
+    p.lora_idx = p0.lora_idx;
+    p.dev_status = p0.dev_status;
+    p.n_segments = p0.n_segments;
+    p.num_adapters = p0.num_adapters;
+    p.T = p0.T;
+    p.H1 = p0.H1;
+    p.ks = ((p0.H1 + C - 1) / C + 63) / 64 * 64;
+    p.share = ((G::TILE + C - 1) / C + 3) / 4 * 4;
+    const int bucket = (p.n_segments + 1 + 1023) / 1024;  // 1..9
+    const size_t smem = G::BASE + 2 * G::x_bytes(p.ks) + size_t(bucket) * 1024 * 4;
+    DeviceFacts f;
+    if (device_facts(f) != LORA_SGMV_OK) return LORA_SGMV_ERR_CUDA;
+    if (smem + 2048 > static_cast<size_t>(f.max_smem_optin)) return LORA_SGMV_ERR_DIM;
+    auto kernel = sgmv::sgmv_shrink_tma_kernel<T, R>;
+    if (ensure_smem(kernel, smem, smem_granted) != LORA_SGMV_OK) return LORA_SGMV_ERR_CUDA;
+    int dev = 0;
+    if (record(cudaGetDevice(&dev)) != cudaSuccess) return LORA_SGMV_ERR_CUDA;
+    if (dev < 0 || dev >= 64) return LORA_SGMV_ERR_UNSUPPORTED;
+    const int lc = C == 1 ? 0 : (C == 2 ? 1 : (C == 4 ? 2 : 3));
+    int clusters_max = 0;
+    {
+        std::lock_guard<std::mutex> lock(g_mu);
+        clusters_max = resident[dev][lc][bucket - 1];
+    }
+    if (clusters_max <= 0) {
+        lora_sgmv_status st = max_active_clusters(kernel, C, smem, &clusters_max, sgmv::kSTThreads);
+        if (st != LORA_SGMV_OK) return st;
+        std::lock_guard<std::mutex> lock(g_mu);
+        resident[dev][lc][bucket - 1] = clusters_max;
+    }
+    CUtensorMap tmX;
+    if (!sgmv::make_shrink_x_map(&tmX, p0.X, p.T, p.H1, p.ks,
+                                 std::is_same<T, __half>::value ? LORA_SGMV_F16 : LORA_SGMV_BF16)) {
+        t_last_error = cudaErrorInvalidValue;
+        return LORA_SGMV_ERR_CUDA;
+    }
+    // units: at most one chunk per token and one partial chunk per segment
+    const long long units = std::max<long long>(
+        1, std::min<long long>(static_cast<long long>(p.n_segments) + (p.T + sgmv::kSTTokens - 1) / sgmv::kSTTokens,
+                               p.T));
+    int clusters = static_cast<int>(std::min<long long>(units, clusters_max));
+    const long long rounds = (units + clusters - 1) / clusters;
+    clusters = static_cast<int>((units + rounds - 1) / rounds);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(clusters * C, 1, 1);
+    cfg.blockDim = dim3(sgmv::kSTThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = C;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return counted(cudaLaunchKernelEx(&cfg, kernel, tmX, p));
+}
+
+// Whether the TMA shrink takes a call: H1 a multiple of 64, its unit list and X buffers in
+// shared memory (at most 8192 segments, at most kSTMaxKs rows of A_i per CTA).
+template <int R>
+bool shrink_tma_fits(int H1, int n_segments, int max_smem_optin) {
+    if (H1 % 64 != 0 || n_segments > sgmv::kSTMaxSegments) return false;
+    const int C = shrink_tma_cluster(H1);
+    const int ks = ((H1 + C - 1) / C + 63) / 64 * 64;
+    if (ks > sgmv::kSTMaxKs) return false;
+    const int bucket = (n_segments + 1 + 1023) / 1024;
+    using G = sgmv::ShrinkTmaGeom<R>;
+    return G::BASE + 2 * G::x_bytes(ks) + size_t(bucket) * 1024 * 4 + 2048 <= size_t(max_smem_optin);
+}
+
 template <typename T, int R>
 lora_sgmv_status launch_shrink(const ShrinkParams& p0, int max_len, cudaStream_t stream) {
+    {
+        DeviceFacts f;
+        if (device_facts(f) != LORA_SGMV_OK) return LORA_SGMV_ERR_CUDA;
+        if (shrink_tma_fits<R>(p0.H1, p0.n_segments, f.max_smem_optin)) return launch_shrink_tma<T, R>(p0, stream);
+    }
     static int smem_granted[64] = {};
     ShrinkParams p = p0;
     const int C = cluster_size_for(p.H1);
@@ -197,10 +314,30 @@ lora_sgmv_status expand_dispatch(const ExpandParams& p, int r, lora_sgmv_dtype d
 
 // ---- grouped tensor-core path ------------------------------------------------------------------
 
+template <bool V_OUT>
+cudaError_t grouped_launch_r(int r, bool bf, const CUtensorMap& tmX, const CUtensorMap& tmY, const CUtensorMap& tmA,
+                             const CUtensorMap& tmB, const sgmv::GroupedParams& P, int blocks, cudaStream_t stream) {
+    switch (r) {
+        case 16:
+            return bf ? sgmv::launch_grouped_tc_kernel<__nv_bfloat16, 16, V_OUT>(tmX, tmY, tmA, tmB, P, blocks, stream)
+                      : sgmv::launch_grouped_tc_kernel<__half, 16, V_OUT>(tmX, tmY, tmA, tmB, P, blocks, stream);
+        case 32:
+            return bf ? sgmv::launch_grouped_tc_kernel<__nv_bfloat16, 32, V_OUT>(tmX, tmY, tmA, tmB, P, blocks, stream)
+                      : sgmv::launch_grouped_tc_kernel<__half, 32, V_OUT>(tmX, tmY, tmA, tmB, P, blocks, stream);
+        case 64:
+            return bf ? sgmv::launch_grouped_tc_kernel<__nv_bfloat16, 64, V_OUT>(tmX, tmY, tmA, tmB, P, blocks, stream)
+                      : sgmv::launch_grouped_tc_kernel<__half, 64, V_OUT>(tmX, tmY, tmA, tmB, P, blocks, stream);
+    }
+    return cudaErrorInvalidValue;
+}
+
+// The grouped tensor-core kernel: the whole SGMV (v_out null), or only the shrink, V = X@A_i
+// (fp32) into v_out, with Y unused (the whole-layer path).
 lora_sgmv_status launch_grouped(void* Y, const void* X, const void* const* A_ptrs, const void* const* B_ptrs,
                                 const int32_t* seg_starts, const int32_t* lora_idx, int n_segments, int num_adapters,
                                 int T, int H1, int r, int H2, float scale, lora_sgmv_dtype dt, uint32_t* dev_status,
-                                cudaStream_t stream) {
+                                cudaStream_t stream, float* v_out = nullptr, const int32_t* ranks = nullptr) {
+    if (r != 16 && r != 32 && r != 64) return LORA_SGMV_ERR_UNSUPPORTED;
     DeviceFacts f;
     if (device_facts(f) != LORA_SGMV_OK) return LORA_SGMV_ERR_CUDA;
     // Rows per M-tile: the fewest that keep every tile in one wave (at most ceil(T/tm) + n tiles
@@ -211,7 +348,8 @@ lora_sgmv_status launch_grouped(void* Y, const void* X, const void* const* A_ptr
     int tm = static_cast<int>(std::min<long long>(sgmv::kGM, ((static_cast<long long>(T) + sms_avail - 1) / sms_avail + 7) / 8 * 8));
     tm = std::max(tm, 64);
     CUtensorMap tmX, tmY;
-    if (!sgmv::make_tile_map(&tmX, X, T, H1, dt, tm) || !sgmv::make_tile_map(&tmY, Y, T, H2, dt, tm)) {
+    if (!sgmv::make_tile_map(&tmX, X, T, H1, dt, tm) ||
+        !sgmv::make_tile_map(&tmY, v_out ? X : Y, T, v_out ? H1 : H2, dt, tm)) {  // (unused with v_out)
         t_last_error = cudaErrorInvalidValue;
         return LORA_SGMV_ERR_CUDA;
     }
@@ -228,6 +366,8 @@ lora_sgmv_status launch_grouped(void* Y, const void* X, const void* const* A_ptr
     P.H1 = H1;
     P.H2 = H2;
     P.scale = scale;
+    P.v_out = v_out;
+    P.ranks = ranks;
     // templates of the A_i and B_i maps; each CTA replaces the address with its adapter's
     CUtensorMap tmA, tmB;
     {
@@ -267,28 +407,15 @@ lora_sgmv_status launch_grouped(void* Y, const void* X, const void* const* A_ptr
             }
         }
     }
+    if (v_out) nsplit = 1;  // the shrink alone: one CTA per M-tile
     const int span_tiles = ((H2 + sgmv::kGN - 1) / sgmv::kGN + nsplit - 1) / nsplit;
     P.nspan = span_tiles * sgmv::kGN;
     P.nsplit = (H2 + P.nspan - 1) / P.nspan;
     const long long blocks = tiles_ub * P.nsplit;
     if (blocks > (1ll << 31) - 1) return LORA_SGMV_ERR_DIM;
-    cudaError_t e = cudaSuccess;
     const bool bf = dt == LORA_SGMV_BF16;
-    switch (r) {
-        case 16:
-            e = bf ? sgmv::launch_grouped_tc_kernel<__nv_bfloat16, 16>(tmX, tmY, tmA, tmB, P, int(blocks), stream)
-                   : sgmv::launch_grouped_tc_kernel<__half, 16>(tmX, tmY, tmA, tmB, P, int(blocks), stream);
-            break;
-        case 32:
-            e = bf ? sgmv::launch_grouped_tc_kernel<__nv_bfloat16, 32>(tmX, tmY, tmA, tmB, P, int(blocks), stream)
-                   : sgmv::launch_grouped_tc_kernel<__half, 32>(tmX, tmY, tmA, tmB, P, int(blocks), stream);
-            break;
-        case 64:
-            e = bf ? sgmv::launch_grouped_tc_kernel<__nv_bfloat16, 64>(tmX, tmY, tmA, tmB, P, int(blocks), stream)
-                   : sgmv::launch_grouped_tc_kernel<__half, 64>(tmX, tmY, tmA, tmB, P, int(blocks), stream);
-            break;
-        default: return LORA_SGMV_ERR_UNSUPPORTED;
-    }
+    const cudaError_t e = v_out ? grouped_launch_r<true>(r, bf, tmX, tmY, tmA, tmB, P, int(blocks), stream)
+                                : grouped_launch_r<false>(r, bf, tmX, tmY, tmA, tmB, P, int(blocks), stream);
     return counted(e);
 }
 
@@ -300,26 +427,6 @@ int estimate_max_len(int max_seg_len, int T, int n) {
 // ---- fused path ---------------------------------------------------------------------------
 
 int round8(int v) { return (v + 7) / 8 * 8; }
-
-// Largest number of clusters of `cluster` CTAs with `smem` bytes each that can be resident at once.
-template <typename K>
-lora_sgmv_status max_active_clusters(K kernel, int cluster, size_t smem, int* out, int threads = sgmv::kFusedThreads) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(cluster, 1, 1);
-    cfg.blockDim = dim3(threads, 1, 1);
-    cfg.dynamicSmemBytes = smem;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = cluster;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    int n = 0;
-    if (record(cudaOccupancyMaxActiveClusters(&n, kernel, &cfg)) != cudaSuccess || n <= 0) return LORA_SGMV_ERR_CUDA;
-    *out = n;
-    return LORA_SGMV_OK;
-}
 
 template <typename T, int R>
 lora_sgmv_status launch_fused(sgmv::FusedParams P, int max_len, cudaStream_t stream) {
@@ -802,13 +909,14 @@ lora_sgmv_status lora_sgmv_expand(void* Y, const float* V, const void* const* B_
     return expand_dispatch(p, r, dtype, max_len, false, static_cast<cudaStream_t>(stream));
 }
 
-lora_sgmv_status lora_sgmv_apply_ex(void* Y, const void* X, const void* const* A_ptrs,
-                                    const void* const* B_ptrs, const int32_t* seg_starts,
-                                    const int32_t* lora_idx, int32_t n_segments, int32_t num_adapters,
-                                    int32_t T, int32_t H1, int32_t r, int32_t H2, float scale,
-                                    lora_sgmv_dtype dtype, int32_t max_seg_len, void* workspace,
-                                    size_t workspace_bytes, uint32_t* dev_status, lora_sgmv_variant variant,
-                                    void* stream) {
+lora_sgmv_status lora_sgmv_apply_flags(void* Y, const void* X, const void* const* A_ptrs,
+                                       const void* const* B_ptrs, const int32_t* seg_starts,
+                                       const int32_t* lora_idx, int32_t n_segments, int32_t num_adapters,
+                                       int32_t T, int32_t H1, int32_t r, int32_t H2, float scale,
+                                       lora_sgmv_dtype dtype, int32_t max_seg_len, void* workspace,
+                                       size_t workspace_bytes, uint32_t* dev_status, lora_sgmv_variant variant,
+                                       uint32_t flags, void* stream) {
+    if (flags & ~uint32_t(LORA_SGMV_FLAG_EARLY_READS)) return LORA_SGMV_ERR_UNSUPPORTED;
     lora_sgmv_status st = check_common(n_segments, num_adapters, T, dtype);
     if (st != LORA_SGMV_OK) return st;
     if (H1 <= 0 || H2 <= 0 || r <= 0) return LORA_SGMV_ERR_DIM;
@@ -852,6 +960,7 @@ lora_sgmv_status lora_sgmv_apply_ex(void* Y, const void* X, const void* const* A
         P.n_problems = 1;
         P.n_segments = n_segments;
         P.T = T;
+        P.early = (flags & LORA_SGMV_FLAG_EARLY_READS) ? 1 : 0;
         if (v == LORA_SGMV_VARIANT_FUSED_TC) return decode_tc_dispatch(P, r, dtype, max_len, s);
         if (v == LORA_SGMV_VARIANT_SPLIT_TC) {
             // V first (split-K shrink kernel, fp32 into the workspace), then the expand spread
@@ -915,6 +1024,18 @@ lora_sgmv_status lora_sgmv_apply_ex(void* Y, const void* X, const void* const* A
     return expand_dispatch(ep, r, dtype, max_len, true, s);
 }
 
+lora_sgmv_status lora_sgmv_apply_ex(void* Y, const void* X, const void* const* A_ptrs,
+                                    const void* const* B_ptrs, const int32_t* seg_starts,
+                                    const int32_t* lora_idx, int32_t n_segments, int32_t num_adapters,
+                                    int32_t T, int32_t H1, int32_t r, int32_t H2, float scale,
+                                    lora_sgmv_dtype dtype, int32_t max_seg_len, void* workspace,
+                                    size_t workspace_bytes, uint32_t* dev_status, lora_sgmv_variant variant,
+                                    void* stream) {
+    return lora_sgmv_apply_flags(Y, X, A_ptrs, B_ptrs, seg_starts, lora_idx, n_segments, num_adapters, T, H1, r,
+                                 H2, scale, dtype, max_seg_len, workspace, workspace_bytes, dev_status, variant, 0u,
+                                 stream);
+}
+
 lora_sgmv_status lora_sgmv_apply(void* Y, const void* X, const void* const* A_ptrs,
                                  const void* const* B_ptrs, const int32_t* seg_starts,
                                  const int32_t* lora_idx, int32_t n_segments, int32_t num_adapters,
@@ -928,10 +1049,12 @@ lora_sgmv_status lora_sgmv_apply(void* Y, const void* X, const void* const* A_pt
 
 }  // extern "C"
 
-extern "C" lora_sgmv_status lora_sgmv_apply_batched(const lora_sgmv_problem* problems, int32_t n_problems,
-                                                    const int32_t* seg_starts, const int32_t* lora_idx,
-                                                    int32_t n_segments, int32_t T, int32_t r, lora_sgmv_dtype dtype,
-                                                    int32_t max_seg_len, uint32_t* dev_status, void* stream) {
+extern "C" lora_sgmv_status lora_sgmv_apply_batched_flags(const lora_sgmv_problem* problems, int32_t n_problems,
+                                                          const int32_t* seg_starts, const int32_t* lora_idx,
+                                                          int32_t n_segments, int32_t T, int32_t r,
+                                                          lora_sgmv_dtype dtype, int32_t max_seg_len, uint32_t flags,
+                                                          uint32_t* dev_status, void* stream) {
+    if (flags & ~uint32_t(LORA_SGMV_FLAG_EARLY_READS)) return LORA_SGMV_ERR_UNSUPPORTED;
     if (dtype != LORA_SGMV_F16 && dtype != LORA_SGMV_BF16) return LORA_SGMV_ERR_DTYPE;
     if (!problems) return LORA_SGMV_ERR_NULL;
     if (n_problems < 1 || n_problems > LORA_SGMV_MAX_PROBLEMS || n_segments < 0 || T < 0 || r <= 0)
@@ -963,11 +1086,142 @@ extern "C" lora_sgmv_status lora_sgmv_apply_batched(const lora_sgmv_problem* pro
     P.n_problems = n_problems;
     P.n_segments = n_segments;
     P.T = T;
+    P.early = (flags & LORA_SGMV_FLAG_EARLY_READS) ? 1 : 0;
     const int max_len = estimate_max_len(max_seg_len, T, n_segments);
     bool tc = decode_tc_preferred(r, max_len);
     for (int i = 0; i < n_problems; ++i) tc = tc && decode_tc_supported(r, problems[i].H1, problems[i].H2);
     if (tc) return decode_tc_dispatch(P, r, dtype, max_len, static_cast<cudaStream_t>(stream));
     return fused_dispatch(P, r, dtype, max_len, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" lora_sgmv_status lora_sgmv_apply_batched(const lora_sgmv_problem* problems, int32_t n_problems,
+                                                    const int32_t* seg_starts, const int32_t* lora_idx,
+                                                    int32_t n_segments, int32_t T, int32_t r, lora_sgmv_dtype dtype,
+                                                    int32_t max_seg_len, uint32_t* dev_status, void* stream) {
+    return lora_sgmv_apply_batched_flags(problems, n_problems, seg_starts, lora_idx, n_segments, T, r, dtype,
+                                         max_seg_len, 0u, dev_status, stream);
+}
+
+// ---- adapters of different ranks, unpadded ------------------------------------------------------
+
+extern "C" lora_sgmv_status lora_sgmv_apply_ranks(void* Y, const void* X, const void* const* A_ptrs,
+                                                  const void* const* B_ptrs, const int32_t* ranks,
+                                                  const int32_t* seg_starts, const int32_t* lora_idx,
+                                                  int32_t n_segments, int32_t num_adapters, int32_t T, int32_t H1,
+                                                  int32_t r_max, int32_t H2, float scale, lora_sgmv_dtype dtype,
+                                                  uint32_t* dev_status, void* stream) {
+    lora_sgmv_status st = check_common(n_segments, num_adapters, T, dtype);
+    if (st != LORA_SGMV_OK) return st;
+    if (H1 <= 0 || H2 <= 0 || r_max <= 0) return LORA_SGMV_ERR_DIM;
+    if (!sgmv::grouped_tc_rank(r_max)) return LORA_SGMV_ERR_UNSUPPORTED;
+    if (H1 < 64 || H2 < 64) return LORA_SGMV_ERR_UNSUPPORTED;
+    if (n_segments == 0 || T == 0) return LORA_SGMV_OK;
+    if (!Y || !X || !A_ptrs || !B_ptrs || !ranks || !seg_starts || !lora_idx) return LORA_SGMV_ERR_NULL;
+    if (num_adapters < 1) return LORA_SGMV_ERR_DIM;
+    if (!aligned16(Y) || !aligned16(X) || H1 % 8 || H2 % 8) return LORA_SGMV_ERR_ALIGN;
+    return launch_grouped(Y, X, A_ptrs, B_ptrs, seg_starts, lora_idx, n_segments, num_adapters, T, H1, r_max, H2,
+                          scale, dtype, dev_status, static_cast<cudaStream_t>(stream), nullptr, ranks);
+}
+
+// ---- the whole layer: Y = X@W + scale * (X@A_i)@B_i ------------------------------------------
+
+namespace {
+
+template <int R>
+lora_sgmv_status launch_gemm_r(const CUtensorMap& tmX, const CUtensorMap& tmW, const CUtensorMap& tmB,
+                               const sgmv::GemmParams& P, lora_sgmv_dtype dt, int grid, cudaStream_t s) {
+    return counted(dt == LORA_SGMV_BF16 ? sgmv::launch_gemm_delta_kernel<__nv_bfloat16, R>(tmX, tmW, tmB, P, grid, s)
+                                        : sgmv::launch_gemm_delta_kernel<__half, R>(tmX, tmW, tmB, P, grid, s));
+}
+
+}  // namespace
+
+extern "C" lora_sgmv_status lora_sgmv_gemm_apply(void* Y, const void* X, const void* W, const void* const* A_ptrs,
+                                                 const void* const* B_ptrs, const int32_t* seg_starts,
+                                                 const int32_t* lora_idx, int32_t n_segments, int32_t num_adapters,
+                                                 int32_t T, int32_t H1, int32_t r, int32_t H2, float scale,
+                                                 lora_sgmv_dtype dtype, int32_t max_seg_len, void* workspace,
+                                                 size_t workspace_bytes, uint32_t* dev_status, void* stream) {
+    lora_sgmv_status st = check_common(n_segments, num_adapters, T, dtype);
+    if (st != LORA_SGMV_OK) return st;
+    if (H1 <= 0 || H2 <= 0 || r <= 0) return LORA_SGMV_ERR_DIM;
+    if (!sgmv::gemm_tc_supported(r, H1, H2)) return (H1 % 8 || H2 % 8) ? LORA_SGMV_ERR_ALIGN : LORA_SGMV_ERR_UNSUPPORTED;
+    if (T == 0) return LORA_SGMV_OK;
+    if (!Y || !X || !W) return LORA_SGMV_ERR_NULL;
+    if (n_segments > 0 && (!A_ptrs || !B_ptrs || !seg_starts || !lora_idx)) return LORA_SGMV_ERR_NULL;
+    if (n_segments > 0 && num_adapters < 1) return LORA_SGMV_ERR_DIM;
+    if (!aligned16(Y) || !aligned16(X) || !aligned16(W)) return LORA_SGMV_ERR_ALIGN;
+    const size_t need = lora_sgmv_workspace_bytes(T, r);
+    if (n_segments > 0 && (!workspace || workspace_bytes < need)) return LORA_SGMV_ERR_WORKSPACE;
+    if (n_segments > 0 && !aligned16(workspace)) return LORA_SGMV_ERR_ALIGN;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    DeviceFacts f;
+    if (device_facts(f) != LORA_SGMV_OK) return LORA_SGMV_ERR_CUDA;
+    float* V = static_cast<float*>(workspace);
+    const int max_len = estimate_max_len(max_seg_len, T, n_segments);
+    if (n_segments > 0) {
+        // V = X@A_i first: the grouped tensor-core kernel's shrink for long segments, else the
+        // split-K shrink kernel
+        if (max_len >= sgmv::kGroupedMinSegment && H1 >= 64 && H2 >= 64) {
+            st = launch_grouped(Y, X, A_ptrs, B_ptrs, seg_starts, lora_idx, n_segments, num_adapters, T, H1, r, H2,
+                                scale, dtype, dev_status, s, V);
+        } else {
+            ShrinkParams sp = {};
+            sp.V = V;
+            sp.X = X;
+            sp.A_ptrs = A_ptrs;
+            sp.B_check = B_ptrs;
+            sp.seg_starts = seg_starts;
+            sp.lora_idx = lora_idx;
+            sp.dev_status = nullptr;  // the layer kernel reports this call's bad segments
+            sp.n_segments = n_segments;
+            sp.num_adapters = num_adapters;
+            sp.T = T;
+            sp.H1 = H1;
+            st = shrink_dispatch(sp, r, dtype, max_len, s);
+        }
+        if (st != LORA_SGMV_OK) return st;
+    }
+    CUtensorMap tmX, tmW, tmB;
+    {
+        const uint64_t dw[2] = {uint64_t(H2), uint64_t(H1)};
+        const uint64_t sw[1] = {uint64_t(H2) * 2};
+        const uint32_t bw[2] = {64, uint32_t(sgmv::kLK)};
+        const uint64_t db[2] = {uint64_t(H2), uint64_t(r)};
+        const uint64_t sb[1] = {uint64_t(H2) * 2};
+        const uint32_t bb[2] = {64, uint32_t(r)};
+        if (!sgmv::make_tile_map(&tmX, X, T, H1, dtype, sgmv::kLM) ||
+            !sgmv::encode_map(&tmW, W, dtype, 2, dw, sw, bw, CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !sgmv::encode_map(&tmB, W, dtype, 2, db, sb, bb, CU_TENSOR_MAP_SWIZZLE_128B)) {
+            t_last_error = cudaErrorInvalidValue;
+            return LORA_SGMV_ERR_CUDA;
+        }
+    }
+    sgmv::GemmParams P = {};
+    P.Y = Y;
+    P.V = V;
+    P.A_ptrs = n_segments > 0 ? A_ptrs : nullptr;
+    P.B_ptrs = n_segments > 0 ? B_ptrs : nullptr;
+    P.seg_starts = seg_starts;
+    P.lora_idx = lora_idx;
+    P.dev_status = dev_status;
+    P.n_segments = n_segments;
+    P.num_adapters = num_adapters;
+    P.T = T;
+    P.H1 = H1;
+    P.H2 = H2;
+    P.scale = scale;
+    P.m_tiles = (T + sgmv::kLM - 1) / sgmv::kLM;
+    P.n_tiles = (H2 + sgmv::kLN - 1) / sgmv::kLN;
+    const long long units = static_cast<long long>(P.m_tiles) * P.n_tiles;
+    if (units > (1ll << 31) - 1) return LORA_SGMV_ERR_DIM;
+    const int grid = static_cast<int>(std::max<long long>(1, std::min<long long>(units, f.sms)));
+    switch (r) {
+        case 16: return launch_gemm_r<16>(tmX, tmW, tmB, P, dtype, grid, s);
+        case 32: return launch_gemm_r<32>(tmX, tmW, tmB, P, dtype, grid, s);
+        case 64: return launch_gemm_r<64>(tmX, tmW, tmB, P, dtype, grid, s);
+    }
+    return LORA_SGMV_ERR_UNSUPPORTED;
 }
 
 // ---- apply for callers that cannot allocate device memory -----------------------------------

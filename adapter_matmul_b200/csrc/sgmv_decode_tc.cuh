@@ -40,7 +40,8 @@
 // Warps: 0 producer of X, A_i and B_i, 1 TMEM owner and MMA issuer, 2..9 epilogue (two per
 // TMEM lane quarter, each taking every other 128-column group of a stage; one of them also
 // runs the V exchange), 10 producer of Y. Programmatic dependent launch: X and Y are read only after
-// griddepcontrol.wait. Every wait is bounded in time.
+// griddepcontrol.wait; so are the segment arrays, tables and adapters unless the caller allows
+// reading them earlier (P.early) or the kernel runs in pre-V mode. Every wait is bounded in time.
 //
 // Pre-V mode (template flag PRE_V, the split form): V [T, r] (fp32) comes from an earlier
 // kernel (the split-K shrink) through global memory. There is no shrink and no cluster: each
@@ -216,6 +217,11 @@ __global__ void __launch_bounds__(kDThreads, 1)
         table_s = claim_map_table();
         if (table_s < 0) report(P.dev_status, LORA_SGMV_DEV_TIMEOUT);
     }
+    // Early reads (segment arrays, tables, adapters before the previous kernel completes) only
+    // where allowed: asked for by the caller, or in pre-V mode, whose previous kernel is this
+    // library's shrink, which writes none of them.
+    const bool early = pre_v || P.early;
+    if (!early) pdl_wait();
     int entries;
     if (P.one_chunk) {
         __syncthreads();
@@ -247,7 +253,9 @@ __global__ void __launch_bounds__(kDThreads, 1)
 #pragma unroll
         for (int e = 0; e < kMapRing; ++e) last_use[e] = -1;
         int jc = 0;
-        bool waited = false;
+        // X is read only after the wait; in pre-V mode there is no X to read, so the producer
+        // never waits and B_i streams while the shrink kernel finishes
+        bool waited = !early || pre_v;
         int deferred = 0;  // shrink stages of the first job still missing their X box
         int d_p = 0, d_t0 = 0, d_k0 = 0;
         auto flush_deferred = [&]() {
@@ -337,7 +345,8 @@ __global__ void __launch_bounds__(kDThreads, 1)
             }
         }
         if (!waited) pdl_wait();
-        // every copy issued lands before the CTA may exit
+        // every copy issued lands before the CTA may exit (pre-V mode: the epilogue's and the Y
+        // producer's waits keep this grid behind the shrink)
         if (lane == 0)
             for (uint32_t i = it > uint32_t(S) ? it - S : 0u; i < it; ++i) drain_wait(&full[i % S], (i / S) & 1u);
         __syncwarp();

@@ -38,10 +38,13 @@
 // stores to global memory.
 //
 // Programmatic dependent launch: the kernel lets the next kernel on the stream
-// launch at once, and reads X and Y only after griddepcontrol.wait (which
-// returns when the previous kernel has completed). Segment metadata, pointer
-// tables and adapter weights are read before it: they must not be written by
-// the kernel that immediately precedes the call on the stream.
+// launch at once. By default every thread waits (griddepcontrol.wait, which
+// returns when the previous kernel has completed) before it reads anything the
+// caller passed, so only the prologue overlaps the previous kernel. When the
+// caller states that the segment arrays, pointer tables and adapters are not
+// written by the kernel immediately before this one (P.early), those are read
+// at once and the first A_i copies stream while that kernel finishes; X and Y
+// are then read only after the wait.
 //
 // Every mbarrier wait is bounded in time; a wait that gives up sets
 // LORA_SGMV_DEV_TIMEOUT in the status word and the thread's later waits
@@ -91,6 +94,7 @@ struct FusedParams {
     int n_segments;
     int T;
     int one_chunk;  // host hint: every segment fits one chunk (job j is segment j; correct either way)
+    int early;      // 1: segment arrays, tables and adapters may be read before griddepcontrol.wait
 };
 
 // compile-time geometry per rank
@@ -643,6 +647,9 @@ __global__ void __launch_bounds__(kFusedThreads, SGMV_FUSED_MIN_BLOCKS) sgmv_fus
         mbar_init(vfree, C);   // one arrival per receiver
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
+    // nothing the caller passed is read before the previous kernel completes, unless the
+    // caller allows the early reads
+    if (!P.early) pdl_wait();
     int entries;
     if (P.one_chunk) {
         __syncthreads();
@@ -658,11 +665,11 @@ __global__ void __launch_bounds__(kFusedThreads, SGMV_FUSED_MIN_BLOCKS) sgmv_fus
     bool dead = false;
     if (warp == 0) {
         // ------------------------------ producer ------------------------------
-        // Adapter weights and segment metadata are not written by the previous kernel on the
-        // stream, so the first job's A rows are requested before griddepcontrol.wait; X and Y
-        // (which the previous kernel may produce) only after it.
+        // With early reads allowed, adapter weights and segment metadata are not written by the
+        // previous kernel on the stream, so the first job's A rows are requested before
+        // griddepcontrol.wait; X and Y (which the previous kernel may produce) only after it.
         uint32_t it = 0;
-        bool waited = false;
+        bool waited = !P.early;
         for (int j = cluster_id; j < entries; j += n_clusters) {
             int p, s, q0, nq;
             entry_at(P, pref, j, p, s, q0, nq);

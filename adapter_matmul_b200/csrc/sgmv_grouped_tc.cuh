@@ -75,7 +75,20 @@ struct GroupedParams {
     int nsplit;  // N-slices of H2
     int nspan;   // columns per N-slice (multiple of kGN)
     int tm;      // rows per M-tile, 8..128 (the MMA's M stays 128; rows past tm are never used)
+    float* v_out;  // V-only mode: V [T, r] fp32 written here, no expand
+    const int32_t* ranks;  // rank of each adapter (device), or null: every adapter has rank R
 };
+
+// Rank of the adapter of segment s when a rank table is given: 8 <= rank <= R, a multiple of 8
+// (A_i rows of 16-byte multiples); 0 when it is not valid.
+template <int R>
+__device__ __forceinline__ int segment_rank(const GroupedParams& P, int s) {
+    if (!P.ranks) return R;
+    const int i = __ldg(P.lora_idx + s);
+    if (i < 0 || i >= P.num_adapters) return 0;
+    const int rs = __ldg(P.ranks + i);
+    return (rs >= 8 && rs <= R && rs % 8 == 0) ? rs : 0;
+}
 
 template <int R>
 struct GroupedGeom {
@@ -226,7 +239,9 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
 
 // grid.x = tiles (upper bound) * nsplit; block kGThreads. tmA and tmB are templates of the
 // A_i and B_i maps (shape, box, swizzle); each CTA makes its adapter's maps from them.
-template <typename T, int R>
+// V_OUT: the shrink alone -- V = X@A_i (fp32) of the tile's rows goes to P.v_out and there is
+// no expand (nsplit must be 1); the whole-layer kernel (sgmv_gemm_tc.cuh) takes V from there.
+template <typename T, int R, bool V_OUT = false>
 __global__ void __launch_bounds__(kGThreads, 1)
     sgmv_grouped_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmY,
                            const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -260,12 +275,15 @@ __global__ void __launch_bounds__(kGThreads, 1)
             Segment seg;
             if (ok && load_segment(P.seg_starts, P.lora_idx, P.A_ptrs, P.B_ptrs, s, P.T, P.num_adapters, seg))
                 job_s[0] = -1;  // rejected segment: reported by CTA 0 below
+            job_s[2] = job_s[0] >= 0 ? segment_rank<R>(P, s) : 0;
+            if (job_s[2] == 0) job_s[0] = -1;  // a rank the kernel cannot take: reported below
         }
         if (blockIdx.x == 0) {  // report every rejected segment once
             for (int s2 = lane; s2 < P.n_segments; s2 += 32) {
                 Segment seg;
-                report(P.dev_status,
-                       load_segment(P.seg_starts, P.lora_idx, P.A_ptrs, P.B_ptrs, s2, P.T, P.num_adapters, seg));
+                const uint32_t bad =
+                    load_segment(P.seg_starts, P.lora_idx, P.A_ptrs, P.B_ptrs, s2, P.T, P.num_adapters, seg);
+                report(P.dev_status, bad ? bad : (segment_rank<R>(P, s2) ? 0u : LORA_SGMV_DEV_BAD_RANK));
             }
         }
     }
@@ -302,7 +320,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
     const int rows = min(P.tm, seg.end - t0);  // valid rows of this tile
     const int n_lo = nsl * P.nspan;
     const int n_hi = min(P.H2, n_lo + P.nspan);
-    const int n_tiles = n_lo < n_hi ? (n_hi - n_lo + kGN - 1) / kGN : 0;
+    const int n_tiles = (!V_OUT && n_lo < n_hi) ? (n_hi - n_lo + kGN - 1) / kGN : 0;
     const int k_steps = (P.H1 + kGK - 1) / kGK;
     const int s_stages = (k_steps + 1) / 2;  // shrink stages of two K-steps (the last may hold one)
 
@@ -330,6 +348,12 @@ __global__ void __launch_bounds__(kGThreads, 1)
         if (lane == 0) {
             map_set_address(&map_build[0], seg.a);
             map_set_address(&map_build[1], seg.b);
+            if (P.ranks) {  // this adapter's own rank: columns (rows of B_i) past it read as zeros
+                const int rs = job_s[2];
+                map_set_dim<0>(&map_build[0], uint32_t(rs));
+                map_set_stride<0>(&map_build[0], uint64_t(rs) * 2);
+                map_set_dim<1>(&map_build[1], uint32_t(rs));
+            }
         }
         __syncwarp();
         map_publish(gA, &map_build[0]);
@@ -442,20 +466,29 @@ __global__ void __launch_bounds__(kGThreads, 1)
         for (int c0 = 32 * half; c0 < R; c0 += 64) {  // the two halves share V's columns
             float v[32];
             tmem_ld32(lane_addr + c0, v);
+            if (V_OUT) {
+                if (m < rows) {
+                    float* dst = P.v_out + size_t(t0 + m) * R + c0;
 #pragma unroll
-            for (int ch = 0; ch < 4; ++ch) {
-                if (c0 + ch * 8 >= R) break;
-                float hi[8], lo[8];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const float x = v[ch * 8 + i];
-                    const float h = Storage<T>::round(x);
-                    hi[i] = h;
-                    lo[i] = x - h;
+                    for (int i = 0; i < 32; i += 4)
+                        if (c0 + i < R) *reinterpret_cast<float4*>(dst + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
                 }
-                const uint32_t off = swz(m, c0 / 8 + ch, G::SW_BITS);
-                st_vec(vhi + off, pack8<T>(hi));
-                st_vec(vlo + off, pack8<T>(lo));
+            } else {
+#pragma unroll
+                for (int ch = 0; ch < 4; ++ch) {
+                    if (c0 + ch * 8 >= R) break;
+                    float hi[8], lo[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const float x = v[ch * 8 + i];
+                        const float h = Storage<T>::round(x);
+                        hi[i] = h;
+                        lo[i] = x - h;
+                    }
+                    const uint32_t off = swz(m, c0 / 8 + ch, G::SW_BITS);
+                    st_vec(vhi + off, pack8<T>(hi));
+                    st_vec(vlo + off, pack8<T>(lo));
+                }
             }
         }
         fence_proxy_async();  // generic-proxy writes of V -> tensor-core reads
@@ -558,7 +591,7 @@ inline bool make_tile_map(CUtensorMap* map, const void* base, int rows, int cols
     return r == CUDA_SUCCESS;
 }
 
-template <typename T, int R>
+template <typename T, int R, bool V_OUT = false>
 inline cudaError_t launch_grouped_tc_kernel(const CUtensorMap& tmX, const CUtensorMap& tmY, const CUtensorMap& tmA,
                                             const CUtensorMap& tmB, const GroupedParams& P, int blocks,
                                             cudaStream_t stream) {
@@ -566,11 +599,11 @@ inline cudaError_t launch_grouped_tc_kernel(const CUtensorMap& tmX, const CUtens
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(once, [] {
-        attr_err = cudaFuncSetAttribute(sgmv_grouped_tc_kernel<T, R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        static_cast<int>(G::SMEM));
+        attr_err = cudaFuncSetAttribute(sgmv_grouped_tc_kernel<T, R, V_OUT>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(G::SMEM));
     });
     if (attr_err != cudaSuccess) return attr_err;
-    sgmv_grouped_tc_kernel<T, R><<<blocks, kGThreads, G::SMEM, stream>>>(tmX, tmY, tmA, tmB, P);
+    sgmv_grouped_tc_kernel<T, R, V_OUT><<<blocks, kGThreads, G::SMEM, stream>>>(tmX, tmY, tmA, tmB, P);
     return cudaGetLastError();
 }
 

@@ -77,6 +77,25 @@ __device__ __forceinline__ void map_set_address(CUtensorMap* smem_map, const voi
                  : "memory");
 }
 
+// One thread: set the extent of dimension ORD (elements) of a map held in shared memory.
+template <int ORD>
+__device__ __forceinline__ void map_set_dim(CUtensorMap* smem_map, uint32_t extent) {
+    asm volatile("tensormap.replace.tile.global_dim.shared::cta.b1024.b32 [%0], %1, %2;" ::"r"(
+                     static_cast<uint32_t>(__cvta_generic_to_shared(smem_map))),
+                 "n"(ORD), "r"(extent)
+                 : "memory");
+}
+
+// One thread: set the byte stride of dimension ORD + 1 of a map held in shared memory (a
+// multiple of 16).
+template <int ORD>
+__device__ __forceinline__ void map_set_stride(CUtensorMap* smem_map, uint64_t stride_bytes) {
+    asm volatile("tensormap.replace.tile.global_stride.shared::cta.b1024.b64 [%0], %1, %2;" ::"r"(
+                     static_cast<uint32_t>(__cvta_generic_to_shared(smem_map))),
+                 "n"(ORD), "l"(stride_bytes)
+                 : "memory");
+}
+
 // Whole warp: copy the map from shared memory to its global slot and release it to the
 // tensormap proxy.
 __device__ __forceinline__ void map_publish(CUtensorMap* gmem_map, const CUtensorMap* smem_map) {

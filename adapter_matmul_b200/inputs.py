@@ -33,7 +33,7 @@ import numpy as np
 F16 = "f16"
 BF16 = "bf16"
 
-_TAGS = {"ids": 1, "x": 2, "a": 3, "b": 4, "y": 5, "len": 6}
+_TAGS = {"ids": 1, "x": 2, "a": 3, "b": 4, "y": 5, "len": 6, "w": 7}
 
 
 def _stream(seed: int, tag: str, index: int = 0) -> np.random.Generator:
@@ -117,6 +117,10 @@ class Workload:
     def y_random(self, proj: int = 0) -> np.ndarray:
         """A non-zero base output, N(0,1), used to exercise the in-place add."""
         return _normal_bits(_stream(self.seed, "y", proj), (self.T, self.H2), 1.0, self.dtype)
+
+    def base_weight(self, proj: int = 0) -> np.ndarray:
+        """The frozen base weight W of shape [H1, H2], entries N(0, 1/H1) (so X@W ~ N(0, 1))."""
+        return _normal_bits(_stream(self.seed, "w", proj), (self.H1, self.H2), 1.0 / math.sqrt(self.H1), self.dtype)
 
     def adapter_a(self, i: int, proj: int = 0) -> np.ndarray:
         """A_i of shape [H1, r], entries N(0, 1/H1)."""

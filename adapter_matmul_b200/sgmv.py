@@ -34,6 +34,9 @@ DEV_BAD_SEGMENT = 0x1
 DEV_BAD_ADAPTER = 0x2
 DEV_BAD_POINTER = 0x4
 DEV_TIMEOUT = 0x8
+DEV_BAD_RANK = 0x10
+
+FLAG_EARLY_READS = 0x1
 
 STATUS_NAMES = {0: "OK", 1: "ERR_NULL", 2: "ERR_DIM", 3: "ERR_ALIGN", 4: "ERR_DTYPE", 5: "ERR_UNSUPPORTED",
                 6: "ERR_CUDA", 7: "ERR_WORKSPACE", 8: "ERR_RANGE"}
@@ -43,7 +46,8 @@ EXPORTS = [
     "lora_sgmv_last_error",
     "lora_sgmv_group_segments", "lora_sgmv_shrink", "lora_sgmv_expand", "lora_sgmv_workspace_bytes",
     "lora_sgmv_apply", "lora_sgmv_apply_ex", "lora_sgmv_apply_batched", "lora_sgmv_apply_noalloc",
-    "lora_sgmv_pad_rank", "lora_sgmv_auto_variant",
+    "lora_sgmv_pad_rank", "lora_sgmv_auto_variant", "lora_sgmv_apply_flags", "lora_sgmv_apply_batched_flags",
+    "lora_sgmv_gemm_apply", "lora_sgmv_apply_ranks",
 ]
 
 
@@ -105,6 +109,18 @@ def load(path: Optional[str] = None):
         lib.lora_sgmv_apply_ex.restype = ctypes.c_int
         lib.lora_sgmv_apply_ex.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, ctypes.c_float,
                                            ctypes.c_int, i32, P, u64, P, ctypes.c_int, P]
+        lib.lora_sgmv_apply_flags.restype = ctypes.c_int
+        lib.lora_sgmv_apply_flags.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, ctypes.c_float,
+                                              ctypes.c_int, i32, P, u64, P, ctypes.c_int, ctypes.c_uint32, P]
+        lib.lora_sgmv_apply_batched_flags.restype = ctypes.c_int
+        lib.lora_sgmv_apply_batched_flags.argtypes = [P, i32, P, P, i32, i32, i32, ctypes.c_int, i32,
+                                                      ctypes.c_uint32, P, P]
+        lib.lora_sgmv_apply_ranks.restype = ctypes.c_int
+        lib.lora_sgmv_apply_ranks.argtypes = [P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, ctypes.c_float,
+                                              ctypes.c_int, P, P]
+        lib.lora_sgmv_gemm_apply.restype = ctypes.c_int
+        lib.lora_sgmv_gemm_apply.argtypes = [P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, ctypes.c_float,
+                                             ctypes.c_int, i32, P, u64, P, P]
         lib.lora_sgmv_apply_batched.restype = ctypes.c_int
         lib.lora_sgmv_apply_batched.argtypes = [P, i32, P, P, i32, i32, i32, ctypes.c_int, i32, P, P]
         lib.lora_sgmv_apply_noalloc.restype = ctypes.c_int
@@ -214,9 +230,18 @@ def lora_sgmv_apply_ex(Y, X, A_ptrs, B_ptrs, seg_starts, lora_idx, n_segments: i
            "lora_sgmv_apply_ex")
 
 
-def lora_sgmv_apply_batched(problems, seg_starts, lora_idx, n_segments: int, T: int, r: int, dtype: int,
-                            max_seg_len: int, dev_status=None, stream=None) -> None:
-    """problems: sequence of dicts (Y, X, A_ptrs, B_ptrs, num_adapters, H1, H2, scale) or Problem structs."""
+def lora_sgmv_apply_flags(Y, X, A_ptrs, B_ptrs, seg_starts, lora_idx, n_segments: int, num_adapters: int, T: int,
+                          H1: int, r: int, H2: int, scale: float, dtype: int, max_seg_len: int, workspace,
+                          workspace_bytes: int, dev_status=None, variant: int = VARIANT_AUTO, flags: int = 0,
+                          stream=None) -> None:
+    _check(load().lora_sgmv_apply_flags(_p(Y), _p(X), _p(A_ptrs), _p(B_ptrs), _p(seg_starts), _p(lora_idx),
+                                        n_segments, num_adapters, T, H1, r, H2, float(scale), dtype, max_seg_len,
+                                        _p(workspace), workspace_bytes, _p(dev_status), variant, flags,
+                                        _stream(stream)),
+           "lora_sgmv_apply_flags")
+
+
+def _problem_array(problems):
     arr = (Problem * max(1, len(problems)))()
     for i, q in enumerate(problems):
         if isinstance(q, Problem):
@@ -224,9 +249,25 @@ def lora_sgmv_apply_batched(problems, seg_starts, lora_idx, n_segments: int, T: 
         else:
             arr[i] = Problem(_p(q["Y"]), _p(q["X"]), _p(q["A_ptrs"]), _p(q["B_ptrs"]), int(q["num_adapters"]),
                              int(q["H1"]), int(q["H2"]), float(q.get("scale", 1.0)))
+    return arr
+
+
+def lora_sgmv_apply_batched(problems, seg_starts, lora_idx, n_segments: int, T: int, r: int, dtype: int,
+                            max_seg_len: int, dev_status=None, stream=None) -> None:
+    """problems: sequence of dicts (Y, X, A_ptrs, B_ptrs, num_adapters, H1, H2, scale) or Problem structs."""
+    arr = _problem_array(problems)
     _check(load().lora_sgmv_apply_batched(ctypes.addressof(arr), len(problems), _p(seg_starts), _p(lora_idx),
                                           n_segments, T, r, dtype, max_seg_len, _p(dev_status), _stream(stream)),
            "lora_sgmv_apply_batched")
+
+
+def lora_sgmv_apply_batched_flags(problems, seg_starts, lora_idx, n_segments: int, T: int, r: int, dtype: int,
+                                  max_seg_len: int, flags: int = 0, dev_status=None, stream=None) -> None:
+    arr = _problem_array(problems)
+    _check(load().lora_sgmv_apply_batched_flags(ctypes.addressof(arr), len(problems), _p(seg_starts),
+                                                _p(lora_idx), n_segments, T, r, dtype, max_seg_len, flags,
+                                                _p(dev_status), _stream(stream)),
+           "lora_sgmv_apply_batched_flags")
 
 
 def lora_sgmv_apply_noalloc(Y, X, A_ptrs, B_ptrs, seg_starts, lora_idx, n_segments: int, num_adapters: int,
@@ -237,6 +278,26 @@ def lora_sgmv_apply_noalloc(Y, X, A_ptrs, B_ptrs, seg_starts, lora_idx, n_segmen
                                           n_segments, num_adapters, T, H1, r, H2, float(scale), dtype, max_seg_len,
                                           _p(dev_status), _stream(stream)),
            "lora_sgmv_apply_noalloc")
+
+
+def lora_sgmv_apply_ranks(Y, X, A_ptrs, B_ptrs, ranks, seg_starts, lora_idx, n_segments: int, num_adapters: int,
+                          T: int, H1: int, r_max: int, H2: int, scale: float, dtype: int, dev_status=None,
+                          stream=None) -> None:
+    """SGMV over adapters of their own ranks (ranks: device int32 per adapter), unpadded."""
+    _check(load().lora_sgmv_apply_ranks(_p(Y), _p(X), _p(A_ptrs), _p(B_ptrs), _p(ranks), _p(seg_starts),
+                                        _p(lora_idx), n_segments, num_adapters, T, H1, r_max, H2, float(scale), dtype,
+                                        _p(dev_status), _stream(stream)),
+           "lora_sgmv_apply_ranks")
+
+
+def lora_sgmv_gemm_apply(Y, X, W, A_ptrs, B_ptrs, seg_starts, lora_idx, n_segments: int, num_adapters: int, T: int,
+                         H1: int, r: int, H2: int, scale: float, dtype: int, max_seg_len: int, workspace,
+                         workspace_bytes: int, dev_status=None, stream=None) -> None:
+    """The whole layer Y = X@W + scale * (X@A_i)@B_i (Y written, not read)."""
+    _check(load().lora_sgmv_gemm_apply(_p(Y), _p(X), _p(W), _p(A_ptrs), _p(B_ptrs), _p(seg_starts), _p(lora_idx),
+                                       n_segments, num_adapters, T, H1, r, H2, float(scale), dtype, max_seg_len,
+                                       _p(workspace), workspace_bytes, _p(dev_status), _stream(stream)),
+           "lora_sgmv_gemm_apply")
 
 
 def lora_sgmv_auto_variant(T: int, n_segments: int, H1: int, r: int, H2: int, dtype: int, max_seg_len: int = 0,

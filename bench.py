@@ -2,30 +2,40 @@
 """SGMV benchmark: LoRA-delta tokens/s and achieved HBM bandwidth on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+                    [--no-per-config] [--no-e2e] [--no-cpu-baseline]
 
-Default workload ("distinct"): Llama-7B-shaped decode with the Distinct
-adapter distribution of the throughput benchmark on page “Punica：多 LoRA 模型统一服务框架” (the Punica
-README): 32 tokens,
-each on its own rank-16 adapter, H1 = H2 = 4096, fp16. One step is one decoder
-layer's LoRA work: four SGMV calls (q, k, v, o projections), each with its
-own adapters, input and output. Steps rotate over 32 layers, each with its own
-weights and activations (1.1 GiB in all, far above the 126 MB L2), so every
-step reads cold data, as a model's layers would.
+Default workload ("distinct"): Llama-7B-shaped decode with the Distinct adapter
+distribution of the throughput benchmark on page "Punica：多 LoRA 模型统一服务框架" (the
+Punica README): 32 tokens, each on its own rank-16 adapter, H1 = H2 = 4096, fp16. One step
+is one decoder layer's LoRA work: four SGMV problems (q, k, v, o projections), each with
+its own adapters, input and output, sharing one token grouping, run as one
+lora_sgmv_apply_batched launch. Steps rotate over layers that each have their own weights
+and activations (far above the 126 MB L2), so every step reads cold data, as a model's
+layers would.
 
-Each layer's four projections share one token grouping, so a step is one
-lora_sgmv_apply_batched launch. The timed region replays CUDA graphs: one
-graph holding a whole rotation of layers back to back (consecutive launches
-overlap through programmatic dependent launch, as a captured decode step
-would), plus single-layer graphs for a remainder, so host launch latency does
-not stand in for kernel time. ``e2e`` repeats the measurement through the
-public calls with host buffers: each step groups the token batch on the host,
-copies the segment arrays and the four projections' X and Y from pinned host
-memory, runs one lora_sgmv_apply_batched launch, and reads Y back. Other
-workloads (--workload) run one lora_sgmv_apply per step, the dispatcher
-choosing the kernels.
+Timing. The K timed steps are one CUDA graph of exactly K launches (layer i mod L at step
+i), replayed once untimed and then once between CUDA events on the launching stream; so
+the timed work does not depend on K beyond its length. Consecutive launches are chained
+by programmatic dependent launch with the library's default contract: a launch's prologue
+(barriers, tensor memory, tensor-map tables) overlaps the end of the previous launch, and
+it reads nothing of its inputs (segments, tables, adapters, X, Y) before the previous
+launch has completed. The line also carries ("early_reads") the same K steps with
+LORA_SGMV_FLAG_EARLY_READS, under which each launch streams its adapter weights while the
+previous one finishes; the statement that flag makes holds here (segments and adapters
+are written by copies before the timed region).
 
-Multi-GPU (torchrun): every rank runs its own replica of the workload (the
-path has no cross-GPU data exchange); value = all ranks' tokens / max time.
+"per_config" times every configuration the same way (the Distinct, Uniform, Skewed and
+Identical decode batches per layer of four projections and per single call, the prefill
+and the 70B-shaped decode per call), each with its dispatched kernels, algorithmic bytes
+and roofline fraction.
+
+"e2e" is the same metric through the public calls with host buffers: each step groups
+the token batch on the host, copies the segment arrays and the projections' X and Y from
+pinned host memory, runs the SGMV launch and copies Y back, double-buffered on three
+streams so that one step's copies overlap the next step's. Timed by the host clock.
+
+Multi-GPU (torchrun): every rank runs its own replica of the workload (the path has no
+cross-GPU data exchange); value = all ranks' tokens / max time.
 """
 from __future__ import annotations
 
@@ -49,21 +59,14 @@ from adapter_matmul_b200 import inputs  # noqa: E402
 METRIC = "LoRA-delta tokens/s (SGMV)"
 UNIT = "tokens/s"
 L2_BYTES = 126 * 1024 * 1024
+PER_CONFIG_MAX_STEPS = 500
 
 
 # DRAM bytes (read + write) of one launch of the dominant kernel, from one ncu capture of the
 # same launch (summaries under profiles/). A figure holds only while the kernel's sources are
 # those it was taken from: their SHA-256 is stored with it and checked here, else "traffic"
-# is null. (The 70B-shaped decode runs two kernels per call, the split form, and has no
-# capture of both yet.)
-TRAFFIC = {
-    "distinct": {"bytes": 35724288 + 2048, "profile": "profiles/fused_kernel_distinct_decode.md",
-                 "sources": ["sgmv_common.cuh", "sgmv_fused.cuh"],
-                 "sha256": "e2d41ed385c1ba3b023529a9127f563df5317aa29af52d1bb8a4398c386b2c2b"},
-    "prefill": {"bytes": 168609024 + 21820416, "profile": "profiles/grouped_kernel_prefill.md",
-                "sources": ["sgmv_common.cuh", "sgmv_fused.cuh", "sgmv_tmap.cuh", "sgmv_grouped_tc.cuh"],
-                "sha256": "ac9d51d05a761e2b4057b75a73f86a10c89895e1982478c529ca7b3a8ff7df66"},
-}
+# is null. For a call of two launches (the split forms) the figure is the pair's.
+TRAFFIC = {}
 
 
 def kernel_sources_sha(files) -> str:
@@ -122,16 +125,40 @@ class Spec:
         self.name, self.w, self.P, self.L, self.desc = name, workload, projections, layers, desc
 
 
+LAYER_CONFIGS = ("distinct", "uniform_h4096", "uniform_h11008", "skewed_h4096", "skewed_h11008",
+                 "identical_h4096", "identical_h11008")
+
+
+def workload_names():
+    """--workload values: a configuration name (a layer of four projections for the decode
+    batches, one call otherwise), or a decode batch name with ':call' (one SGMV call)."""
+    return list(inputs.CONFIGS) + [n + ":call" for n in LAYER_CONFIGS]
+
+
 def make_spec(name: str) -> Spec:
-    if name == "distinct":
-        w = inputs.distinct()
-        return Spec(name, w, 4, 32, "Distinct decode, Llama-7B shape: H1=H2=4096, r=16, fp16, 32 tokens each on "
-                                    "its own adapter; step = one layer = 4 SGMV calls (q,k,v,o)")
-    w = inputs.make(name)
-    per_call = w.algorithmic_bytes()
-    layers = max(1, min(64, math.ceil(3 * L2_BYTES / per_call)))
-    return Spec(name, w, 1, layers, f"{name}: H1={w.H1}, H2={w.H2}, r={w.r}, {w.dtype}, T={w.T}, "
-                                    f"{len(w.touched_adapters())} adapters touched; step = 1 SGMV call")
+    base, _, mode = name.partition(":")
+    w = inputs.make(base)
+    P = 4 if (base in LAYER_CONFIGS and mode != "call") else 1
+    per_step = w.algorithmic_bytes() * P
+    layers = max(1, min(64, math.ceil(3 * L2_BYTES / per_step)))
+    U = len(w.touched_adapters())
+    shape = f"H1={w.H1}, H2={w.H2}, r={w.r}, {w.dtype}, T={w.T}, {U} adapters touched"
+    if base == "distinct" and P == 4:
+        desc = ("Distinct decode, Llama-7B shape: H1=H2=4096, r=16, fp16, 32 tokens each on its own adapter; "
+                "step = one layer = 4 SGMV calls (q,k,v,o) in one launch")
+    elif P == 4:
+        desc = f"{base}: {shape}; step = one layer = 4 SGMV problems of this shape in one launch"
+    else:
+        desc = f"{base}: {shape}; step = 1 SGMV call"
+    return Spec(name, w, P, layers, desc)
+
+
+def config_dict(spec: Spec, world: int) -> dict:
+    """The line's `config`: the workload alone (the same in both arms)."""
+    w = spec.w
+    return {"workload": spec.desc, "name": spec.name, "T": w.T, "H1": w.H1, "H2": w.H2, "r": w.r,
+            "adapters_touched": len(w.touched_adapters()), "sgmv_calls_per_step": spec.P,
+            "parallelism": f"replicas x{world}"}
 
 
 VARIANT_NAMES = {1: "SPLIT", 2: "GROUPED_TC", 3: "FUSED", 4: "FUSED_TC", 5: "SPLIT_TC"}
@@ -400,15 +427,270 @@ def oracle_all_cores(spec: Spec, seconds: float, max_procs: int = 64) -> dict:
         return {"unavailable": f"{type(e).__name__}: {e}"}
 
 
+
 # ---------------------------------------------------------------------------------------------
 # our arm
 # ---------------------------------------------------------------------------------------------
 
-def run_ours(args, spec: Spec, rank: int, world: int, local: int):
+class DeviceSpec:
+    """One workload on the device: L layers x P projections, each with its own resident adapter
+    pool (every adapter of the pool drawn on the device: A ~ N(0, 1/H1), B ~ N(0, 1/r)), its
+    own X ~ N(0, 1) and Y = 0, and pointer tables; the grouping of the token batch (host
+    lora_sgmv_group_segments) is shared by all."""
+
+    def __init__(self, spec: Spec, dev, seed: int):
+        import torch
+
+        from adapter_matmul_b200 import sgmv
+
+        self.spec, self.sgmv = spec, sgmv
+        w = spec.w
+        self.dt = sgmv.F16 if w.dtype == "f16" else sgmv.BF16
+        self.tdt = torch.float16 if w.dtype == "f16" else torch.bfloat16
+        self.seg, self.idx, _ = sgmv.lora_sgmv_group_segments(w.ids, w.num_adapters)
+        self.n = len(self.idx)
+        self.max_len = int(np.max(np.diff(self.seg)))
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(seed)
+        self.calls, self.keep = [], []
+        a_bytes, b_bytes = w.H1 * w.r * 2, w.r * w.H2 * 2
+        for _ in range(spec.L):
+            layer = []
+            for _ in range(spec.P):
+                A = torch.empty((w.num_adapters, w.H1, w.r), dtype=self.tdt, device=dev)
+                A.normal_(0.0, 1.0 / math.sqrt(w.H1), generator=gen)
+                B = torch.empty((w.num_adapters, w.r, w.H2), dtype=self.tdt, device=dev)
+                B.normal_(0.0, 1.0 / math.sqrt(w.r), generator=gen)
+                ids = torch.arange(w.num_adapters, dtype=torch.int64, device=dev)
+                A_ptrs = ids * a_bytes + A.data_ptr()
+                B_ptrs = ids * b_bytes + B.data_ptr()
+                X = torch.empty((w.T, w.H1), dtype=self.tdt, device=dev).normal_(generator=gen)
+                Y = torch.zeros((w.T, w.H2), dtype=self.tdt, device=dev)
+                layer.append((X, Y, A_ptrs, B_ptrs))
+                self.keep += [A, B]
+            self.calls.append(layer)
+        self.d_seg = torch.from_numpy(self.seg).to(dev)
+        self.d_idx = torch.from_numpy(self.idx).to(dev)
+        self.ws_bytes = sgmv.lora_sgmv_workspace_bytes(w.T, w.r)
+        self.ws = torch.empty(self.ws_bytes // 4 + 64, dtype=torch.float32, device=dev)
+        self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.problems = [[sgmv.Problem(Y.data_ptr(), X.data_ptr(), Ap.data_ptr(), Bp.data_ptr(), w.num_adapters,
+                                       w.H1, w.H2, w.scale) for (X, Y, Ap, Bp) in layer] for layer in self.calls]
+
+    def enqueue(self, l: int, flags: int, sh) -> None:
+        """Step l: one batched launch of the layer's projections, or one lora_sgmv_apply call."""
+        sgmv, w = self.sgmv, self.spec.w
+        if self.spec.P > 1:
+            sgmv.lora_sgmv_apply_batched_flags(self.problems[l], self.d_seg, self.d_idx, self.n, w.T, w.r, self.dt,
+                                               self.max_len, flags, self.status, sh)
+            return
+        X, Y, A_ptrs, B_ptrs = self.calls[l][0]
+        sgmv.lora_sgmv_apply_flags(Y, X, A_ptrs, B_ptrs, self.d_seg, self.d_idx, self.n, w.num_adapters, w.T, w.H1,
+                                   w.r, w.H2, w.scale, self.dt, self.max_len, self.ws, self.ws_bytes, self.status,
+                                   sgmv.VARIANT_AUTO, flags, sh)
+
+
+def time_steps(ds: DeviceSpec, steps: int, flags: int, stream, world: int, dev, clocks=None) -> float:
+    """Milliseconds of `steps` steps captured as one CUDA graph (step i runs layer i mod L),
+    replayed once untimed, then once between CUDA events on the launching stream, with a
+    barrier and a device synchronize on both sides; the slowest rank's time."""
+    import torch
+    import torch.distributed as dist
+
+    sh = stream.cuda_stream
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(steps):
+            ds.enqueue(i % ds.spec.L, flags, sh)
+    with torch.cuda.stream(stream):  # a graph replays on the current stream
+        g.replay()
+    stream.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if clocks is not None:
+        clocks.__enter__()
+    with torch.cuda.stream(stream):
+        ev0.record(stream)
+        g.replay()
+        ev1.record(stream)
+    stream.synchronize()
+    if clocks is not None:
+        clocks.__exit__(None, None, None)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms = ev0.elapsed_time(ev1)
+    del g
+    return max_over_ranks(ms, world, dev)
+
+
+def launches_per_step(ds: DeviceSpec, stream) -> int:
+    before = ds.sgmv.lora_sgmv_launch_count()
+    ds.enqueue(0, 0, stream.cuda_stream)
+    stream.synchronize()
+    return int(ds.sgmv.lora_sgmv_launch_count() - before)
+
+
+def measure(spec: Spec, args, steps: int, stream, world: int, dev, rank: int, clocks=None):
+    """Times one workload: default flags (the headline form) and with early reads."""
+    from adapter_matmul_b200 import sgmv
+
+    ds = DeviceSpec(spec, dev, 1234 + rank)
+    sh = stream.cuda_stream
+    for l in range(spec.L):  # eager pass: kernel attributes, first touch
+        ds.enqueue(l, 0, sh)
+    for i in range(args.warmup):
+        ds.enqueue(i % spec.L, 0, sh)
+    stream.synchronize()
+    lps = launches_per_step(ds, stream)
+    ms = time_steps(ds, steps, 0, stream, world, dev, clocks)
+    ms_early = time_steps(ds, steps, sgmv.FLAG_EARLY_READS, stream, world, dev)
+    st = int(ds.status.item())
+    if st != 0:
+        raise RuntimeError(f"{spec.name}: device status {st:#x}")
+    return ds, ms, ms_early, lps
+
+
+def summarize(spec: Spec, ds: DeviceSpec, ms: float, ms_early: float, lps: int, steps: int, dev) -> dict:
+    """One per_config entry: the step's time, throughput and roofline (algorithmic bytes over
+    the step's time: a step is one launch, or one call of two launches for the split forms)."""
+    hbm, tc, _ = peaks()
+    w = spec.w
+    bytes_step = w.algorithmic_bytes() * spec.P
+    s = ms / 1e3 / steps
+    se = ms_early / 1e3 / steps
+    return {"name": spec.name, "workload": spec.desc,
+            "dispatch": dispatch_name(spec, ds.n, ds.max_len, ds.dt, dev),
+            "T": w.T, "adapters_touched": len(w.touched_adapters()), "calls_per_step": spec.P,
+            "launches_per_step": lps, "steps": steps, "layers_rotated": spec.L,
+            "us_per_step": round(s * 1e6, 3), "tokens_per_s": round(w.T / s, 1),
+            "algorithmic_bytes_per_step": int(bytes_step), "gbs": round(bytes_step / s / 1e9, 1),
+            "frac": round(bytes_step / s / 1e9 / hbm, 4),
+            "tflops": round(w.flops() * spec.P / s / 1e12, 3),
+            "tensor_frac": round(w.flops() * spec.P / s / 1e12 / tc, 4),
+            "early_reads": {"us_per_step": round(se * 1e6, 3),
+                            "frac": round(bytes_step / se / 1e9 / hbm, 4)}}
+
+
+def measure_layer(args, steps: int, stream, world: int, dev, rank: int) -> dict:
+    """The whole layer at the prefill shape, Y = X@W + scale*(X@A_i)@B_i, through
+    lora_sgmv_gemm_apply (the grouped kernel's shrink into the workspace, then the tcgen05 base
+    product with the delta as extra K-steps; Y written once), timed like the other entries
+    (two layers rotated: 2 x 200 MB). Beside it: the same layer unfused (torch.matmul for X@W,
+    i.e. cuBLAS, then lora_sgmv_apply adding the delta onto Y), the base product alone through
+    lora_sgmv_gemm_apply without segments, and torch.matmul alone."""
     import torch
     import torch.distributed as dist
 
     from adapter_matmul_b200 import sgmv
+
+    w = inputs.make("prefill")
+    L = 2
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(4321 + rank)
+    seg, idx, _ = sgmv.lora_sgmv_group_segments(w.ids, w.num_adapters)
+    n, max_len = len(idx), int(np.max(np.diff(seg)))
+    d_seg, d_idx = torch.from_numpy(seg).to(dev), torch.from_numpy(idx).to(dev)
+    layers = []
+    for _ in range(L):
+        X = torch.empty((w.T, w.H1), dtype=torch.bfloat16, device=dev).normal_(generator=gen)
+        W = torch.empty((w.H1, w.H2), dtype=torch.bfloat16, device=dev).normal_(0, 1 / math.sqrt(w.H1), generator=gen)
+        A = torch.empty((w.num_adapters, w.H1, w.r), dtype=torch.bfloat16, device=dev)
+        A.normal_(0, 1 / math.sqrt(w.H1), generator=gen)
+        B = torch.empty((w.num_adapters, w.r, w.H2), dtype=torch.bfloat16, device=dev)
+        B.normal_(0, 1 / math.sqrt(w.r), generator=gen)
+        ids = torch.arange(w.num_adapters, dtype=torch.int64, device=dev)
+        Ap, Bp = ids * (w.H1 * w.r * 2) + A.data_ptr(), ids * (w.r * w.H2 * 2) + B.data_ptr()
+        Y = torch.empty((w.T, w.H2), dtype=torch.bfloat16, device=dev)
+        layers.append((X, W, A, B, Ap, Bp, Y))
+    ws_bytes = sgmv.lora_sgmv_workspace_bytes(w.T, w.r)
+    ws = torch.empty(ws_bytes // 4 + 64, dtype=torch.float32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    sh = stream.cuda_stream
+
+    def fused(i):
+        X, W, _, _, Ap, Bp, Y = layers[i % L]
+        sgmv.lora_sgmv_gemm_apply(Y, X, W, Ap, Bp, d_seg, d_idx, n, w.num_adapters, w.T, w.H1, w.r, w.H2, w.scale,
+                                  sgmv.BF16, max_len, ws, ws_bytes, status, sh)
+
+    def base_only(i):
+        X, W, _, _, Ap, Bp, Y = layers[i % L]
+        sgmv.lora_sgmv_gemm_apply(Y, X, W, None, None, None, None, 0, w.num_adapters, w.T, w.H1, w.r, w.H2, w.scale,
+                                  sgmv.BF16, 0, None, 0, status, sh)
+
+    def unfused(i):
+        X, W, _, _, Ap, Bp, Y = layers[i % L]
+        torch.matmul(X, W, out=Y)
+        sgmv.lora_sgmv_apply(Y, X, Ap, Bp, d_seg, d_idx, n, w.num_adapters, w.T, w.H1, w.r, w.H2, w.scale, sgmv.BF16,
+                             max_len, ws, ws_bytes, status, sh)
+
+    def cublas(i):
+        X, W, _, _, _, _, Y = layers[i % L]
+        torch.matmul(X, W, out=Y)
+
+    def timed(fn):
+        with torch.cuda.stream(stream):
+            for i in range(max(3, args.warmup)):
+                fn(i)
+        stream.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(steps):
+                fn(i)
+        with torch.cuda.stream(stream):
+            g.replay()
+        stream.synchronize()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            g.replay()
+            e1.record(stream)
+        stream.synchronize()
+        del g
+        return max_over_ranks(e0.elapsed_time(e1), world, dev) * 1e3 / steps  # us per step
+
+    t_fused = timed(fused)
+    if int(status.item()) != 0:
+        raise RuntimeError(f"prefill layer: device status {int(status.item()):#x}")
+    t_base, t_unfused, t_cublas = timed(base_only), timed(unfused), timed(cublas)
+    hbm, tc, _ = peaks()
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            tc_sus = float(json.load(f)["bf16_tflops_sustained"])
+    except Exception:
+        tc_sus = 1400.0
+    base_fl = 2.0 * w.T * w.H1 * w.H2
+    fl = base_fl + w.flops()
+    return {"name": "prefill_layer",
+            "workload": f"Y = X@W + scale*(X@A_i)@B_i at the prefill shape: T={w.T}, H1={w.H1}, H2={w.H2}, "
+                        f"r={w.r}, bf16, {w.num_adapters} segments; step = 1 lora_sgmv_gemm_apply call",
+            "dispatch": "grouped tcgen05 shrink (V to the workspace), then sgmv_gemm_delta_kernel",
+            "T": w.T, "steps": steps, "layers_rotated": L,
+            "us_per_step": round(t_fused, 3), "tokens_per_s": round(w.T / t_fused * 1e6, 1),
+            "tflops": round(fl / t_fused / 1e6, 2), "bound": "tensor",
+            "tensor_frac": round(fl / t_fused / 1e6 / tc, 4),
+            "tensor_frac_sustained": round(fl / t_fused / 1e6 / tc_sus, 4),
+            "peaks_tflops": {"burst": tc, "sustained": tc_sus},
+            "base_only_us": round(t_base, 3), "base_only_tflops": round(base_fl / t_base / 1e6, 2),
+            "unfused_us": round(t_unfused, 3),
+            "unfused": "torch.matmul (cuBLAS) for X@W, then lora_sgmv_apply (grouped) adding the delta onto Y",
+            "cublas_us": round(t_cublas, 3), "cublas_tflops": round(base_fl / t_cublas / 1e6, 2)}
+
+
+PER_CONFIG = ["llama70b_decode_h28672", "llama70b_decode_h8192", "prefill", "distinct",
+              "uniform_h4096", "uniform_h11008", "skewed_h4096", "skewed_h11008", "identical_h4096",
+              "identical_h11008", "uniform_h4096:call", "uniform_h11008:call", "skewed_h4096:call",
+              "skewed_h11008:call", "identical_h4096:call", "identical_h11008:call"]
+
+
+def run_ours(args, spec: Spec, rank: int, world: int, local: int):
+    import torch
+    import torch.distributed as dist
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
@@ -416,234 +698,171 @@ def run_ours(args, spec: Spec, rank: int, world: int, local: int):
         from datetime import timedelta
 
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
-
-    w = spec.w
-    dt = sgmv.F16 if w.dtype == "f16" else sgmv.BF16
-    tdt = torch.float16 if w.dtype == "f16" else torch.bfloat16
-    seg, idx, _ = sgmv.lora_sgmv_group_segments(w.ids, w.num_adapters)
-    n = len(idx)
-    max_len = int(np.max(np.diff(seg)))
-    touched = w.touched_adapters()
-
-    def dev_bits(bits):
-        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(tdt).to(dev)
-
-    # per (layer, projection): adapters (pool), X, Y; adapters drawn from the seeded generator
-    gen = torch.Generator(device=dev)
-    gen.manual_seed(1234 + rank)
-    calls = []
-    keep = []
-    for l in range(spec.L):
-        for p in range(spec.P):
-            proj = l * spec.P + p
-            A_pool = torch.empty((w.num_adapters, w.H1, w.r), dtype=tdt, device=dev)
-            B_pool = torch.empty((w.num_adapters, w.r, w.H2), dtype=tdt, device=dev)
-            if len(touched) < w.num_adapters:  # resident but unused by this batch
-                A_pool.normal_(0.0, 1.0 / math.sqrt(w.H1), generator=gen)
-                B_pool.normal_(0.0, 1.0 / math.sqrt(w.r), generator=gen)
-            for i in touched:
-                A_pool[i] = dev_bits(w.adapter_a(i, proj))
-                B_pool[i] = dev_bits(w.adapter_b(i, proj))
-            A_ptrs = torch.tensor([A_pool[i].data_ptr() for i in range(w.num_adapters)], dtype=torch.int64, device=dev)
-            B_ptrs = torch.tensor([B_pool[i].data_ptr() for i in range(w.num_adapters)], dtype=torch.int64, device=dev)
-            X = dev_bits(w.x(proj))
-            Y = torch.zeros((w.T, w.H2), dtype=tdt, device=dev)
-            keep += [A_pool, B_pool]
-            calls.append((l, p, X, Y, A_ptrs, B_ptrs))
-    d_seg = torch.from_numpy(seg).to(dev)
-    d_idx = torch.from_numpy(idx).to(dev)
-    ws_bytes = sgmv.lora_sgmv_workspace_bytes(w.T, w.r)
-    ws = torch.empty(ws_bytes // 4, dtype=torch.float32, device=dev)
-    status = torch.zeros(1, dtype=torch.int32, device=dev)
-
     stream = torch.cuda.Stream(device=dev)
-    sh = stream.cuda_stream
+    w = spec.w
 
-    # one launch per step: the layer's projections share the token grouping
-    batched = {}
-    for l in range(spec.L):
-        batched[l] = [sgmv.Problem(Y.data_ptr(), X.data_ptr(), A_ptrs.data_ptr(), B_ptrs.data_ptr(),
-                                   w.num_adapters, w.H1, w.H2, w.scale)
-                      for (ll, p, X, Y, A_ptrs, B_ptrs) in calls[l * spec.P:(l + 1) * spec.P]]
-
-    def enqueue_layer(l):
-        if spec.P > 1:
-            sgmv.lora_sgmv_apply_batched(batched[l], d_seg, d_idx, n, w.T, w.r, dt, max_len, status, sh)
-            return
-        for (ll, p, X, Y, A_ptrs, B_ptrs) in calls[l * spec.P:(l + 1) * spec.P]:
-            sgmv.lora_sgmv_apply(Y, X, A_ptrs, B_ptrs, d_seg, d_idx, n, w.num_adapters, w.T, w.H1, w.r, w.H2,
-                                 w.scale, dt, max_len, ws, ws_bytes, status, sh)
-
-    # one CUDA graph per layer
-    torch.cuda.synchronize()
-    with torch.cuda.stream(stream):
-        for l in range(spec.L):  # eager warm-up (attributes, first-touch)
-            enqueue_layer(l)
-    stream.synchronize()
-    # one graph per layer, and one graph holding a whole rotation of layers back to back
-    # (as a decode step's forward pass would be captured): consecutive kernels in that graph
-    # overlap through programmatic dependent launch
-    graphs = []
-    for l in range(spec.L):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
-            enqueue_layer(l)
-        graphs.append(g)
-    rotation = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(rotation, stream=stream):
-        for l in range(spec.L):
-            enqueue_layer(l)
-
-    def run_steps(k):
-        full, rest = divmod(k, spec.L)
-        for _ in range(full):
-            rotation.replay()
-        for i in range(rest):
-            graphs[i].replay()
-
-    launches_per_step = None
-    with torch.cuda.stream(stream):
-        run_steps(args.warmup)
-    stream.synchronize()
-
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
-    # ---- timed region: K steps ----
-    barrier()
-    torch.cuda.synchronize()
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local) as clocks:
-        with torch.cuda.stream(stream):
-            ev0.record(stream)
-            run_steps(args.steps)
-            ev1.record(stream)
-        stream.synchronize()
-    torch.cuda.synchronize()
-    barrier()
-    ms = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
+    # ---- the headline: K steps of the workload ----
+    clocks = ClockSampler(local)
+    ds, ms, ms_early, lps = measure(spec, args, args.steps, stream, world, dev, rank, clocks)
     ms_per_step = ms / args.steps
+    entry = summarize(spec, ds, ms, ms_early, lps, args.steps, dev)
 
-    # kernels per step: count the launches of one eager layer
-    c0 = sgmv.lora_sgmv_launch_count()
-    with torch.cuda.stream(stream):
-        enqueue_layer(0)
-    stream.synchronize()
-    launches_per_step = sgmv.lora_sgmv_launch_count() - c0
-    gpu_launches = launches_per_step * args.steps
-
-    st = int(status.item())
-    if st != 0:
-        raise RuntimeError(f"device status {st:#x}: a segment was rejected")
-
-    # ---- roofline of the dominant kernel, per launch ----
-    # One launch per call: that kernel. Several launches per call (the split forms: a shrink
-    # kernel, then an expand kernel): the whole call, its algorithmic bytes over its duration.
+    # roofline of the dominant kernel: one launch per step (batched, fused, grouped), or the
+    # whole call where a call runs two kernels (the split forms)
     hbm, tc, which = peaks()
-    bytes_call = w.algorithmic_bytes()
-    if launches_per_step > spec.P:
-        bytes_launch = bytes_call
-        launch_s = ms_per_step / 1e3 / spec.P
-        kernel_name = ("lora_sgmv_apply, dispatcher's choice: %d launches per call, roofline over the whole call"
-                       % (launches_per_step // spec.P))
-    else:
-        bytes_launch = bytes_call * spec.P // launches_per_step
-        launch_s = ms_per_step / 1e3 / launches_per_step
-        kernel_name = ("sgmv_fused_kernel (lora_sgmv_apply_batched: %d projections per launch)" % spec.P
-                       if spec.P > 1 else "lora_sgmv_apply kernels (dispatcher's choice)")
-    roofline = make_roofline(bytes_launch, w.flops() * bytes_launch / bytes_call, launch_s, hbm, tc, which,
+    bytes_step = w.algorithmic_bytes() * spec.P
+    launch_s = ms_per_step / 1e3 / (lps if lps <= spec.P else spec.P)
+    bytes_launch = bytes_step / (lps if lps <= spec.P else spec.P)
+    kernel_name = (f"sgmv_fused_kernel (lora_sgmv_apply_batched: {spec.P} projections per launch)" if spec.P > 1
+                   else "lora_sgmv_apply, dispatcher's choice" +
+                   (f": {lps} launches per call, roofline over the whole call" if lps > 1 else ""))
+    roofline = make_roofline(bytes_launch, w.flops() * spec.P * bytes_launch / bytes_step, launch_s, hbm, tc, which,
                              measured_traffic(spec.name), kernel_name)
 
-    # ---- e2e through the public call with host buffers ----
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(args, spec, torch, sgmv, dev, stream, calls, dt, tdt, world)
+        e2e = run_e2e(args, ds, stream, world, dev)
+    del ds
+    torch.cuda.empty_cache()
+
+    # ---- every configuration ----
+    per_config = {}
+    if not args.no_per_config:
+        steps_cfg = max(args.warmup, min(args.steps, PER_CONFIG_MAX_STEPS))
+        for name in PER_CONFIG:
+            if name == spec.name:
+                per_config[name] = entry
+                continue
+            sp = make_spec(name)
+            d2, m2, m2e, l2 = measure(sp, args, steps_cfg, stream, world, dev, rank)
+            per_config[name] = summarize(sp, d2, m2, m2e, l2, steps_cfg, dev)
+            del d2
+            torch.cuda.empty_cache()
+        per_config["prefill_layer"] = measure_layer(args, min(steps_cfg, 50), stream, world, dev, rank)
+        torch.cuda.empty_cache()
 
     result = None
     if rank == 0:
         value = job_tokens_per_s(w.T * args.steps, world, ms / 1e3)
+        cfg = config_dict(spec, world)
+        cfg.update({"layers_rotated": spec.L,
+                    "l2": f"inputs larger than L2: {spec.L} layers rotated, "
+                          f"{spec.L * bytes_step / 2**30:.2f} GiB of algorithmic bytes per rotation",
+                    "timing": "CUDA events on the launching stream around one replay of a CUDA graph of exactly "
+                              "K steps (step i on layer i mod L), after one untimed replay",
+                    "overlap": "launches chained by programmatic dependent launch under the default contract: the "
+                               "next launch's prologue overlaps the end of the previous one; it reads none of its "
+                               "inputs before the previous launch completes (early_reads: the same with "
+                               "LORA_SGMV_FLAG_EARLY_READS, adapters streamed during the previous launch)"})
         result = {
             "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
-            "config": {"workload": spec.desc, "name": spec.name, "T": w.T, "H1": w.H1, "H2": w.H2, "r": w.r,
-                       "adapters_touched": len(touched), "segments": n, "sgmv_calls_per_step": spec.P,
-                       "dispatch": dispatch_name(spec, n, max_len, dt, dev),
-                       "layers_rotated": spec.L,
-                       "l2": f"inputs larger than L2: {spec.L} layers rotated, "
-                             f"{spec.L * spec.P * bytes_call / 2**30:.2f} GiB of algorithmic bytes per rotation",
-                       "timing": "CUDA events on the launching stream; K layer steps replayed as CUDA graphs "
-                                 "of whole layer rotations (plus single-layer graphs for the remainder)",
-                       "parallelism": f"replicas x{world}"},
+            "config": cfg,
+            "dispatch": entry["dispatch"],
             "roofline": roofline,
-            "gpu_launches": int(gpu_launches),
+            "early_reads": entry["early_reads"],
+            "gpu_launches": int(lps * args.steps),
             "clocks": clocks.summary(),
         }
         if e2e:
             result["e2e"] = e2e
+        if per_config:
+            result["per_config"] = per_config
     if world > 1:
         dist.barrier()
-        del graphs, rotation
         dist.destroy_process_group()
     return result
 
 
-def run_e2e(args, spec, torch, sgmv, dev, stream, calls, dt, tdt, world=1):
-    """Same metric through the public calls with host buffers: lora_sgmv_group_segments on the
-    host, then one lora_sgmv_apply_batched launch for the step's projections (lora_sgmv_apply
-    for one projection). Per step the segment arrays, X and Y of every projection go host ->
-    device (one pinned copy each, the projections packed), and the step's Y comes back."""
-    w = spec.w
-    P = spec.P
+def run_e2e(args, ds: DeviceSpec, stream, world: int, dev) -> dict:
+    """The metric through the public calls with host buffers. Per step: group the batch's adapter
+    ids on the host (lora_sgmv_group_segments), copy the segment arrays and every projection's X
+    and Y from pinned host memory (one packed copy), run the step's SGMV launch
+    (lora_sgmv_apply_batched, or lora_sgmv_apply for one projection), copy Y back to pinned host
+    memory and read it there. Two buffer sets and three streams (host-to-device copies, compute,
+    device-to-host copies): step i's copy in overlaps step i-1's launch and copy out; a buffer
+    set is reused only after its previous step's result has been read. Host wall clock."""
+    import torch
+
+    sgmv, spec, w = ds.sgmv, ds.spec, ds.spec.w
+    P, NB = spec.P, 2
     steps = max(3, min(args.steps, 200))
-    hX = torch.empty((P, w.T, w.H1), dtype=tdt, pin_memory=True)
-    hY = torch.empty((P, w.T, w.H2), dtype=tdt, pin_memory=True)
-    for p in range(P):
-        hX[p].copy_(calls[p][2].cpu())
-        hY[p].copy_(calls[p][3].cpu())
-    outY = torch.empty((P, w.T, w.H2), dtype=tdt, pin_memory=True)
-    ids = np.ascontiguousarray(w.ids, dtype=np.int32)
     meta_len = 2 * w.num_adapters + 1
-    h_meta = torch.empty(meta_len, dtype=torch.int32, pin_memory=True)  # seg_starts, then lora_idx
-    h_meta_np = h_meta.numpy()
-    d_meta = torch.empty(meta_len, dtype=torch.int32, device=dev)
-    dX = torch.empty((P, w.T, w.H1), dtype=tdt, device=dev)
-    dY = torch.empty((P, w.T, w.H2), dtype=tdt, device=dev)
-    ws_bytes = sgmv.lora_sgmv_workspace_bytes(w.T, w.r)
-    ws = torch.empty(ws_bytes // 4, dtype=torch.float32, device=dev)
-    problems = [[sgmv.Problem(dY[p].data_ptr(), dX[p].data_ptr(), calls[l * P + p][4].data_ptr(),
-                              calls[l * P + p][5].data_ptr(), w.num_adapters, w.H1, w.H2, w.scale)
-                 for p in range(P)] for l in range(spec.L)]
-    sh = stream.cuda_stream
+    meta_bytes = (meta_len * 4 + 255) // 256 * 256
+    x_bytes, y_bytes = P * w.T * w.H1 * 2, P * w.T * w.H2 * 2
+    in_bytes = meta_bytes + x_bytes + y_bytes
+    h_in = torch.empty((NB, in_bytes), dtype=torch.uint8, pin_memory=True)
+    d_in = torch.empty((NB, in_bytes), dtype=torch.uint8, device=dev)
+    outY = torch.empty((NB, y_bytes), dtype=torch.uint8, pin_memory=True)
+    hX = torch.stack([ds.calls[0][p][0] for p in range(P)]).cpu().view(torch.uint8).reshape(-1)
+    hY = torch.stack([ds.calls[0][p][1] for p in range(P)]).cpu().view(torch.uint8).reshape(-1)
+    for b in range(NB):  # the step's inputs, staged once in pinned memory (copied every step)
+        h_in[b, meta_bytes:meta_bytes + x_bytes].copy_(hX)
+        h_in[b, meta_bytes + x_bytes:].copy_(hY)
+    h_meta = [h_in[b, :meta_bytes].numpy().view(np.int32) for b in range(NB)]
+    ids = np.ascontiguousarray(w.ids, dtype=np.int32)
+    ws = torch.empty((NB, ds.ws_bytes // 4 + 64), dtype=torch.float32, device=dev)
+    base = [d_in[b].data_ptr() for b in range(NB)]
+    xs = [[base[b] + meta_bytes + p * w.T * w.H1 * 2 for p in range(P)] for b in range(NB)]
+    ys = [[base[b] + meta_bytes + x_bytes + p * w.T * w.H2 * 2 for p in range(P)] for b in range(NB)]
+    problems = [[[sgmv.Problem(ys[b][p], xs[b][p], ds.calls[l][p][2].data_ptr(), ds.calls[l][p][3].data_ptr(),
+                               w.num_adapters, w.H1, w.H2, w.scale) for p in range(P)] for l in range(spec.L)]
+                for b in range(NB)]
+    s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    ev_in = [torch.cuda.Event() for _ in range(NB)]
+    ev_run = [torch.cuda.Event() for _ in range(NB)]
+    ev_out = [torch.cuda.Event() for _ in range(NB)]
+    used = [False] * NB
+    sink = [0]
     h2d = d2h = 0
+    out_np = [outY[b].numpy() for b in range(NB)]
+
+    def read_back(b):
+        ev_out[b].synchronize()
+        sink[0] ^= int(out_np[b][0])  # the host reads the step's result
 
     def one(i):
         nonlocal h2d, d2h
-        l = i % spec.L
+        b, l = i % NB, i % spec.L
+        if used[b]:
+            read_back(b)  # step i-2: its result read, its buffers free
+        used[b] = True
         seg, idx, _ = sgmv.lora_sgmv_group_segments(ids, w.num_adapters)
         n = len(idx)
-        h_meta_np[: n + 1] = seg
-        h_meta_np[n + 1: 2 * n + 1] = idx
+        h_meta[b][: n + 1] = seg
+        h_meta[b][n + 1: 2 * n + 1] = idx
         max_len = int(np.max(np.diff(seg)))
-        d_seg, d_idx = d_meta.data_ptr(), d_meta.data_ptr() + 4 * (n + 1)
-        with torch.cuda.stream(stream):
-            d_meta[: 2 * n + 1].copy_(h_meta[: 2 * n + 1], non_blocking=True)
-            dX.copy_(hX, non_blocking=True)
-            dY.copy_(hY, non_blocking=True)
-            if P > 1:
-                sgmv.lora_sgmv_apply_batched(problems[l], d_seg, d_idx, n, w.T, w.r, dt, max_len, None, sh)
-            else:
-                q = problems[l][0]
-                sgmv.lora_sgmv_apply(q.Y, q.X, q.A_ptrs, q.B_ptrs, d_seg, d_idx, n, w.num_adapters, w.T, w.H1, w.r,
-                                     w.H2, w.scale, dt, max_len, ws, ws_bytes, None, sh)
-            outY.copy_(dY, non_blocking=True)
-        stream.synchronize()
-        h2d = (2 * n + 1) * 4 + hX.numel() * 2 + hY.numel() * 2
-        d2h = outY.numel() * 2
+        d_seg, d_idx = base[b], base[b] + 4 * (n + 1)
+        s_in.wait_event(ev_out[b])  # step i-2's copy out of this buffer set (recorded, or never)
+        with torch.cuda.stream(s_in):
+            d_in[b].copy_(h_in[b], non_blocking=True)
+        ev_in[b].record(s_in)
+        stream.wait_event(ev_in[b])
+        if P > 1:
+            sgmv.lora_sgmv_apply_batched(problems[b][l], d_seg, d_idx, n, w.T, w.r, ds.dt, max_len, None, stream)
+        else:
+            q = problems[b][l][0]
+            sgmv.lora_sgmv_apply(q.Y, q.X, q.A_ptrs, q.B_ptrs, d_seg, d_idx, n, w.num_adapters, w.T, w.H1, w.r,
+                                 w.H2, w.scale, ds.dt, max_len, ws[b], ds.ws_bytes, None, stream)
+        ev_run[b].record(stream)
+        s_out.wait_event(ev_run[b])
+        with torch.cuda.stream(s_out):
+            outY[b].copy_(d_in[b, meta_bytes + x_bytes:], non_blocking=True)
+        ev_out[b].record(s_out)
+        h2d = in_bytes
+        d2h = y_bytes
+
+    def drain():
+        for b in range(NB):
+            if used[b]:
+                read_back(b)
+                used[b] = False
 
     for i in range(3):
         one(i)
+    drain()
+    torch.cuda.synchronize()
     if world > 1:
         import torch.distributed as dist
 
@@ -651,13 +870,15 @@ def run_e2e(args, spec, torch, sgmv, dev, stream, calls, dt, tdt, world=1):
     t0 = time.perf_counter()
     for i in range(steps):
         one(i)
+    drain()
     el = max_over_ranks(time.perf_counter() - t0, world, dev)
     call = "1 lora_sgmv_apply_batched launch" if P > 1 else "1 lora_sgmv_apply call"
     return {"value": round(job_tokens_per_s(w.T * steps, world, el), 1), "unit": UNIT,
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": steps,
-            "note": "host wall clock (the host's grouping is part of the step), slowest rank; per step: host "
-                    f"grouping, pinned H2D of the segment arrays and of X and Y ({P} projections), {call}, "
-                    "D2H of Y, stream sync"}
+            "note": "host wall clock, slowest rank; per step: host grouping, one pinned H2D of the segment "
+                    f"arrays with X and Y ({P} projections), {call}, D2H of Y read on the host; two buffer "
+                    "sets on three streams, so one step's copy in overlaps the previous step's launch and "
+                    "copy out"}
 
 
 # ---------------------------------------------------------------------------------------------
@@ -684,7 +905,7 @@ def run_reference(args, spec: Spec, rank: int):
         "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": 0, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(el * 1e3 / max(1, args.steps), 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": spec.w.dtype, "data": "synthetic",
-        "config": {"workload": spec.desc, "name": spec.name, "T": spec.w.T},
+        "config": config_dict(spec, int(os.environ.get("WORLD_SIZE", "1"))),
         "impl": "reference",
         "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": 1, "kind": "oracle",
                          "sample": runs[0]["sample"]},
@@ -695,16 +916,19 @@ def run_reference(args, spec: Spec, rank: int):
 def main():
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20000)
-    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="distinct", choices=["distinct"] + list(inputs.CONFIGS))
+    ap.add_argument("--workload", default="distinct", choices=workload_names())
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.steps < 1:
+        ap.error("--steps must be >= 1")
     rank, world, local = dist_env()
     spec = make_spec(args.workload)
     if args.impl == "reference":

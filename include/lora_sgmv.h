@@ -48,15 +48,19 @@
  *   - Alignment: X, Y, V and workspace must be 16-byte aligned; H1 and H2
  *     must be multiples of 8.
  *   - Overlap with the previous kernel: the fused kernels (variants FUSED
- *     and FUSED_TC, which AUTO picks for short segments, and
- *     lora_sgmv_apply_batched) are launched with programmatic dependent
- *     launch. It reads segment arrays,
- *     pointer tables and adapter weights while the kernel before it on the
- *     stream may still run, and reads X and Y only after that kernel has
- *     completed. So seg_starts, lora_idx, the tables and the adapters of a
- *     call must not be written by the kernel launched immediately before it
- *     on the same stream (copies and earlier kernels are fine); X and Y may
- *     be. Use LORA_SGMV_VARIANT_SPLIT where that does not hold.
+ *     and FUSED_TC, which AUTO picks for short segments, and the batched
+ *     call) are launched with programmatic dependent launch, so their
+ *     prologue (barriers, tensor memory, tables of tensor maps) overlaps the
+ *     end of the kernel before them on the stream. By default they read
+ *     nothing the caller passed until that kernel has completed, so any
+ *     kernel may write any of a call's inputs right before it. With
+ *     LORA_SGMV_FLAG_EARLY_READS (lora_sgmv_apply_flags,
+ *     lora_sgmv_apply_batched_flags) the caller states that seg_starts,
+ *     lora_idx, the pointer tables and the adapters are not written by the
+ *     kernel launched immediately before the call on the same stream (copies
+ *     and earlier kernels may write them); the kernels then start streaming
+ *     adapter weights while that kernel still runs. X and Y are always read
+ *     only after it has completed.
  *   - Thread safety: calls on different streams may run concurrently. The
  *     library keeps no mutable global state other than a lazily filled,
  *     mutex-guarded cache of device facts and kernel attributes, an atomic
@@ -98,6 +102,11 @@ typedef enum {
 #define LORA_SGMV_DEV_BAD_ADAPTER 0x2u  /* lora_idx[s] outside [0, num_adapters): skipped */
 #define LORA_SGMV_DEV_BAD_POINTER 0x4u  /* table entry NULL or not 16-byte aligned: skipped */
 #define LORA_SGMV_DEV_TIMEOUT 0x8u      /* a bounded wait inside a kernel gave up: results invalid */
+#define LORA_SGMV_DEV_BAD_RANK 0x10u    /* lora_sgmv_apply_ranks: the adapter's rank is not usable: skipped */
+
+/* Flags of lora_sgmv_apply_flags and lora_sgmv_apply_batched_flags. */
+#define LORA_SGMV_FLAG_EARLY_READS 0x1u /* segment arrays, tables and adapters are not written by the
+                                           kernel launched right before the call: read them early */
 
 /* Which kernels lora_sgmv_apply_ex runs. AUTO lets the dispatcher choose. */
 typedef enum {
@@ -179,7 +188,10 @@ lora_sgmv_status lora_sgmv_group_segments(const int32_t* ids, int32_t T, int32_t
  *   r_src, r     1 <= r_src <= r; r_src == r copies.
  *   dtype        16-bit storage type of the four matrices.
  *   stream       cudaStream_t as void*; one kernel launch per matrix given.
- * A destination must not overlap its source. Returns LORA_SGMV_ERR_DTYPE,
+ * A destination must not overlap its source. The padding kernel writes
+ * adapters, so an SGMV call right after it on the same stream must not pass
+ * LORA_SGMV_FLAG_EARLY_READS (the default calls wait for it to complete).
+ * Returns LORA_SGMV_ERR_DTYPE,
  * _NULL (no pair given, or half a pair) or _DIM before any launch, _CUDA if a
  * launch fails, else LORA_SGMV_OK. Runs at adapter load time, not per call.
  */
@@ -278,6 +290,19 @@ lora_sgmv_status lora_sgmv_apply_ex(void* Y, const void* X, const void* const* A
                                     int32_t max_seg_len, void* workspace, size_t workspace_bytes,
                                     uint32_t* dev_status, lora_sgmv_variant variant, void* stream);
 
+/* lora_sgmv_apply_ex with flags: 0 or LORA_SGMV_FLAG_EARLY_READS (see
+ * "Overlap with the previous kernel" above). Other bits return
+ * LORA_SGMV_ERR_UNSUPPORTED. Flags change timing only, never results, as long
+ * as the caller's statement holds. */
+lora_sgmv_status lora_sgmv_apply_flags(void* Y, const void* X, const void* const* A_ptrs,
+                                       const void* const* B_ptrs, const int32_t* seg_starts,
+                                       const int32_t* lora_idx, int32_t n_segments,
+                                       int32_t num_adapters, int32_t T, int32_t H1, int32_t r,
+                                       int32_t H2, float scale, lora_sgmv_dtype dtype,
+                                       int32_t max_seg_len, void* workspace, size_t workspace_bytes,
+                                       uint32_t* dev_status, lora_sgmv_variant variant,
+                                       uint32_t flags, void* stream);
+
 /* One projection of a batched call (see lora_sgmv_apply_batched). */
 typedef struct {
     void* Y;                      /* device, [T, H2], in/out */
@@ -316,6 +341,75 @@ lora_sgmv_status lora_sgmv_apply_batched(const lora_sgmv_problem* problems, int3
                                          lora_sgmv_dtype dtype, int32_t max_seg_len,
                                          uint32_t* dev_status, void* stream);
 
+/* lora_sgmv_apply_batched with flags, as for lora_sgmv_apply_flags. */
+lora_sgmv_status lora_sgmv_apply_batched_flags(const lora_sgmv_problem* problems, int32_t n_problems,
+                                               const int32_t* seg_starts, const int32_t* lora_idx,
+                                               int32_t n_segments, int32_t T, int32_t r,
+                                               lora_sgmv_dtype dtype, int32_t max_seg_len,
+                                               uint32_t flags, uint32_t* dev_status, void* stream);
+
+/*
+ * lora_sgmv_apply_ranks -- lora_sgmv_apply for adapters of different ranks, unpadded.
+ *
+ * The authors' reply on adapters of different ranks (page "Punica: Serving
+ * multiple LoRA finetuned LLM as one", the Hacker News thread) names a grouped
+ * GEMM whose groups have their own sizes. Here adapter i keeps its own rank
+ * r_i: A_i is [H1, r_i] and B_i is [r_i, H2], dense, no padded copy. The
+ * grouped tensor-core kernel runs at rank r_max; each tile's tensor maps take
+ * the adapter's own extent and row pitch, so the columns of A_i (rows of B_i)
+ * past r_i are read as zeros by the copy engine and add nothing. The result is
+ * the adapter's own product at its own rank.
+ *   ranks        device, int32[num_adapters]: r_i, with 8 <= r_i <= r_max
+ *                and r_i a multiple of 8 (rows of A_i in whole 16-byte units).
+ *                A segment whose adapter has another rank is skipped and
+ *                LORA_SGMV_DEV_BAD_RANK is set in *dev_status.
+ *   r_max        16, 32 or 64 (LORA_SGMV_ERR_UNSUPPORTED otherwise).
+ *   H1, H2       at least 64, multiples of 8.
+ *   other arguments as for lora_sgmv_apply; no workspace (V stays on chip).
+ * The grouped kernel is built for long segments (prefill); it is correct for
+ * any segment length, but decode batches run faster padded to one rank
+ * (lora_sgmv_pad_rank) through lora_sgmv_apply.
+ */
+lora_sgmv_status lora_sgmv_apply_ranks(void* Y, const void* X, const void* const* A_ptrs,
+                                       const void* const* B_ptrs, const int32_t* ranks,
+                                       const int32_t* seg_starts, const int32_t* lora_idx,
+                                       int32_t n_segments, int32_t num_adapters, int32_t T, int32_t H1,
+                                       int32_t r_max, int32_t H2, float scale, lora_sgmv_dtype dtype,
+                                       uint32_t* dev_status, void* stream);
+
+/*
+ * lora_sgmv_gemm_apply -- the whole LoRA layer: Y = X@W + scale * (X@A_i)@B_i.
+ *
+ * The README's multi-LoRA paragraph writes the batch as Y = X@W plus the
+ * per-row adapter terms, and its LoRA paragraph gives x@(W + A@B) = x@W +
+ * x@A@B. This call computes both terms in one tensor-core accumulation: after
+ * V = X@A_i (fp32, into the workspace, by the grouped kernel's shrink for
+ * long segments or the split-K shrink), each output tile of X@W takes 2r more
+ * K-steps per adapter whose segment touches the tile, with scale * V carried
+ * as two 16-bit operands (about 16 significant bits). Y is rounded once to the
+ * storage type and written; it is an output, not read. So the delta costs no
+ * read and no write of Y beyond the base product's own write.
+ *   Y            device, [T, H2] out: every row written; rows in no valid
+ *                segment get round(X@W).
+ *   X            device, [T, H1].
+ *   W            device, [H1, H2] row-major, the frozen base weight.
+ *   A_ptrs, B_ptrs, seg_starts, lora_idx, n_segments, num_adapters, T,
+ *   scale, dtype, max_seg_len, dev_status, stream: as for lora_sgmv_apply.
+ *   H1, H2       multiples of 8 (LORA_SGMV_ERR_ALIGN otherwise).
+ *   r            16, 32 or 64 (LORA_SGMV_ERR_UNSUPPORTED otherwise).
+ *   workspace    device scratch of lora_sgmv_workspace_bytes(T, r) bytes for V
+ *                (may be NULL when n_segments is 0).
+ * X, Y and W must be 16-byte aligned. Runs two kernels on `stream` (one when
+ * n_segments is 0). Rejected segments are reported in *dev_status and their
+ * rows get the base product alone.
+ */
+lora_sgmv_status lora_sgmv_gemm_apply(void* Y, const void* X, const void* W, const void* const* A_ptrs,
+                                      const void* const* B_ptrs, const int32_t* seg_starts,
+                                      const int32_t* lora_idx, int32_t n_segments, int32_t num_adapters,
+                                      int32_t T, int32_t H1, int32_t r, int32_t H2, float scale,
+                                      lora_sgmv_dtype dtype, int32_t max_seg_len, void* workspace,
+                                      size_t workspace_bytes, uint32_t* dev_status, void* stream);
+
 /*
  * lora_sgmv_apply_noalloc -- lora_sgmv_apply for callers that cannot allocate.
  *
@@ -334,7 +428,9 @@ lora_sgmv_status lora_sgmv_apply_batched(const lora_sgmv_problem* problems, int3
  *
  * The first call on each device looks up the array's device address (once
  * per device, with that device current); make that first call before any
- * stream capture. Every call on a device shares the one array and leaves
+ * stream capture. The address is kept until the process exits: after a
+ * cudaDeviceReset the array may move, so do not call this entry point again
+ * on a device that was reset. Every call on a device shares the one array and leaves
  * its last contents there (nothing in it needs to start at zero: each call
  * writes every V row it reads). Calls whose kernels overlap on the GPU --
  * on different streams, or from different threads -- race on the array and

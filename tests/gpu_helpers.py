@@ -89,11 +89,11 @@ class DeviceProblem:
 
     def oracle_apply(self, scale=None):
         w = self.w
-        A = [self.A.get(i, np.zeros((w.H1, w.r), np.uint16)) for i in range(w.num_adapters)]
-        B = [self.B.get(i, np.zeros((w.r, w.H2), np.uint16)) for i in range(w.num_adapters)]
-        out, _ = oracle.apply_f32(self.y_bits, self.x_bits, A, B, self.seg, self.idx,
-                                  w.scale if scale is None else scale, w.dtype)
-        return out
+        zA, zB = np.zeros((w.H1, w.r), np.uint16), np.zeros((w.r, w.H2), np.uint16)
+        A = [self.A.get(i, zA) for i in range(w.num_adapters)]
+        B = [self.B.get(i, zB) for i in range(w.num_adapters)]
+        return oracle_apply_rows(self.y_bits, self.x_bits, A, B, self.seg, self.idx,
+                                 w.scale if scale is None else scale, w.dtype)
 
 
 def assert_close(got_bits, ref_bits, dtype, what=""):
@@ -106,3 +106,34 @@ def assert_close(got_bits, ref_bits, dtype, what=""):
         raise AssertionError(f"{what}: {int(bad.sum())} elements out of tolerance; first at {tuple(i)}: "
                              f"gpu={g[tuple(i)]} oracle={o[tuple(i)]}; max abs err {err.max():.3e}")
     return float(err.max())
+
+
+def oracle_apply_rows(y_bits, x_bits, A, B, seg, idx, scale, dtype, threads=None):
+    """The whole-batch oracle over all rows, run on row shares in threads (the C oracle
+    releases the GIL): each thread takes rows [a, b) with the segments cut to that range.
+    Rows are independent in the definition, so the stitched result is the oracle's own."""
+    import os
+    from concurrent.futures import ThreadPoolExecutor
+
+    from bench import rows_share
+
+    T = y_bits.shape[0]
+    seg = np.asarray(seg, np.int64)
+    if len(seg) < 2 or seg[0] != 0 or seg[-1] != T or np.any(np.diff(seg) < 0):
+        out, _ = oracle.apply_f32(y_bits, x_bits, A, B, seg, idx, scale, dtype)  # not a plain grouping
+        return out
+    n = max(1, min(threads or os.cpu_count() or 1, 64, T))
+    bounds = [round(k * T / n) for k in range(n + 1)]
+    out = np.array(y_bits, copy=True)
+
+    def one(k):
+        a, b = bounds[k], bounds[k + 1]
+        if a == b:
+            return
+        sub_seg, sub_idx = rows_share(seg, idx, a, b)
+        res, _ = oracle.apply_f32(y_bits[a:b], x_bits[a:b], A, B, sub_seg, sub_idx, scale, dtype)
+        out[a:b] = res
+
+    with ThreadPoolExecutor(n) as ex:
+        list(ex.map(one, range(n)))
+    return out

@@ -97,3 +97,62 @@ def test_mixed_rank_sgmv_matches_oracle(dtn, variant):
     g, o = f64(_host(dY)), f64(ref)
     err = np.abs(g - o)
     assert np.all(err <= 2e-2 + 1e-2 * np.abs(o)), f"max abs err {err.max()}"
+
+
+# ---- adapters of different ranks without padding: lora_sgmv_apply_ranks ---------------------
+
+def _own_rank_reference(X, Y, A, B, seg, idx, scale, dt, ranks_ok):
+    """The oracle segment by segment, each at its adapter's own rank (unpadded matrices)."""
+    out = np.array(Y, copy=True)
+    for s in range(len(idx)):
+        b, e, i = int(seg[s]), int(seg[s + 1]), int(idx[s])
+        if e <= b or not ranks_ok(i):
+            continue
+        res, _ = oracle.apply_f32(Y[b:e], X[b:e], [A[i]], [B[i]], [0, e - b], [0], scale, dt)
+        out[b:e] = res
+    return out
+
+
+@pytest.mark.parametrize("dt", ["bf16", "f16"])
+@pytest.mark.parametrize("r_max,ranks", [(64, [8, 16, 24, 40, 64, 12, 72]), (32, [8, 16, 24, 32]), (16, [8, 16])])
+def test_apply_ranks_unpadded_matches_each_adapters_own_product(dt, r_max, ranks):
+    import torch
+
+    H1, H2 = 320, 392
+    lens = [130, 3, 200, 0, 64, 129, 1, 90]
+    seg = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    nA = len(ranks)
+    idx = np.array([k % nA for k in range(len(lens))], np.int32)[::-1].copy()
+    T = int(seg[-1])
+    base = inputs.small_random(T, nA, H1, H2, 8, dt, seed=r_max)
+    X, Y = base.x(), base.y_random()
+    A = [inputs.small_random(T, nA, H1, H2, rk, dt, seed=100 + k).adapter_a(k) for k, rk in enumerate(ranks)]
+    B = [inputs.small_random(T, nA, H1, H2, rk, dt, seed=100 + k).adapter_b(k) for k, rk in enumerate(ranks)]
+    dA = [_dev(a) for a in A]
+    dB = [_dev(b) for b in B]
+    A_ptrs = torch.tensor([t.data_ptr() for t in dA], dtype=torch.int64, device="cuda")
+    B_ptrs = torch.tensor([t.data_ptr() for t in dB], dtype=torch.int64, device="cuda")
+    d_ranks = torch.tensor(ranks, dtype=torch.int32, device="cuda")
+    dX, dY = _dev(X), _dev(Y)
+    d_seg = torch.from_numpy(seg).cuda()
+    d_idx = torch.from_numpy(idx).cuda()
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    code = sgmv.F16 if dt == "f16" else sgmv.BF16
+    sgmv.lora_sgmv_apply_ranks(dY, dX, A_ptrs, B_ptrs, d_ranks, d_seg, d_idx, len(idx), nA, T, H1, r_max, H2, 0.8,
+                               code, status)
+    torch.cuda.synchronize()
+
+    def ok(i):
+        return 8 <= ranks[i] <= r_max and ranks[i] % 8 == 0
+
+    ref = _own_rank_reference(X, Y, A, B, seg, idx, 0.8, dt, ok)
+    got = _host(dY)
+    st = int(status.item())
+    used_bad = any(not ok(int(idx[s])) and seg[s + 1] > seg[s] for s in range(len(idx)))
+    assert bool(st & sgmv.DEV_BAD_RANK) == used_bad and not (st & ~sgmv.DEV_BAD_RANK)
+    from gpu_helpers import assert_close
+
+    assert_close(got, ref, dt, f"ranks {ranks} at r_max {r_max}")
+    for s in range(len(idx)):  # rows of skipped segments are untouched, bit for bit
+        if not ok(int(idx[s])):
+            assert np.array_equal(got[seg[s]:seg[s + 1]], Y[seg[s]:seg[s + 1]])
