@@ -18,7 +18,6 @@
 #include "sgmv_gemm_tc.cuh"
 #include "sgmv_grouped_tc.cuh"
 #include "sgmv_pad.cuh"
-#include "sgmv_shrink_tma.cuh"
 #include "sgmv_split.cuh"
 
 namespace {
@@ -129,103 +128,8 @@ lora_sgmv_status max_active_clusters(K kernel, int cluster, size_t smem, int* ou
     return LORA_SGMV_OK;
 }
 
-// Cluster size of the TMA shrink: slices of A_i of at least 512 rows, at most 8 CTAs.
-int shrink_tma_cluster(int H1) {
-    int C = 1;
-    while (C < 8 && H1 / (C * 2) >= 512) C *= 2;
-    return C;
-}
-
-// The shrink with every operand staged by TMA (sgmv_shrink_tma.cuh).
-template <typename T, int R>
-lora_sgmv_status launch_shrink_tma(const ShrinkParams& p0, cudaStream_t stream) {
-    using G = sgmv::ShrinkTmaGeom<R>;
-    static int smem_granted[64] = {};
-    static int resident[64][4][9] = {};  // (device, log2 cluster size, prefix bucket)
-    const int C = shrink_tma_cluster(p0.H1);
-    sgmv::ShrinkTmaParams p = {};
-    p.V = p0.V;
-    p.A_ptrs = p0.A_ptrs;
-    p.B_check = p0.B_check;
-    p.seg_starts = p0.seg_starts;
-    p.lora_idx = p0.lora_idx;
-    p.dev_status = p0.dev_status;
-    p.n_segments = p0.n_segments;
-    p.num_adapters = p0.num_adapters;
-    p.T = p0.T;
-    p.H1 = p0.H1;
-    p.ks = ((p0.H1 + C - 1) / C + 63) / 64 * 64;
-    p.share = ((G::TILE + C - 1) / C + 3) / 4 * 4;
-    const int bucket = (p.n_segments + 1 + 1023) / 1024;  // 1..9
-    const size_t smem = G::BASE + 2 * G::x_bytes(p.ks) + size_t(bucket) * 1024 * 4;
-    DeviceFacts f;
-    if (device_facts(f) != LORA_SGMV_OK) return LORA_SGMV_ERR_CUDA;
-    if (smem + 2048 > static_cast<size_t>(f.max_smem_optin)) return LORA_SGMV_ERR_DIM;
-    auto kernel = sgmv::sgmv_shrink_tma_kernel<T, R>;
-    if (ensure_smem(kernel, smem, smem_granted) != LORA_SGMV_OK) return LORA_SGMV_ERR_CUDA;
-    int dev = 0;
-    if (record(cudaGetDevice(&dev)) != cudaSuccess) return LORA_SGMV_ERR_CUDA;
-    if (dev < 0 || dev >= 64) return LORA_SGMV_ERR_UNSUPPORTED;
-    const int lc = C == 1 ? 0 : (C == 2 ? 1 : (C == 4 ? 2 : 3));
-    int clusters_max = 0;
-    {
-        std::lock_guard<std::mutex> lock(g_mu);
-        clusters_max = resident[dev][lc][bucket - 1];
-    }
-    if (clusters_max <= 0) {
-        lora_sgmv_status st = max_active_clusters(kernel, C, smem, &clusters_max, sgmv::kSTThreads);
-        if (st != LORA_SGMV_OK) return st;
-        std::lock_guard<std::mutex> lock(g_mu);
-        resident[dev][lc][bucket - 1] = clusters_max;
-    }
-    CUtensorMap tmX;
-    if (!sgmv::make_shrink_x_map(&tmX, p0.X, p.T, p.H1, p.ks,
-                                 std::is_same<T, __half>::value ? LORA_SGMV_F16 : LORA_SGMV_BF16)) {
-        t_last_error = cudaErrorInvalidValue;
-        return LORA_SGMV_ERR_CUDA;
-    }
-    // units: at most one chunk per token and one partial chunk per segment
-    const long long units = std::max<long long>(
-        1, std::min<long long>(static_cast<long long>(p.n_segments) + (p.T + sgmv::kSTTokens - 1) / sgmv::kSTTokens,
-                               p.T));
-    int clusters = static_cast<int>(std::min<long long>(units, clusters_max));
-    const long long rounds = (units + clusters - 1) / clusters;
-    clusters = static_cast<int>((units + rounds - 1) / rounds);
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(clusters * C, 1, 1);
-    cfg.blockDim = dim3(sgmv::kSTThreads, 1, 1);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = C;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return counted(cudaLaunchKernelEx(&cfg, kernel, tmX, p));
-}
-
-// Whether the TMA shrink takes a call: H1 a multiple of 64, its unit list and X buffers in
-// shared memory (at most 8192 segments, at most kSTMaxKs rows of A_i per CTA).
-template <int R>
-bool shrink_tma_fits(int H1, int n_segments, int max_smem_optin) {
-    if (H1 % 64 != 0 || n_segments > sgmv::kSTMaxSegments) return false;
-    const int C = shrink_tma_cluster(H1);
-    const int ks = ((H1 + C - 1) / C + 63) / 64 * 64;
-    if (ks > sgmv::kSTMaxKs) return false;
-    const int bucket = (n_segments + 1 + 1023) / 1024;
-    using G = sgmv::ShrinkTmaGeom<R>;
-    return G::BASE + 2 * G::x_bytes(ks) + size_t(bucket) * 1024 * 4 + 2048 <= size_t(max_smem_optin);
-}
-
 template <typename T, int R>
 lora_sgmv_status launch_shrink(const ShrinkParams& p0, int max_len, cudaStream_t stream) {
-    {
-        DeviceFacts f;
-        if (device_facts(f) != LORA_SGMV_OK) return LORA_SGMV_ERR_CUDA;
-        if (shrink_tma_fits<R>(p0.H1, p0.n_segments, f.max_smem_optin)) return launch_shrink_tma<T, R>(p0, stream);
-    }
     static int smem_granted[64] = {};
     ShrinkParams p = p0;
     const int C = cluster_size_for(p.H1);
@@ -705,6 +609,7 @@ lora_sgmv_status decode_tc_maps_and_launch(sgmv::FusedParams& P, lora_sgmv_dtype
                                 : launch_decode_tc<__half, R>(P, maps, max_len, s, v_in);
 }
 
+// v_in: V from an earlier kernel (the split form)
 lora_sgmv_status decode_tc_dispatch(sgmv::FusedParams& P, int r, lora_sgmv_dtype dt, int max_len, cudaStream_t s,
                                     const float* v_in = nullptr) {
     switch (r) {
@@ -749,6 +654,12 @@ lora_sgmv_status launch_pad(void* dst, const void* src, int64_t rows_dst, int64_
     cfg.numAttrs = 0;
     return counted(cudaLaunchKernelEx(&cfg, sgmv::sgmv_pad_kernel, static_cast<uint16_t*>(dst),
                                       static_cast<const uint16_t*>(src), rows_dst, cols_dst, rows_src, cols_src));
+}
+
+// Bytes of the fp32 V [T, r] a workspace holds (padded to 256 bytes).
+size_t v_bytes_for(int32_t T, int32_t r) {
+    const size_t v = static_cast<size_t>(T) * static_cast<size_t>(r) * sizeof(float);
+    return (v + 255) / 256 * 256;
 }
 
 lora_sgmv_status check_common(int32_t n_segments, int32_t num_adapters, int32_t T, lora_sgmv_dtype dtype) {
@@ -830,8 +741,7 @@ lora_sgmv_status lora_sgmv_group_segments(const int32_t* ids, int32_t T, int32_t
 
 size_t lora_sgmv_workspace_bytes(int32_t T, int32_t r) {
     if (T <= 0 || r <= 0) return 0;
-    const size_t v = static_cast<size_t>(T) * static_cast<size_t>(r) * sizeof(float);
-    return (v + 255) / 256 * 256;
+    return v_bytes_for(T, r);
 }
 
 lora_sgmv_status lora_sgmv_pad_rank(void* A_dst, const void* A_src, void* B_dst, const void* B_src, int32_t H1,
@@ -929,8 +839,7 @@ lora_sgmv_status lora_sgmv_apply_flags(void* Y, const void* X, const void* const
     if (!Y || !X || !A_ptrs || !B_ptrs || !seg_starts || !lora_idx) return LORA_SGMV_ERR_NULL;
     if (num_adapters < 1) return LORA_SGMV_ERR_DIM;
     if (!aligned16(Y) || !aligned16(X) || H1 % 8 || H2 % 8) return LORA_SGMV_ERR_ALIGN;
-    const size_t need = lora_sgmv_workspace_bytes(T, r);
-    if (!workspace || workspace_bytes < need) return LORA_SGMV_ERR_WORKSPACE;
+    if (!workspace || workspace_bytes < lora_sgmv_workspace_bytes(T, r)) return LORA_SGMV_ERR_WORKSPACE;
     if (!aligned16(workspace)) return LORA_SGMV_ERR_ALIGN;
     const int max_len = estimate_max_len(max_seg_len, T, n_segments);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -964,7 +873,8 @@ lora_sgmv_status lora_sgmv_apply_flags(void* Y, const void* X, const void* const
         if (v == LORA_SGMV_VARIANT_FUSED_TC) return decode_tc_dispatch(P, r, dtype, max_len, s);
         if (v == LORA_SGMV_VARIANT_SPLIT_TC) {
             // V first (split-K shrink kernel, fp32 into the workspace), then the expand spread
-            // over every SM, each job's N split among independent CTAs
+            // over every SM, each job's N split among independent CTAs (its B_i stages stream
+            // while the shrink finishes)
             float* V = static_cast<float*>(workspace);
             ShrinkParams sp = {};
             sp.V = V;
@@ -1213,6 +1123,7 @@ extern "C" lora_sgmv_status lora_sgmv_gemm_apply(void* Y, const void* X, const v
     P.scale = scale;
     P.m_tiles = (T + sgmv::kLM - 1) / sgmv::kLM;
     P.n_tiles = (H2 + sgmv::kLN - 1) / sgmv::kLN;
+    P.v_after_wait = n_segments > 0 ? 1 : 0;  // V from the shrink just launched
     const long long units = static_cast<long long>(P.m_tiles) * P.n_tiles;
     if (units > (1ll << 31) - 1) return LORA_SGMV_ERR_DIM;
     const int grid = static_cast<int>(std::max<long long>(1, std::min<long long>(units, f.sms)));

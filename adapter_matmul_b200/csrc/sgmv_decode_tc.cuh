@@ -221,7 +221,10 @@ __global__ void __launch_bounds__(kDThreads, 1)
     // where allowed: asked for by the caller, or in pre-V mode, whose previous kernel is this
     // library's shrink, which writes none of them.
     const bool early = pre_v || P.early;
-    if (!early) pdl_wait();
+    if (!early) {
+        prefetch_metadata(P);  // L2 only: no value is read before the wait
+        pdl_wait();
+    }
     int entries;
     if (P.one_chunk) {
         __syncthreads();

@@ -260,6 +260,28 @@ __device__ __forceinline__ uint32_t cluster_size() {
 
 // ---- job list --------------------------------------------------------------------------
 
+// Warm L2 with the small arrays the first jobs read (segment bounds, adapter ids, pointer
+// tables) while the previous kernel on the stream may still run. A prefetch reads no value into
+// the kernel (L2 stays coherent with later writes), so it is safe under the default contract;
+// the CTAs of the grid split the table lines between them.
+__device__ __forceinline__ void prefetch_metadata(const FusedParams& P) {
+    const int tid = threadIdx.x, nth = blockDim.x;
+    const int n = P.n_segments;
+    const int lines_seg = (n + 1 + 31) / 32;  // 128-byte lines of seg_starts (and of lora_idx)
+    for (int l = tid; l < 2 * lines_seg; l += nth) {
+        const int32_t* base = l < lines_seg ? P.seg_starts : P.lora_idx;
+        const int off = (l < lines_seg ? l : l - lines_seg) * 32;
+        if (off < n + 1) asm volatile("prefetch.global.L2 [%0];" ::"l"(base + off));
+    }
+    for (int p = 0; p < P.n_problems; ++p) {
+        const int lines_tab = (P.prob[p].num_adapters + 15) / 16;  // 16 pointers per line
+        for (int l = blockIdx.x + gridDim.x * tid; l < 2 * lines_tab; l += gridDim.x * nth) {
+            const void* const* tab = l < lines_tab ? P.prob[p].A_ptrs : P.prob[p].B_ptrs;
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(tab + (l < lines_tab ? l : l - lines_tab) * 16));
+        }
+    }
+}
+
 // Number of CH-token chunks of segment s, or 0 if the segment is empty or invalid.
 template <int CH = kFusedTokens>
 __device__ __forceinline__ int segment_chunks(const FusedParams& P, int s) {
@@ -648,8 +670,11 @@ __global__ void __launch_bounds__(kFusedThreads, SGMV_FUSED_MIN_BLOCKS) sgmv_fus
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     // nothing the caller passed is read before the previous kernel completes, unless the
-    // caller allows the early reads
-    if (!P.early) pdl_wait();
+    // caller allows the early reads (the metadata is only prefetched into L2 before)
+    if (!P.early) {
+        prefetch_metadata(P);
+        pdl_wait();
+    }
     int entries;
     if (P.one_chunk) {
         __syncthreads();

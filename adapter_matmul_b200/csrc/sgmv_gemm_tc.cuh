@@ -22,10 +22,17 @@
 // per SM, tiles taken round-robin in row-major order so that the CTAs in flight share W and a
 // few X panels in L2). One ring of four 48 KB stages: a base stage holds an X tile [128 x 64]
 // (K-major, 128-byte swizzle) and a W tile [64 x 256] (four MN-major 64-column boxes); a delta
-// stage holds a V'_hi or V'_lo operand [128 x r] in the X slot (written by the epilogue warps)
-// and the B_i tile [r x 256] in the W slot (TMA through a tensor map made on the device, as B_i
-// is reached through a pointer table). The fp32 accumulator lives in TMEM, two buffers of 256
-// columns, so the epilogue of one tile overlaps the main loop of the next.
+// stage holds the B_i tile [r x 256] in the W slot (TMA through a tensor map made on the device,
+// as B_i is reached through a pointer table). The V'_hi and V'_lo operands [128 x r] of a pass
+// have a buffer of their own, written by the epilogue warps as soon as the previous pass's MMAs
+// have read it -- for a tile in one segment, during the main loop of the tile, well before its
+// delta stage. The fp32 accumulator lives in TMEM, two buffers of 256 columns, so the epilogue of
+// one tile overlaps the main loop of the next.
+//
+// The kernel that makes V runs just before this one on the stream; this kernel is launched with
+// programmatic dependent launch after it, so its CTAs start on the SMs that kernel leaves free
+// and stream X and W (which that kernel does not write) while it finishes; only the epilogue
+// warps wait (griddepcontrol.wait) before they read V.
 //
 // Warps: 0 producer (TMA), 1 TMEM owner and MMA issuer (one thread), 2..9 epilogue (two per
 // TMEM lane quarter, one per 128-column half of the tile), which also build the V' operands.
@@ -46,7 +53,8 @@ constexpr int kLTmemCols = 512;  // two accumulators of 256 columns
 constexpr int kLXBytes = kLM * kLK * 2;         // 16 KB
 constexpr int kLWBytes = kLK * kLN * 2;         // 32 KB (four 8 KB boxes)
 constexpr int kLStage = kLXBytes + kLWBytes;    // 48 KB
-constexpr size_t kLSmem = size_t(kLStages) * kLStage + 1024;  // + alignment slack
+constexpr int kLVBytes = kLM * 64 * 2;          // one V' operand [128 x r <= 64], 128-byte rows
+constexpr size_t kLSmem = size_t(kLStages) * kLStage + 2 * kLVBytes + 1024;  // + alignment slack
 
 inline bool gemm_tc_supported(int r, int H1, int H2) {
     return (r == 16 || r == 32 || r == 64) && H1 >= 8 && H2 >= 8 && H1 % 8 == 0 && H2 % 8 == 0;
@@ -68,6 +76,7 @@ struct GemmParams {
     float scale;
     int m_tiles;
     int n_tiles;
+    int v_after_wait;  // 1: V comes from the kernel just before (read only after griddepcontrol.wait)
 };
 
 // Next valid segment at or after s that intersects rows [m0, m1); n_segments if none. The
@@ -87,8 +96,10 @@ __global__ void __launch_bounds__(kLThreads, 1)
     extern __shared__ __align__(1024) unsigned char lsm_raw[];
     unsigned char* ring =
         reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(lsm_raw) + 1023) & ~uintptr_t(1023));
-    __shared__ __align__(8) uint64_t full[kLStages], empty[kLStages], vslot[kLStages], vdone[kLStages];
+    __shared__ __align__(8) uint64_t full[kLStages], empty[kLStages], vfull, vempty;
     __shared__ __align__(8) uint64_t acc_full[2], acc_empty[2];
+    unsigned char* vhi = ring + kLStages * kLStage;  // V' operands of the current delta pass
+    unsigned char* vlo = vhi + kLVBytes;
     __shared__ __align__(128) CUtensorMap map_build;
     __shared__ uint32_t tmem_base_s;
     __shared__ int table_s;
@@ -101,9 +112,9 @@ __global__ void __launch_bounds__(kLThreads, 1)
         for (int i = 0; i < kLStages; ++i) {
             mbar_init(&full[i], 1);    // producer's expect_tx; the copies complete the bytes
             mbar_init(&empty[i], 1);   // MMA commit
-            mbar_init(&vslot[i], 1);           // the stage's slot is free for a V' operand (producer)
-            mbar_init(&vdone[i], kLEpiWarps);  // V' operand written into the stage
         }
+        mbar_init(&vfull, kLEpiWarps);  // V' operands of the next pass written
+        mbar_init(&vempty, 1);          // MMA commit: the pass's MMAs have read them
         for (int i = 0; i < 2; ++i) {
             mbar_init(&acc_full[i], 1);
             mbar_init(&acc_empty[i], kLEpiWarps);
@@ -137,7 +148,7 @@ __global__ void __launch_bounds__(kLThreads, 1)
     if (warp == 0) {
         // ---------------------------------- producer ----------------------------------
         MapTable* tab = g_map_tables + (table < 0 ? 0 : table);
-        uint32_t it = 0, vpar = 0;
+        uint32_t it = 0;
         int passes = 0;
         for (int u = first_unit; u < units; u += gridDim.x) {
             const int m0 = (u / P.n_tiles) * kLM, n0 = (u % P.n_tiles) * kLN;
@@ -157,8 +168,8 @@ __global__ void __launch_bounds__(kLThreads, 1)
             Segment seg;
             for (int s = next_pass(P, 0, m0, m0 + kLM, seg); s < P.n_segments;
                  s = next_pass(P, s + 1, m0, m0 + kLM, seg)) {
-                // the B_i map of this pass goes to ring entry e; the stages that last used the
-                // entry are at least eight stages back, so their copies have landed
+                // the B_i map of this pass goes to ring entry e; the stage that last used the
+                // entry is at least eight stages back, so its copies have landed
                 CUtensorMap* gB = &tab->m[passes % (2 * kMapRing)];
                 ++passes;
                 map_template_to_smem(&map_build, &tmB);
@@ -167,15 +178,9 @@ __global__ void __launch_bounds__(kLThreads, 1)
                 map_publish(gB, &map_build);
                 if (lane == 0) map_acquire(gB);
                 __syncwarp();
-                for (int h = 0; h < 2; ++h, ++it) {  // V'_hi stage, then V'_lo stage
+                {  // the delta stage: B_i's tile in the W slot
                     const uint32_t st = it % kLStages;
                     if (it >= kLStages) mbar_wait<false>(&empty[st], ((it / kLStages) - 1) & 1u, P.dev_status, dead);
-                    // hand the free slot to the epilogue warps, which write the V' operand into it (they
-                    // wait on vslot, not on empty: a waiter may be at most one phase ahead of a barrier,
-                    // and the epilogue warps would be many phases of `empty` ahead)
-                    if (lane == 0) mbar_arrive_local(&vslot[st]);
-                    mbar_wait<false>(&vdone[st], (vpar >> st) & 1u, P.dev_status, dead);
-                    vpar ^= 1u << st;
                     unsigned char* bs = ring + st * kLStage + kLXBytes;
                     if (lane == 0) {
                         mbar_arrive_expect_tx(&full[st], 4 * R * 128);
@@ -183,6 +188,7 @@ __global__ void __launch_bounds__(kLThreads, 1)
                         for (int j = 0; j < 4; ++j) tma_load_2d(bs + j * (R * 128), gB, n0 + j * 64, 0, &full[st]);
                     }
                     __syncwarp();
+                    ++it;
                 }
             }
         }
@@ -194,7 +200,7 @@ __global__ void __launch_bounds__(kLThreads, 1)
         // ---------------------------------- MMA issuer ----------------------------------
         const uint32_t fmt = std::is_same<T, __nv_bfloat16>::value ? 1u : 0u;
         const uint32_t idesc = instr_desc(fmt, 0, 1, kLN, kLM);  // A K-major, B MN-major, N = 256
-        uint32_t it = 0;
+        uint32_t it = 0, pk = 0;
         int local = 0;
         for (int u = first_unit; u < units; u += gridDim.x, ++local) {
             const int m0 = (u / P.n_tiles) * kLM;
@@ -222,22 +228,25 @@ __global__ void __launch_bounds__(kLThreads, 1)
             Segment seg;
             for (int s = next_pass(P, 0, m0, m0 + kLM, seg); s < P.n_segments;
                  s = next_pass(P, s + 1, m0, m0 + kLM, seg)) {
-                for (int h = 0; h < 2; ++h, ++it) {
+                {
                     const uint32_t st = it % kLStages;
                     mbar_wait<false>(&full[st], (it / kLStages) & 1u, P.dev_status, dead);
+                    mbar_wait<false>(&vfull, pk & 1u, P.dev_status, dead);
                     tc_fence_after();
                     if (lane == 0) {
-                        const uint32_t va = smem_u32(ring + st * kLStage);
-                        const uint32_t ba = va + kLXBytes;
+                        const uint32_t ba = smem_u32(ring + st * kLStage + kLXBytes);
 #pragma unroll
                         for (int kk = 0; kk < R / 16; ++kk) {
-                            const uint64_t adesc = smem_desc(va + kk * 32, 16, 1024, 2);
                             const uint64_t bdesc = smem_desc(ba + kk * 16 * 128, R * 128, 1024, 2);
-                            tc_mma(acc, adesc, bdesc, idesc, 1u);
+                            tc_mma(acc, smem_desc(smem_u32(vhi) + kk * 32, 16, 1024, 2), bdesc, idesc, 1u);
+                            tc_mma(acc, smem_desc(smem_u32(vlo) + kk * 32, 16, 1024, 2), bdesc, idesc, 1u);
                         }
                         tc_commit(&empty[st]);
+                        tc_commit(&vempty);
                     }
                     __syncwarp();
+                    ++it;
+                    ++pk;
                 }
             }
             if (lane == 0) tc_commit(&acc_full[buf]);
@@ -252,18 +261,23 @@ __global__ void __launch_bounds__(kLThreads, 1)
         const int vrow = et >> 1;            // V' operand: row vrow, columns [vcol0, vcol0 + R/2)
         const int vcol0 = (et & 1) * (R / 2);
         T* __restrict__ Y = static_cast<T*>(P.Y);
-        uint32_t it = 0, vpar = 0;
+        uint32_t pk = 0;
+        bool waited = !P.v_after_wait;
         int local = 0;
         for (int u = first_unit; u < units; u += gridDim.x, ++local) {
             const int m0 = (u / P.n_tiles) * kLM, n0 = (u % P.n_tiles) * kLN;
             const int buf = local & 1;
-            it += k_steps;
-            // the V' operands of this tile's delta passes, written into the stages' X slots
+            // the V' operands of this tile's delta passes, each written once the previous pass's
+            // MMAs have read the buffer
             Segment seg;
             for (int s = next_pass(P, 0, m0, m0 + kLM, seg); s < P.n_segments;
-                 s = next_pass(P, s + 1, m0, m0 + kLM, seg)) {
+                 s = next_pass(P, s + 1, m0, m0 + kLM, seg), ++pk) {
                 const int g = m0 + vrow;
                 const bool in = g >= seg.begin && g < seg.end;
+                if (!waited) {  // V is written by the kernel just before this one
+                    pdl_wait();
+                    waited = true;
+                }
                 float v[R / 2];
 #pragma unroll
                 for (int j = 0; j < R / 2; j += 4) {
@@ -274,26 +288,23 @@ __global__ void __launch_bounds__(kLThreads, 1)
                     v[j + 2] = __fmul_rn(P.scale, q.z);
                     v[j + 3] = __fmul_rn(P.scale, q.w);
                 }
-                for (int h = 0; h < 2; ++h, ++it) {
-                    const uint32_t st = it % kLStages;
-                    mbar_wait<false>(&vslot[st], (vpar >> st) & 1u, P.dev_status, dead);
-                    unsigned char* vs = ring + st * kLStage;
+                if (pk >= 1) mbar_wait<false>(&vempty, (pk - 1) & 1u, P.dev_status, dead);
 #pragma unroll
-                    for (int c8 = 0; c8 < R / 16; ++c8) {
-                        float o[8];
+                for (int c8 = 0; c8 < R / 16; ++c8) {
+                    float hi[8], lo[8];
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            const float x = v[c8 * 8 + i];
-                            const float hi = Storage<T>::round(x);
-                            o[i] = h == 0 ? hi : x - hi;
-                        }
-                        st_vec(vs + swz(vrow, (vcol0 / 8) + c8, 3), pack8<T>(o));
+                    for (int i = 0; i < 8; ++i) {
+                        const float x = v[c8 * 8 + i];
+                        hi[i] = Storage<T>::round(x);
+                        lo[i] = x - hi[i];
                     }
-                    fence_proxy_async();  // generic-proxy writes -> tensor-core reads
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive_local(&vdone[st]);
-                    vpar ^= 1u << st;
+                    const uint32_t off = swz(vrow, (vcol0 / 8) + c8, 3);
+                    st_vec(vhi + off, pack8<T>(hi));
+                    st_vec(vlo + off, pack8<T>(lo));
                 }
+                fence_proxy_async();  // generic-proxy writes -> tensor-core reads
+                __syncwarp();
+                if (lane == 0) mbar_arrive_local(&vfull);
             }
             // epilogue: row m of the tile, this warp's 128 columns
             mbar_wait<false>(&acc_full[buf], (local >> 1) & 1u, P.dev_status, dead);
@@ -323,6 +334,7 @@ __global__ void __launch_bounds__(kLThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive_relaxed(&acc_empty[buf]);
         }
+        if (!waited) pdl_wait();  // keep this grid behind its predecessor even without delta passes
     }
     tc_fence_before();
     __syncthreads();
@@ -342,8 +354,17 @@ inline cudaError_t launch_gemm_delta_kernel(const CUtensorMap& tmX, const CUtens
                                         static_cast<int>(kLSmem));
     });
     if (attr_err != cudaSuccess) return attr_err;
-    sgmv_gemm_delta_kernel<T, R><<<grid, kLThreads, kLSmem, stream>>>(tmX, tmW, tmB, P);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid, 1, 1);
+    cfg.blockDim = dim3(kLThreads, 1, 1);
+    cfg.dynamicSmemBytes = kLSmem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = P.v_after_wait ? 1 : 0;  // overlap only the kernel that makes V
+    return cudaLaunchKernelEx(&cfg, sgmv_gemm_delta_kernel<T, R>, tmX, tmW, tmB, P);
 }
 
 }  // namespace sgmv

@@ -264,6 +264,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int tile = blockIdx.x / P.nsplit;
+    if (V_OUT) pdl_launch_dependents();  // the whole-layer kernel may start on free SMs
     const int nsl = blockIdx.x - tile * P.nsplit;
 
     if (warp == 0) {
