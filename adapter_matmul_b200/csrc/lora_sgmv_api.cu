@@ -15,7 +15,7 @@
 #include "../../include/lora_sgmv.h"
 #include "sgmv_decode_tc.cuh"
 #include "sgmv_fused.cuh"
-#include "sgmv_gemm_tc.cuh"
+#include "sgmv_gemm_tc2.cuh"
 #include "sgmv_grouped_tc.cuh"
 #include "sgmv_pad.cuh"
 #include "sgmv_split.cuh"
@@ -49,7 +49,10 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 bool split_rank(int r) { return r == 8 || r == 16 || r == 32 || r == 64 || r == 128; }
 
 // Lazily filled per-device facts, guarded by a mutex.
+constexpr int kMaxDevices = 64;
+
 struct DeviceFacts {
+    int dev = 0;
     int sms = 0;
     int max_smem_optin = 0;
 };
@@ -62,6 +65,7 @@ lora_sgmv_status device_facts(DeviceFacts& out) {
     std::lock_guard<std::mutex> lock(g_mu);
     if (dev >= static_cast<int>(g_devices.size())) g_devices.resize(dev + 1);
     DeviceFacts& f = g_devices[dev];
+    f.dev = dev;
     if (f.sms == 0) {
         if (cudaDeviceGetAttribute(&f.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
             cudaDeviceGetAttribute(&f.max_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
@@ -1037,11 +1041,63 @@ extern "C" lora_sgmv_status lora_sgmv_apply_ranks(void* Y, const void* X, const 
 
 namespace {
 
+// Rows from which the layer runs on SM pairs (256 x 256 tiles) rather than single SMs (128 x 256).
+#ifndef SGMV_GEMM_PAIR_MIN_T
+#define SGMV_GEMM_PAIR_MIN_T 256
+#endif
+
 template <int R>
 lora_sgmv_status launch_gemm_r(const CUtensorMap& tmX, const CUtensorMap& tmW, const CUtensorMap& tmB,
                                const sgmv::GemmParams& P, lora_sgmv_dtype dt, int grid, cudaStream_t s) {
     return counted(dt == LORA_SGMV_BF16 ? sgmv::launch_gemm_delta_kernel<__nv_bfloat16, R>(tmX, tmW, tmB, P, grid, s)
                                         : sgmv::launch_gemm_delta_kernel<__half, R>(tmX, tmW, tmB, P, grid, s));
+}
+
+// Pairs of SMs that can be resident at once for the pair kernel (cached per device).
+template <typename T, int R>
+lora_sgmv_status gemm_pairs_resident(int dev, int* out) {
+    static int cached[kMaxDevices] = {};
+    if (dev < 0 || dev >= kMaxDevices) return LORA_SGMV_ERR_UNSUPPORTED;
+    {
+        std::lock_guard<std::mutex> lock(g_mu);
+        if (cached[dev] > 0) {
+            *out = cached[dev];
+            return LORA_SGMV_OK;
+        }
+    }
+    static std::once_flag once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(once, [] {
+        attr_err = cudaFuncSetAttribute(sgmv::sgmv_gemm_delta_pair_kernel<T, R>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(sgmv::kL2Smem));
+    });
+    if (record(attr_err) != cudaSuccess) return LORA_SGMV_ERR_CUDA;
+    int n = 0;
+    lora_sgmv_status st = max_active_clusters(sgmv::sgmv_gemm_delta_pair_kernel<T, R>, 2, sgmv::kL2Smem, &n,
+                                              sgmv::kLThreads);
+    if (st != LORA_SGMV_OK) return st;
+    std::lock_guard<std::mutex> lock(g_mu);
+    cached[dev] = n;
+    *out = n;
+    return LORA_SGMV_OK;
+}
+
+template <typename T, int R>
+lora_sgmv_status launch_gemm_pair_t(const CUtensorMap& tmX, const CUtensorMap& tmW, const CUtensorMap& tmB,
+                                    const sgmv::GemmParams& P, int dev, cudaStream_t s) {
+    int resident = 0;
+    lora_sgmv_status st = gemm_pairs_resident<T, R>(dev, &resident);
+    if (st != LORA_SGMV_OK) return st;
+    const long long units = static_cast<long long>(P.m_tiles) * P.n_tiles;
+    const int pairs = static_cast<int>(std::max<long long>(1, std::min<long long>(units, resident)));
+    return counted(sgmv::launch_gemm_delta_pair_kernel<T, R>(tmX, tmW, tmB, P, pairs, s));
+}
+
+template <int R>
+lora_sgmv_status launch_gemm_pair_r(const CUtensorMap& tmX, const CUtensorMap& tmW, const CUtensorMap& tmB,
+                                    const sgmv::GemmParams& P, lora_sgmv_dtype dt, int dev, cudaStream_t s) {
+    return dt == LORA_SGMV_BF16 ? launch_gemm_pair_t<__nv_bfloat16, R>(tmX, tmW, tmB, P, dev, s)
+                                : launch_gemm_pair_t<__half, R>(tmX, tmW, tmB, P, dev, s);
 }
 
 }  // namespace
@@ -1121,9 +1177,20 @@ extern "C" lora_sgmv_status lora_sgmv_gemm_apply(void* Y, const void* X, const v
     P.H1 = H1;
     P.H2 = H2;
     P.scale = scale;
+    P.v_after_wait = n_segments > 0 ? 1 : 0;  // V from the shrink just launched
+    if (T >= SGMV_GEMM_PAIR_MIN_T) {
+        P.m_tiles = (T + sgmv::kL2M - 1) / sgmv::kL2M;
+        P.n_tiles = (H2 + sgmv::kL2N - 1) / sgmv::kL2N;
+        if (static_cast<long long>(P.m_tiles) * P.n_tiles > (1ll << 31) - 1) return LORA_SGMV_ERR_DIM;
+        switch (r) {
+            case 16: return launch_gemm_pair_r<16>(tmX, tmW, tmB, P, dtype, f.dev, s);
+            case 32: return launch_gemm_pair_r<32>(tmX, tmW, tmB, P, dtype, f.dev, s);
+            case 64: return launch_gemm_pair_r<64>(tmX, tmW, tmB, P, dtype, f.dev, s);
+        }
+        return LORA_SGMV_ERR_UNSUPPORTED;
+    }
     P.m_tiles = (T + sgmv::kLM - 1) / sgmv::kLM;
     P.n_tiles = (H2 + sgmv::kLN - 1) / sgmv::kLN;
-    P.v_after_wait = n_segments > 0 ? 1 : 0;  // V from the shrink just launched
     const long long units = static_cast<long long>(P.m_tiles) * P.n_tiles;
     if (units > (1ll << 31) - 1) return LORA_SGMV_ERR_DIM;
     const int grid = static_cast<int>(std::max<long long>(1, std::min<long long>(units, f.sms)));
