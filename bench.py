@@ -66,7 +66,23 @@ PER_CONFIG_MAX_STEPS = 500
 # same launch (summaries under profiles/). A figure holds only while the kernel's sources are
 # those it was taken from: their SHA-256 is stored with it and checked here, else "traffic"
 # is null. For a call of two launches (the split forms) the figure is the pair's.
-TRAFFIC = {}
+TRAFFIC = {
+    # profiles/fused_kernel_distinct_decode.md
+    "distinct": {"bytes": 35724544, "sources": ["sgmv_fused.cuh", "sgmv_common.cuh"],
+        "sha256": "4da228808e6c7cdb3a144776e48bbe2e01fc0fad7bd074f571a15c5d55da95e8"},
+    # profiles/split_tc_llama70b_decode_h28672.md
+    "llama70b_decode_h28672": {"bytes": 489211648,
+        "sources": ["sgmv_split.cuh", "sgmv_decode_tc.cuh", "sgmv_tmap.cuh", "sgmv_common.cuh"],
+        "sha256": "94643e8ccf1b2c58e2973670a7d4d1b87452ab65a2e06e6cc508dd9d2dfe354d"},
+    # profiles/decode_tc_kernel_llama70b_decode_h8192.md
+    "llama70b_decode_h8192": {"bytes": 211907328,
+        "sources": ["sgmv_decode_tc.cuh", "sgmv_tmap.cuh", "sgmv_common.cuh"],
+        "sha256": "3671ea9eccd0479c921c3020ee059879a38f1fa771078784b0a3d687574eea47"},
+    # profiles/grouped_kernel_prefill.md
+    "prefill": {"bytes": 190034176,
+        "sources": ["sgmv_grouped_tc.cuh", "sgmv_tmap.cuh", "sgmv_common.cuh"],
+        "sha256": "2193ad68fae5fefb2b7868384a1ed95506a46235078f0bb38709c7f2f1e56fb7"},
+}
 
 
 def kernel_sources_sha(files) -> str:
@@ -571,7 +587,8 @@ def summarize(spec: Spec, ds: DeviceSpec, ms: float, ms_early: float, lps: int, 
             "tflops": round(w.flops() * spec.P / s / 1e12, 3),
             "tensor_frac": round(w.flops() * spec.P / s / 1e12 / tc, 4),
             "early_reads": {"us_per_step": round(se * 1e6, 3),
-                            "frac": round(bytes_step / se / 1e9 / hbm, 4)}}
+                            "frac": round(bytes_step / se / 1e9 / hbm, 4)},
+            "traffic_per_step": measured_traffic(spec.name)}
 
 
 def measure_layer(args, steps: int, stream, world: int, dev, rank: int) -> dict:
