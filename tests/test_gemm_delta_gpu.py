@@ -2,10 +2,12 @@
 the oracle's base_plus_delta_f32 (README page "Punica：多 LoRA 模型统一服务框架", LoRA and
 multi-LoRA paragraphs), element by element.
 
-Small cases cover ragged tiles (T, H1 and H2 not multiples of the 128 x 256 tile or of the
-64-wide K step), tiles that span several segments, empty and rejected segments, rows in no
-segment, both storage types, every rank the kernel takes, and both shrink kernels that make V
-(segments shorter and longer than 128 rows). The prefill-sized layer (T = 9771, H1 = H2 =
+Small cases cover both forms of the layer kernel (single SMs with 128 x 256 tiles below 256
+rows, SM pairs with 256 x 256 tiles from 256 rows, on either side of that boundary), ragged
+tiles (T, H1 and H2 not multiples of the tile or of the 64-wide K step, down to a pair whose
+second SM holds no column of H2), tiles that span several segments, empty and rejected
+segments, rows in no segment, both storage types, every rank the kernel takes, and both
+shrink kernels that make V (segments shorter and longer than 128 rows). The prefill-sized layer (T = 9771, H1 = H2 =
 4096, r = 64, bf16) is checked on whole rows: the first and last row of every segment and a
 random sample, every column. Tolerance: |gpu - oracle| <= 2e-2 + 1e-2 |oracle|.
 """
@@ -103,6 +105,26 @@ def test_layer_long_segments_grouped_shrink(r):
     assert int(L.status.item()) == 0
     ref, _ = oracle.base_plus_delta_f32(L.x_bits, L.w_bits, L.A, L.B, seg, idx, -1.25, "bf16")
     assert_close(got, ref, "bf16", f"layer long segments r={r}")
+
+
+@pytest.mark.parametrize("T", [255, 256, 257, 700])
+@pytest.mark.parametrize("r", [16, 64])
+def test_layer_short_segments_around_the_pair_boundary(T, r):
+    # segments of 0..57 rows over the whole batch (split-K shrink), adapters reused out of
+    # order; H2 = 264 leaves the second SM of the last column pair without a valid column
+    rng = np.random.default_rng(T * 7 + r)
+    lens, left = [], T - 3
+    while left > 0:
+        lens.append(int(min(left, rng.integers(0, 58))))
+        left -= lens[-1]
+    seg = np.concatenate([[3], 3 + np.cumsum(lens)]).astype(np.int32)
+    idx = rng.integers(0, 5, len(lens)).astype(np.int32)
+    w = inputs.small_random(T, 5, 136, 264, r, "f16", seed=T + r)
+    L = Layer(w, seg, idx)
+    got = L.run(0.5)
+    assert int(L.status.item()) == 0
+    ref, _ = oracle.base_plus_delta_f32(L.x_bits, L.w_bits, L.A, L.B, seg, idx, 0.5, "f16")
+    assert_close(got, ref, "f16", f"layer T={T} r={r}")
 
 
 def test_layer_without_segments_is_the_base_product():
