@@ -475,9 +475,13 @@ __global__ void __launch_bounds__(kDThreads, 1)
             const int cw = pre_v ? w - j * n_sl : c;  // N slice (and K slice)
             int p, s, q0, nq;
             entry_at<kDTokens>(P, pref, j, p, s, q0, nq);
+            // rejected segments are reported as the jobs meet them: one thread of the first CTA
+            // of the visiting cluster (of the first N slice in pre-V mode)
+            const bool reporter = c == 0 && cw == 0 && warp == 9 && lane == 0;
+            if (nq == 0 && reporter) report(P.dev_status, segment_bounds_check(P, s));
             for (int q = q0; q < q0 + nq; ++q) {
                 Job job;
-                if (!job_at<kDTokens>(P, p, s, q, cw, job)) break;
+                if (!job_at_reporting<kDTokens>(P, p, s, q, cw, job, reporter)) break;
                 const FusedProblem& pr = P.prob[job.p];
                 const int nA = (job.nk + G::KS - 1) / G::KS;
                 const int nB = (job.nc + G::NW - 1) / G::NW;
@@ -615,14 +619,6 @@ __global__ void __launch_bounds__(kDThreads, 1)
         if (quarter == 0 && half == 0) {
             pdl_wait();
             if (!pre_v && u >= 1) mbar_wait<true>(&vfree, (u - 1) & 1u, P.dev_status, dead);
-            if (c == 0 && lane == 0) {  // report each rejected segment once
-                for (int j = cluster_id; j < P.n_problems * P.n_segments; j += n_clusters) {
-                    const int p2 = j / P.n_segments, s2 = j - p2 * P.n_segments;
-                    Segment seg;
-                    report(P.dev_status, load_segment(P.seg_starts, P.lora_idx, P.prob[p2].A_ptrs, P.prob[p2].B_ptrs,
-                                                      s2, P.T, P.prob[p2].num_adapters, seg));
-                }
-            }
         }
     }
     tc_fence_before();

@@ -282,6 +282,12 @@ __device__ __forceinline__ void prefetch_metadata(const FusedParams& P) {
     }
 }
 
+// LORA_SGMV_DEV_BAD_SEGMENT if the bounds of segment s break the contract, else 0.
+__device__ __forceinline__ uint32_t segment_bounds_check(const FusedParams& P, int s) {
+    const int b = __ldg(P.seg_starts + s), e = __ldg(P.seg_starts + s + 1);
+    return (b < 0 || b > e || e > P.T) ? LORA_SGMV_DEV_BAD_SEGMENT : 0u;
+}
+
 // Number of CH-token chunks of segment s, or 0 if the segment is empty or invalid.
 template <int CH = kFusedTokens>
 __device__ __forceinline__ int segment_chunks(const FusedParams& P, int s) {
@@ -303,6 +309,8 @@ __device__ void build_job_prefix(const FusedParams& P, int* pref) {
     int local = 0;
     for (int s = s0; s < s1; ++s) {
         local += segment_chunks<CH>(P, s);
+        // a segment with invalid bounds has no chunk, so no job reports it: CTA 0 does, here
+        if (blockIdx.x == 0) report(P.dev_status, segment_bounds_check(P, s));
         // warm L1 for the lookups job_at() makes next: adapter id, then its table entries
         const int i = __ldg(P.lora_idx + s);
         for (int p = 0; p < P.n_problems; ++p) {
@@ -372,12 +380,14 @@ __device__ __forceinline__ void entry_at(const FusedParams& P, const int* pref, 
     nq = 1;
 }
 
-// Chunk q (of CH tokens) of segment s of problem p: false if the segment fails the device-side checks.
+// Chunk q (of CH tokens) of segment s of problem p: 0, or the LORA_SGMV_DEV_* bits of the
+// device-side checks the segment fails (then the job is not filled in).
 template <int CH = kFusedTokens>
-__device__ __forceinline__ bool job_at(const FusedParams& P, int p, int s, int q, int c, Job& job) {
+__device__ __forceinline__ uint32_t job_check(const FusedParams& P, int p, int s, int q, int c, Job& job) {
     const FusedProblem& pr = P.prob[p];
     Segment seg;
-    if (load_segment(P.seg_starts, P.lora_idx, pr.A_ptrs, pr.B_ptrs, s, P.T, pr.num_adapters, seg)) return false;
+    const uint32_t bad = load_segment(P.seg_starts, P.lora_idx, pr.A_ptrs, pr.B_ptrs, s, P.T, pr.num_adapters, seg);
+    if (bad) return bad;
     job.p = p;
     job.t0 = seg.begin + q * CH;
     job.nt = min(CH, seg.end - job.t0);
@@ -387,7 +397,23 @@ __device__ __forceinline__ bool job_at(const FusedParams& P, int p, int s, int q
     job.nk = max(0, min(pr.ks, pr.H1 - job.k0));
     job.c0 = c * pr.ns;
     job.nc = max(0, min(pr.ns, pr.H2 - job.c0));
-    return true;
+    return 0u;
+}
+
+template <int CH = kFusedTokens>
+__device__ __forceinline__ bool job_at(const FusedParams& P, int p, int s, int q, int c, Job& job) {
+    return job_check<CH>(P, p, s, q, c, job) == 0u;
+}
+
+// A rejected segment is reported by the one thread that meets it first as a job (`reporter`:
+// one thread of the first CTA of the visiting cluster); a one-chunk-mode entry without chunks
+// may be a segment with invalid bounds.
+template <int CH = kFusedTokens>
+__device__ __forceinline__ bool job_at_reporting(const FusedParams& P, int p, int s, int q, int c, Job& job,
+                                                 bool reporter) {
+    const uint32_t bad = job_check<CH>(P, p, s, q, c, job);
+    if (bad && reporter) report(P.dev_status, bad);
+    return bad == 0u;
 }
 
 // ---- consumer body ----------------------------------------------------------------------
@@ -710,13 +736,17 @@ __global__ void __launch_bounds__(kFusedThreads, SGMV_FUSED_MIN_BLOCKS) sgmv_fus
         // ------------------------------ consumers ------------------------------
         if (C > 1) cluster_wait();
         const int ct = threadIdx.x - 32;
+        // rejected segments are reported as the jobs meet them (no pass over the segments at
+        // the end, which the next kernel on the stream would wait for)
+        const bool reporter = c == 0 && ct == 0;
         uint32_t it = 0, u = 0;
         for (int j = cluster_id; j < entries; j += n_clusters) {
             int p, s, q0, nq;
             entry_at(P, pref, j, p, s, q0, nq);
+            if (nq == 0 && reporter) report(P.dev_status, segment_bounds_check(P, s));
             for (int q = q0; q < q0 + nq; ++q) {
                 Job job;
-                if (!job_at(P, p, s, q, c, job)) break;
+                if (!job_at_reporting(P, p, s, q, c, job, reporter)) break;
                 if (job.nt == 1)
                     consume_job<T, R, 1>(P, job, S, it, u, C, c, ct, dead);
                 else if (job.nt <= 2)
@@ -732,16 +762,6 @@ __global__ void __launch_bounds__(kFusedThreads, SGMV_FUSED_MIN_BLOCKS) sgmv_fus
         pdl_wait();
         // every receiver has consumed this CTA's last tile before its shared memory goes away
         if (u >= 1) mbar_wait<true>(vfree, (u - 1) & 1u, P.dev_status, dead);
-        // report each rejected segment once
-        if (ct == 0 && c == 0) {
-            for (int j = cluster_id; j < P.n_problems * P.n_segments; j += n_clusters) {
-                const int p = j / P.n_segments, s = j - p * P.n_segments;
-                Segment seg;
-                const uint32_t bad = load_segment(P.seg_starts, P.lora_idx, P.prob[p].A_ptrs, P.prob[p].B_ptrs, s,
-                                                  P.T, P.prob[p].num_adapters, seg);
-                if (bad) report(P.dev_status, bad);
-            }
-        }
     }
 }
 

@@ -122,13 +122,6 @@ __global__ void __launch_bounds__(kLThreads, 1)
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         table_s = claim_map_table();
         if (table_s < 0) report(P.dev_status, LORA_SGMV_DEV_TIMEOUT);
-        if (blockIdx.x == 0) {  // report every rejected segment once
-            for (int s = 0; s < P.n_segments; ++s) {
-                Segment seg;
-                report(P.dev_status,
-                       load_segment(P.seg_starts, P.lora_idx, P.A_ptrs, P.B_ptrs, s, P.T, P.num_adapters, seg));
-            }
-        }
     }
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tmem_base_s)),
@@ -261,6 +254,12 @@ __global__ void __launch_bounds__(kLThreads, 1)
         const int vrow = et >> 1;            // V' operand: row vrow, columns [vcol0, vcol0 + R/2)
         const int vcol0 = (et & 1) * (R / 2);
         T* __restrict__ Y = static_cast<T*>(P.Y);
+        if (blockIdx.x == 0 && warp == 9)  // report every rejected segment once, one lane per segment
+            for (int s = lane; s < P.n_segments; s += 32) {
+                Segment seg;
+                report(P.dev_status,
+                       load_segment(P.seg_starts, P.lora_idx, P.A_ptrs, P.B_ptrs, s, P.T, P.num_adapters, seg));
+            }
         uint32_t pk = 0;
         bool waited = !P.v_after_wait;
         int local = 0;

@@ -279,15 +279,18 @@ __global__ void __launch_bounds__(kGThreads, 1)
             job_s[2] = job_s[0] >= 0 ? segment_rank<R>(P, s) : 0;
             if (job_s[2] == 0) job_s[0] = -1;  // a rank the kernel cannot take: reported below
         }
-        if (blockIdx.x == 0) {  // report every rejected segment once
-            for (int s2 = lane; s2 < P.n_segments; s2 += 32) {
-                Segment seg;
-                const uint32_t bad =
-                    load_segment(P.seg_starts, P.lora_idx, P.A_ptrs, P.B_ptrs, s2, P.T, P.num_adapters, seg);
-                report(P.dev_status, bad ? bad : (segment_rank<R>(P, s2) ? 0u : LORA_SGMV_DEV_BAD_RANK));
-            }
-        }
     }
+    // every rejected segment reported once: by CTA 0's last epilogue warp, one lane per segment,
+    // where that warp waits anyway (before its first expand tile, or on leaving without a tile)
+    auto report_rejected = [&]() {
+        if (blockIdx.x != 0 || warp != 9) return;
+        for (int s2 = lane; s2 < P.n_segments; s2 += 32) {
+            Segment seg;
+            const uint32_t bad =
+                load_segment(P.seg_starts, P.lora_idx, P.A_ptrs, P.B_ptrs, s2, P.T, P.num_adapters, seg);
+            report(P.dev_status, bad ? bad : (segment_rank<R>(P, s2) ? 0u : LORA_SGMV_DEV_BAD_RANK));
+        }
+    };
     if (threadIdx.x == 0) {
         for (int i = 0; i < kGStages; ++i) {
             mbar_init(&full[i], 1);       // producer expect_tx; the TMA copies complete the bytes
@@ -312,7 +315,10 @@ __global__ void __launch_bounds__(kGThreads, 1)
     }
     __syncthreads();
     const int seg_id = job_s[0];
-    if (seg_id < 0) return;  // no tile here, or a rejected segment (reported once)
+    if (seg_id < 0) {  // no tile here, or a rejected segment
+        report_rejected();
+        return;
+    }
     const int mt = job_s[1];
 
     Segment seg;
@@ -457,6 +463,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
         }
     } else {
         // ---------------------------------- epilogue ----------------------------------
+        report_rejected();
         const int quarter = warp & 3;       // TMEM lanes [32*quarter, 32*quarter + 32)
         const int half = (warp - 2) >> 2;   // columns [64*half, 64*half + 64) of each N-tile
         const int m = quarter * 32 + lane;

@@ -179,10 +179,11 @@ __device__ __forceinline__ void shrink_chunk(const ShrinkParams& p, cg::cluster_
     cluster.sync();  // partial tiles and the X slice may be overwritten only after every read
 }
 
-// Token chunks of segment s (0 for a segment the checks reject).
-__device__ __forceinline__ int shrink_segment_chunks(const ShrinkParams& p, int s) {
+// Token chunks of segment s (0 for a segment the checks reject, whose reasons go to *bad).
+__device__ __forceinline__ int shrink_segment_chunks(const ShrinkParams& p, int s, uint32_t* bad) {
     Segment seg;
-    if (load_segment(p.seg_starts, p.lora_idx, p.A_ptrs, p.B_check, s, p.T, p.num_adapters, seg)) return 0;
+    *bad = load_segment(p.seg_starts, p.lora_idx, p.A_ptrs, p.B_check, s, p.T, p.num_adapters, seg);
+    if (*bad) return 0;
     return (seg.end - seg.begin + kShrinkTokens - 1) / kShrinkTokens;
 }
 
@@ -226,8 +227,13 @@ __global__ void __launch_bounds__(kShrinkThreads) sgmv_shrink_cluster_kernel(con
         const int per_thr = (n + NT - 1) / NT;
         const int s0 = min(n, tid * per_thr), s1 = min(n, s0 + per_thr);
         int local = 0;
-        for (int s = s0; s < s1; ++s) {  // chunk counts, parked in the prefix slots
-            const int k = shrink_segment_chunks(p, s);
+        // chunk counts, parked in the prefix slots; one CTA reports each rejected segment (while
+        // the list is built, not after the chunks, so that no CTA's end waits on it)
+        const bool reporter = blockIdx.y == 0 && c == 0;
+        for (int s = s0; s < s1; ++s) {
+            uint32_t bad;
+            const int k = shrink_segment_chunks(p, s, &bad);
+            if (reporter) report(p.dev_status, bad);
             pref[s + 1] = k;
             local += k;
         }
@@ -263,12 +269,6 @@ __global__ void __launch_bounds__(kShrinkThreads) sgmv_shrink_cluster_kernel(con
             const int t0 = seg.begin + (u - pref[lo]) * TC;
             run_chunk(static_cast<const T*>(seg.a), t0, min(TC, seg.end - t0));
         }
-        if (c == 0 && tid == 0)  // report each rejected segment once
-            for (int s = blockIdx.y; s < n; s += gridDim.y) {
-                Segment seg;
-                report(p.dev_status, load_segment(p.seg_starts, p.lora_idx, p.A_ptrs, p.B_check, s, p.T,
-                                                  p.num_adapters, seg));
-            }
         return;
     }
 

@@ -192,15 +192,17 @@ def test_empty_repeated_unsorted_segments_and_uncovered_rows():
 
 @pytest.mark.parametrize("variant", [sgmv.VARIANT_SPLIT, sgmv.VARIANT_FUSED, sgmv.VARIANT_FUSED_TC,
                                      sgmv.VARIANT_SPLIT_TC])
-def test_bad_segments_are_skipped_and_reported(variant):
-    # [4,2) reversed; adapter 9 out of range; adapter 2 has a null table entry; [20,30) past T
+@pytest.mark.parametrize("hint", [4, 40])
+def test_bad_segments_are_skipped_and_reported(variant, hint):
+    # [4,2) reversed; adapter 9 out of range; adapter 2 has a null table entry; [20,30) past T.
+    # The length hint 4 makes the fused kernels take one entry per segment, 40 the chunk list.
     seg = np.array([0, 4, 2, 8, 12, 16, 20, 30], np.int32)
     idx = np.array([0, 1, 9, 3, 2, 4, 1], np.int32)
     tc = variant in (sgmv.VARIANT_FUSED_TC, sgmv.VARIANT_SPLIT_TC)
     p = _custom(seg, idx, H2=256 if tc else 264)
     p.A_ptrs[2] = 0
     before = from_dev(p.Y)
-    got = p.apply(variant=variant)
+    got = p.apply(variant=variant, max_seg_len=hint)
     st = int(p.status.item())
     assert st & sgmv.DEV_BAD_SEGMENT and st & sgmv.DEV_BAD_ADAPTER and st & sgmv.DEV_BAD_POINTER
     # valid segments: [0,4) adapter 0, [8,12) adapter 3, [16,20) adapter 4
