@@ -136,21 +136,29 @@ template <typename T, int R>
 lora_sgmv_status launch_shrink(const ShrinkParams& p0, int max_len, cudaStream_t stream) {
     static int smem_granted[64] = {};
     ShrinkParams p = p0;
-    const int C = cluster_size_for(p.H1);
-    p.ks = ((p.H1 + C - 1) / C + 7) / 8 * 8;
-    p.flat = p.n_segments <= sgmv::kShrinkFlatMaxSegments ? 1 : 0;
-    const size_t smem = sgmv::shrink_smem_bytes(p.ks, R, p.flat ? p.n_segments : 0);
     DeviceFacts f;
     if (device_facts(f) != LORA_SGMV_OK) return LORA_SGMV_ERR_CUDA;
+    p.flat = p.n_segments <= sgmv::kShrinkFlatMaxSegments ? 1 : 0;
+    // at most one chunk per token, and at most one partial chunk per segment
+    const long long units = std::min<long long>(
+        static_cast<long long>(p.n_segments) + (p.T + sgmv::kShrinkTokens - 1) / sgmv::kShrinkTokens, p.T);
+    int C = cluster_size_for(p.H1);
+    // Fewer, longer CTAs when clusters of 8 would need more than two waves (the SM count's
+    // worth of CTA pairs, two CTAs per SM): each chunk's fixed steps (the chunk list, X, the
+    // cluster reduction) are then paid by half as many CTAs. Measured on the 70B-shaped decode
+    // (127 chunks, H1 = 8192): 8 CTAs per chunk 41.8 us, 4 CTAs 39.5 us, 2 CTAs 49.8 us.
+    if (p.flat && C == 8 && units * 8 > 4ll * f.sms) C = 4;
+#ifdef SGMV_SHRINK_CLUSTER
+    C = std::min(C, SGMV_SHRINK_CLUSTER);
+#endif
+    p.ks = ((p.H1 + C - 1) / C + 7) / 8 * 8;
+    const size_t smem = sgmv::shrink_smem_bytes(p.ks, R, p.flat ? p.n_segments : 0);
     if (smem > static_cast<size_t>(f.max_smem_optin)) return LORA_SGMV_ERR_DIM;
     auto kernel = sgmv::sgmv_shrink_cluster_kernel<T, R>;
     if (ensure_smem(kernel, smem, smem_granted) != LORA_SGMV_OK) return LORA_SGMV_ERR_CUDA;
 
     cudaLaunchConfig_t cfg = {};
     if (p.flat) {
-        // at most one chunk per token, and at most one partial chunk per segment
-        const long long units = std::min<long long>(
-            static_cast<long long>(p.n_segments) + (p.T + sgmv::kShrinkTokens - 1) / sgmv::kShrinkTokens, p.T);
         cfg.gridDim = dim3(C, static_cast<unsigned>(std::max<long long>(1, std::min<long long>(units, 65535))), 1);
     } else {
         cfg.gridDim = dim3(C, clamp_grid_y(p.n_segments), chunk_slots(max_len, sgmv::kShrinkTokens, 8));
@@ -420,11 +428,12 @@ bool decode_tc_preferred(int r, int max_len) { return max_len > 2 && r >= 32; }
 // The split form of the tensor-core decode (V by the split-K shrink kernel, then an expand that
 // spreads each job's N over independent CTAs) pays a second launch and a V round trip through
 // the workspace, and wins when the fused form would leave SMs idle: fewer jobs than SMs, each
-// with a large B_i (several MB) to stream.
+// with a large B_i to stream (measured on the 70B-shaped decode, 111 jobs: split 135 vs fused
+// 177 us at 3.7 MB per B_i, 80 vs 83 us at 1 MB).
 bool split_tc_preferred(int T, int n_segments, int max_len, int H2, int r, int sms) {
     const long long chunks = std::min<long long>(n_segments + (T + 15) / 16, std::max(T, 1));
     const long long jobs = max_len <= 16 ? n_segments : chunks;
-    return jobs < sms && double(H2) * r * 2 >= 2e6;
+    return jobs < sms && double(H2) * r * 2 >= 1e6;
 }
 
 bool decode_tc_supported(int r, int H1, int H2) {

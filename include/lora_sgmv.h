@@ -272,7 +272,7 @@ lora_sgmv_status lora_sgmv_apply(void* Y, const void* X, const void* const* A_pt
  * 8192 segments -> SPLIT; else segments of more than 2 tokens, r >= 32 and
  * H1, H2 multiples of 64 -> SPLIT_TC when there are fewer jobs (16-token
  * chunks, or segments when none is longer than 16) than SMs and each B_i
- * holds at least 2 MB, else FUSED_TC; else FUSED.
+ * holds at least 1,000,000 bytes (r * H2 * 2), else FUSED_TC; else FUSED.
  * Returns LORA_SGMV_VARIANT_AUTO when a size or sm_count is not positive or
  * dtype is unknown.
  */

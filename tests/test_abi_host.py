@@ -183,7 +183,7 @@ def test_batched_validation_codes():
     ("tiny", "FUSED"), ("distinct", "FUSED"), ("uniform_h4096", "FUSED"), ("uniform_h11008", "FUSED"),
     ("skewed_h4096", "FUSED"), ("skewed_h11008", "FUSED"), ("identical_h4096", "FUSED"),
     ("identical_h11008", "FUSED"), ("prefill", "GROUPED_TC"), ("llama70b_decode_h28672", "SPLIT_TC"),
-    ("llama70b_decode_h8192", "FUSED_TC")])
+    ("llama70b_decode_h8192", "SPLIT_TC")])
 def test_auto_variant_on_the_configurations(name, want):
     # the dispatcher's choice for each benchmark configuration on a 148-SM B200 (host only)
     w = inputs.make(name)
@@ -208,11 +208,12 @@ def test_auto_variant_rule_edges():
     assert auto(256, 95, 8192, 64, 28672, BF16, 2) == V.VARIANT_FUSED
     assert auto(256, 95, 8192, 16, 28672, BF16, 56) == V.VARIANT_FUSED
     assert auto(256, 95, 8192, 64, 28680, BF16, 56) == V.VARIANT_FUSED
-    # the split form: fewer jobs than SMs and B_i of 2 MB or more
+    # the split form: fewer jobs than SMs and B_i of 1,000,000 bytes or more
     assert auto(256, 95, 8192, 64, 28672, BF16, 56, 148) == V.VARIANT_SPLIT_TC
     assert auto(256, 95, 8192, 64, 28672, BF16, 56, 100) == V.VARIANT_FUSED_TC   # 111 jobs, 100 SMs
-    assert auto(256, 95, 8192, 64, 16384, BF16, 56, 148) == V.VARIANT_SPLIT_TC   # 2.1 MB
-    assert auto(256, 95, 8192, 64, 8192, BF16, 56, 148) == V.VARIANT_FUSED_TC    # 1 MB
+    assert auto(256, 95, 8192, 64, 8192, BF16, 56, 148) == V.VARIANT_SPLIT_TC    # 1,048,576 bytes
+    assert auto(256, 95, 8192, 64, 7808, BF16, 56, 148) == V.VARIANT_FUSED_TC    # 999,424 bytes
+    assert auto(256, 95, 8192, 32, 8192, BF16, 56, 148) == V.VARIANT_FUSED_TC    # 524,288 bytes
     # invalid sizes
     assert auto(0, 1, 64, 16, 64, F16, 1) == V.VARIANT_AUTO
     assert auto(8, 1, 64, 16, 64, 7, 1) == V.VARIANT_AUTO

@@ -23,7 +23,7 @@ pytestmark = pytest.mark.gpu
     ("llama70b_decode_h28672", sgmv.VARIANT_AUTO),
     ("llama70b_decode_h28672", sgmv.VARIANT_FUSED_TC),
     ("llama70b_decode_h8192", sgmv.VARIANT_AUTO),
-    ("llama70b_decode_h8192", sgmv.VARIANT_SPLIT_TC),
+    ("llama70b_decode_h8192", sgmv.VARIANT_FUSED_TC),
     ("llama70b_decode_h8192", sgmv.VARIANT_FUSED),
 ])
 def test_full_size_every_element(name, variant):

@@ -45,7 +45,7 @@ def _documented_rule(T, n, H1, r, H2, max_seg_len, sms):
         return sgmv.VARIANT_SPLIT
     if L > 2 and r in (32, 64) and H1 % 64 == 0 and H2 % 64 == 0:
         jobs = n if L <= 16 else min(n + -(-T // 16), T)
-        if jobs < sms and r * H2 * 2 >= 2e6:
+        if jobs < sms and r * H2 * 2 >= 1e6:
             return sgmv.VARIANT_SPLIT_TC
         return sgmv.VARIANT_FUSED_TC
     return sgmv.VARIANT_FUSED
