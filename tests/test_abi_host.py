@@ -218,3 +218,61 @@ def test_auto_variant_rule_edges():
     assert auto(0, 1, 64, 16, 64, F16, 1) == V.VARIANT_AUTO
     assert auto(8, 1, 64, 16, 64, 7, 1) == V.VARIANT_AUTO
     assert auto(8, 1, 64, 16, 64, F16, 1, 0) == V.VARIANT_AUTO
+
+
+def gemm(**kw):
+    a = dict(Y=FAKE, X=FAKE, W=FAKE, A=FAKE, B=FAKE, seg=FAKE, idx=FAKE, n=2, na=4, T=300, H1=256, r=64, H2=264,
+             scale=1.0, dt=1, mx=0, ws=FAKE, wsb=1 << 20, st=None)
+    a.update(kw)
+    return sgmv.load().lora_sgmv_gemm_apply(a["Y"], a["X"], a["W"], a["A"], a["B"], a["seg"], a["idx"], a["n"],
+                                            a["na"], a["T"], a["H1"], a["r"], a["H2"], a["scale"], a["dt"], a["mx"],
+                                            a["ws"], a["wsb"], a["st"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(dt=7), 4), (dict(n=-1), 2), (dict(T=-1), 2), (dict(na=-1), 2), (dict(H1=0), 2), (dict(H2=-8), 2),
+    (dict(r=0), 2), (dict(r=8), 5), (dict(r=128), 5), (dict(H1=260), 3), (dict(H2=100), 3),
+    (dict(Y=None), 1), (dict(X=None), 1), (dict(W=None), 1), (dict(A=None), 1), (dict(seg=None), 1),
+    (dict(na=0), 2), (dict(Y=MIS), 3), (dict(W=MIS), 3),
+    (dict(ws=None), 7), (dict(wsb=300 * 64 * 4 - 4), 7), (dict(ws=MIS), 3),
+])
+def test_gemm_apply_validation_codes(kw, code):
+    # the whole-layer entry point rejects bad arguments on the host, before any CUDA call
+    assert gemm(**kw) == code
+
+
+def test_gemm_apply_empty_batch_is_a_noop_without_gpu():
+    assert gemm(T=0, Y=None, X=None, W=None) == 0
+
+
+def ranks(**kw):
+    a = dict(Y=FAKE, X=FAKE, A=FAKE, B=FAKE, rk=FAKE, seg=FAKE, idx=FAKE, n=2, na=4, T=300, H1=256, rmax=64,
+             H2=264, scale=1.0, dt=1, st=None)
+    a.update(kw)
+    return sgmv.load().lora_sgmv_apply_ranks(a["Y"], a["X"], a["A"], a["B"], a["rk"], a["seg"], a["idx"], a["n"],
+                                             a["na"], a["T"], a["H1"], a["rmax"], a["H2"], a["scale"], a["dt"],
+                                             a["st"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(dt=7), 4), (dict(n=-1), 2), (dict(H1=0), 2), (dict(rmax=0), 2), (dict(rmax=8), 5), (dict(rmax=128), 5),
+    (dict(H1=32), 5), (dict(H2=56), 5), (dict(rk=None), 1), (dict(Y=None), 1), (dict(idx=None), 1),
+    (dict(na=0), 2), (dict(X=MIS), 3), (dict(H1=260), 3),
+])
+def test_apply_ranks_validation_codes(kw, code):
+    assert ranks(**kw) == code
+
+
+def test_apply_ranks_empty_batch_is_a_noop_without_gpu():
+    assert ranks(n=0, Y=None, rk=None) == 0
+
+
+def test_flags_other_than_early_reads_are_refused():
+    lib = sgmv.load()
+    for flags in (0x2, 0x80000000, 0x3):
+        assert lib.lora_sgmv_apply_flags(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 2, 4, 8, 256, 16, 256, 1.0, 0, 0, FAKE,
+                                         1 << 20, None, 0, flags, None) == 5
+        assert lib.lora_sgmv_apply_batched_flags(None, 1, FAKE, FAKE, 2, 8, 16, 0, 0, flags, None, None) == 5
+    # the one defined flag passes validation (an empty batch then returns OK with no CUDA call)
+    assert lib.lora_sgmv_apply_flags(None, None, None, None, None, None, 0, 4, 8, 256, 16, 256, 1.0, 0, 0, None, 0,
+                                     None, 0, sgmv.FLAG_EARLY_READS, None) == 0
