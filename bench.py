@@ -68,20 +68,21 @@ PER_CONFIG_MAX_STEPS = 500
 # is null. For a call of two launches (the split forms) the figure is the pair's.
 TRAFFIC = {
     # profiles/fused_kernel_distinct_decode.md
-    "distinct": {"bytes": 35724544, "sources": ["sgmv_fused.cuh", "sgmv_common.cuh"],
-        "sha256": "4da228808e6c7cdb3a144776e48bbe2e01fc0fad7bd074f571a15c5d55da95e8"},
+    "distinct": {"bytes": 35721728,
+        "sources": ["sgmv_fused.cuh", "sgmv_common.cuh"],
+        "sha256": "97079d473b93cca612249920e720b9ecdd8da2060a5ceca86fd764c41d0db04c"},
     # profiles/split_tc_llama70b_decode_h28672.md
-    "llama70b_decode_h28672": {"bytes": 489211648,
+    "llama70b_decode_h28672": {"bytes": 487882240,
         "sources": ["sgmv_split.cuh", "sgmv_decode_tc.cuh", "sgmv_tmap.cuh", "sgmv_common.cuh"],
-        "sha256": "94643e8ccf1b2c58e2973670a7d4d1b87452ab65a2e06e6cc508dd9d2dfe354d"},
-    # profiles/decode_tc_kernel_llama70b_decode_h8192.md
-    "llama70b_decode_h8192": {"bytes": 211907328,
-        "sources": ["sgmv_decode_tc.cuh", "sgmv_tmap.cuh", "sgmv_common.cuh"],
-        "sha256": "3671ea9eccd0479c921c3020ee059879a38f1fa771078784b0a3d687574eea47"},
+        "sha256": "2f4ca4bccd23f9e27a7a0882206b3f1e56ab53ed9fd8d1ff33e14bff919d4ba2"},
+    # profiles/split_tc_llama70b_decode_h8192.md
+    "llama70b_decode_h8192": {"bytes": 214965248,
+        "sources": ["sgmv_split.cuh", "sgmv_decode_tc.cuh", "sgmv_tmap.cuh", "sgmv_common.cuh"],
+        "sha256": "2f4ca4bccd23f9e27a7a0882206b3f1e56ab53ed9fd8d1ff33e14bff919d4ba2"},
     # profiles/grouped_kernel_prefill.md
-    "prefill": {"bytes": 190034176,
+    "prefill": {"bytes": 191557632,
         "sources": ["sgmv_grouped_tc.cuh", "sgmv_tmap.cuh", "sgmv_common.cuh"],
-        "sha256": "2193ad68fae5fefb2b7868384a1ed95506a46235078f0bb38709c7f2f1e56fb7"},
+        "sha256": "d53cce5554111c3e8dcfa0032527bc110d620edeab4f8db89b87783a60599e2f"},
 }
 
 
