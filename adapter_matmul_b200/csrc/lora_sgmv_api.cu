@@ -382,9 +382,15 @@ lora_sgmv_status launch_fused(sgmv::FusedParams P, int max_len, cudaStream_t str
     int ctas = 0;
     lora_sgmv_status st = resident_for(0, &ctas);
     if (st != LORA_SGMV_OK) return st;
-    // cluster size: the largest C whose jobs*C CTAs are all resident at once; 1 if even that is too many
+    // cluster size: the largest C whose jobs*C CTAs are all resident at once, counting both the
+    // CTA slots and the clusters of C the GPU places at once (clusters of 8 fit fewer times than
+    // the CTA count suggests: a cluster's CTAs share a GPC); 1 if even that is too many
     int lc = 3;
-    while (lc > 0 && jobs * (1ll << lc) > ctas) --lc;
+    while (lc > 0) {
+        int cm = 0;
+        if (jobs * (1ll << lc) <= ctas && resident_for(lc, &cm) == LORA_SGMV_OK && jobs <= cm) break;
+        --lc;
+    }
 #ifdef SGMV_FORCE_CLUSTER_LOG2
     lc = SGMV_FORCE_CLUSTER_LOG2;
 #endif
