@@ -344,16 +344,16 @@ int estimate_max_len(int max_seg_len, int T, int n) {
 
 int round8(int v) { return (v + 7) / 8 * 8; }
 
-template <typename T, int R>
+template <typename T, int R, int CH>
 lora_sgmv_status launch_fused(sgmv::FusedParams P, int max_len, cudaStream_t stream) {
     static int smem_granted[64] = {};
     // resident clusters per (device, log2 cluster size, job-prefix size bucket)
     static int resident[64][4][9] = {};
-    using G = sgmv::FusedGeom<R>;
+    using G = sgmv::FusedGeom<R, CH>;
     if (P.n_segments > sgmv::kFusedMaxSegments) return LORA_SGMV_ERR_DIM;
     const int bucket = (P.n_segments + 1 + 1023) / 1024;  // 1..9
     const size_t smem = G::BASE + size_t(bucket) * 1024 * 4;
-    auto kernel = sgmv::sgmv_fused_kernel<T, R>;
+    auto kernel = sgmv::sgmv_fused_kernel<T, R, CH>;
     if (ensure_smem(kernel, smem, smem_granted) != LORA_SGMV_OK) return LORA_SGMV_ERR_CUDA;
     int dev = 0;
     if (record(cudaGetDevice(&dev)) != cudaSuccess) return LORA_SGMV_ERR_CUDA;
@@ -374,11 +374,10 @@ lora_sgmv_status launch_fused(sgmv::FusedParams P, int max_len, cudaStream_t str
         *out = n;
         return LORA_SGMV_OK;
     };
-    // jobs: token chunks of <= 8 over all segments and problems (upper bound from T and n)
-    const long long chunks = std::min<long long>(P.n_segments + (P.T + sgmv::kFusedTokens - 1) / sgmv::kFusedTokens,
-                                                 std::max(P.T, 1));
-    const long long jobs = std::max<long long>(
-        1, (max_len <= sgmv::kFusedTokens ? static_cast<long long>(P.n_segments) : chunks) * P.n_problems);
+    // jobs: token chunks of <= CH over all segments and problems (upper bound from T and n)
+    const long long chunks = std::min<long long>(P.n_segments + (P.T + CH - 1) / CH, std::max(P.T, 1));
+    const long long jobs =
+        std::max<long long>(1, (max_len <= CH ? static_cast<long long>(P.n_segments) : chunks) * P.n_problems);
     int ctas = 0;
     lora_sgmv_status st = resident_for(0, &ctas);
     if (st != LORA_SGMV_OK) return st;
@@ -398,7 +397,7 @@ lora_sgmv_status launch_fused(sgmv::FusedParams P, int max_len, cudaStream_t str
     st = resident_for(lc, &clusters_max);
     if (st != LORA_SGMV_OK) return st;
     const int C = 1 << lc;
-    P.one_chunk = max_len <= sgmv::kFusedTokens ? 1 : 0;
+    P.one_chunk = max_len <= CH ? 1 : 0;
     for (int i = 0; i < P.n_problems; ++i) {
         P.prob[i].ks = round8((P.prob[i].H1 + C - 1) / C);
         P.prob[i].ns = round8((P.prob[i].H2 + C - 1) / C);
@@ -639,16 +638,28 @@ lora_sgmv_status decode_tc_dispatch(sgmv::FusedParams& P, int r, lora_sgmv_dtype
     return LORA_SGMV_ERR_UNSUPPORTED;
 }
 
-template <typename T>
-lora_sgmv_status fused_dispatch_r(const sgmv::FusedParams& P, int r, int max_len, cudaStream_t s) {
+// Tokens per job of the fused kernel: 8, or 4 when segments reach 16 tokens, whose chunks would
+// otherwise each stream 8 Y rows and do 8 tokens' fp32 expand on one cluster. Measured on the
+// Skewed layer (H2 = 11008): 44.0 -> 26.9 us; Identical: 25.0 -> 16.4 us; the Uniform layer,
+// whose segments hold 1-9 tokens, is better with 8 (25.4 vs 26.0 us).
+constexpr int kFusedLongSegment = 16;
+
+template <typename T, int CH>
+lora_sgmv_status fused_dispatch_rc(const sgmv::FusedParams& P, int r, int max_len, cudaStream_t s) {
     switch (r) {
-        case 8: return launch_fused<T, 8>(P, max_len, s);
-        case 16: return launch_fused<T, 16>(P, max_len, s);
-        case 32: return launch_fused<T, 32>(P, max_len, s);
-        case 64: return launch_fused<T, 64>(P, max_len, s);
-        case 128: return launch_fused<T, 128>(P, max_len, s);
+        case 8: return launch_fused<T, 8, CH>(P, max_len, s);
+        case 16: return launch_fused<T, 16, CH>(P, max_len, s);
+        case 32: return launch_fused<T, 32, CH>(P, max_len, s);
+        case 64: return launch_fused<T, 64, CH>(P, max_len, s);
+        case 128: return launch_fused<T, 128, CH>(P, max_len, s);
     }
     return LORA_SGMV_ERR_UNSUPPORTED;
+}
+
+template <typename T>
+lora_sgmv_status fused_dispatch_r(const sgmv::FusedParams& P, int r, int max_len, cudaStream_t s) {
+    return max_len >= kFusedLongSegment ? fused_dispatch_rc<T, 4>(P, r, max_len, s)
+                                        : fused_dispatch_rc<T, sgmv::kFusedTokens>(P, r, max_len, s);
 }
 
 lora_sgmv_status fused_dispatch(const sgmv::FusedParams& P, int r, lora_sgmv_dtype dt, int max_len,

@@ -5,7 +5,9 @@
 // with adapter i and each row t of it, Y[t,:] += scale * (X[t,:] @ A_i) @ B_i,
 // A_i [H1, r], B_i [r, H2], row-major.
 //
-// Jobs. A job is (problem p, segment s, chunk of <= 8 tokens of s). At start
+// Jobs. A job is (problem p, segment s, chunk of <= CH tokens of s), CH = 8, or 4 when the
+// call's segments reach 16 tokens (the host's choice: a long segment's jobs then carry half the
+// Y rows and expand work each and spread over twice as many clusters). At start
 // every CTA reads seg_starts once and builds the exact job list (a prefix sum
 // of the segments' chunk counts in shared memory), so long segments split
 // into as many jobs as they have chunks and no slot is empty. Clusters are
@@ -62,7 +64,7 @@ constexpr int kFusedMaxProblems = 8;
 #ifndef SGMV_FUSED_MIN_BLOCKS
 #define SGMV_FUSED_MIN_BLOCKS 2
 #endif
-constexpr int kFusedTokens = 8;                  // tokens per job (chunk)
+constexpr int kFusedTokens = 8;                  // tokens per job (chunk); 4 for calls with long segments
 constexpr int kFusedStages = SGMV_FUSED_STAGES;  // ring depth
 constexpr int kFusedConsumerWarps = 4;
 constexpr int kFusedConsumers = 32 * kFusedConsumerWarps;
@@ -97,21 +99,21 @@ struct FusedParams {
     int early;      // 1: segment arrays, tables and adapters may be read before griddepcontrol.wait
 };
 
-// compile-time geometry per rank
-template <int R>
+// compile-time geometry per rank and chunk size (tokens per job)
+template <int R, int CH = kFusedTokens>
 struct FusedGeom {
     static constexpr int RG = R / 8;                                   // expand row groups (8 rows each)
     static constexpr int NTC = (1024 / RG) < 512 ? (1024 / RG) : 512;  // B columns per stage
     static constexpr int GC = NTC / 8;                                 // expand column groups
     static_assert(RG * GC <= kFusedConsumers, "expand tile too wide");
     static constexpr int BPITCH = NTC * 2 + 16;                        // bytes per staged B row
-    static constexpr int BSTAGE = R * BPITCH + kFusedTokens * NTC * 2;  // B rows + Y rows
+    static constexpr int BSTAGE = R * BPITCH + CH * NTC * 2;          // B rows + Y rows
     static constexpr int STAGE = (BSTAGE > 16384 ? BSTAGE : 16384);
     static constexpr int CG = R / 8;                                   // 8-column groups of A
     static constexpr int RLN = kFusedConsumers / CG;                   // shrink row lanes
     static constexpr size_t RING = size_t(kFusedStages) * STAGE;
-    static constexpr size_t RED = size_t(kFusedConsumerWarps) * kFusedTokens * R * 4;
-    static constexpr size_t TILE = size_t(kFusedTokens) * R * 4;  // one partial V tile
+    static constexpr size_t RED = size_t(kFusedConsumerWarps) * CH * R * 4;
+    static constexpr size_t TILE = size_t(CH) * R * 4;            // one partial V tile
     static constexpr size_t RECV = kFusedMaxCluster * TILE;
     static constexpr size_t BASE = RING + RED + RECV + TILE;      // + the job prefix (n+1 ints)
     // A rows per shrink stage for a chunk of nt tokens (A rows plus X columns fill a stage)
@@ -429,10 +431,10 @@ struct FusedSmem {
     float* vs;
 };
 
-template <typename T, int R, int NTOK>
+template <typename T, int R, int NTOK, int CH>
 __device__ __forceinline__ void consume_job(const FusedParams& P, const Job& job, const FusedSmem& S, uint32_t& it,
                                             uint32_t u, int C, int c, int ct, bool& dead) {
-    using G = FusedGeom<R>;
+    using G = FusedGeom<R, CH>;
     const int lane = ct & 31;
     const int cw = ct >> 5;
     const int nt = job.nt;
@@ -480,7 +482,7 @@ __device__ __forceinline__ void consume_job(const FusedParams& P, const Job& job
         for (int t = 0; t < NTOK; ++t)
             if (t < nt) {
 #pragma unroll
-                for (int i = 0; i < 8; ++i) S.red[(cw * kFusedTokens + t) * R + cg * 8 + i] = acc[t][i];
+                for (int i = 0; i < 8; ++i) S.red[(cw * CH + t) * R + cg * 8 + i] = acc[t][i];
             }
     }
     consumer_sync();
@@ -494,18 +496,18 @@ __device__ __forceinline__ void consume_job(const FusedParams& P, const Job& job
         float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
         for (int w = 0; w < kFusedConsumerWarps; ++w) {
-            const float4 q = *reinterpret_cast<const float4*>(S.red + w * kFusedTokens * R + e4 * 4);
+            const float4 q = *reinterpret_cast<const float4*>(S.red + w * CH * R + e4 * 4);
             v.x += q.x;
             v.y += q.y;
             v.z += q.z;
             v.w += q.w;
         }
-        for (int q = 0; q < C; ++q) st_async_v4(S.recv + size_t(c) * kFusedTokens * R + e4 * 4, v, S.vready, q);
+        for (int q = 0; q < C; ++q) st_async_v4(S.recv + size_t(c) * CH * R + e4 * 4, v, S.vready, q);
     }
     mbar_wait<true>(S.vready, u & 1u, P.dev_status, dead);
     for (int e = ct; e < nt * R; e += kFusedConsumers) {
         float sum = 0.f;
-        for (int q = 0; q < C; ++q) sum += S.recv[size_t(q) * kFusedTokens * R + e];
+        for (int q = 0; q < C; ++q) sum += S.recv[size_t(q) * CH * R + e];
         S.vs[e] = sum;
     }
     consumer_sync();
@@ -571,10 +573,10 @@ __device__ __forceinline__ void consume_job(const FusedParams& P, const Job& job
 
 // X columns of the first job's shrink stages (stages 0 .. tiles-1), requested once the
 // previous kernel on the stream has completed.
-template <typename T, int R>
+template <typename T, int R, int CH>
 __device__ __forceinline__ void issue_deferred_x(unsigned char* ring, uint64_t* full, const void* Xv, int H1, int t0,
                                                  int nt, int k0, int KT, int nk, int tiles, int lane) {
-    using G = FusedGeom<R>;
+    using G = FusedGeom<R, CH>;
     const T* X = static_cast<const T*>(Xv);
     for (int ta = 0; ta < tiles; ++ta) {
         unsigned char* st = ring + size_t(ta) * G::STAGE;
@@ -587,10 +589,10 @@ __device__ __forceinline__ void issue_deferred_x(unsigned char* ring, uint64_t* 
 }
 
 // Producer side of one job: shrink stages (A rows + X columns), then expand stages (B rows + Y rows).
-template <typename T, int R>
+template <typename T, int R, int CH>
 __device__ __forceinline__ void produce_job(const FusedParams& P, const Job& job, unsigned char* smem, uint64_t* full,
                                             uint64_t* empty, uint32_t& it, bool& waited, int lane, bool& dead) {
-    using G = FusedGeom<R>;
+    using G = FusedGeom<R, CH>;
     const FusedProblem& pr = P.prob[job.p];
     const T* X = static_cast<const T*>(pr.X);
     const T* Yg = static_cast<const T*>(pr.Y);
@@ -605,7 +607,7 @@ __device__ __forceinline__ void produce_job(const FusedParams& P, const Job& job
             if (!waited) {  // the ring is full: the deferred X must come first
                 pdl_wait();
                 waited = true;
-                issue_deferred_x<T, R>(smem, full, X, pr.H1, job.t0, job.nt, job.k0, KT, job.nk, deferred, lane);
+                issue_deferred_x<T, R, CH>(smem, full, X, pr.H1, job.t0, job.nt, job.k0, KT, job.nk, deferred, lane);
             }
             mbar_wait<false>(&empty[stage], ((it / kFusedStages) - 1) & 1u, P.dev_status, dead);
         }
@@ -632,7 +634,7 @@ __device__ __forceinline__ void produce_job(const FusedParams& P, const Job& job
     if (!waited) {
         pdl_wait();
         waited = true;
-        issue_deferred_x<T, R>(smem, full, X, pr.H1, job.t0, job.nt, job.k0, KT, job.nk, deferred, lane);
+        issue_deferred_x<T, R, CH>(smem, full, X, pr.H1, job.t0, job.nt, job.k0, KT, job.nk, deferred, lane);
     }
     if (job.nc > 0 && lane < job.nt) bulk_prefetch_l2(Yg + size_t(job.t0 + lane) * pr.H2 + job.c0, uint32_t(job.nc) * 2);
     const int nB = (job.nc + G::NTC - 1) / G::NTC;
@@ -657,9 +659,11 @@ __device__ __forceinline__ void produce_job(const FusedParams& P, const Job& job
 // ---- the kernel ----------------------------------------------------------------------------
 
 // grid.x = C * clusters, cluster (C,1,1), C in {1,2,4,8}. Warp 0 produces, warps 1..4 consume.
-template <typename T, int R>
+// CH: tokens per job (8, or 4 for calls with long segments, whose jobs then carry half the Y
+// rows and expand work each and spread over twice as many clusters).
+template <typename T, int R, int CH = kFusedTokens>
 __global__ void __launch_bounds__(kFusedThreads, SGMV_FUSED_MIN_BLOCKS) sgmv_fused_kernel(const FusedParams P) {
-    using G = FusedGeom<R>;
+    using G = FusedGeom<R, CH>;
     extern __shared__ __align__(128) unsigned char smem[];
     __shared__ __align__(8) uint64_t full[kFusedStages];
     __shared__ __align__(8) uint64_t empty[kFusedStages];
@@ -706,7 +710,7 @@ __global__ void __launch_bounds__(kFusedThreads, SGMV_FUSED_MIN_BLOCKS) sgmv_fus
         __syncthreads();
         entries = P.n_problems * P.n_segments;
     } else {
-        build_job_prefix(P, pref);  // ends with __syncthreads
+        build_job_prefix<CH>(P, pref);  // ends with __syncthreads
         entries = P.n_problems * pref[P.n_segments];
     }
     // Barriers of every CTA exist before any remote operation: each CTA arrives here and
@@ -723,11 +727,11 @@ __global__ void __launch_bounds__(kFusedThreads, SGMV_FUSED_MIN_BLOCKS) sgmv_fus
         bool waited = !P.early;
         for (int j = cluster_id; j < entries; j += n_clusters) {
             int p, s, q0, nq;
-            entry_at(P, pref, j, p, s, q0, nq);
+            entry_at<CH>(P, pref, j, p, s, q0, nq);
             for (int q = q0; q < q0 + nq; ++q) {
                 Job job;
-                if (!job_at(P, p, s, q, c, job)) break;
-                produce_job<T, R>(P, job, smem, full, empty, it, waited, lane, dead);
+                if (!job_at<CH>(P, p, s, q, c, job)) break;
+                produce_job<T, R, CH>(P, job, smem, full, empty, it, waited, lane, dead);
             }
         }
         if (!waited) pdl_wait();
@@ -742,19 +746,19 @@ __global__ void __launch_bounds__(kFusedThreads, SGMV_FUSED_MIN_BLOCKS) sgmv_fus
         uint32_t it = 0, u = 0;
         for (int j = cluster_id; j < entries; j += n_clusters) {
             int p, s, q0, nq;
-            entry_at(P, pref, j, p, s, q0, nq);
+            entry_at<CH>(P, pref, j, p, s, q0, nq);
             if (nq == 0 && reporter) report(P.dev_status, segment_bounds_check(P, s));
             for (int q = q0; q < q0 + nq; ++q) {
                 Job job;
-                if (!job_at_reporting(P, p, s, q, c, job, reporter)) break;
+                if (!job_at_reporting<CH>(P, p, s, q, c, job, reporter)) break;
                 if (job.nt == 1)
-                    consume_job<T, R, 1>(P, job, S, it, u, C, c, ct, dead);
+                    consume_job<T, R, 1, CH>(P, job, S, it, u, C, c, ct, dead);
                 else if (job.nt <= 2)
-                    consume_job<T, R, 2>(P, job, S, it, u, C, c, ct, dead);
-                else if (job.nt <= 4)
-                    consume_job<T, R, 4>(P, job, S, it, u, C, c, ct, dead);
+                    consume_job<T, R, 2, CH>(P, job, S, it, u, C, c, ct, dead);
+                else if (CH == 4 || job.nt <= 4)
+                    consume_job<T, R, 4, CH>(P, job, S, it, u, C, c, ct, dead);
                 else
-                    consume_job<T, R, 8>(P, job, S, it, u, C, c, ct, dead);
+                    consume_job<T, R, (CH > 4 ? 8 : 4), CH>(P, job, S, it, u, C, c, ct, dead);
                 ++u;
             }
         }
