@@ -70,7 +70,7 @@ TRAFFIC = {
     # profiles/fused_kernel_distinct_decode.md
     "distinct": {"bytes": 35721728,
         "sources": ["sgmv_fused.cuh", "sgmv_common.cuh"],
-        "sha256": "97079d473b93cca612249920e720b9ecdd8da2060a5ceca86fd764c41d0db04c"},
+        "sha256": "6552c4033b5e2540a7d033f2b197baf0c9ddf3269fb04823340175560c568ce3"},
     # profiles/split_tc_llama70b_decode_h28672.md
     "llama70b_decode_h28672": {"bytes": 487882240,
         "sources": ["sgmv_split.cuh", "sgmv_decode_tc.cuh", "sgmv_tmap.cuh", "sgmv_common.cuh"],
