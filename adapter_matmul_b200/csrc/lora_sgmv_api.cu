@@ -148,9 +148,6 @@ lora_sgmv_status launch_shrink(const ShrinkParams& p0, int max_len, cudaStream_t
     // cluster reduction) are then paid by half as many CTAs. Measured on the 70B-shaped decode
     // (127 chunks, H1 = 8192): 8 CTAs per chunk 41.8 us, 4 CTAs 39.5 us, 2 CTAs 49.8 us.
     if (p.flat && C == 8 && units * 8 > 4ll * f.sms) C = 4;
-#ifdef SGMV_SHRINK_CLUSTER
-    C = std::min(C, SGMV_SHRINK_CLUSTER);
-#endif
     p.ks = ((p.H1 + C - 1) / C + 7) / 8 * 8;
     const size_t smem = sgmv::shrink_smem_bytes(p.ks, R, p.flat ? p.n_segments : 0);
     if (smem > static_cast<size_t>(f.max_smem_optin)) return LORA_SGMV_ERR_DIM;
@@ -390,9 +387,6 @@ lora_sgmv_status launch_fused(sgmv::FusedParams P, int max_len, cudaStream_t str
         if (jobs * (1ll << lc) <= ctas && resident_for(lc, &cm) == LORA_SGMV_OK && jobs <= cm) break;
         --lc;
     }
-#ifdef SGMV_FORCE_CLUSTER_LOG2
-    lc = SGMV_FORCE_CLUSTER_LOG2;
-#endif
     int clusters_max = 0;
     st = resident_for(lc, &clusters_max);
     if (st != LORA_SGMV_OK) return st;

@@ -152,7 +152,6 @@ template <int N>
 __device__ __forceinline__ void bulk_wait() {
     asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
 }
-__device__ __forceinline__ void epilogue_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
 // The rows [t0, t0 + nt) of a chunk are moved as boxes of 16, 8, 4, 2 and 1 rows (the binary
 // digits of nt), so Y rows of other segments are never read or written. Box m (rows 2^m) of
