@@ -452,21 +452,21 @@ lora_sgmv_variant auto_variant(int T, int n_segments, int max_len, int H1, int H
     return LORA_SGMV_VARIANT_FUSED;
 }
 
-template <typename T, int R>
+// PRE_V: V comes from an earlier kernel (v_in); else the clusters compute it
+template <typename T, int R, bool PRE_V>
 lora_sgmv_status launch_decode_tc(sgmv::FusedParams P, const sgmv::DecodeMaps& maps, int max_len, cudaStream_t stream,
                                   const float* v_in) {
-    static int smem_granted[2][64] = {};  // per kernel mode
+    static int smem_granted[64] = {};
     // resident clusters per (device, cluster size, job-prefix size bucket)
     static int resident[64][sgmv::kFusedMaxCluster + 1][9] = {};
-    using G = sgmv::DecodeTCGeom<R>;
+    using G = sgmv::DecodeTCGeom<R, PRE_V>;
     constexpr int CH = sgmv::kDTokens;
     if (P.n_segments > sgmv::kFusedMaxSegments) return LORA_SGMV_ERR_DIM;
     const int bucket = (P.n_segments + 1 + 1023) / 1024;  // 1..9
     auto smem_for = [&](int C) {
         return G::BASE + size_t(C) * G::TILE + size_t(bucket) * 1024 * 4 + 1024 /* alignment slack */;
     };
-    // one kernel per mode: with V from the workspace, or computed by the cluster
-    auto kernel = v_in ? sgmv::sgmv_decode_tc_kernel<T, R, true> : sgmv::sgmv_decode_tc_kernel<T, R, false>;
+    auto kernel = sgmv::sgmv_decode_tc_kernel<T, R, PRE_V>;
     DeviceFacts f;
     if (device_facts(f) != LORA_SGMV_OK) return LORA_SGMV_ERR_CUDA;
     // the largest cluster whose shared memory (ring + one partial V tile per CTA of the cluster
@@ -475,7 +475,7 @@ lora_sgmv_status launch_decode_tc(sgmv::FusedParams P, const sgmv::DecodeMaps& m
     int c_fit = sgmv::kFusedMaxCluster;
     while (c_fit > 0 && smem_for(c_fit) > smem_cap) --c_fit;
     if (c_fit == 0) return LORA_SGMV_ERR_DIM;
-    if (ensure_smem(kernel, smem_for(c_fit), smem_granted[v_in ? 1 : 0]) != LORA_SGMV_OK) return LORA_SGMV_ERR_CUDA;
+    if (ensure_smem(kernel, smem_for(c_fit), smem_granted) != LORA_SGMV_OK) return LORA_SGMV_ERR_CUDA;
     int dev = 0;
     if (record(cudaGetDevice(&dev)) != cudaSuccess) return LORA_SGMV_ERR_CUDA;
     if (dev < 0 || dev >= 64) return LORA_SGMV_ERR_UNSUPPORTED;
@@ -500,7 +500,7 @@ lora_sgmv_status launch_decode_tc(sgmv::FusedParams P, const sgmv::DecodeMaps& m
         std::min<long long>(P.n_segments + (P.T + CH - 1) / CH, std::max(P.T, 1));
     const long long jobs = std::max<long long>(1, (one_chunk ? static_cast<long long>(P.n_segments) : chunks) *
                                                       P.n_problems);
-    if (v_in) {
+    if constexpr (PRE_V) {
         // V is precomputed: each job's N is cut into S slices and the jobs x S units are walked
         // by independent CTAs, all resident at once. Estimated time = rounds x (slice bytes at
         // the ~24 GB/s one CTA of this kernel streams + a fixed cost per unit).
@@ -612,13 +612,21 @@ lora_sgmv_status decode_tc_maps_and_launch(sgmv::FusedParams& P, lora_sgmv_dtype
                                            const float* v_in) {
     sgmv::DecodeMaps maps;
     std::memset(&maps, 0, sizeof(maps));
-    for (int i = 0; i < P.n_problems; ++i)
-        if (!sgmv::make_decode_maps<R>(maps, i, P.prob[i].X, P.prob[i].Y, P.T, P.prob[i].H1, P.prob[i].H2, dt)) {
+    for (int i = 0; i < P.n_problems; ++i) {
+        const bool ok = v_in ? sgmv::make_decode_maps<R, true>(maps, i, P.prob[i].X, P.prob[i].Y, P.T, P.prob[i].H1,
+                                                               P.prob[i].H2, dt)
+                             : sgmv::make_decode_maps<R, false>(maps, i, P.prob[i].X, P.prob[i].Y, P.T, P.prob[i].H1,
+                                                                P.prob[i].H2, dt);
+        if (!ok) {
             t_last_error = cudaErrorInvalidValue;
             return LORA_SGMV_ERR_CUDA;
         }
-    return dt == LORA_SGMV_BF16 ? launch_decode_tc<__nv_bfloat16, R>(P, maps, max_len, s, v_in)
-                                : launch_decode_tc<__half, R>(P, maps, max_len, s, v_in);
+    }
+    if (v_in)
+        return dt == LORA_SGMV_BF16 ? launch_decode_tc<__nv_bfloat16, R, true>(P, maps, max_len, s, v_in)
+                                    : launch_decode_tc<__half, R, true>(P, maps, max_len, s, v_in);
+    return dt == LORA_SGMV_BF16 ? launch_decode_tc<__nv_bfloat16, R, false>(P, maps, max_len, s, v_in)
+                                : launch_decode_tc<__half, R, false>(P, maps, max_len, s, v_in);
 }
 
 // v_in: V from an earlier kernel (the split form)

@@ -73,18 +73,22 @@ struct DecodeMaps {
 __host__ __device__ constexpr int round1024(int v) { return (v + 1023) / 1024 * 1024; }
 __host__ __device__ constexpr int cmax(int a, int b) { return a > b ? a : b; }
 
-template <int R>
+template <int R, bool PRE_V = false>
 struct DecodeTCGeom {
     static constexpr int KS = R == 16 ? 256 : 128;        // rows of A_i per shrink stage
     static constexpr int A_BYTES = KS * R * 2;            // 16, 8, 8 KB (r = 64, 32, 16)
     static constexpr int XB = KS / 64;                    // X column blocks per shrink stage
     static constexpr int X_BYTES = XB * kDTokens * 128;   // 16 rows per block
     // 64-column blocks of B_i per expand stage: a stage carries 32 KB of B_i at r = 64, 16 KB
-    // otherwise (the per-stage costs of the MMA and the epilogue are paid per stage)
-    static constexpr int NB = (R == 64 ? 32768 : 16384) / (R * 128);
-    static constexpr int NW = NB * 64;                    // columns per expand stage: 256, 256, 512
-    static constexpr int B_BYTES = R * NW * 2;            // 32, 16, 16 KB
-    static constexpr int STAGES = R == 64 ? 4 : 6;        // main ring depth
+    // otherwise (the per-stage costs of the MMA and the epilogue are paid per stage). With V
+    // precomputed the ring holds B_i alone, and at r = 64 it takes two 64 KB stages of 512
+    // columns: the same bytes in flight as four 32 KB stages, half the per-stage costs (the
+    // fused form keeps 32 KB, since its shrink stages would leave most of a 64 KB slot unused).
+    static constexpr bool WIDE = PRE_V && R == 64;
+    static constexpr int NB = (WIDE ? 65536 : (R == 64 ? 32768 : 16384)) / (R * 128);
+    static constexpr int NW = NB * 64;                    // columns per expand stage: 256 (512 wide), 256, 512
+    static constexpr int B_BYTES = R * NW * 2;            // 32 (64 wide), 16, 16 KB
+    static constexpr int STAGES = WIDE ? 2 : (R == 64 ? 4 : 6);  // main ring depth
     static constexpr int YW = NW < 256 ? NW : 256;        // Y box width
     static constexpr int YBOXES = NW / YW;
     static constexpr int Y_BYTES = round1024(kDTokens * NW * 2);  // one Y stage: [YBOXES][16 rows][YW]
@@ -162,7 +166,7 @@ template <typename T, int R, bool PRE_V>
 __global__ void __launch_bounds__(kDThreads, 1)
     sgmv_decode_tc_kernel(const __grid_constant__ DecodeMaps maps, const FusedParams P, const float* v_in,
                           int n_slices) {
-    using G = DecodeTCGeom<R>;
+    using G = DecodeTCGeom<R, PRE_V>;
     constexpr int S = G::STAGES;
     constexpr int SY = kDYStages;
     constexpr int ND2 = G::ND2;
@@ -652,10 +656,11 @@ inline bool encode_map(CUtensorMap* map, const void* base, lora_sgmv_dtype dt, i
     return r == CUDA_SUCCESS;
 }
 
-// All maps of problem p for the tensor-core decode kernel at rank R (H1, H2 multiples of 64).
-template <int R>
+// All maps of problem p for the tensor-core decode kernel at rank R (H1, H2 multiples of 64),
+// for the kernel's form PRE_V.
+template <int R, bool PRE_V>
 inline bool make_decode_maps(DecodeMaps& m, int p, const void* X, void* Y, int T, int H1, int H2, lora_sgmv_dtype dt) {
-    using G = DecodeTCGeom<R>;
+    using G = DecodeTCGeom<R, PRE_V>;
     {  // X view {64, T, H1/64}: element (k, t, b) at X + t*H1 + 64*b + k
         const uint64_t d[3] = {64, uint64_t(T), uint64_t(H1 / 64)};
         const uint64_t s[2] = {uint64_t(H1) * 2, 128};
