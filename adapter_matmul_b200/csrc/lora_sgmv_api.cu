@@ -143,19 +143,35 @@ lora_sgmv_status launch_shrink(const ShrinkParams& p0, int max_len, cudaStream_t
     const long long units = std::min<long long>(
         static_cast<long long>(p.n_segments) + (p.T + sgmv::kShrinkTokens - 1) / sgmv::kShrinkTokens, p.T);
     int C = cluster_size_for(p.H1);
-    // Fewer, longer CTAs when clusters of 8 would need more than two waves (the SM count's
-    // worth of CTA pairs, two CTAs per SM): each chunk's fixed steps (the chunk list, X, the
-    // cluster reduction) are then paid by half as many CTAs. Measured on the 70B-shaped decode
-    // (127 chunks, H1 = 8192): 8 CTAs per chunk 41.8 us, 4 CTAs 39.5 us, 2 CTAs 49.8 us.
+    // Fewer, longer CTAs when clusters of 8 would fill the SMs several times over: each chunk's
+    // fixed steps (the chunk list, the first copies, the cluster reduction) are then paid by
+    // half as many CTAs. Measured on the 70B-shaped decode (106 chunks, H1 = 8192, three CTAs
+    // per SM): 8 CTAs per chunk 44.4 us, 4 CTAs 37.5 us.
     if (p.flat && C == 8 && units * 8 > 4ll * f.sms) C = 4;
     p.ks = ((p.H1 + C - 1) / C + 7) / 8 * 8;
-    const size_t smem = sgmv::shrink_smem_bytes(p.ks, R, p.flat ? p.n_segments : 0);
+    const size_t smem = sgmv::shrink_smem_bytes(R, p.flat ? p.n_segments : 0);
     if (smem > static_cast<size_t>(f.max_smem_optin)) return LORA_SGMV_ERR_DIM;
     auto kernel = sgmv::sgmv_shrink_cluster_kernel<T, R>;
     if (ensure_smem(kernel, smem, smem_granted) != LORA_SGMV_OK) return LORA_SGMV_ERR_CUDA;
 
+    // X [T, H1] as boxes of {XB columns, 8 rows}; rows past T read as zeros
+    CUtensorMap xmap;
+    {
+        const uint64_t d[2] = {uint64_t(p.H1), uint64_t(p.T)};
+        const uint64_t st[1] = {uint64_t(p.H1) * 2};
+        const uint32_t b[2] = {uint32_t(sgmv::shrink_x_box(R)), uint32_t(sgmv::kShrinkTokens)};
+        const lora_sgmv_dtype dt = std::is_same<T, __half>::value ? LORA_SGMV_F16 : LORA_SGMV_BF16;
+        if (!sgmv::encode_map(&xmap, p.X, dt, 2, d, st, b, CU_TENSOR_MAP_SWIZZLE_NONE)) {
+            t_last_error = cudaErrorInvalidValue;
+            return LORA_SGMV_ERR_CUDA;
+        }
+    }
+
     cudaLaunchConfig_t cfg = {};
     if (p.flat) {
+        // one cluster per chunk: clusters beyond those resident at once start as others end,
+        // which evens out the chunks' unequal durations (measured on the 70B-shaped decode:
+        // 37.5 us, against 47.8 us with the grid cut to the resident clusters walking the list)
         cfg.gridDim = dim3(C, static_cast<unsigned>(std::max<long long>(1, std::min<long long>(units, 65535))), 1);
     } else {
         cfg.gridDim = dim3(C, clamp_grid_y(p.n_segments), chunk_slots(max_len, sgmv::kShrinkTokens, 8));
@@ -170,7 +186,7 @@ lora_sgmv_status launch_shrink(const ShrinkParams& p0, int max_len, cudaStream_t
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return counted(cudaLaunchKernelEx(&cfg, kernel, p));
+    return counted(cudaLaunchKernelEx(&cfg, kernel, xmap, p));
 }
 
 template <typename T, int R>

@@ -119,6 +119,25 @@ __device__ __forceinline__ void unpack8(const uint4& v, float (&f)[8]) {
     p = Storage<T>::to2(v.w); f[6] = p.x; f[7] = p.y;
 }
 
+// Two fp32 lanes in one 64-bit register pair, for the paired fp32 arithmetic of sm_100
+// (fma.rn.f32x2: each lane is one fused multiply-add rounded to nearest, the result fmaf gives).
+__device__ __forceinline__ uint64_t f32x2(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ float2 f32x2_split(uint64_t v) {
+    float2 r;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
+    return r;
+}
+// a * b + c per lane
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
 template <typename T>
 __device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
     uint4 v;

@@ -8,15 +8,15 @@
 // Shrink. One thread-block cluster of C CTAs per token chunk (8 tokens of one segment;
 // the clusters walk a flat list of the chunks, or segment and chunk slots when there are
 // too many segments for the list's prefix to fit in shared memory).
-// CTA c of the cluster owns rows [c*KS, (c+1)*KS) of A_i; that slice of A_i
-// is one contiguous run of KS*r*2 bytes, read once with 128-bit coalesced
-// loads. Each CTA stages its slice of the chunk's X rows in shared memory,
-// accumulates fp32 partial sums per thread (one token row for a one-token chunk, with twice
-// the loads of A_i in flight, else eight), reduces them with warp shuffles
-// and then across warps in shared memory. The C partial V tiles are summed in
-// a fixed order through distributed shared memory (DSMEM), and each CTA
-// stores its share of the reduced V with plain stores: no atomics, no
-// zero-fill of V, bit-reproducible.
+// CTA c of the cluster owns rows [c*KS, (c+1)*KS) of A_i; that slice of A_i is one
+// contiguous run of KS*r*2 bytes. One thread streams it through a ring of shared-memory
+// slots with 1-D bulk copies (16 KB each), and with each slot a tensor-map copy of the
+// chunk's X columns for the same rows, so the copies run ahead of the arithmetic. All
+// threads accumulate fp32 partial sums from the ring (paired FMAs, two columns per
+// instruction), reduce them with warp shuffles and then across warps in shared memory. The
+// C partial V tiles are summed in a fixed order through distributed shared memory (DSMEM),
+// and each CTA stores its share of the reduced V with plain stores: no atomics, no
+// zero-fill of V, bit-reproducible. 128 threads per CTA and three CTAs per SM.
 //
 // Expand. One CTA per (column block of 8*NT columns, segment, token-chunk
 // slot). Each thread owns 8 consecutive columns: it streams B_i[j, cols] for
@@ -31,6 +31,7 @@
 #include <cooperative_groups.h>
 
 #include "sgmv_common.cuh"
+#include "sgmv_grouped_tc.cuh"  // PTX wrappers (mbarriers, bulk and tensor-map copies)
 
 namespace sgmv {
 
@@ -67,83 +68,127 @@ struct ExpandParams {
     float scale;
 };
 
-constexpr int kShrinkThreads = 256;
-constexpr int kShrinkTokens = 8;   // tokens per chunk
-constexpr int kShrinkUnroll = 8;   // 16-byte loads in flight per thread
+constexpr int kShrinkThreads = 128;
+constexpr int kShrinkTokens = 8;     // tokens per chunk
+constexpr int kShrinkSlotA = 16384;  // bytes of A_i per ring slot (one bulk copy)
+constexpr int kShrinkSlots = 3;      // ring depth
 constexpr int kExpandThreads = 128;
 constexpr int kExpandTokens = 8;
 
 constexpr int kShrinkFlatMaxSegments = 8192;  // flat grid: the chunk prefix fits in shared memory
 
-__host__ __device__ constexpr size_t shrink_smem_bytes(int ks, int R, int flat_segments = 0) {
-    // X slice [TC][ks] (16-bit) + per-warp partials [NW][TC*R] + CTA partial [TC*R]
-    // (+ flat grid: chunk prefix [n_segments + 1] and per-warp totals [NW])
-    return size_t(kShrinkTokens) * ks * 2 + size_t(kShrinkThreads / 32) * kShrinkTokens * R * 4 +
-           size_t(kShrinkTokens) * R * 4 +
+// A ring slot: SR rows of A_i (16 KB), then the chunk's X columns for those rows, [8][SR]
+// (16-bit), loaded by NXB tensor-map boxes of {XB columns, 8 rows}.
+__host__ __device__ constexpr int shrink_slot_rows(int R) { return kShrinkSlotA / (R * 2); }
+__host__ __device__ constexpr int shrink_x_box(int R) { return shrink_slot_rows(R) < 256 ? shrink_slot_rows(R) : 256; }
+__host__ __device__ constexpr int shrink_slot_bytes(int R) {
+    return kShrinkSlotA + kShrinkTokens * shrink_slot_rows(R) * 2;
+}
+__host__ __device__ constexpr size_t shrink_ring_bytes(int R) {
+    // the ring, which after a chunk's last slot holds the per-warp partials [NW][TC*R]
+    return size_t(kShrinkSlots) * shrink_slot_bytes(R) > size_t(kShrinkThreads / 32) * kShrinkTokens * R * 4
+               ? size_t(kShrinkSlots) * shrink_slot_bytes(R)
+               : size_t(kShrinkThreads / 32) * kShrinkTokens * R * 4;
+}
+
+__host__ __device__ constexpr size_t shrink_smem_bytes(int R, int flat_segments = 0) {
+    // ring + CTA partial [TC*R] (+ flat grid: chunk prefix [n_segments + 1] and per-warp totals [NW])
+    return shrink_ring_bytes(R) + size_t(kShrinkTokens) * R * 4 +
            (flat_segments > 0 ? size_t(flat_segments + 1 + kShrinkThreads / 32) * 4 : 0);
 }
 
 // One token chunk [t0, t0 + nt) of a segment, this CTA's rows [k0, k0 + nk) of its A_i:
-// stage the chunk's X slice, accumulate TCN token rows (rows past nt are zero) with U
-// 16-byte loads of A_i in flight per thread, reduce over the CTA, sum the C partial tiles
-// across the cluster in rank order and store this CTA's share of V. Every CTA of the cluster
-// calls it for the same chunk.
-template <typename T, int R, int TCN, int U>
-__device__ __forceinline__ void shrink_chunk(const ShrinkParams& p, cg::cluster_group& cluster, const T* __restrict__ A,
-                                             int t0, int nt, int k0, int nk, T* xs, float* red, float* part) {
+// stream the rows, and the chunk's X columns beside them, through the ring, accumulate TCN
+// token rows, reduce over the CTA, sum the C partial tiles across the cluster in rank order
+// and store this CTA's share of V. X rows past nt (the next segment's tokens, or zeros past T)
+// only reach sums that are never stored. Every CTA of the cluster calls it for the same
+// chunk; `it` counts the ring slots this CTA has used.
+template <typename T, int R, int TCN>
+__device__ __forceinline__ void shrink_chunk(const CUtensorMap* xmap, const ShrinkParams& p, cg::cluster_group& cluster,
+                                             const T* __restrict__ A, int t0, int nt, int k0, int nk,
+                                             unsigned char* ring, uint64_t* full, uint32_t& it, bool& dead,
+                                             float* part) {
     constexpr int NT = kShrinkThreads;
-    constexpr int G = R / 8;     // 16-byte vectors per row of A_i
-    constexpr int RL = NT / G;   // row lanes
+    constexpr int G = R / 8;                     // 16-byte vectors per row of A_i
+    constexpr int RL = NT / G;                   // row lanes
     constexpr int NW = NT / 32;
+    constexpr int SR = shrink_slot_rows(R);      // rows of A_i per slot
+    constexpr int RPT = SR / RL;                 // rows per thread per slot
+    constexpr int XB = shrink_x_box(R);
+    constexpr int SLOT = shrink_slot_bytes(R);
+    static_assert(SR % RL == 0 && SR % XB == 0, "a slot must hold whole rows for every row lane");
     const int tid = threadIdx.x;
     const int lane = tid & 31;
     const int warp = tid >> 5;
     const int cgi = tid % G;
     const int rl = tid / G;
-    const int KS = p.ks;
     const int c = static_cast<int>(cluster.block_rank());
     const int C = static_cast<int>(cluster.num_blocks());
-    const T* __restrict__ X = static_cast<const T*>(p.X);
-
-    // stage X[t0 .. t0+TCN, k0 .. k0+nk) (rows past the chunk are zero)
-    const int vpr = nk / 8;
-    for (int v = tid; v < TCN * vpr; v += NT) {
-        const int row = v / vpr;
-        const int col = (v - row * vpr) * 8;
-        uint4 val = make_uint4(0, 0, 0, 0);
-        if (row < nt) val = ld_vec(X + size_t(t0 + row) * p.H1 + k0 + col);
-        st_vec(xs + size_t(row) * KS + col, val);
+    const int nslot = (nk + SR - 1) / SR;
+    const unsigned char* Ab = reinterpret_cast<const unsigned char*>(A + size_t(k0) * R);
+    auto issue = [&](int i) {  // slot i of this chunk
+        const uint32_t a_bytes = static_cast<uint32_t>(min(SR, nk - i * SR)) * R * 2;
+        const uint32_t b = (it + i) % kShrinkSlots;
+        unsigned char* dst = ring + size_t(b) * SLOT;
+        mbar_arrive_expect_tx(&full[b], a_bytes + kShrinkTokens * SR * 2);
+        bulk_g2s(dst, Ab + size_t(i) * kShrinkSlotA, a_bytes, &full[b]);
+#pragma unroll
+        for (int xb = 0; xb < SR / XB; ++xb)
+            tma_load_2d(dst + kShrinkSlotA + xb * kShrinkTokens * XB * 2, xmap, k0 + i * SR + xb * XB, t0, &full[b]);
+    };
+    if (tid == 0) {
+        // the ring last held the previous chunk's partials, written by generic stores
+        fence_proxy_async();
+        for (int i = 0; i < min(nslot, kShrinkSlots); ++i) issue(i);
     }
-    __syncthreads();
 
+    // column pairs (2q, 2q + 1) of the 8 sums per token row, updated by paired FMAs
+    uint64_t acc2[TCN][4];
+#pragma unroll
+    for (int t = 0; t < TCN; ++t)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) acc2[t][q] = 0;
+
+#pragma unroll 1
+    for (int i = 0; i < nslot; ++i) {
+        const uint32_t g = it + i;
+        mbar_wait<false>(&full[g % kShrinkSlots], (g / kShrinkSlots) & 1u, p.dev_status, dead);
+        const unsigned char* sl = ring + size_t(g % kShrinkSlots) * SLOT;
+        const T* xs = reinterpret_cast<const T*>(sl + kShrinkSlotA);
+#pragma unroll
+        for (int m = 0; m < RPT; ++m) {
+            const int row = rl + m * RL;
+            if (i * SR + row < nk) {
+                float a[8];
+                unpack8<T>(ld_vec(sl + size_t(row) * (R * 2) + cgi * 16), a);
+                uint64_t a2[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) a2[q] = f32x2(a[2 * q], a[2 * q + 1]);
+                // X box xb holds columns [xb*XB, (xb+1)*XB) of the slot as [8][XB]
+                const T* xr = xs + (row / XB) * (kShrinkTokens * XB) + (row % XB);
+#pragma unroll
+                for (int t = 0; t < TCN; ++t) {
+                    const float x = Storage<T>::to1(xr[t * XB]);
+                    const uint64_t x2 = f32x2(x, x);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) acc2[t][q] = ffma2(x2, a2[q], acc2[t][q]);
+                }
+            }
+        }
+        __syncthreads();  // every thread is done with the slot before it is refilled
+        if (tid == 0 && i + kShrinkSlots < nslot) issue(i + kShrinkSlots);
+    }
+    it += static_cast<uint32_t>(nslot);
     float acc[TCN][8];
 #pragma unroll
     for (int t = 0; t < TCN; ++t)
 #pragma unroll
-        for (int i = 0; i < 8; ++i) acc[t][i] = 0.f;
-
-    for (int kb = rl; kb < nk; kb += RL * U) {
-        uint4 av[U];
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const int kr = kb + u * RL;
-            av[u] = kr < nk ? ld_stream(A + size_t(k0 + kr) * R + cgi * 8) : make_uint4(0, 0, 0, 0);
+        for (int q = 0; q < 4; ++q) {
+            const float2 v = f32x2_split(acc2[t][q]);
+            acc[t][2 * q] = v.x;
+            acc[t][2 * q + 1] = v.y;
         }
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const int kr = kb + u * RL;
-            if (kr < nk) {
-                float a[8];
-                unpack8<T>(av[u], a);
-#pragma unroll
-                for (int t = 0; t < TCN; ++t) {
-                    const float x = Storage<T>::to1(xs[size_t(t) * KS + kr]);
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) acc[t][i] = fmaf(x, a[i], acc[t][i]);
-                }
-            }
-        }
-    }
+    float* red = reinterpret_cast<float*>(ring);  // no copy is in flight after the last slot
     // reduce over the row lanes of this warp (lanes sharing cgi)
 #pragma unroll
     for (int off = G; off < 32; off <<= 1)
@@ -192,11 +237,11 @@ __device__ __forceinline__ int shrink_segment_chunks(const ShrinkParams& p, int 
 // every CTA builds the list's prefix (chunks before each segment) in shared memory, so the
 // grid holds no CTA without a chunk.
 template <typename T, int R>
-__global__ void __launch_bounds__(kShrinkThreads) sgmv_shrink_cluster_kernel(const ShrinkParams p) {
+__global__ void __launch_bounds__(kShrinkThreads, 3)
+    sgmv_shrink_cluster_kernel(const __grid_constant__ CUtensorMap xmap, const ShrinkParams p) {
     constexpr int NT = kShrinkThreads;
     constexpr int TC = kShrinkTokens;
     constexpr int G = R / 8;
-    constexpr int NW = NT / 32;
     static_assert(R % 8 == 0 && G <= 32 && (32 % G) == 0, "rank must be 8..256, power of two");
 
     cg::cluster_group cluster = cg::this_cluster();
@@ -204,9 +249,16 @@ __global__ void __launch_bounds__(kShrinkThreads) sgmv_shrink_cluster_kernel(con
     const int tid = threadIdx.x;
 
     extern __shared__ __align__(128) unsigned char smem[];
-    T* xs = reinterpret_cast<T*>(smem);
-    float* red = reinterpret_cast<float*>(smem + size_t(TC) * p.ks * 2);
-    float* part = red + NW * TC * R;
+    unsigned char* ring = smem;
+    float* part = reinterpret_cast<float*>(smem + shrink_ring_bytes(R));
+    __shared__ __align__(8) uint64_t full[kShrinkSlots];
+    if (tid == 0) {
+        for (int i = 0; i < kShrinkSlots; ++i) mbar_init(&full[i], 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    uint32_t it = 0;    // ring slots used
+    bool dead = false;  // a wait on the ring gave up (reported; the results are invalid)
 
     // The expand kernel may be scheduled as soon as every shrink CTA is running.
     pdl_launch_dependents();
@@ -215,9 +267,9 @@ __global__ void __launch_bounds__(kShrinkThreads) sgmv_shrink_cluster_kernel(con
     const int nk = max(0, min(k0 + p.ks, p.H1) - k0);
     auto run_chunk = [&](const T* A, int t0, int nt) {
         if (nt == 1)
-            shrink_chunk<T, R, 1, 2 * kShrinkUnroll>(p, cluster, A, t0, nt, k0, nk, xs, red, part);
+            shrink_chunk<T, R, 1>(&xmap, p, cluster, A, t0, nt, k0, nk, ring, full, it, dead, part);
         else
-            shrink_chunk<T, R, TC, kShrinkUnroll>(p, cluster, A, t0, nt, k0, nk, xs, red, part);
+            shrink_chunk<T, R, TC>(&xmap, p, cluster, A, t0, nt, k0, nk, ring, full, it, dead, part);
     };
 
     if (p.flat) {
