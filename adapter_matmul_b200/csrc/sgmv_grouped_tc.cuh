@@ -22,8 +22,10 @@
 // canonical layout the MMA descriptors describe: X and Y through tensor maps built per
 // call, A_i and B_i (reached through a device table of pointers) through maps each CTA
 // makes from a per-call template (sgmv_tmap.cuh). Warp roles: warp 0 producer, warp 1
-// allocates TMEM and issues tcgen05.mma (one thread), warps 2..9 epilogue (one TMEM lane
-// quarter and one 64-column half of each N-tile each). The host picks the number of
+// allocates TMEM and issues tcgen05.mma (one thread), warps 2..17 epilogue in two groups of
+// eight (one TMEM lane quarter and one 64-column half of an N-tile per warp): group 0 makes
+// V and takes the even N-tiles, group 1 the odd ones, so two tiles' epilogues (TMEM reads,
+// the add onto the staged Y rows, the stores) overlap; each group owns one D2 buffer. The host picks the number of
 // N-slices per M-tile from the bytes the busiest SM streams (every slice re-reads its tile's
 // X rows and A_i).
 //
@@ -48,8 +50,10 @@ constexpr int kGM = 128;                 // rows per M-tile (UMMA M)
 constexpr int kGK = 64;                  // K per shrink stage (one 128-byte swizzle atom of 16-bit values)
 constexpr int kGN = 128;                 // columns per expand N-tile
 constexpr int kGStages = 4;              // one ring for both phases: 2 K-steps or 1 N-tile per stage
-constexpr int kGThreads = 320;           // 10 warps: producer, MMA issuer, 8 epilogue warps
-constexpr int kGEpiWarps = 8;            // two per TMEM lane quarter, one per 64-column half of a tile
+constexpr int kGEpiWarps = 8;            // per group: two per TMEM lane quarter, one per 64-column half
+constexpr int kGEpiGroups = 2;           // epilogue groups, taking alternate N-tiles (one D2 buffer each)
+constexpr int kGThreads = 32 * (2 + kGEpiGroups * kGEpiWarps);  // producer, MMA issuer, epilogue groups
+static_assert(kGEpiGroups == 2, "each epilogue group owns one of the two D2 buffers");
 constexpr int kGTmemCols = 512;
 
 inline bool grouped_tc_rank(int r) { return r == 16 || r == 32 || r == 64; }
@@ -464,14 +468,15 @@ __global__ void __launch_bounds__(kGThreads, 1)
     } else {
         // ---------------------------------- epilogue ----------------------------------
         report_rejected();
-        const int quarter = warp & 3;       // TMEM lanes [32*quarter, 32*quarter + 32)
-        const int half = (warp - 2) >> 2;   // columns [64*half, 64*half + 64) of each N-tile
+        const int grp = (warp - 2) / kGEpiWarps;         // this warp's group: N-tiles grp, grp + 2, ...
+        const int quarter = warp & 3;                     // TMEM lanes [32*quarter, 32*quarter + 32)
+        const int half = ((warp - 2) % kGEpiWarps) >> 2;  // columns [64*half, 64*half + 64) of its N-tiles
         const int m = quarter * 32 + lane;
         const uint32_t lane_addr = tmem + (uint32_t(quarter * 32) << 16);
-        // V = D1 -> V_hi + V_lo (K-major, swizzled rows of R values)
-        mbar_wait<false>(&d1_full, 0, P.dev_status, dead);
+        // V = D1 -> V_hi + V_lo (K-major, swizzled rows of R values), by group 0
+        if (grp == 0) mbar_wait<false>(&d1_full, 0, P.dev_status, dead);
         tc_fence_after();
-        for (int c0 = 32 * half; c0 < R; c0 += 64) {  // the two halves share V's columns
+        for (int c0 = 32 * half; grp == 0 && c0 < R; c0 += 64) {  // the two halves share V's columns
             float v[32];
             tmem_ld32(lane_addr + c0, v);
             if (V_OUT) {
@@ -499,17 +504,19 @@ __global__ void __launch_bounds__(kGThreads, 1)
                 }
             }
         }
-        fence_proxy_async();  // generic-proxy writes of V -> tensor-core reads
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_local(&v_full);
+        if (grp == 0) {
+            fence_proxy_async();  // generic-proxy writes of V -> tensor-core reads
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_local(&v_full);
+        }
 
         T* __restrict__ Y = static_cast<T*>(P.Y);
         const bool row_ok = m < rows;
-        for (int nt = 0; nt < n_tiles; ++nt) {
+        for (int nt = grp; nt < n_tiles; nt += kGEpiGroups) {
             const uint32_t it = uint32_t(s_stages + nt);
             const uint32_t st = it % kGStages;
-            const int buf = nt & 1;
+            const int buf = nt & 1;  // == grp
             mbar_wait<false>(&full[st], (it / kGStages) & 1u, P.dev_status, dead);
             mbar_wait<false>(&d2_full[buf], (nt >> 1) & 1u, P.dev_status, dead);
             tc_fence_after();
