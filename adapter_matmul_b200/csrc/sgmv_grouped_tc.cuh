@@ -13,7 +13,7 @@
 //           the expand sees V to about 16 significant bits (the MMA takes 16-bit
 //           operands; V itself is never rounded to one 16-bit value);
 //   expand  D2[128 x 128] (TMEM, fp32) = V_hi @ B_tile + V_lo @ B_tile per N-tile,
-//           double-buffered in TMEM; the epilogue adds scale * D2 to the Y tile,
+//           in four TMEM buffers; the epilogue adds scale * D2 to the Y tile,
 //           rounds once to the storage type and stores only rows inside the segment.
 // Rows of a tile past the segment's end belong to the next segment (or past T, where
 // TMA fills zeros); their results are discarded, so tiles never write across segments.
@@ -25,9 +25,9 @@
 // allocates TMEM and issues tcgen05.mma (one thread), warps 2..17 epilogue in two groups of
 // eight (one TMEM lane quarter and one 64-column half of an N-tile per warp): group 0 makes
 // V and takes the even N-tiles, group 1 the odd ones, so two tiles' epilogues (TMEM reads,
-// the add onto the staged Y rows, the stores) overlap; each group owns one D2 buffer. The host picks the number of
-// N-slices per M-tile from the bytes the busiest SM streams (every slice re-reads its tile's
-// X rows and A_i).
+// the add onto the staged Y rows, the stores) overlap, and the MMAs run up to four N-tiles
+// ahead of the epilogues (four D2 buffers). The host picks the number of N-slices per M-tile
+// from the bytes the busiest SM streams (every slice re-reads its tile's X rows and A_i).
 //
 // Every mbarrier wait is bounded in time; a wait that gives up sets
 // LORA_SGMV_DEV_TIMEOUT and the kernel runs to its end (TMEM is always freed).
@@ -49,11 +49,12 @@ constexpr int kGroupedMinSegment = 128;  // dispatcher: longest segment at least
 constexpr int kGM = 128;                 // rows per M-tile (UMMA M)
 constexpr int kGK = 64;                  // K per shrink stage (one 128-byte swizzle atom of 16-bit values)
 constexpr int kGN = 128;                 // columns per expand N-tile
-constexpr int kGStages = 4;              // one ring for both phases: 2 K-steps or 1 N-tile per stage
+constexpr int kGMaxStages = 8;           // one ring for both phases: 2 K-steps or 1 N-tile per stage
+constexpr int kGSmemMax = 225 * 1024;    // dynamic shared memory the ring and V may fill (+1 KB static)
 constexpr int kGEpiWarps = 8;            // per group: two per TMEM lane quarter, one per 64-column half
-constexpr int kGEpiGroups = 2;           // epilogue groups, taking alternate N-tiles (one D2 buffer each)
+constexpr int kGEpiGroups = 2;           // epilogue groups, taking alternate N-tiles
 constexpr int kGThreads = 32 * (2 + kGEpiGroups * kGEpiWarps);  // producer, MMA issuer, epilogue groups
-static_assert(kGEpiGroups == 2, "each epilogue group owns one of the two D2 buffers");
+constexpr int kGD2Bufs = 4;              // D2 accumulators in TMEM (128 columns each; D1 shares buffer 0)
 constexpr int kGTmemCols = 512;
 
 inline bool grouped_tc_rank(int r) { return r == 16 || r == 32 || r == 64; }
@@ -78,7 +79,7 @@ struct GroupedParams {
     float scale;
     int nsplit;  // N-slices of H2
     int nspan;   // columns per N-slice (multiple of kGN)
-    int tm;      // rows per M-tile, 8..128 (the MMA's M stays 128; rows past tm are never used)
+    int tm;      // rows per M-tile, 64..128, a multiple of 8 (the MMA's M stays 128; rows past tm are never used)
     float* v_out;  // V-only mode: V [T, r] fp32 written here, no expand
     const int32_t* ranks;  // rank of each adapter (device), or null: every adapter has rank R
 };
@@ -94,21 +95,37 @@ __device__ __forceinline__ int segment_rank(const GroupedParams& P, int s) {
     return (rs >= 8 && rs <= R && rs % 8 == 0) ? rs : 0;
 }
 
+// Ring stages are sized for the M-tile's tm rows (a multiple of 8), so short tiles give a
+// deeper ring. Shrink stage: two K-steps, [X box 0][X box 1][A tile 0][A tile 1]: X boxes of
+// tm rows x 64 columns (TMA, 128B swizzle, tm * 128 bytes each), A_i tiles [64 x R]
+// (MN-major). Expand stage: [Y box 0][Y box 1][B_i tile]: the N-tile's Y rows as two boxes of
+// tm rows x 64 columns, and B_i [R x 128] (MN-major). Every part starts on a 1024-byte
+// boundary. The MMAs still read 128 rows (M = 128): an X operand spans 16 KB from its box,
+// past the tm loaded rows into the rest of the ring or the V buffers after it, and the rows
+// past tm only reach results that are discarded.
+__host__ __device__ constexpr int grouped_a_slot(int r) { return (64 * r * 2 + 1023) / 1024 * 1024; }
+__host__ __device__ constexpr int grouped_stage_bytes(int r, int tm) {
+    return 2 * tm * 128 + (2 * grouped_a_slot(r) > r * kGN * 2 ? 2 * grouped_a_slot(r) : r * kGN * 2);
+}
+__host__ __device__ constexpr int grouped_stages(int r, int tm) {
+    return (kGSmemMax - 1024 - 2 * kGM * r * 2) / grouped_stage_bytes(r, tm) < kGMaxStages
+               ? (kGSmemMax - 1024 - 2 * kGM * r * 2) / grouped_stage_bytes(r, tm)
+               : kGMaxStages;
+}
+__host__ __device__ constexpr size_t grouped_smem_bytes(int r, int tm) {
+    return size_t(grouped_stages(r, tm)) * grouped_stage_bytes(r, tm) + 2 * size_t(kGM) * r * 2 +
+           1024 /* alignment slack */;
+}
+static_assert(grouped_stages(64, 128) >= 4 && grouped_stages(16, 128) >= 4, "the ring holds at least four stages");
+// the X operand read from box 1 of the last stage stays inside the allocation
+static_assert(64 * 128 + kGM * 128 <= grouped_stage_bytes(16, 64) + 2 * kGM * 16 * 2, "X operand span");
+
 template <int R>
 struct GroupedGeom {
-    // shrink stage: two K-steps, [X tile 0][X tile 1][A tile 0][A tile 1]: X tiles [128 x 64]
-    // (TMA, 128B swizzle; tm rows loaded), A_i tiles [64 x R] (MN-major)
-    static constexpr int X_BYTES = kGM * kGK * 2;
     static constexpr int A_BYTES = kGK * R * 2;
-    static constexpr int A_SLOT = ((A_BYTES + 1023) / 1024) * 1024;
-    static constexpr int SSTAGE = 2 * X_BYTES + 2 * A_SLOT;
-    // expand stage: Y tile [128 x 128] as two 64-column TMA boxes + B_i tile [R x 128] (MN-major)
-    static constexpr int Y_BYTES = kGM * kGN * 2;
+    static constexpr int A_SLOT = grouped_a_slot(R);
     static constexpr int B_BYTES = R * kGN * 2;
-    static constexpr int ESTAGE = Y_BYTES + B_BYTES;
-    static constexpr int STAGE = SSTAGE > ESTAGE ? SSTAGE : ESTAGE;
     static constexpr int V_BYTES = kGM * R * 2;  // one of V_hi, V_lo
-    static constexpr size_t SMEM = size_t(kGStages) * STAGE + 2 * size_t(V_BYTES) + 1024 /* alignment slack */;
     // swizzle of an MN-major A_i tile (rows of R 16-bit values) and of K-major V rows
     static constexpr int SW_BITS = R == 64 ? 3 : (R == 32 ? 2 : 1);           // 128B, 64B, 32B
     static constexpr uint64_t SW_TYPE = R == 64 ? 2 : (R == 32 ? 4 : 6);      // descriptor layout type
@@ -254,12 +271,15 @@ __global__ void __launch_bounds__(kGThreads, 1)
     extern __shared__ __align__(1024) unsigned char gsmem_raw[];
     // 1024-byte alignment for the swizzled tiles
     unsigned char* gsmem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(gsmem_raw) + 1023) & ~uintptr_t(1023));
+    const int NS = grouped_stages(R, P.tm);           // ring stages
+    const int SB = grouped_stage_bytes(R, P.tm);      // bytes per stage
+    const int BOX = P.tm * 128;                       // one X or Y box of tm rows
     unsigned char* ring = gsmem;
-    unsigned char* vhi = ring + kGStages * G::STAGE;
+    unsigned char* vhi = ring + size_t(NS) * SB;
     unsigned char* vlo = vhi + G::V_BYTES;
 
-    __shared__ __align__(8) uint64_t full[kGStages], empty[kGStages];
-    __shared__ __align__(8) uint64_t d1_full, v_full, d2_full[2], d2_empty[2];
+    __shared__ __align__(8) uint64_t full[kGMaxStages], empty[kGMaxStages];
+    __shared__ __align__(8) uint64_t d1_full, v_full, d2_full[kGD2Bufs], d2_empty[kGD2Bufs];
     __shared__ __align__(128) CUtensorMap map_build[2];
     __shared__ uint32_t tmem_base_s;
     __shared__ int job_s[3];
@@ -296,14 +316,14 @@ __global__ void __launch_bounds__(kGThreads, 1)
         }
     };
     if (threadIdx.x == 0) {
-        for (int i = 0; i < kGStages; ++i) {
+        for (int i = 0; i < NS; ++i) {
             mbar_init(&full[i], 1);       // producer expect_tx; the TMA copies complete the bytes
             mbar_init(&empty[i], 1 + kGEpiWarps);  // MMA commit + 8 arrivals (the MMA thread for shrink
                                           // stages, the epilogue warps for expand stages)
         }
         mbar_init(&d1_full, 1);
         mbar_init(&v_full, kGEpiWarps);
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < kGD2Bufs; ++i) {
             mbar_init(&d2_full[i], 1);
             mbar_init(&d2_empty[i], kGEpiWarps);
         }
@@ -335,7 +355,8 @@ __global__ void __launch_bounds__(kGThreads, 1)
     const int k_steps = (P.H1 + kGK - 1) / kGK;
     const int s_stages = (k_steps + 1) / 2;  // shrink stages of two K-steps (the last may hold one)
 
-    // TMEM: D1 at columns [0, R), D2 buffers at 128 and 256
+    // TMEM: D2 buffers at columns 0, 128, 256 and 384; D1 at [0, R), inside buffer 0, which
+    // the first expand MMA overwrites only after V has been read from it (v_full)
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tmem_base_s)),
                      "r"(kGTmemCols)
@@ -376,30 +397,30 @@ __global__ void __launch_bounds__(kGThreads, 1)
         __syncwarp();
         uint32_t it = 0;
         for (int ss = 0; ss < s_stages; ++ss, ++it) {
-            const uint32_t st = it % kGStages;
-            if (it >= kGStages) mbar_wait<false>(&empty[st], ((it / kGStages) - 1) & 1u, P.dev_status, dead);
-            unsigned char* xs = ring + st * G::STAGE;
+            const uint32_t st = it % NS;
+            if (it >= uint32_t(NS)) mbar_wait<false>(&empty[st], ((it / NS) - 1) & 1u, P.dev_status, dead);
+            unsigned char* xs = ring + size_t(st) * SB;
             const int nks = min(2, k_steps - 2 * ss);
             if (lane == 0) {
                 mbar_arrive_expect_tx(&full[st], uint32_t(nks) * (uint32_t(P.tm) * kGK * 2 + G::A_BYTES));
                 for (int h = 0; h < nks; ++h) {
                     const int ks = 2 * ss + h;
-                    tma_load_2d(xs + h * G::X_BYTES, &tmX, ks * kGK, t0, &full[st]);
-                    tma_load_2d(xs + 2 * G::X_BYTES + h * G::A_SLOT, gA, 0, ks * kGK, &full[st]);
+                    tma_load_2d(xs + h * BOX, &tmX, ks * kGK, t0, &full[st]);
+                    tma_load_2d(xs + 2 * BOX + h * G::A_SLOT, gA, 0, ks * kGK, &full[st]);
                 }
             }
             __syncwarp();
         }
         for (int nt = 0; nt < n_tiles; ++nt, ++it) {
-            const uint32_t st = it % kGStages;
-            if (it >= kGStages) mbar_wait<false>(&empty[st], ((it / kGStages) - 1) & 1u, P.dev_status, dead);
-            unsigned char* ys = ring + st * G::STAGE;
-            unsigned char* bs = ys + G::Y_BYTES;
+            const uint32_t st = it % NS;
+            if (it >= uint32_t(NS)) mbar_wait<false>(&empty[st], ((it / NS) - 1) & 1u, P.dev_status, dead);
+            unsigned char* ys = ring + size_t(st) * SB;
+            unsigned char* bs = ys + 2 * BOX;
             const int n0 = n_lo + nt * kGN;
             if (lane == 0) {
                 mbar_arrive_expect_tx(&full[st], 2u * P.tm * 64 * 2 + G::B_BYTES);
                 tma_load_2d(ys, &tmY, n0, t0, &full[st]);
-                tma_load_2d(ys + G::Y_BYTES / 2, &tmY, n0 + 64, t0, &full[st]);
+                tma_load_2d(ys + BOX, &tmY, n0 + 64, t0, &full[st]);
                 tma_load_2d(bs, gB, n0, 0, &full[st]);
                 tma_load_2d(bs + R * 128, gB, n0 + 64, 0, &full[st]);
             }
@@ -407,8 +428,8 @@ __global__ void __launch_bounds__(kGThreads, 1)
         }
         // every copy issued lands before the CTA may exit
         if (lane == 0)
-            for (uint32_t i = it > uint32_t(kGStages) ? it - kGStages : 0u; i < it; ++i)
-                drain_wait(&full[i % kGStages], (i / kGStages) & 1u);
+            for (uint32_t i = it > uint32_t(NS) ? it - NS : 0u; i < it; ++i)
+                drain_wait(&full[i % NS], (i / NS) & 1u);
         __syncwarp();
     } else if (warp == 1) {
         // ---------------------------------- MMA issuer ----------------------------------
@@ -417,15 +438,15 @@ __global__ void __launch_bounds__(kGThreads, 1)
         const uint32_t idesc_e = instr_desc(fmt, 0, 1, kGN, kGM);  // V K-major, B_i MN-major, N = 128
         uint32_t it = 0;
         for (int ss = 0; ss < s_stages; ++ss, ++it) {
-            const uint32_t st = it % kGStages;
-            mbar_wait<false>(&full[st], (it / kGStages) & 1u, P.dev_status, dead);
+            const uint32_t st = it % NS;
+            mbar_wait<false>(&full[st], (it / NS) & 1u, P.dev_status, dead);
             tc_fence_after();
             if (lane == 0) {
                 const int nks = min(2, k_steps - 2 * ss);
-                const uint32_t xa0 = smem_u32(ring + st * G::STAGE);
+                const uint32_t xa0 = smem_u32(ring + size_t(st) * SB);
                 for (int h = 0; h < nks; ++h) {
-                    const uint32_t xa = xa0 + h * G::X_BYTES;
-                    const uint32_t aa = xa0 + 2 * G::X_BYTES + h * G::A_SLOT;
+                    const uint32_t xa = xa0 + h * BOX;
+                    const uint32_t aa = xa0 + 2 * BOX + h * G::A_SLOT;
 #pragma unroll
                     for (int kk = 0; kk < kGK / 16; ++kk) {
                         const uint64_t adesc = smem_desc(xa + kk * 32, 16, 1024, 2);
@@ -444,14 +465,14 @@ __global__ void __launch_bounds__(kGThreads, 1)
         mbar_wait<false>(&v_full, 0, P.dev_status, dead);
         tc_fence_after();
         for (int nt = 0; nt < n_tiles; ++nt, ++it) {
-            const uint32_t st = it % kGStages;
-            const int buf = nt & 1;
-            if (nt >= 2) mbar_wait<false>(&d2_empty[buf], ((nt >> 1) - 1) & 1u, P.dev_status, dead);
-            mbar_wait<false>(&full[st], (it / kGStages) & 1u, P.dev_status, dead);
+            const uint32_t st = it % NS;
+            const int buf = nt % kGD2Bufs;
+            if (nt >= kGD2Bufs) mbar_wait<false>(&d2_empty[buf], ((nt / kGD2Bufs) - 1) & 1u, P.dev_status, dead);
+            mbar_wait<false>(&full[st], (it / NS) & 1u, P.dev_status, dead);
             tc_fence_after();
             if (lane == 0) {
-                const uint32_t ba = smem_u32(ring + st * G::STAGE + G::Y_BYTES);
-                const uint32_t d2 = tmem + 128u + 128u * buf;
+                const uint32_t ba = smem_u32(ring + size_t(st) * SB + 2 * BOX);
+                const uint32_t d2 = tmem + 128u * buf;
 #pragma unroll
                 for (int kk = 0; kk < R / 16; ++kk) {
                     const uint64_t bdesc = smem_desc(ba + kk * 16 * 128, R * 128, 1024, 2);
@@ -515,20 +536,20 @@ __global__ void __launch_bounds__(kGThreads, 1)
         const bool row_ok = m < rows;
         for (int nt = grp; nt < n_tiles; nt += kGEpiGroups) {
             const uint32_t it = uint32_t(s_stages + nt);
-            const uint32_t st = it % kGStages;
-            const int buf = nt & 1;  // == grp
-            mbar_wait<false>(&full[st], (it / kGStages) & 1u, P.dev_status, dead);
-            mbar_wait<false>(&d2_full[buf], (nt >> 1) & 1u, P.dev_status, dead);
+            const uint32_t st = it % NS;
+            const int buf = nt % kGD2Bufs;
+            mbar_wait<false>(&full[st], (it / NS) & 1u, P.dev_status, dead);
+            mbar_wait<false>(&d2_full[buf], (nt / kGD2Bufs) & 1u, P.dev_status, dead);
             tc_fence_after();
-            unsigned char* ys = ring + st * G::STAGE;
+            unsigned char* ys = ring + size_t(st) * SB;
             const int n0 = n_lo + nt * kGN;
             // row m of the tile: y + scale * D2, written back over the staged Y row
 #pragma unroll 1
             for (int c0 = 64 * half; c0 < 64 * half + 64; c0 += 32) {
                 float acc[32];
-                tmem_ld32(lane_addr + 128u + 128u * buf + c0, acc);
+                tmem_ld32(lane_addr + 128u * buf + c0, acc);
                 if (row_ok) {
-                    unsigned char* yb = ys + (c0 / 64) * (G::Y_BYTES / 2);
+                    unsigned char* yb = ys + (c0 / 64) * BOX;
 #pragma unroll
                     for (int ch = 0; ch < 4; ++ch) {
                         if (n0 + c0 + ch * 8 < n_hi) {
@@ -552,7 +573,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
                 const int col = n0 + half * 64 + c * 8;
                 if (rr < rows && col < n_hi)
                     st_vec(Y + size_t(t0 + rr) * P.H2 + col,
-                           *reinterpret_cast<const uint4*>(ys + half * (G::Y_BYTES / 2) + swz(rr, c, 3)));
+                           *reinterpret_cast<const uint4*>(ys + half * BOX + swz(rr, c, 3)));
             }
             // the TMEM reads completed at tcgen05.wait::ld; no tcgen05 fence here (it would also
             // wait for the Y stores just issued)
@@ -610,15 +631,16 @@ template <typename T, int R, bool V_OUT = false>
 inline cudaError_t launch_grouped_tc_kernel(const CUtensorMap& tmX, const CUtensorMap& tmY, const CUtensorMap& tmA,
                                             const CUtensorMap& tmB, const GroupedParams& P, int blocks,
                                             cudaStream_t stream) {
-    using G = GroupedGeom<R>;
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(once, [] {
         attr_err = cudaFuncSetAttribute(sgmv_grouped_tc_kernel<T, R, V_OUT>,
-                                        cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(G::SMEM));
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, kGSmemMax);
     });
     if (attr_err != cudaSuccess) return attr_err;
-    sgmv_grouped_tc_kernel<T, R, V_OUT><<<blocks, kGThreads, G::SMEM, stream>>>(tmX, tmY, tmA, tmB, P);
+    if (P.tm < 64 || P.tm > kGM || P.tm % 8 != 0) return cudaErrorInvalidValue;  // the X span assumes tm >= 64
+    sgmv_grouped_tc_kernel<T, R, V_OUT><<<blocks, kGThreads, grouped_smem_bytes(R, P.tm), stream>>>(tmX, tmY, tmA, tmB,
+                                                                                                    P);
     return cudaGetLastError();
 }
 
