@@ -63,26 +63,27 @@ PER_CONFIG_MAX_STEPS = 500
 
 
 # DRAM bytes (read + write) of one launch of the dominant kernel, from one ncu capture of the
-# same launch (summaries under profiles/). A figure holds only while the kernel's sources are
-# those it was taken from: their SHA-256 is stored with it and checked here, else "traffic"
-# is null. For a call of two launches (the split forms) the figure is the pair's.
+# same launch (summaries under profiles/). A figure holds only while the sources it was taken
+# from (the kernel's headers, those they include, and the host code that sizes its launch) are
+# unchanged: their SHA-256 is stored with it and checked here, else "traffic" is null. For a
+# call of two launches (the split forms) the figure is the pair's.
 TRAFFIC = {
     # profiles/fused_kernel_distinct_decode.md
-    "distinct": {"bytes": 35721728,
-        "sources": ["sgmv_fused.cuh", "sgmv_common.cuh"],
-        "sha256": "6552c4033b5e2540a7d033f2b197baf0c9ddf3269fb04823340175560c568ce3"},
+    "distinct": {"bytes": 35721472,
+        "sources": ["sgmv_fused.cuh", "sgmv_common.cuh", "lora_sgmv_api.cu"],
+        "sha256": "c75727b99e65aad5eaf86614ba92741c19238003af87b656d7bfbc5676c5f0d1"},
     # profiles/split_tc_llama70b_decode_h28672.md
-    "llama70b_decode_h28672": {"bytes": 487882240,
-        "sources": ["sgmv_split.cuh", "sgmv_decode_tc.cuh", "sgmv_tmap.cuh", "sgmv_common.cuh"],
-        "sha256": "2f4ca4bccd23f9e27a7a0882206b3f1e56ab53ed9fd8d1ff33e14bff919d4ba2"},
+    "llama70b_decode_h28672": {"bytes": 489396992,
+        "sources": ["sgmv_split.cuh", "sgmv_decode_tc.cuh", "sgmv_grouped_tc.cuh", "sgmv_fused.cuh", "sgmv_tmap.cuh", "sgmv_common.cuh", "lora_sgmv_api.cu"],
+        "sha256": "f7220a666f350c3aefb70827ba5912fbf3de7d8457f1a6c1bb946c4cbf30d08a"},
     # profiles/split_tc_llama70b_decode_h8192.md
-    "llama70b_decode_h8192": {"bytes": 214965248,
-        "sources": ["sgmv_split.cuh", "sgmv_decode_tc.cuh", "sgmv_tmap.cuh", "sgmv_common.cuh"],
-        "sha256": "2f4ca4bccd23f9e27a7a0882206b3f1e56ab53ed9fd8d1ff33e14bff919d4ba2"},
+    "llama70b_decode_h8192": {"bytes": 216834304,
+        "sources": ["sgmv_split.cuh", "sgmv_decode_tc.cuh", "sgmv_grouped_tc.cuh", "sgmv_fused.cuh", "sgmv_tmap.cuh", "sgmv_common.cuh", "lora_sgmv_api.cu"],
+        "sha256": "f7220a666f350c3aefb70827ba5912fbf3de7d8457f1a6c1bb946c4cbf30d08a"},
     # profiles/grouped_kernel_prefill.md
-    "prefill": {"bytes": 191557632,
-        "sources": ["sgmv_grouped_tc.cuh", "sgmv_tmap.cuh", "sgmv_common.cuh"],
-        "sha256": "d53cce5554111c3e8dcfa0032527bc110d620edeab4f8db89b87783a60599e2f"},
+    "prefill": {"bytes": 190224128,
+        "sources": ["sgmv_grouped_tc.cuh", "sgmv_fused.cuh", "sgmv_tmap.cuh", "sgmv_common.cuh", "lora_sgmv_api.cu"],
+        "sha256": "6b1175797d7915a676608b429a5a65442a18742c4b9603669442de2fbc5d4973"},
 }
 
 
