@@ -47,7 +47,7 @@ EXPORTS = [
     "lora_sgmv_group_segments", "lora_sgmv_shrink", "lora_sgmv_expand", "lora_sgmv_workspace_bytes",
     "lora_sgmv_apply", "lora_sgmv_apply_ex", "lora_sgmv_apply_batched", "lora_sgmv_apply_noalloc",
     "lora_sgmv_pad_rank", "lora_sgmv_auto_variant", "lora_sgmv_apply_flags", "lora_sgmv_apply_batched_flags",
-    "lora_sgmv_gemm_apply", "lora_sgmv_apply_ranks",
+    "lora_sgmv_gemm_apply", "lora_sgmv_apply_ranks", "lora_sgmv_step_host",
 ]
 
 
@@ -56,6 +56,12 @@ class Problem(ctypes.Structure):
     _fields_ = [("Y", ctypes.c_void_p), ("X", ctypes.c_void_p), ("A_ptrs", ctypes.c_void_p),
                 ("B_ptrs", ctypes.c_void_p), ("num_adapters", ctypes.c_int32), ("H1", ctypes.c_int32),
                 ("H2", ctypes.c_int32), ("scale", ctypes.c_float)]
+
+
+class Copy(ctypes.Structure):
+    """Mirror of lora_sgmv_copy."""
+    _fields_ = [("src", ctypes.c_void_p), ("dst", ctypes.c_void_p), ("bytes", ctypes.c_size_t)]
+
 
 _lock = threading.Lock()
 _lib = None
@@ -130,6 +136,9 @@ def load(path: Optional[str] = None):
         lib.lora_sgmv_auto_variant.argtypes = [i32, i32, i32, i32, i32, ctypes.c_int, i32, i32]
         lib.lora_sgmv_pad_rank.restype = ctypes.c_int
         lib.lora_sgmv_pad_rank.argtypes = [P, P, P, P, i32, i32, i32, i32, ctypes.c_int, P]
+        lib.lora_sgmv_step_host.restype = ctypes.c_int
+        lib.lora_sgmv_step_host.argtypes = [P, i32, i32, P, P, P, P, i32, P, i32, i32, ctypes.c_int,
+                                            ctypes.c_uint32, P, i32, P, P, P]
         if path is None:
             _lib = lib
         return lib
@@ -321,3 +330,30 @@ def pointer_table(tensors: Sequence, device=None):
     ptrs = [t.data_ptr() for t in tensors]
     dev = device if device is not None else (tensors[0].device if tensors else "cuda")
     return torch.tensor(ptrs, dtype=torch.int64, device=dev)
+
+
+class HostStep:
+    """lora_sgmv_step_host with its arguments marshalled once: a serving loop calls run(stream)
+    per step. ids_host, meta_host (pinned) and perm are host arrays (numpy, or pointers);
+    meta_dev is device memory; h2d and d2h are sequences of (src, dst, bytes); problems as for
+    lora_sgmv_apply_batched. The contents of ids_host are read at each run."""
+
+    def __init__(self, ids_host, T: int, num_adapters: int, meta_host, meta_dev, h2d, problems, r: int,
+                 dtype: int, d2h, flags: int = 0, perm=None, dev_status=None):
+        self._lib = load()
+        self._probs = _problem_array(problems)
+        self._h2d = (Copy * max(1, len(h2d)))(*[Copy(_p(a), _p(b), int(n)) for a, b, n in h2d])
+        self._d2h = (Copy * max(1, len(d2h)))(*[Copy(_p(a), _p(b), int(n)) for a, b, n in d2h])
+        self._n = ctypes.c_int32(0)
+        self._args = [_p(ids_host), int(T), int(num_adapters), _p(meta_host), _p(meta_dev), _p(perm),
+                      ctypes.addressof(self._h2d), len(h2d), ctypes.addressof(self._probs), len(problems), int(r),
+                      int(dtype), int(flags), ctypes.addressof(self._d2h), len(d2h), _p(dev_status),
+                      ctypes.addressof(self._n)]
+        self._fn = self._lib.lora_sgmv_step_host
+
+    def run(self, stream) -> int:
+        """Enqueue one step on `stream` (a cudaStream_t as int, or a torch stream); returns n."""
+        st = self._fn(*self._args, _stream(stream))
+        if st != 0:
+            raise SGMVError(st, "lora_sgmv_step_host")
+        return self._n.value

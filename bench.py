@@ -29,10 +29,12 @@ Identical decode batches per layer of four projections and per single call, the 
 and the 70B-shaped decode per call), each with its dispatched kernels, algorithmic bytes
 and roofline fraction.
 
-"e2e" is the same metric through the public calls with host buffers: each step groups
-the token batch on the host, copies the segment arrays and the projections' X and Y from
-pinned host memory, runs the SGMV launch and copies Y back, double-buffered on three
-streams so that one step's copies overlap the next step's. Timed by the host clock.
+"e2e" is the same metric through the public calls with host buffers: each step is one
+lora_sgmv_step_host call, which groups the token batch on the host, copies the segment arrays
+and the projections' X and Y from pinned host memory, runs the batched SGMV launch and copies Y
+back, after which the host reads Y; three buffer sets on their own streams, so that one step's
+copies overlap the previous steps'. Timed by the host clock. (A workload of one projection runs
+lora_sgmv_apply between the copies instead.)
 
 Multi-GPU (torchrun): every rank runs its own replica of the workload (the path has no
 cross-GPU data exchange); value = all ranks' tokens / max time.
@@ -795,13 +797,97 @@ def run_ours(args, spec: Spec, rank: int, world: int, local: int):
 
 
 def run_e2e(args, ds: DeviceSpec, stream, world: int, dev) -> dict:
-    """The metric through the public calls with host buffers. Per step: group the batch's adapter
-    ids on the host (lora_sgmv_group_segments), copy the segment arrays and every projection's X
-    and Y from pinned host memory (one packed copy), run the step's SGMV launch
-    (lora_sgmv_apply_batched, or lora_sgmv_apply for one projection), copy Y back to pinned host
-    memory and read it there. Two buffer sets and three streams (host-to-device copies, compute,
-    device-to-host copies): step i's copy in overlaps step i-1's launch and copy out; a buffer
-    set is reused only after its previous step's result has been read. Host wall clock."""
+    if ds.spec.P > 1:
+        return run_e2e_step_host(args, ds, world, dev)
+    return run_e2e_single(args, ds, stream, world, dev)
+
+
+def run_e2e_step_host(args, ds: DeviceSpec, world: int, dev) -> dict:
+    """The metric through the library's host-memory serving call, lora_sgmv_step_host, one call
+    per step: it groups the batch's adapter ids on the host, copies the segment arrays and every
+    projection's X and Y from pinned host memory (one packed copy), runs the batched SGMV launch
+    and copies Y back to pinned host memory, all enqueued on one stream; the host then reads the
+    result. Three buffer sets, each with its own stream: step i's copy in overlaps the launches
+    and copies out of steps i-1 and i-2, and a buffer set is reused only after its previous
+    step's result has been read. Host wall clock."""
+    import torch
+
+    sgmv, spec, w = ds.sgmv, ds.spec, ds.spec.w
+    P, NB = spec.P, 3
+    steps = max(3, min(args.steps, 200))
+    meta_bytes = ((2 * w.num_adapters + 1) * 4 + 255) // 256 * 256
+    x_bytes, y_bytes = P * w.T * w.H1 * 2, P * w.T * w.H2 * 2
+    in_bytes = meta_bytes + x_bytes + y_bytes
+    h_in = torch.empty((NB, in_bytes), dtype=torch.uint8, pin_memory=True)
+    d_in = torch.empty((NB, in_bytes), dtype=torch.uint8, device=dev)
+    outY = torch.empty((NB, y_bytes), dtype=torch.uint8, pin_memory=True)
+    hX = torch.stack([ds.calls[0][p][0] for p in range(P)]).cpu().view(torch.uint8).reshape(-1)
+    hY = torch.stack([ds.calls[0][p][1] for p in range(P)]).cpu().view(torch.uint8).reshape(-1)
+    for b in range(NB):  # the step's inputs, staged once in pinned memory (copied every step)
+        h_in[b, meta_bytes:meta_bytes + x_bytes].copy_(hX)
+        h_in[b, meta_bytes + x_bytes:].copy_(hY)
+    ids = np.ascontiguousarray(w.ids, dtype=np.int32)
+    hb = [h_in[b].data_ptr() for b in range(NB)]
+    db = [d_in[b].data_ptr() for b in range(NB)]
+    ob = [outY[b].data_ptr() for b in range(NB)]
+    runs = [[sgmv.HostStep(
+        ids, w.T, w.num_adapters, hb[b], db[b], [(hb[b], db[b], in_bytes)],
+        [sgmv.Problem(db[b] + meta_bytes + x_bytes + p * w.T * w.H2 * 2, db[b] + meta_bytes + p * w.T * w.H1 * 2,
+                      ds.calls[l][p][2].data_ptr(), ds.calls[l][p][3].data_ptr(), w.num_adapters, w.H1, w.H2,
+                      w.scale) for p in range(P)],
+        w.r, ds.dt, [(db[b] + meta_bytes + x_bytes, ob[b], y_bytes)]) for l in range(spec.L)] for b in range(NB)]
+    streams = [torch.cuda.Stream(device=dev) for _ in range(NB)]
+    sh = [s.cuda_stream for s in streams]
+    done = [torch.cuda.Event() for _ in range(NB)]
+    used = [False] * NB
+    out_np = [outY[b].numpy() for b in range(NB)]
+    sink = [0]
+
+    def one(i):
+        b, l = i % NB, i % spec.L
+        if used[b]:
+            done[b].synchronize()  # step i-NB: its copies are done, its result is read
+            sink[0] ^= int(out_np[b][0])
+        used[b] = True
+        runs[b][l].run(sh[b])
+        done[b].record(streams[b])
+
+    def drain():
+        for b in range(NB):
+            if used[b]:
+                done[b].synchronize()
+                sink[0] ^= int(out_np[b][0])
+                used[b] = False
+
+    for i in range(3):
+        one(i)
+    drain()
+    torch.cuda.synchronize()
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+    t0 = time.perf_counter()
+    for i in range(steps):
+        one(i)
+    drain()
+    el = max_over_ranks(time.perf_counter() - t0, world, dev)
+    return {"value": round(job_tokens_per_s(w.T * steps, world, el), 1), "unit": UNIT,
+            "h2d_bytes_per_step": int(in_bytes), "d2h_bytes_per_step": int(y_bytes), "steps": steps,
+            "note": "host wall clock, slowest rank; per step one lora_sgmv_step_host call: host grouping, one "
+                    f"pinned H2D of the segment arrays with X and Y ({P} projections), 1 batched SGMV launch, "
+                    "D2H of Y, then the host reads Y; three buffer sets, each on its own stream, so one step's "
+                    "copy in overlaps the previous steps' launches and copies out"}
+
+
+def run_e2e_single(args, ds: DeviceSpec, stream, world: int, dev) -> dict:
+    """The metric through the public calls with host buffers, for a workload of one projection.
+    Per step: group the batch's adapter ids on the host (lora_sgmv_group_segments), copy the
+    segment arrays with X and Y from pinned host memory (one packed copy), run lora_sgmv_apply,
+    copy Y back to pinned host memory and read it there. Two buffer sets and three streams
+    (host-to-device copies, compute, device-to-host copies): step i's copy in overlaps step
+    i-1's launch and copy out; a buffer set is reused only after its previous step's result has
+    been read. Host wall clock."""
     import torch
 
     sgmv, spec, w = ds.sgmv, ds.spec, ds.spec.w
@@ -858,12 +944,9 @@ def run_e2e(args, ds: DeviceSpec, stream, world: int, dev) -> dict:
             d_in[b].copy_(h_in[b], non_blocking=True)
         ev_in[b].record(s_in)
         stream.wait_event(ev_in[b])
-        if P > 1:
-            sgmv.lora_sgmv_apply_batched(problems[b][l], d_seg, d_idx, n, w.T, w.r, ds.dt, max_len, None, stream)
-        else:
-            q = problems[b][l][0]
-            sgmv.lora_sgmv_apply(q.Y, q.X, q.A_ptrs, q.B_ptrs, d_seg, d_idx, n, w.num_adapters, w.T, w.H1, w.r,
-                                 w.H2, w.scale, ds.dt, max_len, ws[b], ds.ws_bytes, None, stream)
+        q = problems[b][l][0]
+        sgmv.lora_sgmv_apply(q.Y, q.X, q.A_ptrs, q.B_ptrs, d_seg, d_idx, n, w.num_adapters, w.T, w.H1, w.r,
+                             w.H2, w.scale, ds.dt, max_len, ws[b], ds.ws_bytes, None, stream)
         ev_run[b].record(stream)
         s_out.wait_event(ev_run[b])
         with torch.cuda.stream(s_out):
@@ -891,11 +974,10 @@ def run_e2e(args, ds: DeviceSpec, stream, world: int, dev) -> dict:
         one(i)
     drain()
     el = max_over_ranks(time.perf_counter() - t0, world, dev)
-    call = "1 lora_sgmv_apply_batched launch" if P > 1 else "1 lora_sgmv_apply call"
     return {"value": round(job_tokens_per_s(w.T * steps, world, el), 1), "unit": UNIT,
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": steps,
             "note": "host wall clock, slowest rank; per step: host grouping, one pinned H2D of the segment "
-                    f"arrays with X and Y ({P} projections), {call}, D2H of Y read on the host; two buffer "
+                    "arrays with X and Y, 1 lora_sgmv_apply call, D2H of Y read on the host; two buffer "
                     "sets on three streams, so one step's copy in overlaps the previous step's launch and "
                     "copy out"}
 

@@ -443,6 +443,55 @@ lora_sgmv_status lora_sgmv_apply_noalloc(void* Y, const void* X, const void* con
                                          int32_t H2, float scale, lora_sgmv_dtype dtype,
                                          int32_t max_seg_len, uint32_t* dev_status, void* stream);
 
+/* One copy for lora_sgmv_step_host: bytes from src to dst. */
+typedef struct {
+    const void* src;
+    void* dst;
+    size_t bytes;
+} lora_sgmv_copy;
+
+/*
+ * lora_sgmv_step_host -- one serving step whose batch lives in host memory.
+ *
+ * The segmented batch of the multi-LoRA paragraph (page "Punica：多 LoRA
+ * 模型统一服务框架", the Punica README) as one call a serving loop makes per
+ * step, with every piece enqueued on `stream` and nothing waited for:
+ *   1. groups ids (host, int32[T], the adapter of each batch token) as
+ *      lora_sgmv_group_segments does, writing seg_starts (n + 1 entries)
+ *      then lora_idx (n entries) to meta_host[0 .. 2n + 1), and perm to
+ *      `perm` (host, int32[T]; NULL: not returned). Rows of every problem's
+ *      X and Y are taken in grouped order: row p belongs to batch token
+ *      perm[p];
+ *   2. copies h2d[0 .. n_h2d) host -> device in order (cudaMemcpyAsync);
+ *      one of them must carry meta_host to meta_dev, and they must fill the
+ *      problems' X and Y;
+ *   3. runs lora_sgmv_apply_batched_flags(problems, n_problems, meta_dev,
+ *      meta_dev + n + 1, n, T, r, dtype, the longest segment, flags,
+ *      dev_status) unless n == 0;
+ *   4. copies d2h[0 .. n_d2h) device -> host in order.
+ *   meta_host    host, int32[2 * num_adapters + 1]; pinned, so that its copy
+ *                is asynchronous.
+ *   meta_dev     device, int32[2 * num_adapters + 1].
+ *   h2d, d2h     host arrays of copies (src, dst, bytes); the host side of
+ *                each should be pinned memory.
+ *   n_segments_out  host, int32 out (may be NULL): n.
+ *   other arguments as for lora_sgmv_apply_batched_flags.
+ * meta_host and every host range must not be written (nor, for d2h, read)
+ * until the step's copies are done: record an event on `stream` after the
+ * call and wait for it. Returns LORA_SGMV_ERR_NULL, _DIM or _RANGE (an id
+ * out of range) before anything is enqueued; LORA_SGMV_ERR_CUDA when a copy
+ * cannot be enqueued (cudaGetLastError holds the cause); a launch error of
+ * step 3 after the copies in were enqueued (the copies out are then not
+ * enqueued); else LORA_SGMV_OK.
+ */
+lora_sgmv_status lora_sgmv_step_host(const int32_t* ids, int32_t T, int32_t num_adapters,
+                                     int32_t* meta_host, const int32_t* meta_dev, int32_t* perm,
+                                     const lora_sgmv_copy* h2d, int32_t n_h2d,
+                                     const lora_sgmv_problem* problems, int32_t n_problems, int32_t r,
+                                     lora_sgmv_dtype dtype, uint32_t flags, const lora_sgmv_copy* d2h,
+                                     int32_t n_d2h, uint32_t* dev_status, int32_t* n_segments_out,
+                                     void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -276,3 +276,29 @@ def test_flags_other_than_early_reads_are_refused():
     # the one defined flag passes validation (an empty batch then returns OK with no CUDA call)
     assert lib.lora_sgmv_apply_flags(None, None, None, None, None, None, 0, 4, 8, 256, 16, 256, 1.0, 0, 0, None, 0,
                                      None, 0, sgmv.FLAG_EARLY_READS, None) == 0
+
+
+def test_step_host_validation_codes_before_any_copy():
+    # every check of lora_sgmv_step_host returns before a copy or launch is enqueued
+    import ctypes
+    lib = sgmv.load()
+    ids = np.array([0, 2, 1, 2], np.int32)
+    meta = np.zeros(2 * 4 + 1, np.int32)
+    probs = (sgmv.Problem * 1)(sgmv.Problem(FAKE, FAKE, FAKE, FAKE, 4, 256, 512, 1.0))
+    cps = (sgmv.Copy * 1)(sgmv.Copy(FAKE, FAKE, 64))
+
+    def call(ids_p=ids.ctypes.data, T=4, na=4, mh=meta.ctypes.data, md=FAKE, h2d=ctypes.addressof(cps), nh=1,
+             pr=ctypes.addressof(probs), npr=1, d2h=ctypes.addressof(cps), nd=1):
+        return lib.lora_sgmv_step_host(ids_p, T, na, mh, md, None, h2d, nh, pr, npr, 16, 0, 0, d2h, nd, None, None,
+                                       None)
+
+    assert call(mh=None) == 1 and call(md=None) == 1 and call(pr=None) == 1 and call(ids_p=None) == 1
+    assert call(T=-1) == 2 and call(na=0) == 2 and call(npr=0) == 2 and call(npr=9) == 2
+    assert call(h2d=None) == 1 and call(d2h=None) == 1 and call(nh=-1) == 1
+    bad = (sgmv.Copy * 1)(sgmv.Copy(None, FAKE, 64))
+    assert call(h2d=ctypes.addressof(bad)) == 1
+    ids[1] = 4  # out of [0, num_adapters)
+    assert call() == 8
+    ids[1] = -1
+    assert call() == 8
+    assert not meta.any()  # nothing was written before the id check failed
