@@ -407,6 +407,52 @@ __device__ __forceinline__ bool job_at(const FusedParams& P, int p, int s, int q
     return job_check<CH>(P, p, s, q, c, job) == 0u;
 }
 
+// One-chunk mode, producer warp: the first chunk of segment s of problem p as a job, with the
+// segment's metadata fetched by the lanes in parallel (its bounds and adapter id, and, when the
+// problem has at most 32 adapters, every entry of both pointer tables), so the adapter's address
+// is known after one round trip instead of three dependent ones. The checks are load_segment's.
+// Returns the segment's chunks; 0 when it is empty or fails a check (the job is then not set).
+template <int CH = kFusedTokens>
+__device__ __forceinline__ int first_job_warp(const FusedParams& P, int p, int s, int c, int lane, Job& job) {
+    const FusedProblem& pr = P.prob[p];
+    int v = 0;
+    if (lane == 0)
+        v = __ldg(P.seg_starts + s);
+    else if (lane == 1)
+        v = __ldg(P.seg_starts + s + 1);
+    else if (lane == 2)
+        v = __ldg(P.lora_idx + s);
+    const bool whole_table = pr.num_adapters <= 32;
+    unsigned long long ta = 0, tb = 0;
+    if (whole_table && lane < pr.num_adapters) {
+        ta = __ldg(reinterpret_cast<const unsigned long long*>(pr.A_ptrs) + lane);
+        tb = __ldg(reinterpret_cast<const unsigned long long*>(pr.B_ptrs) + lane);
+    }
+    const int b = __shfl_sync(0xffffffffu, v, 0);
+    const int e = __shfl_sync(0xffffffffu, v, 1);
+    const int i = __shfl_sync(0xffffffffu, v, 2);
+    if (b < 0 || b > e || e > P.T || i < 0 || i >= pr.num_adapters) return 0;
+    unsigned long long a, bb;
+    if (whole_table) {
+        a = __shfl_sync(0xffffffffu, ta, i);
+        bb = __shfl_sync(0xffffffffu, tb, i);
+    } else {
+        a = __ldg(reinterpret_cast<const unsigned long long*>(pr.A_ptrs) + i);
+        bb = __ldg(reinterpret_cast<const unsigned long long*>(pr.B_ptrs) + i);
+    }
+    if (a == 0 || bb == 0 || ((a | bb) & 15u)) return 0;
+    job.p = p;
+    job.t0 = b;
+    job.nt = min(CH, e - b);
+    job.a = reinterpret_cast<const void*>(a);
+    job.b = reinterpret_cast<const void*>(bb);
+    job.k0 = c * pr.ks;
+    job.nk = max(0, min(pr.ks, pr.H1 - job.k0));
+    job.c0 = c * pr.ns;
+    job.nc = max(0, min(pr.ns, pr.H2 - job.c0));
+    return (e - b + CH - 1) / CH;
+}
+
 // A rejected segment is reported by the one thread that meets it first as a job (`reporter`:
 // one thread of the first CTA of the visiting cluster); a one-chunk-mode entry without chunks
 // may be a segment with invalid bounds.
@@ -726,9 +772,21 @@ __global__ void __launch_bounds__(kFusedThreads, SGMV_FUSED_MIN_BLOCKS) sgmv_fus
         uint32_t it = 0;
         bool waited = !P.early;
         for (int j = cluster_id; j < entries; j += n_clusters) {
-            int p, s, q0, nq;
-            entry_at<CH>(P, pref, j, p, s, q0, nq);
-            for (int q = q0; q < q0 + nq; ++q) {
+            int p, s, q_begin, q_end;
+            if (P.one_chunk) {
+                p = j / P.n_segments;
+                s = j - p * P.n_segments;
+                Job job;
+                q_end = first_job_warp<CH>(P, p, s, c, lane, job);
+                if (q_end > 0) produce_job<T, R, CH>(P, job, smem, full, empty, it, waited, lane, dead);
+                q_begin = 1;  // any further chunk (a longest-segment hint below the truth) as below
+            } else {
+                int q0, nq;
+                entry_at<CH>(P, pref, j, p, s, q0, nq);
+                q_begin = q0;
+                q_end = q0 + nq;
+            }
+            for (int q = q_begin; q < q_end; ++q) {
                 Job job;
                 if (!job_at<CH>(P, p, s, q, c, job)) break;
                 produce_job<T, R, CH>(P, job, smem, full, empty, it, waited, lane, dead);
