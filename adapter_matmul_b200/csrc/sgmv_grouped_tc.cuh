@@ -639,8 +639,10 @@ inline cudaError_t launch_grouped_tc_kernel(const CUtensorMap& tmX, const CUtens
     });
     if (attr_err != cudaSuccess) return attr_err;
     if (P.tm < 64 || P.tm > kGM || P.tm % 8 != 0) return cudaErrorInvalidValue;  // the X span assumes tm >= 64
-    sgmv_grouped_tc_kernel<T, R, V_OUT><<<blocks, kGThreads, grouped_smem_bytes(R, P.tm), stream>>>(tmX, tmY, tmA, tmB,
-                                                                                                    P);
+    // the V-only form has no expand: its second epilogue group would idle, so it is not launched
+    const int threads = V_OUT ? 32 * (2 + kGEpiWarps) : kGThreads;
+    sgmv_grouped_tc_kernel<T, R, V_OUT><<<blocks, threads, grouped_smem_bytes(R, P.tm), stream>>>(tmX, tmY, tmA, tmB,
+                                                                                                  P);
     return cudaGetLastError();
 }
 

@@ -224,14 +224,6 @@ __device__ __forceinline__ void shrink_chunk(const CUtensorMap* xmap, const Shri
     cluster.sync();  // partial tiles and the X slice may be overwritten only after every read
 }
 
-// Token chunks of segment s (0 for a segment the checks reject, whose reasons go to *bad).
-__device__ __forceinline__ int shrink_segment_chunks(const ShrinkParams& p, int s, uint32_t* bad) {
-    Segment seg;
-    *bad = load_segment(p.seg_starts, p.lora_idx, p.A_ptrs, p.B_check, s, p.T, p.num_adapters, seg);
-    if (*bad) return 0;
-    return (seg.end - seg.begin + kShrinkTokens - 1) / kShrinkTokens;
-}
-
 // Two grids. p.flat == 0: x = C (one cluster along x), y = segment slots, z = token-chunk
 // slots. p.flat == 1: x = C, y = slots over the flat list of (segment, chunk) units, z = 1;
 // every CTA builds the list's prefix (chunks before each segment) in shared memory, so the
@@ -279,13 +271,21 @@ __global__ void __launch_bounds__(kShrinkThreads, 3)
         const int per_thr = (n + NT - 1) / NT;
         const int s0 = min(n, tid * per_thr), s1 = min(n, s0 + per_thr);
         int local = 0;
-        // chunk counts, parked in the prefix slots; one CTA reports each rejected segment (while
-        // the list is built, not after the chunks, so that no CTA's end waits on it)
+        // chunk counts from the segment bounds alone (one round trip: the adapter id is read
+        // beside them and its table entries are only prefetched), parked in the prefix slots; one
+        // CTA reports each segment with invalid bounds while the list is built, and a segment
+        // whose adapter or pointers fail is reported and skipped where its first chunk runs
         const bool reporter = blockIdx.y == 0 && c == 0;
         for (int s = s0; s < s1; ++s) {
-            uint32_t bad;
-            const int k = shrink_segment_chunks(p, s, &bad);
-            if (reporter) report(p.dev_status, bad);
+            const int b = __ldg(p.seg_starts + s), e = __ldg(p.seg_starts + s + 1);
+            const int i = __ldg(p.lora_idx + s);
+            const bool ok = b >= 0 && b <= e && e <= p.T;
+            if (reporter && !ok) report(p.dev_status, LORA_SGMV_DEV_BAD_SEGMENT);
+            if (ok && i >= 0 && i < p.num_adapters) {
+                asm volatile("prefetch.global.L1 [%0];" ::"l"(p.A_ptrs + i));
+                if (p.B_check) asm volatile("prefetch.global.L1 [%0];" ::"l"(p.B_check + i));
+            }
+            const int k = ok ? (e - b + TC - 1) / TC : 0;
             pref[s + 1] = k;
             local += k;
         }
@@ -317,7 +317,12 @@ __global__ void __launch_bounds__(kShrinkThreads, 3)
                     hi = mid;
             }
             Segment seg;
-            load_segment(p.seg_starts, p.lora_idx, p.A_ptrs, p.B_check, lo, p.T, p.num_adapters, seg);
+            const uint32_t bad =
+                load_segment(p.seg_starts, p.lora_idx, p.A_ptrs, p.B_check, lo, p.T, p.num_adapters, seg);
+            if (bad) {  // uniform over the cluster: every CTA read the same words
+                if (c == 0 && tid == 0 && u == pref[lo]) report(p.dev_status, bad);
+                continue;
+            }
             const int t0 = seg.begin + (u - pref[lo]) * TC;
             run_chunk(static_cast<const T*>(seg.a), t0, min(TC, seg.end - t0));
         }
