@@ -278,13 +278,26 @@ lora_sgmv_status launch_grouped(void* Y, const void* X, const void* const* A_ptr
     const int sms_avail = std::max(1, f.sms - n_segments);
     int tm = static_cast<int>(std::min<long long>(sgmv::kGM, ((static_cast<long long>(T) + sms_avail - 1) / sms_avail + 7) / 8 * 8));
     tm = std::max(tm, 64);
+    // X and Y as 3-D views {64 columns, T rows, blocks of 64 columns} when the width is a
+    // multiple of 64, so that one copy brings two 64-column blocks; else row-major 2-D maps
+    const bool x3d = H1 % 64 == 0;
+    const bool y3d = !v_out && H2 % 64 == 0;
+    auto view3d = [&](CUtensorMap* m, const void* base, int cols) {
+        const uint64_t d[3] = {64, uint64_t(T), uint64_t(cols / 64)};
+        const uint64_t st[2] = {uint64_t(cols) * 2, 128};
+        const uint32_t b[3] = {64, uint32_t(tm), 2};
+        return sgmv::encode_map(m, base, dt, 3, d, st, b, CU_TENSOR_MAP_SWIZZLE_128B);
+    };
     CUtensorMap tmX, tmY;
-    if (!sgmv::make_tile_map(&tmX, X, T, H1, dt, tm) ||
-        !sgmv::make_tile_map(&tmY, v_out ? X : Y, T, v_out ? H1 : H2, dt, tm)) {  // (unused with v_out)
+    if (!(x3d ? view3d(&tmX, X, H1) : sgmv::make_tile_map(&tmX, X, T, H1, dt, tm)) ||
+        !(y3d ? view3d(&tmY, Y, H2)
+              : sgmv::make_tile_map(&tmY, v_out ? X : Y, T, v_out ? H1 : H2, dt, tm))) {  // (unused with v_out)
         t_last_error = cudaErrorInvalidValue;
         return LORA_SGMV_ERR_CUDA;
     }
     sgmv::GroupedParams P = {};
+    P.x3d = x3d ? 1 : 0;
+    P.y3d = y3d ? 1 : 0;
     P.Y = Y;
     P.A_ptrs = A_ptrs;
     P.B_ptrs = B_ptrs;
@@ -302,16 +315,23 @@ lora_sgmv_status launch_grouped(void* Y, const void* X, const void* const* A_ptr
     // templates of the A_i and B_i maps; each CTA replaces the address with its adapter's
     CUtensorMap tmA, tmB;
     {
+        // A_i boxes of r columns x 128 rows: both K-steps of a shrink stage in one copy
         const uint64_t da[2] = {uint64_t(r), uint64_t(H1)};
         const uint64_t sa[1] = {uint64_t(r) * 2};
-        const uint32_t ba[2] = {uint32_t(r), uint32_t(sgmv::kGK)};
+        const uint32_t ba[2] = {uint32_t(r), uint32_t(2 * sgmv::kGK)};
         const CUtensorMapSwizzle swa =
             r == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : (r == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
+        // B_i: {64 columns, r rows, blocks of 64 columns} with boxes of two blocks, or 2-D boxes
+        // of r rows x 64 columns
+        const uint64_t db3[3] = {64, uint64_t(r), uint64_t(H2 / 64)};
+        const uint64_t sb3[2] = {uint64_t(H2) * 2, 128};
+        const uint32_t bb3[3] = {64, uint32_t(r), 2};
         const uint64_t db[2] = {uint64_t(H2), uint64_t(r)};
         const uint64_t sb[1] = {uint64_t(H2) * 2};
         const uint32_t bb[2] = {64, uint32_t(r)};
         if (!sgmv::encode_map(&tmA, X, dt, 2, da, sa, ba, swa) ||
-            !sgmv::encode_map(&tmB, X, dt, 2, db, sb, bb, CU_TENSOR_MAP_SWIZZLE_128B)) {
+            !(y3d ? sgmv::encode_map(&tmB, X, dt, 3, db3, sb3, bb3, CU_TENSOR_MAP_SWIZZLE_128B)
+                  : sgmv::encode_map(&tmB, X, dt, 2, db, sb, bb, CU_TENSOR_MAP_SWIZZLE_128B))) {
             t_last_error = cudaErrorInvalidValue;
             return LORA_SGMV_ERR_CUDA;
         }

@@ -82,6 +82,8 @@ struct GroupedParams {
     int tm;      // rows per M-tile, 64..128, a multiple of 8 (the MMA's M stays 128; rows past tm are never used)
     float* v_out;  // V-only mode: V [T, r] fp32 written here, no expand
     const int32_t* ranks;  // rank of each adapter (device), or null: every adapter has rank R
+    int x3d;       // tmX is the 3-D view {64, T, H1/64} (H1 a multiple of 64), box {64, tm, 2}
+    int y3d;       // tmY {64, T, H2/64} and the B_i template {64, R, H2/64} are 3-D, boxes of 2 blocks
 };
 
 // Rank of the adapter of segment s when a rank table is given: 8 <= rank <= R, a multiple of 8
@@ -124,6 +126,7 @@ template <int R>
 struct GroupedGeom {
     static constexpr int A_BYTES = kGK * R * 2;
     static constexpr int A_SLOT = grouped_a_slot(R);
+    static_assert(A_SLOT == A_BYTES, "one 128-row copy of A_i lands as the stage's two K-step tiles");
     static constexpr int B_BYTES = R * kGN * 2;
     static constexpr int V_BYTES = kGM * R * 2;  // one of V_hi, V_lo
     // swizzle of an MN-major A_i tile (rows of R 16-bit values) and of K-major V rows
@@ -402,11 +405,16 @@ __global__ void __launch_bounds__(kGThreads, 1)
             unsigned char* xs = ring + size_t(st) * SB;
             const int nks = min(2, k_steps - 2 * ss);
             if (lane == 0) {
-                mbar_arrive_expect_tx(&full[st], uint32_t(nks) * (uint32_t(P.tm) * kGK * 2 + G::A_BYTES));
-                for (int h = 0; h < nks; ++h) {
-                    const int ks = 2 * ss + h;
-                    tma_load_2d(xs + h * BOX, &tmX, ks * kGK, t0, &full[st]);
-                    tma_load_2d(xs + 2 * BOX + h * G::A_SLOT, gA, 0, ks * kGK, &full[st]);
+                // A_i: one box of the stage's 128 rows (rows past H1 read as zeros); X: one 3-D box
+                // of both K-steps when the view allows it (blocks past H1/64 read as zeros), else
+                // one box per K-step
+                const uint32_t xb = uint32_t(P.x3d ? 2 : nks) * uint32_t(BOX);
+                mbar_arrive_expect_tx(&full[st], xb + 2u * G::A_BYTES);
+                tma_load_2d(xs + 2 * BOX, gA, 0, 2 * ss * kGK, &full[st]);
+                if (P.x3d) {
+                    tma_load_3d(xs, &tmX, 0, t0, 2 * ss, &full[st]);
+                } else {
+                    for (int h = 0; h < nks; ++h) tma_load_2d(xs + h * BOX, &tmX, (2 * ss + h) * kGK, t0, &full[st]);
                 }
             }
             __syncwarp();
@@ -419,10 +427,15 @@ __global__ void __launch_bounds__(kGThreads, 1)
             const int n0 = n_lo + nt * kGN;
             if (lane == 0) {
                 mbar_arrive_expect_tx(&full[st], 2u * P.tm * 64 * 2 + G::B_BYTES);
-                tma_load_2d(ys, &tmY, n0, t0, &full[st]);
-                tma_load_2d(ys + BOX, &tmY, n0 + 64, t0, &full[st]);
-                tma_load_2d(bs, gB, n0, 0, &full[st]);
-                tma_load_2d(bs + R * 128, gB, n0 + 64, 0, &full[st]);
+                if (P.y3d) {  // the N-tile's two 64-column blocks of Y and of B_i, one copy each
+                    tma_load_3d(ys, &tmY, 0, t0, n0 / 64, &full[st]);
+                    tma_load_3d(bs, gB, 0, 0, n0 / 64, &full[st]);
+                } else {
+                    tma_load_2d(ys, &tmY, n0, t0, &full[st]);
+                    tma_load_2d(ys + BOX, &tmY, n0 + 64, t0, &full[st]);
+                    tma_load_2d(bs, gB, n0, 0, &full[st]);
+                    tma_load_2d(bs + R * 128, gB, n0 + 64, 0, &full[st]);
+                }
             }
             __syncwarp();
         }
