@@ -71,21 +71,21 @@ PER_CONFIG_MAX_STEPS = 500
 # call of two launches (the split forms) the figure is the pair's.
 TRAFFIC = {
     # profiles/fused_kernel_distinct_decode.md
-    "distinct": {"bytes": 35721472,
+    "distinct": {"bytes": 35726848,
         "sources": ["sgmv_fused.cuh", "sgmv_common.cuh", "lora_sgmv_api.cu"],
-        "sha256": "c75727b99e65aad5eaf86614ba92741c19238003af87b656d7bfbc5676c5f0d1"},
+        "sha256": "b72ac89a6d8e011e06deab07c3c133bad172c3055a215e88d318d91293dce9c0"},
     # profiles/split_tc_llama70b_decode_h28672.md
-    "llama70b_decode_h28672": {"bytes": 489396992,
+    "llama70b_decode_h28672": {"bytes": 488363264,
         "sources": ["sgmv_split.cuh", "sgmv_decode_tc.cuh", "sgmv_grouped_tc.cuh", "sgmv_fused.cuh", "sgmv_tmap.cuh", "sgmv_common.cuh", "lora_sgmv_api.cu"],
-        "sha256": "f7220a666f350c3aefb70827ba5912fbf3de7d8457f1a6c1bb946c4cbf30d08a"},
+        "sha256": "a83197d89687a1795e1980576c3f9146964ee1da5d48e0f3d30c74ee23bd44c7"},
     # profiles/split_tc_llama70b_decode_h8192.md
-    "llama70b_decode_h8192": {"bytes": 216834304,
+    "llama70b_decode_h8192": {"bytes": 215355648,
         "sources": ["sgmv_split.cuh", "sgmv_decode_tc.cuh", "sgmv_grouped_tc.cuh", "sgmv_fused.cuh", "sgmv_tmap.cuh", "sgmv_common.cuh", "lora_sgmv_api.cu"],
-        "sha256": "f7220a666f350c3aefb70827ba5912fbf3de7d8457f1a6c1bb946c4cbf30d08a"},
+        "sha256": "a83197d89687a1795e1980576c3f9146964ee1da5d48e0f3d30c74ee23bd44c7"},
     # profiles/grouped_kernel_prefill.md
-    "prefill": {"bytes": 190224128,
+    "prefill": {"bytes": 190626048,
         "sources": ["sgmv_grouped_tc.cuh", "sgmv_fused.cuh", "sgmv_tmap.cuh", "sgmv_common.cuh", "lora_sgmv_api.cu"],
-        "sha256": "6b1175797d7915a676608b429a5a65442a18742c4b9603669442de2fbc5d4973"},
+        "sha256": "df93b527ca02b7f28efae49add3307fab29847fb686197f089f657234969e355"},
 }
 
 
