@@ -88,7 +88,6 @@ def test_host_step_equals_the_device_launch_and_repeats():
     torch.cuda.synchronize()
     dev = [from_dev(p.Y) for p in hb.probs]
     streams = [torch.cuda.Stream(), torch.cuda.Stream()]
-    first = None
     for i in range(4):
         s = streams[i % 2]
         hb.step.run(s)
@@ -96,8 +95,6 @@ def test_host_step_equals_the_device_launch_and_repeats():
         got = [hb.out(k) for k in range(len(hb.probs))]
         for k in range(len(got)):
             assert np.array_equal(got[k], dev[k]), f"step {i} problem {k} differs from the device launch"
-        if first is None:
-            first = got
     assert int(hb.status.item()) == 0 and int(p0.status.item()) == 0
 
 
@@ -110,3 +107,27 @@ def test_host_step_rejects_an_out_of_range_id_before_anything_runs():
         hb.step.run(torch.cuda.current_stream())
     torch.cuda.synchronize()
     assert np.array_equal(hb.outs[0].numpy(), before)
+
+
+def test_host_step_with_an_empty_batch_only_copies():
+    # T = 0: no segment and no launch; the copies still run in order
+    import ctypes
+    lib = sgmv.load()
+    meta = torch.empty(64, dtype=torch.int32, pin_memory=True)
+    dmeta = torch.zeros(64, dtype=torch.int32, device="cuda")
+    src = torch.arange(256, dtype=torch.uint8).pin_memory()
+    dst = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    back = torch.zeros(256, dtype=torch.uint8, pin_memory=True)
+    h2d = (sgmv.Copy * 1)(sgmv.Copy(src.data_ptr(), dst.data_ptr(), 256))
+    d2h = (sgmv.Copy * 1)(sgmv.Copy(dst.data_ptr(), back.data_ptr(), 256))
+    probs = (sgmv.Problem * 1)(sgmv.Problem(dst.data_ptr(), dst.data_ptr(), dmeta.data_ptr(), dmeta.data_ptr(), 4,
+                                            64, 64, 1.0))
+    n = ctypes.c_int32(-1)
+    s = torch.cuda.Stream()
+    st = lib.lora_sgmv_step_host(None, 0, 4, meta.data_ptr(), dmeta.data_ptr(), None, ctypes.addressof(h2d), 1,
+                                 ctypes.addressof(probs), 1, 16, sgmv.F16, 0, ctypes.addressof(d2h), 1, None,
+                                 ctypes.addressof(n), s.cuda_stream)
+    s.synchronize()
+    assert st == 0 and n.value == 0
+    assert int(meta[0]) == 0
+    assert torch.equal(back, src)

@@ -254,13 +254,16 @@ def test_large_h1_and_many_segments():
 
 @pytest.mark.parametrize("r", [16, 32, 64])
 @pytest.mark.parametrize("dtype", ["bf16", "f16"])
-def test_grouped_tc_ragged_tiles(r, dtype):
-    # segments shorter than, equal to and longer than the 128-row tile; H1 not a multiple of the
-    # 64-wide K step; H2 not a multiple of the 128-wide N tile; an empty segment; Y non-zero
+@pytest.mark.parametrize("H1,H2", [(328, 392), (320, 448)])
+def test_grouped_tc_ragged_tiles(r, dtype, H1, H2):
+    # segments shorter than, equal to and longer than the 128-row tile; an empty segment; Y
+    # non-zero. (328, 392): H1 not a multiple of the 64-wide K step, H2 not a multiple of the
+    # 128-wide N tile (row-major 2-D copies). (320, 448): odd numbers of 64-column blocks, so the
+    # last stage's 3-D copies of two blocks reach one block past H1 and past H2
     lens = [5, 128, 300, 0, 1, 129]
     seg = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
     idx = np.array([2, 0, 1, 3, 2, 4], np.int32)
-    w = inputs.small_random(int(seg[-1]), 5, 328, 392, r, dtype, seed=r)
+    w = inputs.small_random(int(seg[-1]), 5, H1, H2, r, dtype, seed=r)
     p = DeviceProblem(w, y_random=True, adapters=list(range(5)), seg_starts=seg, lora_idx=idx)
     got = p.apply(variant=sgmv.VARIANT_GROUPED_TC)
     assert int(p.status.item()) == 0
