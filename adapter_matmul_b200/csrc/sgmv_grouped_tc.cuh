@@ -378,6 +378,24 @@ __global__ void __launch_bounds__(kGThreads, 1)
         // r rows x 64 columns; columns of B_i past this CTA's slice are loaded but never stored
         CUtensorMap* gA = &g_map_tables[table_s].m[0];
         CUtensorMap* gB = &g_map_tables[table_s].m[1];
+        // the first stages' X tiles (through the host-made map) start before the adapter maps are
+        // made; their A_i halves follow once the maps are published
+        const int pre = min(NS, s_stages);
+        auto issue_x = [&](int ss, unsigned char* xs) {  // lane 0: expect the stage's bytes, copy X
+            const int nks = min(2, k_steps - 2 * ss);
+            // X: one 3-D box of both K-steps when the view allows it (blocks past H1/64 read as
+            // zeros), else one box per K-step; A_i (issued with the maps): one box of 128 rows
+            const uint32_t xb = uint32_t(P.x3d ? 2 : nks) * uint32_t(BOX);
+            mbar_arrive_expect_tx(&full[ss % NS], xb + 2u * G::A_BYTES);
+            if (P.x3d) {
+                tma_load_3d(xs, &tmX, 0, t0, 2 * ss, &full[ss % NS]);
+            } else {
+                for (int h = 0; h < nks; ++h) tma_load_2d(xs + h * BOX, &tmX, (2 * ss + h) * kGK, t0, &full[ss % NS]);
+            }
+        };
+        if (lane == 0)
+            for (int ss = 0; ss < pre; ++ss) issue_x(ss, ring + size_t(ss) * SB);
+        __syncwarp();
         map_template_to_smem(&map_build[0], &tmA);
         map_template_to_smem(&map_build[1], &tmB);
         if (lane == 0) {
@@ -403,19 +421,9 @@ __global__ void __launch_bounds__(kGThreads, 1)
             const uint32_t st = it % NS;
             if (it >= uint32_t(NS)) mbar_wait<false>(&empty[st], ((it / NS) - 1) & 1u, P.dev_status, dead);
             unsigned char* xs = ring + size_t(st) * SB;
-            const int nks = min(2, k_steps - 2 * ss);
             if (lane == 0) {
-                // A_i: one box of the stage's 128 rows (rows past H1 read as zeros); X: one 3-D box
-                // of both K-steps when the view allows it (blocks past H1/64 read as zeros), else
-                // one box per K-step
-                const uint32_t xb = uint32_t(P.x3d ? 2 : nks) * uint32_t(BOX);
-                mbar_arrive_expect_tx(&full[st], xb + 2u * G::A_BYTES);
-                tma_load_2d(xs + 2 * BOX, gA, 0, 2 * ss * kGK, &full[st]);
-                if (P.x3d) {
-                    tma_load_3d(xs, &tmX, 0, t0, 2 * ss, &full[st]);
-                } else {
-                    for (int h = 0; h < nks; ++h) tma_load_2d(xs + h * BOX, &tmX, (2 * ss + h) * kGK, t0, &full[st]);
-                }
+                if (ss >= pre) issue_x(ss, xs);
+                tma_load_2d(xs + 2 * BOX, gA, 0, 2 * ss * kGK, &full[st]);  // rows past H1 read as zeros
             }
             __syncwarp();
         }
