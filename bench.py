@@ -75,17 +75,17 @@ TRAFFIC = {
         "sources": ["sgmv_fused.cuh", "sgmv_common.cuh", "lora_sgmv_api.cu"],
         "sha256": "b72ac89a6d8e011e06deab07c3c133bad172c3055a215e88d318d91293dce9c0"},
     # profiles/split_tc_llama70b_decode_h28672.md
-    "llama70b_decode_h28672": {"bytes": 488363264,
+    "llama70b_decode_h28672": {"bytes": 488989184,
         "sources": ["sgmv_split.cuh", "sgmv_decode_tc.cuh", "sgmv_grouped_tc.cuh", "sgmv_fused.cuh", "sgmv_tmap.cuh", "sgmv_common.cuh", "lora_sgmv_api.cu"],
-        "sha256": "a83197d89687a1795e1980576c3f9146964ee1da5d48e0f3d30c74ee23bd44c7"},
+        "sha256": "6c0a82bc2a9540a24c4be59f5852d5ae96e1792dcbe4fbe4f346567ffe7a9df2"},
     # profiles/split_tc_llama70b_decode_h8192.md
-    "llama70b_decode_h8192": {"bytes": 215355648,
+    "llama70b_decode_h8192": {"bytes": 217230080,
         "sources": ["sgmv_split.cuh", "sgmv_decode_tc.cuh", "sgmv_grouped_tc.cuh", "sgmv_fused.cuh", "sgmv_tmap.cuh", "sgmv_common.cuh", "lora_sgmv_api.cu"],
-        "sha256": "a83197d89687a1795e1980576c3f9146964ee1da5d48e0f3d30c74ee23bd44c7"},
+        "sha256": "6c0a82bc2a9540a24c4be59f5852d5ae96e1792dcbe4fbe4f346567ffe7a9df2"},
     # profiles/grouped_kernel_prefill.md
-    "prefill": {"bytes": 190626048,
+    "prefill": {"bytes": 190149120,
         "sources": ["sgmv_grouped_tc.cuh", "sgmv_fused.cuh", "sgmv_tmap.cuh", "sgmv_common.cuh", "lora_sgmv_api.cu"],
-        "sha256": "df93b527ca02b7f28efae49add3307fab29847fb686197f089f657234969e355"},
+        "sha256": "9b9f31895d43aa41ef27ad13e9b2807746ff134a60d6af1d99cd1eef4554db6c"},
 }
 
 
